@@ -1,0 +1,150 @@
+"""Python front end of the fp64 CPU oracle (``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg are the only callers.  The product path never imports this
+module.  It shares no code with the CUDA library.
+
+``build()`` compiles ``oracle.c`` with gcc into ``liboracle.so`` beside it (on
+demand, when the library is missing or older than its source).  The functions
+take numpy arrays of any float dtype, widen them to float64 (exact for bf16
+and fp32 values) and return float64 results.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc if needed; return the library path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off", "-pthread", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_prefill.restype = ctypes.c_int
+            lib.oracle_prefill.argtypes = [
+                _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, _dp, _ip, ctypes.c_int, _dp, _dp, _dp, _ip,
+                ctypes.c_int, ctypes.c_int]
+            lib.oracle_decode.restype = ctypes.c_int
+            lib.oracle_decode.argtypes = [
+                _dp, _dp, _dp, _dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+            lib.oracle_feature_map.restype = None
+            lib.oracle_feature_map.argtypes = [_dp, ctypes.c_int, _dp]
+            lib.oracle_log_gate.restype = ctypes.c_double
+            lib.oracle_log_gate.argtypes = [_dp, ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, t=_dp):
+    return None if a is None else a.ctypes.data_as(t)
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def feature_map(x):
+    """Softmax over the last axis, row by row, through the oracle's C routine."""
+    lib = _load()
+    x = _f64(x)
+    d = x.shape[-1]
+    flat = x.reshape(-1, d)
+    y = np.empty_like(flat)
+    for i in range(flat.shape[0]):
+        row = np.ascontiguousarray(flat[i])
+        out = np.empty(d)
+        lib.oracle_feature_map(_ptr(row), d, _ptr(out))
+        y[i] = out
+    return y.reshape(x.shape)
+
+
+def log_gate(k):
+    """log sigmoid(mean over the last axis), row by row, through the C routine."""
+    lib = _load()
+    k = _f64(k)
+    d = k.shape[-1]
+    flat = k.reshape(-1, d)
+    res = np.array([lib.oracle_log_gate(_ptr(np.ascontiguousarray(r)), d) for r in flat])
+    return res.reshape(k.shape[:-1])
+
+
+def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_off=False,
+            nthreads=None):
+    """Token-by-token prefill.  Returns (out, final_state, ring, pos).
+
+    q [B, T, Hq, d]; k, v [B, T, Hkv, d]; cu_seqlens (optional, B == 1) lists
+    n_seqs + 1 offsets into T.  out [B, T, Hq, d], final_state [n, Hq, d, d],
+    ring [n, Hkv, 2, w, d], pos [n] int32.
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n = cu.shape[0] - 1
+    else:
+        cu = None
+        n = B
+    s0 = None if initial_state is None else _f64(initial_state)
+    out = np.zeros_like(q)
+    fs = np.zeros((n, Hq, d, d))
+    ring = np.zeros((n, Hkv, 2, w, d))
+    pos = np.zeros(n, dtype=np.int32)
+    rc = lib.oracle_prefill(
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, T, d, w, float(alpha), _ptr(s0),
+        _ptr(cu, _ip), n, _ptr(out), _ptr(fs), _ptr(ring), _ptr(pos, _ip), int(bool(gate_off)),
+        nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_prefill rejected its arguments")
+    return out, fs, ring, pos
+
+
+def decode(q, k, v, state, ring, pos, w=64, alpha=0.5, gate_off=False, nthreads=None):
+    """One decode step.  Returns (out, new_state, new_ring, new_pos); inputs are not modified."""
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    st = _f64(state).copy()
+    rg = _f64(ring).copy()
+    ps = np.ascontiguousarray(np.asarray(pos, dtype=np.int32)).copy()
+    out = np.zeros_like(q)
+    rc = lib.oracle_decode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(st), _ptr(rg), _ptr(out), _ptr(ps, _ip), B, Hq, Hkv, d, w,
+        float(alpha), int(bool(gate_off)), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    return out, st, rg, ps
