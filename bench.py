@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Benchmark of the Liger Attention forward pass on B200.
+
+Workload (Llama-3-8B attention shape, synthetic seeded N(0,1) data):
+  prefill: B=2, T=8192, Hq=32, Hkv=8, d=128, bf16, w=64, alpha=0.5, fp32 final state
+  decode:  B=64, Hq=32, Hkv=8, d=128 after a 1024-token prefill; steps captured in a CUDA graph
+
+One step = one prefill call over the whole batch (the headline `value`,
+tokens/s); the decode loop is timed in the same run and reported under
+"decode".  Inputs are larger than L2 (q, k, v 201 MB; decode states 268 MB),
+so no L2 flush is needed between iterations.  Multi-GPU: one process per GPU,
+every rank runs the same per-GPU workload (weak scaling, no collective on the
+data path); times are the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_linear_attention_liger_b200 import inputs  # noqa: E402
+
+METRIC = "prefill tokens/s & decode tokens/s (8B attn shape), % of roofline"
+PREFILL = inputs.WORKLOADS["llama8b_prefill"]
+DECODE = inputs.WORKLOADS["llama8b_decode"]
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def prefill_algorithmic(wl=PREFILL):
+    """Algorithmic bytes and flops of one prefill call (read q, k, v once, write out and the
+    final state once; flops of readout, causal intra-chunk, state update and window)."""
+    tok = wl.B * wl.T
+    esz = 2 if wl.dtype == torch.bfloat16 else 4
+    bytes_ = tok * (2 * wl.Hq + 2 * wl.Hkv) * wl.d * esz + wl.n_seqs * wl.Hq * wl.d * wl.d * 4
+    C = 64
+    flops = tok * (wl.Hq * 2 * wl.d ** 2 + wl.Hq * 4 * wl.d * (C + 1) / 2 + wl.Hkv * 2 * wl.d ** 2
+                   + wl.Hq * 4 * wl.w * wl.d)
+    return bytes_, flops
+
+
+def decode_algorithmic(wl=DECODE):
+    """Bytes of one decode step: state read + write, window ring read, q/k/v read, out write."""
+    esz = 2
+    state = wl.B * wl.Hq * wl.d * wl.d * 4 * 2
+    ring = wl.B * wl.Hkv * 2 * wl.w * wl.d * esz
+    io = wl.B * (2 * wl.Hq + 2 * wl.Hkv) * wl.d * esz
+    return state + ring + io
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                clk = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((time.perf_counter(), clk, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self._t.join(timeout=2)
+
+    def summary(self, windows):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        sel = [s for s in self.samples if any(a <= s[0] <= b for a, b in windows)]
+        if not sel:  # regions shorter than the sampling period: take the nearest samples
+            mids = [(a + b) / 2 for a, b in windows]
+            sel = [min(self.samples, key=lambda s: abs(s[0] - m)) for m in mids] if self.samples else []
+        reasons = set()
+        for _, _, rs in sel:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in sel]) if sel else None,
+                "sm_max_mhz": self.sm_max, "reasons": sorted(reasons), "samples": len(sel)}
+
+
+# ----------------------------------------------------------------- dist
+
+def timing_events(n, stream):
+    """n timing events whose CUDA handles exist (torch creates them at first record), so the
+    library can record them by handle."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record(stream)
+    return evs
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(target_s: float):
+    """Times the fp64 oracle on a bounded sample of the prefill workload and returns
+    (workload tokens/s, seconds, sample description, threads).  The sample is the first T_s
+    tokens of every sequence, all q heads, with T_s sized by a short calibration so the run
+    takes about target_s; if the whole workload fits in that time it is run whole, repeated
+    until target_s has passed."""
+    from oracle import oracle
+    wl = PREFILL
+    q, k, v = inputs.prefill_inputs(wl)
+    q, k, v = (t.float().numpy().astype(np.float64) for t in (q, k, v))
+    nthr = min(cpu_threads(), wl.B * wl.Hq)
+    t_cal = 128
+    t0 = time.perf_counter()
+    oracle.prefill(q[:, :t_cal], k[:, :t_cal], v[:, :t_cal], w=wl.w, alpha=wl.alpha, nthreads=nthr)
+    dt = time.perf_counter() - t0
+    T_s = int(min(wl.T, max(t_cal, t_cal * target_s / max(dt, 1e-6))))
+    reps, secs = 0, 0.0
+    while reps == 0 or secs < target_s:
+        t0 = time.perf_counter()
+        oracle.prefill(q[:, :T_s], k[:, :T_s], v[:, :T_s], w=wl.w, alpha=wl.alpha, nthreads=nthr)
+        secs += time.perf_counter() - t0
+        reps += 1
+    tokens = wl.B * T_s * reps
+    desc = (f"fp64 oracle, all {wl.B} sequences x {wl.Hq} q heads, first {T_s} of {wl.T} tokens, "
+            f"run {reps}x ({tokens} workload tokens in {secs:.1f} s), {nthr} threads")
+    return tokens / secs, secs, desc, nthr
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle as it stands, on host cores, rank 0 only."""
+    if rank != 0:
+        return
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    vals = []
+    desc = ""
+    nthr = cpu_threads()
+    for i in range(args.warmup + args.steps):
+        tps, secs, desc, nthr = oracle_prefill_sample(per_step)
+        if i >= args.warmup:
+            vals.append(tps)
+    value = float(statistics.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": PREFILL.tokens / value * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1))", "config": workload_config(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config():
+    p, d = PREFILL, DECODE
+    return {"workload": "llama8b_prefill (+ llama8b_decode)",
+            "prefill": {"B": p.B, "T": p.T, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d, "w": p.w,
+                        "alpha": p.alpha},
+            "decode": {"B": d.B, "prefix": d.T, "Hq": d.Hq, "Hkv": d.Hkv, "d": d.d, "w": d.w,
+                       "alpha": d.alpha},
+            "l2": "inputs larger than L2 (prefill q+k+v 201 MB, decode states 268 MB > 126 MB)"}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_ours(args, world, rank, local):
+    from gated_linear_attention_liger_b200 import ops
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ops.load()
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    sampler = ClockSampler(local).start()
+    windows = []
+
+    # ---------------- prefill
+    wl = PREFILL
+    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
+    out = torch.empty_like(q)
+    fs = torch.empty(wl.n_seqs, wl.Hq, wl.d, wl.d, device=dev, dtype=torch.float32)
+    ws_n = ops.prefill_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.n_seqs)
+    ws = torch.empty(max(ws_n, 1), device=dev, dtype=torch.uint8)
+
+    def prefill_call():
+        ops.prefill(q, k, v, alpha=wl.alpha, w=wl.w, out=out, final_state=fs, workspace=ws,
+                    stream=stream)
+
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        prefill_call()
+    ks = timing_events(args.steps, stream)
+    ke = timing_events(args.steps, stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = ops.kernel_launches()
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ops.set_timing_events(ks[i], ke[i])
+        prefill_call()
+    t_end.record(stream)
+    ops.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    prefill_launches = ops.kernel_launches() - launches0
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    ms_step = ms_total / args.steps
+    k_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ks, ke)), world, dev)
+    value = world * wl.tokens / (ms_step * 1e-3)
+    alg_bytes, alg_flops = prefill_algorithmic(wl)
+    achieved = alg_bytes / (k_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "kernel": "prefill chunk pass", "kernel_ms": k_ms,
+                "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+                "tensor_frac": alg_flops / (k_ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
+                "peak_source": pk["source"], "frac_of": f"{pk['source']} HBM copy bandwidth"}
+    traffic = os.environ.get("LIGER_PREFILL_TRAFFIC_BYTES")
+    if traffic:
+        roofline["traffic"] = float(traffic)
+
+    # ---------------- e2e: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hfs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        n_e2e = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                q.copy_(hq, non_blocking=True)
+                k.copy_(hk, non_blocking=True)
+                v.copy_(hv, non_blocking=True)
+            prefill_call()
+            with torch.cuda.stream(stream):
+                ho.copy_(out, non_blocking=True)
+                hfs.copy_(fs, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world, dev)
+        e2e = {"value": world * wl.tokens / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hfs.numel() * hfs.element_size(),
+               "ms_per_step": e_ms, "steps": n_e2e}
+        del hq, hk, hv, ho, hfs
+    del q, k, v, out, ws
+
+    # ---------------- decode
+    dec = run_decode(args, world, dev, stream, pk, windows)
+
+    sampler.stop()
+    clocks = sampler.summary(windows)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, secs, desc, nthr = oracle_prefill_sample(args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": nthr, "kind": "oracle", "sample": desc,
+               "seconds": secs}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1), Llama-3-8B attention shapes)",
+            "config": workload_config(), "roofline": roofline, "decode": dec, "e2e": e2e,
+            "gpu_launches": prefill_launches, "clocks": clocks, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, world, dev, stream, pk, windows):
+    from gated_linear_attention_liger_b200 import ops
+    wl = DECODE
+    n_graph = args.decode_steps
+    # state, ring and pos from a seeded 1024-token prefill through the library
+    pre = inputs.Workload("decode_prefix", "prefill", wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.dtype,
+                          seed=wl.seed)
+    pq, pkk, pv = (t.to(dev) for t in inputs.prefill_inputs(pre))
+    _, state, ring, pos = ops.prefill(pq, pkk, pv, alpha=wl.alpha, w=wl.w, return_ring=True,
+                                      stream=stream)
+    stream.synchronize()
+    del pq, pkk, pv
+    steps_in = [inputs.decode_step_inputs(wl, s) for s in range(n_graph)]
+    dq = torch.stack([s[0] for s in steps_in]).to(dev)
+    dk = torch.stack([s[1] for s in steps_in]).to(dev)
+    dv = torch.stack([s[2] for s in steps_in]).to(dev)
+    dout = torch.empty_like(dq)
+    ks = timing_events(n_graph, stream)
+    ke = timing_events(n_graph, stream)
+
+    def steps(timed):
+        for s in range(n_graph):
+            if timed:
+                ops.set_timing_events(ks[s], ke[s])
+            ops.decode(dq[s], dk[s], dv[s], state, ring, pos, alpha=wl.alpha, out=dout[s], stream=stream)
+        ops.set_timing_events(None, None)
+
+    steps(False)  # warm-up outside the graph
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    l0 = ops.kernel_launches()
+    kernel_events = True
+    try:
+        with torch.cuda.graph(graph, stream=stream):
+            steps(True)
+    except Exception:
+        kernel_events = False
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            steps(False)
+    per_graph_launches = ops.kernel_launches() - l0
+    for _ in range(max(1, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.steps // 10)
+    w0 = time.perf_counter()
+    k_ms = []
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+            if kernel_events:
+                stream.synchronize()
+                try:
+                    k_ms.append(statistics.mean(x.elapsed_time(y) for x, y in zip(ks, ke)))
+                except (RuntimeError, ValueError):
+                    kernel_events = False
+        b.record(stream)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    ms_step = max_over_ranks(a.elapsed_time(b) / (reps * n_graph), world, dev)
+    kms = max_over_ranks(statistics.mean(k_ms), world, dev) if (kernel_events and k_ms) else ms_step
+    alg = decode_algorithmic(wl)
+    achieved = alg / (kms * 1e-3) / 1e9
+    del graph
+    return {"metric": "decode tokens/s (8B attn shape, B=64)", "value": world * wl.B / (ms_step * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms_step, "graph_steps": n_graph, "replays": reps,
+            "gpu_launches": per_graph_launches * reps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "kernel": "decode state stream", "kernel_ms": kms,
+                         "kernel_timing": "events in graph" if kernel_events else "graph step average",
+                         "algorithmic_bytes": alg, "peak_source": pk["source"]}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=200, help="decode steps per captured graph")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: warm-up raised to 3", file=sys.stderr)
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

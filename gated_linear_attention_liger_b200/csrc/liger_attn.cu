@@ -1,0 +1,213 @@
+// liger_attn.cu -- the C ABI (include/liger_attn.h): argument checks, path
+// selection and kernel launches on the caller's stream.  No allocation, no
+// host synchronisation.
+#include "liger_attn.h"
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
+thread_local uint64_t g_launches = 0;
+
+// Bracket the dominant kernel of a call with the caller's timing events.
+void mark_start(cudaStream_t s) { if (g_ev_start) cudaEventRecord(g_ev_start, s); }
+void mark_stop(cudaStream_t s) { if (g_ev_stop) cudaEventRecord(g_ev_stop, s); }
+
+liger_status fail(liger_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+liger_status cuda_check(const char* where) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(LIGER_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+  return LIGER_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Which prefill kernel serves a call.
+enum class PrefillPath { kSimt, kTensorCore };
+
+PrefillPath choose_prefill_path(int Hq, int Hkv, int d, int w, liger_dtype dt,
+                                const float* initial_state) {
+  const char* force = std::getenv("LIGER_PREFILL_PATH");
+  if (force && std::strcmp(force, "simt") == 0) return PrefillPath::kSimt;
+  if (dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && initial_state == nullptr &&
+      liger::tc::supports(d))
+    return PrefillPath::kTensorCore;
+  return PrefillPath::kSimt;
+}
+
+liger_status check_common(int Hq, int Hkv, int d, int w, float alpha, liger_dtype dt) {
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(LIGER_ERR_INVALID_ARG, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (w < 1) return fail(LIGER_ERR_INVALID_ARG, "window w must be >= 1 (w=%d)", w);
+  if (!(alpha >= 0.f && alpha <= 1.f))
+    return fail(LIGER_ERR_INVALID_ARG, "alpha must lie in [0, 1] (alpha=%g)", (double)alpha);
+  if (dt != LIGER_BF16 && dt != LIGER_FP32) return fail(LIGER_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (d != 64 && d != 128) return fail(LIGER_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
+  if (w > 64) return fail(LIGER_ERR_UNSUPPORTED, "window w=%d (supported: 1..64)", w);
+  return LIGER_OK;
+}
+
+template <typename Tin, int D>
+liger_status launch_simt_prefill(const liger::SimtPrefillArgs& a, int n_seqs, cudaStream_t s) {
+  const size_t smem = liger::simt_prefill_smem_bytes<D>();
+  auto kern = liger::prefill_simt_kernel<Tin, D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(prefill_simt)");
+  const long blocks = (long)n_seqs * a.Hq;
+  if (blocks > 0x7fffffffL) return fail(LIGER_ERR_UNSUPPORTED, "too many (sequence, head) units");
+  mark_start(s);
+  kern<<<(unsigned)blocks, liger::kSimtThreads, smem, s>>>(a);
+  mark_stop(s);
+  ++g_launches;
+  return cuda_check("prefill_simt launch");
+}
+
+template <typename Tin>
+liger_status launch_ring(const void* k, const void* v, void* ring, int32_t* pos, const int32_t* cu,
+                         long T, int n_seqs, int Hkv, int d, int w, cudaStream_t s) {
+  if (!ring && !pos) return LIGER_OK;
+  dim3 grid((unsigned)n_seqs, (unsigned)Hkv);
+  liger::prefill_ring_kernel<Tin><<<grid, 256, 0, s>>>(
+      static_cast<const Tin*>(k), static_cast<const Tin*>(v), static_cast<Tin*>(ring), pos, cu, T,
+      Hkv, d, w);
+  ++g_launches;
+  return cuda_check("prefill_ring launch");
+}
+
+template <typename Tin>
+liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, cudaStream_t s) {
+  return d == 64 ? launch_simt_prefill<Tin, 64>(a, n_seqs, s) : launch_simt_prefill<Tin, 128>(a, n_seqs, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int liger_abi_version(void) { return LIGER_ABI_VERSION; }
+
+const char* liger_last_error(void) { return g_last_error.c_str(); }
+
+void liger_set_timing_events(void* start_event, void* stop_event) {
+  g_ev_start = static_cast<cudaEvent_t>(start_event);
+  g_ev_stop = static_cast<cudaEvent_t>(stop_event);
+}
+
+uint64_t liger_kernel_launches(void) { return g_launches; }
+
+size_t liger_attn_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                         liger_dtype dt) {
+  if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return 0;
+  if (dt != LIGER_BF16 || (d != 64 && d != 128) || (Hq / Hkv) % 2) return 0;
+  const int n = n_seqs > 0 ? n_seqs : B;
+  return liger::tc::workspace_bytes(B, Hq, Hkv, (long)T, d, n);
+}
+
+liger_status liger_attn_prefill(const void* q, const void* k, const void* v, void* out,
+                                float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
+                                float alpha, liger_dtype dt, const float* initial_state,
+                                const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
+                                int32_t* pos_out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  g_last_error.clear();
+  liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
+  if (st != LIGER_OK) return st;
+  if (B < 1 || T < 0) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 and T >= 0 (B=%d T=%d)", B, T);
+  if (cu_seqlens) {
+    if (B != 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (B=%d)", B);
+    if (n_seqs < 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires n_seqs >= 1 (n_seqs=%d)", n_seqs);
+  } else if (n_seqs != B) {
+    return fail(LIGER_ERR_INVALID_ARG, "without cu_seqlens n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
+  }
+  const long ntok = (long)B * T;
+  if ((long)T * B * Hq > (1L << 40) / d) return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
+  if (ntok > 0 && (!q || !k || !v || !out))
+    return fail(LIGER_ERR_INVALID_ARG, "q, k, v and out must be non-null");
+  const void* ptrs[] = {q, k, v, out, final_state, initial_state, swa_ring_out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+  if (pos_out && (reinterpret_cast<uintptr_t>(pos_out) & 3u))
+    return fail(LIGER_ERR_INVALID_ARG, "pos_out must be 4-byte aligned");
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const PrefillPath path = choose_prefill_path(Hq, Hkv, d, w, dt, initial_state);
+  if (path == PrefillPath::kTensorCore) {
+    const size_t need = liger::tc::workspace_bytes(B, Hq, Hkv, (long)T, d, n_seqs);
+    if (need > workspace_bytes || (need && !workspace))
+      return fail(LIGER_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, workspace_bytes);
+    liger::tc::PrefillProblem pb{q, k, v, out, final_state, cu_seqlens, B, Hq, Hkv, (long)T, d, n_seqs, alpha};
+    st = liger::tc::run_prefill(pb, workspace, s);
+    if (st != LIGER_OK) return fail(st, "%s", liger::tc::last_message());
+  } else {
+    liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha};
+    st = dt == LIGER_BF16 ? prefill_simt_dispatch<__nv_bfloat16>(a, d, n_seqs, s)
+                          : prefill_simt_dispatch<float>(a, d, n_seqs, s);
+    if (st != LIGER_OK) return st;
+  }
+  if (dt == LIGER_BF16)
+    return launch_ring<__nv_bfloat16>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
+  return launch_ring<float>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
+}
+
+liger_status liger_attn_decode(const void* q, const void* k, const void* v, float* state,
+                               void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                               int d, int w, float alpha, liger_dtype dt, void* stream) {
+  g_last_error.clear();
+  liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
+  if (st != LIGER_OK) return st;
+  if (B < 1) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 (B=%d)", B);
+  if ((long)B * Hq > 0x7fffffffL) return fail(LIGER_ERR_UNSUPPORTED, "too many (sequence, head) units");
+  if (!q || !k || !v || !state || !swa_ring || !out || !pos)
+    return fail(LIGER_ERR_INVALID_ARG, "all decode pointers must be non-null");
+  const void* ptrs[] = {q, k, v, state, swa_ring, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(pos) & 3u) return fail(LIGER_ERR_INVALID_ARG, "pos must be 4-byte aligned");
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha};
+  const unsigned blocks = (unsigned)((long)B * Hq);
+  mark_start(s);
+  if (dt == LIGER_BF16) {
+    if (d == 64) liger::decode_kernel<__nv_bfloat16, 64><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
+    else liger::decode_kernel<__nv_bfloat16, 128><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
+  } else {
+    if (d == 64) liger::decode_kernel<float, 64><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
+    else liger::decode_kernel<float, 128><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
+  }
+  mark_stop(s);
+  ++g_launches;
+  st = cuda_check("decode launch");
+  if (st != LIGER_OK) return st;
+  liger::advance_pos_kernel<<<(B + 255) / 256, 256, 0, s>>>(pos, B);
+  ++g_launches;
+  return cuda_check("advance_pos launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,171 @@
+"""ctypes binding of ``libliger_attn.so`` (C ABI in ``include/liger_attn.h``).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+library.  PyTorch supplies device memory and streams.  The library is loaded
+on first use; if it is missing this raises (there is no CPU fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libliger_attn.so")
+
+LIGER_OK, LIGER_ERR_INVALID_ARG, LIGER_ERR_UNSUPPORTED, LIGER_ERR_CUDA, LIGER_ERR_TIMEOUT = range(5)
+LIGER_BF16, LIGER_FP32 = 0, 1
+STATUS_NAMES = {0: "LIGER_OK", 1: "LIGER_ERR_INVALID_ARG", 2: "LIGER_ERR_UNSUPPORTED",
+                3: "LIGER_ERR_CUDA", 4: "LIGER_ERR_TIMEOUT"}
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_lock = threading.Lock()
+_lib = None
+
+# Entry points and their C signatures (restype, argtypes), as declared in the header.
+SIGNATURES = {
+    "liger_abi_version": (_i, []),
+    "liger_last_error": (ctypes.c_char_p, []),
+    "liger_attn_prefill_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
+    "liger_attn_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _i,
+                                _vp, _vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "liger_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
+                               _i, _vp]),
+    "liger_set_timing_events": (None, [_vp, _vp]),
+    "liger_kernel_launches": (ctypes.c_uint64, []),
+}
+
+
+class LigerError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def load(path: Optional[str] = None):
+    """Load the CUDA library (raises FileNotFoundError if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or LIB_PATH
+            if not os.path.exists(p):
+                raise FileNotFoundError(
+                    f"{p} is missing: build it with `python -m gated_linear_attention_liger_b200.build`"
+                    " (the Liger Attention ops have no CPU fallback)")
+            lib = ctypes.CDLL(p)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def set_timing_events(start=None, stop=None):
+    """Bracket the dominant kernel of later calls (this thread) with two torch.cuda.Events."""
+    load().liger_set_timing_events(None if start is None else ctypes.c_void_p(start.cuda_event),
+                                   None if stop is None else ctypes.c_void_p(stop.cuda_event))
+
+
+def kernel_launches() -> int:
+    """Kernels this thread has launched through the library so far."""
+    return int(load().liger_kernel_launches())
+
+
+def last_error() -> str:
+    return load().liger_last_error().decode()
+
+
+def _check(status: int):
+    if status != LIGER_OK:
+        raise LigerError(status, last_error())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LIGER_BF16
+    if t.dtype == torch.float32:
+        return LIGER_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def prefill_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:
+    return int(load().liger_attn_prefill_workspace_size(
+        B, Hq, Hkv, T, d, n_seqs, LIGER_BF16 if dtype == torch.bfloat16 else LIGER_FP32))
+
+
+def prefill(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seqlens=None,
+            return_ring: bool = False, out=None, final_state=None, ring=None, pos=None,
+            workspace=None, want_final_state: bool = True, stream=None):
+    """Liger Attention prefill.
+
+    q [B, T, Hq, d], k and v [B, T, Hkv, d] (bf16 or fp32, CUDA).  Returns
+    (out, final_state) or, with return_ring, (out, final_state, ring, pos).
+    cu_seqlens: int32 CUDA tensor of n+1 offsets (B must be 1).
+    """
+    lib = load()
+    _need_cuda(q, k, v, initial_state, cu_seqlens)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if final_state is None and want_final_state:
+        final_state = torch.empty(n, Hq, d, d, device=dev, dtype=torch.float32)
+    if return_ring:
+        if ring is None:
+            ring = torch.empty(n, Hkv, 2, w, d, device=dev, dtype=q.dtype)
+        if pos is None:
+            pos = torch.empty(n, device=dev, dtype=torch.int32)
+    need = prefill_workspace_size(B, Hq, Hkv, T, d, n, q.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.liger_attn_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(final_state), B, Hq, Hkv, T, d, w,
+        float(alpha), _dt(q), _ptr(initial_state), _ptr(cu_seqlens), n, _ptr(ring), _ptr(pos),
+        _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check(st)
+    if return_ring:
+        return out, final_state, ring, pos
+    return out, final_state
+
+
+def decode(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None):
+    """One Liger Attention decode step; updates state, ring and pos in place.
+
+    q [B, Hq, d], k and v [B, Hkv, d]; state [B, Hq, d, d] fp32; ring
+    [B, Hkv, 2, w, d]; pos [B] int32.  Returns out [B, Hq, d].
+    """
+    lib = load()
+    _need_cuda(q, k, v, state, ring, pos)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    w = ring.shape[3]
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib.liger_attn_decode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos), B, Hq, Hkv, d, w,
+        float(alpha), _dt(q), _stream_ptr(stream))
+    _check(st)
+    return out

@@ -1,0 +1,149 @@
+/*
+ * liger_attn.h -- C ABI of the Liger Attention forward pass for NVIDIA B200
+ * (sm_100a).  Built into libliger_attn.so.
+ *
+ * The operation.  Liger Attention ("Liger: Linearizing Large Language Models
+ * to Gated Recurrent Structures", Paper-Notes page, sections
+ * "核心思想：Key 投影复用构建门控", "统一的门控线性循环框架" and
+ * "Liger Attention：层内混合注意力"; news article on Liger, section
+ * "手法の説明") mixes, per query head h with key/value head kv = h / (Hq/Hkv):
+ *
+ *   gated recurrent branch (GRM):
+ *     g_t   = sigmoid(mean_d k_t)                 (pooled key gate, kept as log g)
+ *     phi() = softmax over the head dimension d   (applied to q_t and to k_t)
+ *     S_t   = g_t * S_{t-1} + phi(k_t)^T v_t      (d x d, row = key dim, col = value dim)
+ *     grm_t = phi(q_t) S_t                        (state updated before it is read)
+ *   sliding-window branch (SWA), window w (64 on the pages):
+ *     swa_t = sum_{j=t-w+1..t} softmax_j(q_t . k_j / sqrt(d)) v_j   (self included)
+ *   output:
+ *     o_t   = alpha * grm_t + (1 - alpha) * swa_t
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned.  The library never allocates device memory
+ *     and never synchronizes the host; it enqueues kernels on `stream` (a
+ *     cudaStream_t, NULL = legacy default stream) and returns.
+ *   - Errors: a bad argument returns LIGER_ERR_INVALID_ARG, a legal but
+ *     unimplemented combination LIGER_ERR_UNSUPPORTED, a failed CUDA call
+ *     LIGER_ERR_CUDA; nothing is launched in those cases (for LIGER_ERR_CUDA,
+ *     launches made before the failing call stay enqueued).  The message of the
+ *     last failure on the calling thread is returned by liger_last_error().
+ *   - No C++ exception crosses the ABI; calls from several host threads are
+ *     safe as long as they do not share output buffers.
+ *   - dt is the storage type of q, k, v, out and the window ring.  The
+ *     recurrent state is always fp32.  Arithmetic is fp32 (bf16 tensor-core
+ *     operands with fp32 accumulation on the bf16 prefill path).
+ *   - Supported: d in {64, 128}; 1 <= w <= 64 (the bf16 tensor-core prefill
+ *     needs w == 64 and an even Hq/Hkv and falls back to the general kernel
+ *     otherwise); Hq % Hkv == 0; 0 <= alpha <= 1.
+ */
+#ifndef LIGER_ATTN_H
+#define LIGER_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LIGER_OK = 0,
+  LIGER_ERR_INVALID_ARG = 1,
+  LIGER_ERR_UNSUPPORTED = 2,
+  LIGER_ERR_CUDA = 3,
+  LIGER_ERR_TIMEOUT = 4
+} liger_status;
+
+typedef enum { LIGER_BF16 = 0, LIGER_FP32 = 1 } liger_dtype;
+
+/* ABI version of this header (bumped on any signature change). */
+#define LIGER_ABI_VERSION 1
+int liger_abi_version(void);
+
+/*
+ * Bytes of device workspace liger_attn_prefill needs for these sizes
+ * (0 is a valid answer).  T is the tokens per sequence, or the packed total
+ * when cu_seqlens is used (then B == 1 and n_seqs is the number of sequences;
+ * otherwise pass n_seqs = B).  Returns 0 for sizes the prefill would reject.
+ */
+size_t liger_attn_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                         liger_dtype dt);
+
+/*
+ * Prefill: runs the recurrence and the window over whole sequences.
+ * Sources: the recurrence and the hybrid above (Paper-Notes page, sections
+ * 统一的门控线性循环框架 and Liger Attention); the parallel-in-chunk,
+ * recurrent-across-chunk evaluation is the reordering the news article's
+ * section "軽量ファインチューニング" credits for the linear cost.
+ *
+ *   q            [B, T, Hq, d]  dt          (in)
+ *   k, v         [B, T, Hkv, d] dt          (in)
+ *   out          [B, T, Hq, d]  dt          (out)
+ *   final_state  [n, Hq, d, d]  fp32        (out, nullable) state after the last
+ *                token of each sequence; every q head of a group gets its copy.
+ *   initial_state[n, Hq, d, d]  fp32        (in, nullable = zero) seeds the
+ *                recurrence; the window still starts at the first token.
+ *   cu_seqlens   [n + 1]        int32       (in, nullable) packed variable-length
+ *                sequences: offsets into the T axis, first 0, last T, non-
+ *                decreasing; requires B == 1.  The state and the window restart
+ *                at each sequence start.  Without it, n = B sequences of T.
+ *   swa_ring_out [n, Hkv, 2, w, d] dt       (out, nullable) window ring for decode:
+ *                [., ., 0] keys, [., ., 1] values; position p of a sequence at
+ *                slot p mod w for its last min(len, w) positions, zeros elsewhere.
+ *   pos_out      [n]            int32       (out, nullable) sequence lengths.
+ *   workspace    device scratch of at least liger_attn_prefill_workspace_size()
+ *                bytes (nullable when that size is 0); contents on entry are
+ *                ignored; the caller must not touch it until the call's work
+ *                on `stream` is done.
+ */
+liger_status liger_attn_prefill(const void* q, const void* k, const void* v, void* out,
+                                float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
+                                float alpha, liger_dtype dt, const float* initial_state,
+                                const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
+                                int32_t* pos_out, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
+ * Decode: one new token for each of B independent sequences.
+ * Source: the same recurrence and hybrid, stepped once; the constant-size
+ * state replacing the growing key/value cache is the linear-time,
+ * constant-memory decoding both Liger pages describe (news article,
+ * introduction and section "実験分析"; Paper-Notes page, section "亮点与洞察").
+ *
+ *   q            [B, Hq, d]        dt    (in)
+ *   k, v         [B, Hkv, d]       dt    (in)
+ *   state        [B, Hq, d, d]     fp32  (in/out) each q head's state is
+ *                updated independently: S <- g S + phi(k)^T v.
+ *   swa_ring     [B, Hkv, 2, w, d] dt    (in/out) the new key and value are
+ *                written at slot pos mod w.
+ *   out          [B, Hq, d]        dt    (out)
+ *   pos          [B]               int32 (in/out) tokens seen so far; +1 per call.
+ *                The window of the new token covers positions
+ *                max(0, pos - w + 1) .. pos; slots outside it are never read.
+ */
+liger_status liger_attn_decode(const void* q, const void* k, const void* v, float* state,
+                               void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                               int d, int w, float alpha, liger_dtype dt, void* stream);
+
+/* Message of the last failure on the calling thread ("" if none). */
+const char* liger_last_error(void);
+
+/*
+ * Measurement hooks (no counterpart on the pages; they serve the roofline
+ * measurement).  liger_set_timing_events(start, stop) takes two cudaEvent_t
+ * (or NULL, NULL to switch off); while set, every later prefill or decode call
+ * on the calling thread records `start` just before and `stop` just after its
+ * dominant kernel (the prefill's chunk pass, the decode's state stream) on the
+ * call's stream.  liger_kernel_launches() returns how many kernels the calling
+ * thread has launched through this library so far (launches captured into a
+ * CUDA graph are counted once, at capture).
+ */
+void liger_set_timing_events(void* start_event, void* stop_event);
+uint64_t liger_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGER_ATTN_H */

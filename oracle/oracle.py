@@ -112,6 +112,8 @@ def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != (B, T, Hkv, d):
+        raise ValueError("prefill: inconsistent shapes")
     if cu_seqlens is not None:
         cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
         n = cu.shape[0] - 1
@@ -119,6 +121,8 @@ def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_
         cu = None
         n = B
     s0 = None if initial_state is None else _f64(initial_state)
+    if s0 is not None and s0.shape != (n, Hq, d, d):
+        raise ValueError("prefill: initial_state must be [n, Hq, d, d]")
     out = np.zeros_like(q)
     fs = np.zeros((n, Hq, d, d))
     ring = np.zeros((n, Hkv, 2, w, d))
@@ -132,14 +136,24 @@ def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_
     return out, fs, ring, pos
 
 
-def decode(q, k, v, state, ring, pos, w=64, alpha=0.5, gate_off=False, nthreads=None):
-    """One decode step.  Returns (out, new_state, new_ring, new_pos); inputs are not modified."""
+def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthreads=None):
+    """One decode step.  Returns (out, new_state, new_ring, new_pos); inputs are not modified.
+
+    q [B, Hq, d]; k, v [B, Hkv, d]; state [B, Hq, d, d]; ring [B, Hkv, 2, w, d]; pos [B].
+    The window w is the ring's slot count (a w argument, if given, must agree).
+    """
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     st = _f64(state).copy()
     rg = _f64(ring).copy()
+    if w is not None and w != rg.shape[3]:
+        raise ValueError(f"w={w} but the ring has {rg.shape[3]} slots")
+    w = rg.shape[3]
+    if k.shape != (B, Hkv, d) or v.shape != (B, Hkv, d) or st.shape != (B, Hq, d, d) \
+            or rg.shape != (B, Hkv, 2, w, d) or np.asarray(pos).shape != (B,):
+        raise ValueError("decode: inconsistent shapes")
     ps = np.ascontiguousarray(np.asarray(pos, dtype=np.int32)).copy()
     out = np.zeros_like(q)
     rc = lib.oracle_decode(

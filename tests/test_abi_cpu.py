@@ -1,0 +1,115 @@
+"""The C-ABI library: builds for sm_100a, loads without a GPU, exports every
+symbol the header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_linear_attention_liger_b200 import build as libbuild
+from gated_linear_attention_liger_b200 import ops
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "liger_attn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)
+    keywords = {"if", "sizeof", "defined", "return"}
+    return sorted({n for n in names if n.startswith("liger_") and n not in keywords})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return ops.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("liger_attn_prefill", "liger_attn_decode", "liger_attn_prefill_workspace_size",
+                     "liger_last_error", "liger_abi_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in ops.SIGNATURES, f"binding lacks {name}"
+    assert lib.liger_abi_version() == 1
+
+
+def _prefill(lib, **kw):
+    a = dict(q=16, k=16, v=16, out=16, fs=None, B=1, Hq=4, Hkv=2, T=8, d=64, w=64, alpha=0.5, dt=0,
+             s0=None, cu=None, n=1, ring=None, pos=None, ws=None, wsb=0)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.liger_attn_prefill(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["out"]), vp(a["fs"]), a["B"],
+                                  a["Hq"], a["Hkv"], a["T"], a["d"], a["w"], a["alpha"], a["dt"],
+                                  vp(a["s0"]), vp(a["cu"]), a["n"], vp(a["ring"]), vp(a["pos"]),
+                                  vp(a["ws"]), a["wsb"], None)
+
+
+def _decode(lib, **kw):
+    a = dict(q=16, k=16, v=16, st=16, ring=16, out=16, pos=16, B=2, Hq=4, Hkv=2, d=128, w=64,
+             alpha=0.5, dt=0)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.liger_attn_decode(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["st"]), vp(a["ring"]),
+                                 vp(a["out"]), vp(a["pos"]), a["B"], a["Hq"], a["Hkv"], a["d"], a["w"],
+                                 a["alpha"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3, Hkv=2), ops.LIGER_ERR_INVALID_ARG),
+    (dict(Hkv=0), ops.LIGER_ERR_INVALID_ARG),
+    (dict(w=0), ops.LIGER_ERR_INVALID_ARG),
+    (dict(alpha=1.5), ops.LIGER_ERR_INVALID_ARG),
+    (dict(alpha=float("nan")), ops.LIGER_ERR_INVALID_ARG),
+    (dict(dt=7), ops.LIGER_ERR_INVALID_ARG),
+    (dict(d=96), ops.LIGER_ERR_UNSUPPORTED),
+    (dict(w=65), ops.LIGER_ERR_UNSUPPORTED),
+    (dict(B=0), ops.LIGER_ERR_INVALID_ARG),
+    (dict(T=-1), ops.LIGER_ERR_INVALID_ARG),
+    (dict(B=2, cu=16, n=2), ops.LIGER_ERR_INVALID_ARG),
+    (dict(cu=16, n=0), ops.LIGER_ERR_INVALID_ARG),
+    (dict(B=2, n=1), ops.LIGER_ERR_INVALID_ARG),
+    (dict(q=None), ops.LIGER_ERR_INVALID_ARG),
+    (dict(out=8), ops.LIGER_ERR_INVALID_ARG),
+    (dict(fs=24), ops.LIGER_ERR_INVALID_ARG),
+    (dict(cu=18), ops.LIGER_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_arguments(lib, kw, status):
+    assert _prefill(lib, **kw) == status
+    assert lib.liger_last_error().decode() != ""
+
+
+def test_prefill_rejects_short_workspace(lib):
+    need = lib.liger_attn_prefill_workspace_size(2, 32, 8, 8192, 128, 2, 0)
+    if need == 0:
+        pytest.skip("no workspace needed on this path")
+    assert _prefill(lib, B=2, Hq=32, Hkv=8, T=8192, d=128, n=2, ws=16, wsb=need - 16) == \
+        ops.LIGER_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=5), ops.LIGER_ERR_INVALID_ARG),
+    (dict(B=0), ops.LIGER_ERR_INVALID_ARG),
+    (dict(st=None), ops.LIGER_ERR_INVALID_ARG),
+    (dict(pos=None), ops.LIGER_ERR_INVALID_ARG),
+    (dict(pos=18), ops.LIGER_ERR_INVALID_ARG),
+    (dict(ring=40), ops.LIGER_ERR_INVALID_ARG),
+    (dict(d=32), ops.LIGER_ERR_UNSUPPORTED),
+    (dict(alpha=-0.1), ops.LIGER_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments(lib, kw, status):
+    assert _decode(lib, **kw) == status
+    assert lib.liger_last_error().decode() != ""
+
+
+def test_workspace_size_is_zero_for_rejected_sizes(lib):
+    assert lib.liger_attn_prefill_workspace_size(0, 32, 8, 128, 128, 0, 0) == 0
+    assert lib.liger_attn_prefill_workspace_size(1, 3, 2, 128, 128, 1, 0) == 0
+    assert lib.liger_attn_prefill_workspace_size(1, 4, 2, 128, 128, 1, 1) == 0  # fp32 needs none

@@ -1,0 +1,240 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs.
+
+Small cases compare every output; the full workload sizes run the CUDA
+kernels in the same launch configuration the benchmark times and compare
+sampled (batch row, kv-head group) units that the oracle recomputes from
+scratch.  Tolerances: bf16 max-abs 2e-2 and rel-L2 5e-3, fp32 1e-4 for both;
+the window ring and positions are copies and must match bit for bit.
+"""
+import os
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from gated_linear_attention_liger_b200 import inputs, ops
+from oracle import oracle
+from tests.parity_util import assert_close, np64, oracle_group
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # name, B, Hq, Hkv, T, d, dtype, w, alpha, seqlens, key_bias, with_s0
+    ("bf16_d64_ragged", 2, 4, 2, 200, 64, torch.bfloat16, 64, 0.5, (), 0.0, False),
+    ("bf16_d128_ragged", 1, 8, 2, 257, 128, torch.bfloat16, 64, 0.5, (), 0.0, False),
+    ("bf16_d128_one_token", 2, 4, 1, 1, 128, torch.bfloat16, 64, 0.5, (), 0.0, False),
+    ("bf16_d64_one_chunk", 1, 4, 2, 64, 64, torch.bfloat16, 64, 0.5, (), 0.0, False),
+    ("bf16_d128_shorter_than_window", 1, 4, 2, 30, 128, torch.bfloat16, 64, 0.5, (), 0.0, False),
+    ("bf16_d128_varlen", 1, 4, 1, 270, 128, torch.bfloat16, 64, 0.5, (5, 130, 1, 64, 70), 0.0, False),
+    ("bf16_d64_varlen_empty_seq", 1, 4, 2, 150, 64, torch.bfloat16, 64, 0.5, (0, 77, 73, 0), 0.0, False),
+    ("bf16_mha_w16_alpha03", 1, 3, 3, 150, 64, torch.bfloat16, 16, 0.3, (), 0.0, False),
+    ("bf16_d128_grm_only", 1, 4, 2, 190, 128, torch.bfloat16, 64, 1.0, (), 0.0, False),
+    ("bf16_d128_swa_only", 1, 4, 2, 190, 128, torch.bfloat16, 64, 0.0, (), 0.0, False),
+    ("bf16_d128_extreme_gates", 1, 8, 4, 320, 128, torch.bfloat16, 64, 0.5, (), 4.0, False),
+    ("bf16_d64_initial_state", 2, 4, 2, 150, 64, torch.bfloat16, 64, 0.5, (), 0.0, True),
+    ("fp32_d128_ragged", 1, 4, 2, 150, 128, torch.float32, 64, 0.5, (), 0.0, False),
+    ("fp32_d64_varlen_s0", 1, 2, 1, 160, 64, torch.float32, 64, 0.5, (60, 100), 0.0, True),
+]
+
+
+def run_small(case, device, path=None):
+    name, B, Hq, Hkv, T, d, dtype, w, alpha, seqlens, kb, with_s0 = case
+    wl = inputs.small(name, B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, dtype=dtype, seed=zlib.crc32(name.encode()) % 10000,
+                      seqlens=seqlens, key_bias_std=kb)
+    q, k, v = inputs.prefill_inputs(wl)
+    cu = wl.cu_seqlens
+    n = wl.n_seqs
+    s0 = inputs.random_state(n, Hq, d, seed=5, scale=0.05) if with_s0 else None
+    old = os.environ.get("LIGER_PREFILL_PATH")
+    if path:
+        os.environ["LIGER_PREFILL_PATH"] = path
+    try:
+        out, fs, ring, pos = ops.prefill(
+            q.to(device), k.to(device), v.to(device), alpha=alpha, w=w,
+            initial_state=None if s0 is None else s0.to(device),
+            cu_seqlens=None if cu is None else torch.tensor(cu, dtype=torch.int32, device=device),
+            return_ring=True)
+        torch.cuda.synchronize()
+    finally:
+        if path:
+            if old is None:
+                os.environ.pop("LIGER_PREFILL_PATH")
+            else:
+                os.environ["LIGER_PREFILL_PATH"] = old
+    ref = oracle.prefill(np64(q), np64(k), np64(v), w=w, alpha=alpha, cu_seqlens=cu,
+                         initial_state=None if s0 is None else np64(s0))
+    return (out, fs, ring, pos), ref, dtype
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_prefill_small_parity(case, cuda_device):
+    (out, fs, ring, pos), (ro, rfs, rring, rpos), dtype = run_small(case, cuda_device)
+    assert_close(np64(out), ro, dtype, "out")
+    assert_close(np64(fs), rfs, dtype, "final_state")
+    np.testing.assert_array_equal(np64(ring), rring)
+    np.testing.assert_array_equal(pos.cpu().numpy(), rpos)
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[6] == torch.bfloat16][:6],
+                         ids=[c[0] for c in SMALL if c[6] == torch.bfloat16][:6])
+def test_prefill_general_kernel_parity(case, cuda_device):
+    """The general (CUDA-core) prefill kernel, forced for bf16 inputs."""
+    (out, fs, ring, pos), (ro, rfs, rring, rpos), dtype = run_small(case, cuda_device, path="simt")
+    assert_close(np64(out), ro, dtype, "out")
+    assert_close(np64(fs), rfs, dtype, "final_state")
+
+
+def test_prefill_empty_batch(cuda_device):
+    q = torch.zeros(2, 0, 4, 64, dtype=torch.bfloat16, device=cuda_device)
+    k = torch.zeros(2, 0, 2, 64, dtype=torch.bfloat16, device=cuda_device)
+    s0 = inputs.random_state(2, 4, 64, seed=3).to(cuda_device)
+    out, fs, ring, pos = ops.prefill(q, k, k, initial_state=s0, return_ring=True)
+    torch.cuda.synchronize()
+    assert out.shape == q.shape
+    torch.testing.assert_close(fs, s0, rtol=0, atol=0)
+    assert int(pos.abs().sum()) == 0 and float(ring.float().abs().sum()) == 0.0
+
+
+def test_prefill_is_deterministic(cuda_device):
+    wl = inputs.small("det", B=2, Hq=8, Hkv=2, T=600, d=128)
+    q, k, v = (t.to(cuda_device) for t in inputs.prefill_inputs(wl))
+    a, sa = ops.prefill(q, k, v)
+    b, sb = ops.prefill(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(sa, sb)
+
+
+# ----------------------------------------------------------------- full sizes
+
+def _full_prefill_check(name, units, device):
+    wl = inputs.WORKLOADS[name]
+    q, k, v = inputs.prefill_inputs(wl)
+    cu = wl.cu_seqlens
+    cu_t = None if cu is None else torch.tensor(cu, dtype=torch.int32, device=device)
+    out, fs, ring, pos = ops.prefill(q.to(device), k.to(device), v.to(device), alpha=wl.alpha, w=wl.w,
+                                     cu_seqlens=cu_t, return_ring=True)
+    torch.cuda.synchronize()
+    out, fs = out.cpu(), fs.cpu()
+    G = wl.Hq // wl.Hkv
+    for b, kv in units:
+        ro, rfs, rring, rpos = oracle_group(q, k, v, b, kv, G, w=wl.w, alpha=wl.alpha, cu=cu)
+        hs = slice(kv * G, (kv + 1) * G)
+        assert_close(np64(out[b:b + 1, :, hs]), ro, wl.dtype, f"{name} out b={b} kv={kv}")
+        fsel = fs[:, hs] if cu is not None else fs[b:b + 1, hs]
+        assert_close(np64(fsel), rfs, wl.dtype, f"{name} final_state b={b} kv={kv}")
+        rsel = ring[:, kv:kv + 1] if cu is not None else ring[b:b + 1, kv:kv + 1]
+        np.testing.assert_array_equal(np64(rsel), rring)
+    exp_pos = np.diff(cu) if cu is not None else np.full(wl.B, wl.T)
+    np.testing.assert_array_equal(pos.cpu().numpy(), exp_pos)
+
+
+def test_full_llama1b_prefill(cuda_device):
+    _full_prefill_check("llama1b_prefill", [(0, 0), (3, 7), (1, 4)], cuda_device)
+
+
+def test_full_llama8b_prefill(cuda_device):
+    _full_prefill_check("llama8b_prefill", [(0, 2), (1, 7)], cuda_device)
+
+
+def test_full_long_varlen_prefill(cuda_device):
+    _full_prefill_check("long_varlen", [(0, 5)], cuda_device)
+
+
+def test_full_tiny_fp32(cuda_device):
+    wl = inputs.WORKLOADS["tiny_fp32"]
+    q, k, v = inputs.prefill_inputs(wl)
+    out, fs = ops.prefill(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device))
+    torch.cuda.synchronize()
+    ro, rfs, _, _ = oracle.prefill(np64(q), np64(k), np64(v))
+    assert_close(np64(out), ro, torch.float32, "out")
+    assert_close(np64(fs), rfs, torch.float32, "final_state")
+
+
+# ----------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dtype,d,w,T0,G", [
+    (torch.bfloat16, 128, 64, 70, 4),
+    (torch.bfloat16, 64, 64, 0, 2),
+    (torch.bfloat16, 64, 16, 5, 1),
+    (torch.float32, 128, 64, 100, 2),
+    (torch.float32, 64, 64, 3, 4),
+])
+def test_decode_steps_parity(dtype, d, w, T0, G, cuda_device):
+    """Oracle prefix -> identical state/ring/pos on both sides -> several decode steps."""
+    B, Hkv, steps = 3, 2, 12
+    Hq = Hkv * G
+    wl = inputs.small("dec", B=B, Hq=Hq, Hkv=Hkv, T=T0 + steps, d=d, dtype=dtype, seed=17)
+    q, k, v = inputs.prefill_inputs(wl)
+    if T0:
+        _, st, rg, ps = oracle.prefill(np64(q[:, :T0]), np64(k[:, :T0]), np64(v[:, :T0]), w=w)
+    else:
+        st, rg, ps = np.zeros((B, Hq, d, d)), np.zeros((B, Hkv, 2, w, d)), np.zeros(B, np.int32)
+    g_state = torch.tensor(st, dtype=torch.float32)
+    st = np64(g_state)  # the oracle continues from the same fp32 state the GPU holds
+    g_state = g_state.to(cuda_device)
+    g_ring = torch.tensor(rg).to(dtype)
+    rg = np64(g_ring)
+    g_ring = g_ring.to(cuda_device)
+    g_pos = torch.tensor(ps, dtype=torch.int32, device=cuda_device)
+    for t in range(T0, T0 + steps):
+        qt, kt, vt = q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous()
+        o = ops.decode(qt.to(cuda_device), kt.to(cuda_device), vt.to(cuda_device), g_state, g_ring, g_pos)
+        ro, st, rg, ps = oracle.decode(np64(qt), np64(kt), np64(vt), st, rg, ps, w=w)
+        torch.cuda.synchronize()
+        assert_close(np64(o), ro, dtype, f"decode out step {t}")
+    assert_close(np64(g_state), st, dtype, "decode state")
+    np.testing.assert_array_equal(np64(g_ring), rg)
+    np.testing.assert_array_equal(g_pos.cpu().numpy(), ps)
+
+
+def test_prefill_then_decode_matches_longer_prefill(cuda_device):
+    """Cross-path: GPU prefill(T1) + T2 GPU decode steps == GPU prefill(T1 + T2)."""
+    wl = inputs.small("xpath", B=2, Hq=8, Hkv=2, T=300, d=128, seed=23)
+    q, k, v = (t.to(cuda_device) for t in inputs.prefill_inputs(wl))
+    T1 = 260
+    full, fs_full, ring_full, _ = ops.prefill(q, k, v, return_ring=True)
+    _, st, rg, ps = ops.prefill(q[:, :T1].contiguous(), k[:, :T1].contiguous(), v[:, :T1].contiguous(),
+                                return_ring=True)
+    for t in range(T1, wl.T):
+        o = ops.decode(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), st, rg, ps)
+        assert_close(np64(o), np64(full[:, t]), torch.bfloat16, f"step {t}")
+    assert_close(np64(st), np64(fs_full), torch.bfloat16, "state")
+    assert torch.equal(rg, ring_full)
+    assert int(ps.min()) == wl.T == int(ps.max())
+
+
+def test_full_llama8b_decode(cuda_device):
+    """B=64 decode at the full shape after a 1024-token prefix; sampled sequences
+    carry an oracle-built state and ring, 200 steps compared step by step."""
+    wl = inputs.WORKLOADS["llama8b_decode"]
+    B, Hq, Hkv, d, w, G = wl.B, wl.Hq, wl.Hkv, wl.d, wl.w, wl.Hq // wl.Hkv
+    units = [(5, 1), (63, 6)]
+    state = torch.zeros(B, Hq, d, d, dtype=torch.float32)
+    ring = torch.zeros(B, Hkv, 2, w, d, dtype=wl.dtype)
+    pos = torch.full((B,), wl.T, dtype=torch.int32)
+    ref = {}
+    pre = inputs.Workload("pre", "prefill", 1, G, 1, wl.T, d, wl.dtype, seed=wl.seed)
+    for b, kv in units:
+        q, k, v = inputs.prefill_inputs(pre, seed=wl.seed + 97 * b + kv)
+        _, st, rg, ps = oracle.prefill(np64(q), np64(k), np64(v), w=w)
+        hs = slice(kv * G, (kv + 1) * G)
+        state[b, hs] = torch.tensor(st[0], dtype=torch.float32)
+        ring[b, kv] = torch.tensor(rg[0]).to(wl.dtype)
+        ref[(b, kv)] = [np64(state[b:b + 1, hs]), np64(ring[b:b + 1, kv:kv + 1]), np.array([wl.T], np.int32)]
+    g_state, g_ring, g_pos = state.to(cuda_device), ring.to(cuda_device), pos.to(cuda_device)
+    for step in range(200):
+        q, k, v = inputs.decode_step_inputs(wl, step)
+        o = ops.decode(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), g_state, g_ring, g_pos)
+        o = o.cpu()
+        for (b, kv), (st, rg, ps) in ref.items():
+            hs = slice(kv * G, (kv + 1) * G)
+            ro, st, rg, ps = oracle.decode(np64(q[b:b + 1, hs]), np64(k[b:b + 1, kv:kv + 1]),
+                                           np64(v[b:b + 1, kv:kv + 1]), st, rg, ps, w=w)
+            ref[(b, kv)] = [st, rg, ps]
+            assert_close(np64(o[b:b + 1, hs]), ro, wl.dtype, f"decode step {step} b={b} kv={kv}")
+    for (b, kv), (st, rg, ps) in ref.items():
+        hs = slice(kv * G, (kv + 1) * G)
+        assert_close(np64(g_state[b:b + 1, hs]), st, wl.dtype, "state")
+        np.testing.assert_array_equal(np64(g_ring[b:b + 1, kv:kv + 1]), rg)
+    assert int(g_pos.min()) == wl.T + 200 == int(g_pos.max())
