@@ -50,6 +50,22 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
+    kernel's sources have changed since the capture was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    m = hashlib.sha256()
+    for name in rec["source_files"]:
+        with open(os.path.join(ROOT, "gated_linear_attention_liger_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    return float(rec["bytes"]) if m.hexdigest()[:16] == rec["source_sha"] else None
+
+
 def prefill_algorithmic(wl=PREFILL):
     """Algorithmic bytes and flops of one prefill call (read q, k, v once, write out and the
     final state once; flops of readout, causal intra-chunk, state update and window)."""
@@ -261,6 +277,14 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(local).start()
     windows = []
 
+    if args.only == "decode":
+        dec = run_decode(args, world, dev, stream, pk, windows)
+        sampler.stop()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "partial": "decode only", "decode": dec,
+                              "clocks": sampler.summary(windows)}), flush=True)
+        return
+
     # ---------------- prefill
     wl = PREFILL
     q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
@@ -306,13 +330,11 @@ def run_ours(args, world, rank, local):
                 "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
                 "tensor_frac": alg_flops / (k_ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
                 "peak_source": pk["source"], "frac_of": f"{pk['source']} HBM copy bandwidth"}
-    traffic = os.environ.get("LIGER_PREFILL_TRAFFIC_BYTES")
-    if traffic:
-        roofline["traffic"] = float(traffic)
+    roofline["traffic"] = measured_traffic("chunk_kernel<128>")
 
     # ---------------- e2e: host buffers, copies inside the timed region
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.only is None:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         hfs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
@@ -347,12 +369,12 @@ def run_ours(args, world, rank, local):
     del q, k, v, out, ws
 
     # ---------------- decode
-    dec = run_decode(args, world, dev, stream, pk, windows)
+    dec = None if args.only == "prefill" else run_decode(args, world, dev, stream, pk, windows)
 
     sampler.stop()
     clocks = sampler.summary(windows)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
         tps, secs, desc, nthr = oracle_prefill_sample(args.cpu_seconds)
         cpu = {"value": tps, "unit": "tokens/s", "cores": nthr, "kind": "oracle", "sample": desc,
                "seconds": secs}
@@ -440,7 +462,7 @@ def run_decode(args, world, dev, stream, pk, windows):
             "unit": "tokens/s", "ms_per_step": ms_step, "graph_steps": n_graph, "replays": reps,
             "gpu_launches": per_graph_launches * reps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "frac": achieved / pk["hbm_gbs"], "traffic": measured_traffic("decode_kernel<bf16,128>"),
                          "kernel": "decode state stream", "kernel_ms": kms,
                          "kernel_timing": "events in graph" if kernel_events else "graph step average",
                          "algorithmic_bytes": alg, "peak_source": pk["source"]}}
@@ -454,6 +476,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=200, help="decode steps per captured graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU baseline")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part only (for profiling); the JSON line is then partial")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

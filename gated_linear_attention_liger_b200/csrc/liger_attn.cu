@@ -24,9 +24,17 @@ thread_local std::string g_last_error;
 thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
 thread_local uint64_t g_launches = 0;
 
-// Bracket the dominant kernel of a call with the caller's timing events.
-void mark_start(cudaStream_t s) { if (g_ev_start) cudaEventRecord(g_ev_start, s); }
-void mark_stop(cudaStream_t s) { if (g_ev_stop) cudaEventRecord(g_ev_stop, s); }
+// Bracket the dominant kernel of a call with the caller's timing events.  In a
+// stream capture the records become graph nodes of their own (external flag).
+void record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else cudaEventRecord(ev, s);
+}
+void mark_start(cudaStream_t s) { if (g_ev_start) record(g_ev_start, s); }
+void mark_stop(cudaStream_t s) { if (g_ev_stop) record(g_ev_stop, s); }
+void count_launches(int n) { g_launches += (uint64_t)n; }
 
 liger_status fail(liger_status s, const char* fmt, ...) {
   char buf[512];
@@ -50,11 +58,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Which prefill kernel serves a call.
 enum class PrefillPath { kSimt, kTensorCore };
 
-PrefillPath choose_prefill_path(int Hq, int Hkv, int d, int w, liger_dtype dt,
+PrefillPath choose_prefill_path(long ntok, int Hq, int Hkv, int d, int w, liger_dtype dt,
                                 const float* initial_state) {
   const char* force = std::getenv("LIGER_PREFILL_PATH");
   if (force && std::strcmp(force, "simt") == 0) return PrefillPath::kSimt;
-  if (dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && initial_state == nullptr &&
+  if (ntok > 0 && dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && initial_state == nullptr &&
       liger::tc::supports(d))
     return PrefillPath::kTensorCore;
   return PrefillPath::kSimt;
@@ -156,13 +164,14 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
     return fail(LIGER_ERR_INVALID_ARG, "pos_out must be 4-byte aligned");
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const PrefillPath path = choose_prefill_path(Hq, Hkv, d, w, dt, initial_state);
+  const PrefillPath path = choose_prefill_path(ntok, Hq, Hkv, d, w, dt, initial_state);
   if (path == PrefillPath::kTensorCore) {
     const size_t need = liger::tc::workspace_bytes(B, Hq, Hkv, (long)T, d, n_seqs);
     if (need > workspace_bytes || (need && !workspace))
       return fail(LIGER_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, workspace_bytes);
     liger::tc::PrefillProblem pb{q, k, v, out, final_state, cu_seqlens, B, Hq, Hkv, (long)T, d, n_seqs, alpha};
-    st = liger::tc::run_prefill(pb, workspace, s);
+    const liger::tc::LaunchHooks hooks{mark_start, mark_stop, count_launches};
+    st = liger::tc::run_prefill(pb, workspace, s, hooks);
     if (st != LIGER_OK) return fail(st, "%s", liger::tc::last_message());
   } else {
     liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha};

@@ -1,11 +1,64 @@
-// prefill_tc.cuh -- bf16 chunked prefill on the tcgen05 tensor cores (sm_100a).
+// prefill_tc.cuh -- bf16 chunked prefill on the sm_100a tensor cores.
+//
+// The recurrence S_t = g_t S_{t-1} + phi(k_t)^T v_t, o_t = phi(q_t) S_t and the
+// 64-token window ("Liger: Linearizing Large Language Models to Gated Recurrent
+// Structures", Paper-Notes page, sections 统一的门控线性循环框架 and Liger
+// Attention) are evaluated in 64-token chunks: inside a chunk the recurrence is
+// unrolled into decay-masked dense products, across chunks only the d x d fp32
+// state is carried.  With b_i the running sum of log g inside a chunk (b_C at
+// its last token) and S the state entering the chunk:
+//   grm_i  = e^{b_i} phi(q_i) S + sum_{j<=i} e^{b_i-b_j} (phi(q_i).phi(k_j)) v_j
+//   S_next = e^{b_C} S + sum_j (e^{b_C-b_j} phi(k_j))^T v_j
+// Every exponent is a difference of running sums taken later-minus-earlier,
+// so it is <= 0 and cannot overflow however small the gates are.
+//
+// Work split (one GPU):
+//   plan      : segment table from the sequence offsets (device side, so the
+//               launch needs no host synchronisation).
+//   seg_state : per (segment, kv head) the state a segment adds from a zero
+//               start, dS = sum over its chunks, and its total log decay.
+//   scan      : per (sequence, kv head) the state entering every segment and the
+//               final state (written to each q head of the group).
+//   chunk     : per (segment, pair of q heads of one kv head) the fused pass:
+//               TMA stages q/k/v chunks; four warps compute phi, gates and the
+//               window softmax on TMEM rows; one thread issues tcgen05 MMAs:
+//                 Ss = Q [K_prev;K_cur]^T        raw scores of the window band
+//                 Sg = phi(Q) phi(K)^T           recurrent scores
+//                 O  = (alpha e^{b_i}/Z_i e_q) S  inter-chunk readout
+//                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
+//                 O += P_prev V_prev + P_cur V_cur, P_cur = beta*softmax + alpha*decayed Sg
+//               and the epilogue stores bf16 rows.
+// Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
+// is exactly the order a TMA box over (d, head, token) produces.
 #pragma once
 
-#include "liger_attn.h"
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <mutex>
+
 #include "common.cuh"
+#include "liger_attn.h"
+#include "sm100.cuh"
 
 namespace liger {
 namespace tc {
+
+using namespace liger::sm100;
+
+constexpr int C = 64;             // tokens per chunk
+constexpr int ROWS = 128;         // MMA M: two heads x 64 tokens
+constexpr int NTHREADS = 192;     // warps 0-3 rows, warp 4 TMA, warp 5 MMA
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // 2 s per wait
+
+struct SegInfo {
+  int32_t seq, t_begin, t_end, q0;   // tokens [t_begin, t_end) of the sequence starting at q0
+};
+struct SeqInfo {
+  int32_t first_seg, n_seg;
+};
 
 struct PrefillProblem {
   const void* q;
@@ -20,10 +73,882 @@ struct PrefillProblem {
   float alpha;
 };
 
-inline bool supports(int d) { (void)d; return false; }
-inline size_t workspace_bytes(int, int, int, long, int, int) { return 0; }
-inline const char* last_message() { return "tensor-core prefill not built"; }
-inline liger_status run_prefill(const PrefillProblem&, void*, cudaStream_t) { return LIGER_ERR_UNSUPPORTED; }
+// Workspace layout (bytes from its start).
+struct Plan {
+  int L;            // chunks per segment
+  int n_seg_max;    // upper bound on segments
+  size_t off_seqs, off_segs, off_lam, off_ds, total;
+};
+
+struct DevParams {
+  const SegInfo* segs;
+  const SeqInfo* seqs;
+  const int32_t* n_segs;
+  float* lam;            // [n_seg_max][Hkv]
+  float* ds;             // [n_seg_max][Hkv][D][D]: dS, replaced by the entering state by scan
+  uint32_t* err;
+  void* out;
+  float* final_state;
+  const int32_t* cu;
+  long T, NT;
+  int Hq, Hkv, n_seqs, n_seg_max, L;
+  float alpha;
+  uint64_t wait_ns;
+};
+
+// ============================================================== plan kernel
+
+__global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* n_segs) {
+  if (threadIdx.x != 0) return;
+  *p.err = 0u;
+  int seg = 0;
+  const long span = (long)C * p.L;
+  for (int s = 0; s < p.n_seqs; ++s) {
+    long q0, q1;
+    seq_range(p.cu, s, p.T, p.NT, &q0, &q1);
+    const long len = q1 - q0;
+    const int nseg = (int)((len + span - 1) / span);
+    if (seg + nseg > p.n_seg_max) {   // cannot happen with the host's bound; fail safe
+      atomicOr(p.err, 2u);
+      seqs[s] = SeqInfo{seg, 0};
+      continue;
+    }
+    seqs[s] = SeqInfo{seg, nseg};
+    for (int i = 0; i < nseg; ++i) {
+      const long b = q0 + i * span;
+      const long e = b + span < q1 ? b + span : q1;
+      segs[seg++] = SegInfo{s, (int32_t)b, (int32_t)e, (int32_t)q0};
+    }
+  }
+  *n_segs = seg;
+}
+
+// ============================================================== row helpers
+
+// Element e (0..D-1) of 128-byte-swizzled row `row` in a K-major tile whose
+// 64-element blocks are `block_stride` bytes apart.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int e, uint32_t block_stride) {
+  return (uint32_t)(e >> 6) * block_stride + sw128(row, (e & 63) >> 3) + (uint32_t)((e & 7) << 1);
+}
+
+// Load 8 bf16 (one 16-byte chunk) as floats.
+__device__ __forceinline__ void ld_chunk8(const char* base, uint32_t off, float (&x)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(base + off);
+  x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x);
+  x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+  x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z);
+  x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
+}
+__device__ __forceinline__ void st_chunk8(char* base, uint32_t off, const float* x) {
+  uint4 u;
+  u.x = pack_bf16(x[0], x[1]);
+  u.y = pack_bf16(x[2], x[3]);
+  u.z = pack_bf16(x[4], x[5]);
+  u.w = pack_bf16(x[6], x[7]);
+  *reinterpret_cast<uint4*>(base + off) = u;
+}
+
+// Feature map and gate of one chunk of keys, shared by the seg_state and chunk
+// kernels.  Thread r (0..127) owns half of token j = r >> 1: elements
+// [h * D/2, (h+1) * D/2) with h = r & 1.  Writes phi(k) (bf16) to `phik` (may be
+// null), the log gates to bsh[0..63] (0 past the valid tokens), scans them to
+// running sums in bsh, and returns the thread's phi values in ph.
+template <int D>
+__device__ __forceinline__ void key_features(const char* kraw, char* phik, float* bsh, int r, int nv,
+                                             float (&ph)[D / 2]) {
+  constexpr int HALF = D / 2;
+  const int j = r >> 1, h = r & 1;
+  float m = -INFINITY, sum = 0.f;
+#pragma unroll
+  for (int c = 0; c < HALF / 8; ++c) {
+    float x[8];
+    ld_chunk8(kraw, kmajor_off(j, h * HALF + c * 8, C * 128), x);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      ph[c * 8 + u] = x[u];
+      m = fmaxf(m, x[u]);
+      sum += x[u];
+    }
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  float z = 0.f;
+#pragma unroll
+  for (int u = 0; u < HALF; ++u) {
+    ph[u] = __expf(ph[u] - m);
+    z += ph[u];
+  }
+  z += __shfl_xor_sync(0xffffffffu, z, 1);
+  const float iz = 1.0f / z;
+#pragma unroll
+  for (int u = 0; u < HALF; ++u) ph[u] *= iz;
+  if (phik) {
+#pragma unroll
+    for (int c = 0; c < HALF / 8; ++c) st_chunk8(phik, kmajor_off(j, h * HALF + c * 8, C * 128), &ph[c * 8]);
+  }
+  if (h == 0) bsh[j] = j < nv ? log_sigmoid(sum / (float)D) : 0.f;
+  named_bar(1, 128);
+  if (r < 32) {   // inclusive running sum over the 64 tokens, two per lane
+    const float a0 = bsh[2 * r], a1 = bsh[2 * r + 1];
+    float s = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float t = __shfl_up_sync(0xffffffffu, s, o);
+      if (r >= o) s += t;
+    }
+    const float before = s - a0 - a1;
+    __syncwarp();
+    bsh[2 * r] = before + a0;
+    bsh[2 * r + 1] = before + a0 + a1;
+  }
+  named_bar(1, 128);
+}
+
+// Decay-scaled keys e^{b_C - b_j} phi(k_j) (zero past the valid tokens), written
+// in the same swizzled layout; read by the MMA as the MN-major A operand K^T.
+template <int D>
+__device__ __forceinline__ void write_ktilde(char* kt, const float* bsh, int r, int nv, float bC,
+                                             const float (&ph)[D / 2]) {
+  constexpr int HALF = D / 2;
+  const int j = r >> 1, h = r & 1;
+  const float sc = j < nv ? __expf(bC - bsh[j]) : 0.f;
+#pragma unroll
+  for (int c = 0; c < HALF / 8; ++c) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = ph[c * 8 + u] * sc;
+    st_chunk8(kt, kmajor_off(j, h * HALF + c * 8, C * 128), x);
+  }
+}
+
+// ============================================================== seg_state kernel
+
+template <int D>
+struct SegSmem {
+  static constexpr uint32_t KV = C * D * 2;        // one chunk of k (or v)
+  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 4 * KV, SMALL = 5 * KV;
+  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    seg_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                     DevParams p) {
+  using L = SegSmem<D>;
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
+  uint64_t* kv_full = bars;        // [2]
+  uint64_t* kv_empty = bars + 2;   // [2]
+  uint64_t* feat = bars + 4;
+  uint64_t* mma_done = bars + 5;
+  uint64_t* drain = bars + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
+  float* bsh = reinterpret_cast<float*>(bars + 10);   // 64 floats
+
+  const int seg = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  if (seg >= *p.n_segs) return;
+  const SegInfo sg = p.segs[seg];
+  const int nch = (sg.t_end - sg.t_begin + C - 1) / C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr uint32_t TCOLS = D < 32 ? 32 : D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&kv_full[0], 1); mbar_init(&kv_full[1], 1);
+    mbar_init(&kv_empty[0], 1); mbar_init(&kv_empty[1], 1);
+    mbar_init(feat, 128); mbar_init(mma_done, 1); mbar_init(drain, 1);
+    *abort_flag = 0u;
+    *never = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.err, p.wait_ns};
+
+  if (warp == 4) {   // ---------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+      int issued = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int slot = c & 1;
+        if (c >= 2 && !mbar_wait(&kv_empty[slot], ((c >> 1) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&kv_full[slot], 2 * L::KV);
+        const int t = sg.t_begin + c * C;
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &kv_full[slot], kb * 64, kv, t);
+          tma_load_3d(smem + L::V0 + slot * L::KV + kb * C * 128, &tmv, &kv_full[slot], kb * 64, kv, t);
+        }
+        issued = c + 1;
+      }
+      // never leave the CTA with copies in flight
+      for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
+        mbar_wait(&kv_full[c & 1], (c >> 1) & 1, WaitCtx{never, nullptr, p.wait_ns});
+    }
+  } else if (warp == 5) {   // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, D, 1, 1);
+      const uint32_t lbo_a = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
+      for (int c = 0; c < nch; ++c) {
+        const int slot = c & 1;
+        if (!mbar_wait(&kv_full[slot], (c >> 1) & 1, wc)) break;
+        if (!mbar_wait(feat, c & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(smem_u32(smem + L::KT) + kk * 2048, lbo_a, 1024);
+          const uint64_t b = sdesc_sw128(smem_u32(smem + L::V0 + slot * L::KV) + kk * 2048, C * 128, 1024);
+          mma_bf16_ss(tmem, a, b, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(mma_done);
+        mma_commit(&kv_empty[slot]);
+      }
+      mma_commit(drain);
+    }
+  } else {   // ---------------- rows (threads 0..127)
+    const int r = threadIdx.x;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float lam = 0.f;
+    // Row threads never leave the loop early: after a timeout every wait returns
+    // at once (the CTA's abort flag is set), so all rows still meet at each
+    // named barrier and warp-collective TMEM access stays uniform.
+    for (int c = 0; c < nch; ++c) {
+      const int slot = c & 1;
+      const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
+      mbar_wait(&kv_full[slot], (c >> 1) & 1, wc);
+      float ph[D / 2];
+      key_features<D>(smem + L::K0 + slot * L::KV, nullptr, bsh, r, nv, ph);
+      const float bC = bsh[nv - 1];
+      lam += bC;
+      if (c > 0) {
+        mbar_wait(mma_done, (c - 1) & 1, wc);
+        tc_fence_after();
+      }
+      write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+      if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
+        const float dec = __expf(bC);
+#pragma unroll
+        for (int col = 0; col < D; col += 32) {
+          float v[32];
+          tmem_ld32(lane_base + col, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= dec;
+          tmem_st32(lane_base + col, v);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(feat);
+      named_bar(1, 128);   // bsh is rewritten by the next chunk
+    }
+    if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
+      tc_fence_after();
+      float* dst = p.ds + (((size_t)seg * p.Hkv + kv) * D + r) * D;
+#pragma unroll
+      for (int col = 0; col < D; col += 32) {
+        float v[32];
+        tmem_ld32(lane_base + col, v);
+        tmem_wait_ld();
+        if (r < D) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4)
+            *reinterpret_cast<float4*>(dst + col + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        }
+      }
+      if (r == 0) p.lam[(size_t)seg * p.Hkv + kv] = lam;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    mbar_wait(drain, 0, WaitCtx{never, nullptr, p.wait_ns});
+    tc_fence_after();
+    tmem_dealloc(tmem, TCOLS);
+  }
+}
+
+// ============================================================== scan kernel
+
+// Grid (n_seqs * Hkv, D*D / 1024), 256 threads x 4 floats.  Replaces dS of each
+// segment by the state entering it and writes the final state to every q head.
+template <int D>
+__global__ void scan_kernel(DevParams p) {
+  const int seq = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  const size_t e = ((size_t)blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (e >= (size_t)D * D) return;
+  const SeqInfo si = p.seqs[seq];
+  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = si.first_seg; s < si.first_seg + si.n_seg; ++s) {
+    float4* cell = reinterpret_cast<float4*>(p.ds + ((size_t)s * p.Hkv + kv) * D * D + e);
+    const float4 d = *cell;
+    *cell = run;
+    const float g = __expf(p.lam[(size_t)s * p.Hkv + kv]);
+    run = make_float4(fmaf(g, run.x, d.x), fmaf(g, run.y, d.y), fmaf(g, run.z, d.z), fmaf(g, run.w, d.w));
+  }
+  if (p.final_state) {
+    const int G = p.Hq / p.Hkv;
+    for (int h = kv * G; h < (kv + 1) * G; ++h)
+      *reinterpret_cast<float4*>(p.final_state + ((size_t)seq * p.Hq + h) * D * D + e) = run;
+  }
+}
+
+// ============================================================== chunk kernel
+
+template <int D>
+struct ChunkSmem {
+  static constexpr uint32_t QB = ROWS * D * 2;    // q tile (two heads)
+  static constexpr uint32_t KV = C * D * 2;       // one chunk of k or v
+  static constexpr uint32_t PQB = ROWS * D * 2 > 2 * ROWS * 64 * 2 ? ROWS * D * 2 : 2 * ROWS * 64 * 2;
+  static constexpr uint32_t Q0 = 0;
+  static constexpr uint32_t K0 = Q0 + QB;         // 3 slots
+  static constexpr uint32_t V0 = K0 + 3 * KV;     // 3 slots
+  static constexpr uint32_t PQ = V0 + 3 * KV;     // phi(q) (unnormalised), later P
+  static constexpr uint32_t PK = PQ + PQB;        // phi(k)
+  static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
+  static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
+  static constexpr uint32_t SMALL = SB + D * D * 2;
+  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
+};
+
+// TMEM columns of the chunk kernel.
+constexpr uint32_t kColSs = 0, kColSg = 128, kColO = 192;
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                 const __grid_constant__ CUtensorMap tmv, DevParams p) {
+  using L = ChunkSmem<D>;
+  constexpr uint32_t kColS = kColO + D;
+  constexpr uint32_t TCOLS = 512;
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
+  uint64_t* kv_full = bars;          // [3]
+  uint64_t* kv_empty = bars + 3;     // [3]
+  uint64_t* q_full = bars + 6;
+  uint64_t* q_empty = bars + 7;
+  uint64_t* ss_done = bars + 8;
+  uint64_t* feat = bars + 9;
+  uint64_t* sg_done = bars + 10;
+  uint64_t* p_ready = bars + 11;
+  uint64_t* o_done = bars + 12;
+  uint64_t* o_free = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
+  float* bsh = reinterpret_cast<float*>(bars + 18);   // 64 floats
+
+  const int npairs = p.Hq / 2;
+  const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
+  if (seg >= *p.n_segs) return;
+  const SegInfo sg = p.segs[seg];
+  const int G = p.Hq / p.Hkv;
+  const int h0 = pair * 2, kv = h0 / G;
+  const int nch = (sg.t_end - sg.t_begin + C - 1) / C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    mbar_init(q_full, 1); mbar_init(q_empty, 1);
+    mbar_init(ss_done, 1); mbar_init(feat, 128); mbar_init(sg_done, 1);
+    mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128); mbar_init(drain, 1);
+    *abort_flag = 0u;
+    *never = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.err, p.wait_ns};
+
+  if (warp == 4) {   // ---------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmq);
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+      auto load_kv = [&](int u) {   // u-th key/value chunk: tokens t_begin + 64 (u - 1)
+        const int slot = u % 3;
+        const int t = sg.t_begin + (u - 1) * C;
+        mbar_arrive_expect_tx(&kv_full[slot], 2 * L::KV);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb) {
+          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &kv_full[slot], kb * 64, kv, t);
+          tma_load_3d(smem + L::V0 + slot * L::KV + kb * C * 128, &tmv, &kv_full[slot], kb * 64, kv, t);
+        }
+      };
+      auto load_q = [&](int c) {
+        mbar_arrive_expect_tx(q_full, L::QB);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(smem + L::Q0 + kb * ROWS * 128, &tmq, q_full, kb * 64, h0, sg.t_begin + c * C);
+      };
+      int kv_issued = 2, q_issued = 1;
+      load_kv(0);
+      load_kv(1);
+      load_q(0);
+      for (int c = 0; c + 1 < nch; ++c) {
+        const int u = c + 2;
+        if (u >= 3 && !mbar_wait(&kv_empty[u % 3], (u / 3 - 1) & 1, wc)) break;
+        load_kv(u);
+        kv_issued = u + 1;
+        if (!mbar_wait(q_empty, c & 1, wc)) break;
+        load_q(c + 1);
+        q_issued = c + 2;
+      }
+      const WaitCtx drain_wc{never, nullptr, p.wait_ns};
+      for (int u = (kv_issued > 3 ? kv_issued - 3 : 0); u < kv_issued; ++u)
+        mbar_wait(&kv_full[u % 3], (u / 3) & 1, drain_wc);
+      mbar_wait(q_full, (q_issued - 1) & 1, drain_wc);
+    }
+  } else if (warp == 5) {   // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
+      const uint32_t id_inter = idesc_bf16(128, D, 0, 1);
+      const uint32_t id_state = idesc_bf16(128, D, 1, 1);
+      const uint32_t lbo_kt = D == 128 ? C * 128 : 0;
+      const uint32_t q_base = smem_u32(smem + L::Q0);
+      const uint32_t pq_base = smem_u32(smem + L::PQ);
+      const uint32_t pk_base = smem_u32(smem + L::PK);
+      const uint32_t kt_base = smem_u32(smem + L::KT);
+      const uint32_t sb_base = smem_u32(smem + L::SB);
+      for (int c = 0; c < nch; ++c) {
+        const int ks = (c + 1) % 3, ps = c % 3;
+        const uint32_t kc = smem_u32(smem + L::K0 + ks * L::KV), kp = smem_u32(smem + L::K0 + ps * L::KV);
+        const uint32_t vc = smem_u32(smem + L::V0 + ks * L::KV), vp = smem_u32(smem + L::V0 + ps * L::KV);
+        if (c == 0 && !mbar_wait(&kv_full[0], 0, wc)) break;
+        if (!mbar_wait(&kv_full[ks], ((c + 1) / 3) & 1, wc)) break;
+        if (!mbar_wait(q_full, c & 1, wc)) break;
+        tc_fence_after();
+        // window scores against the previous and the current chunk of keys
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+          const uint64_t a = sdesc_sw128(q_base + (kk >> 2) * (ROWS * 128) + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + kColSs, a, sdesc_sw128(kp + ko, 16, 1024), id_n64, kk > 0);
+          mma_bf16_ss(tmem + kColSs + 64, a, sdesc_sw128(kc + ko, 16, 1024), id_n64, kk > 0);
+        }
+        mma_commit(ss_done);
+        if (!mbar_wait(feat, c & 1, wc)) break;
+        if (c > 0 && !mbar_wait(o_free, (c - 1) & 1, wc)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
+          const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
+          // recurrent scores phi(Q) phi(K)^T
+          mma_bf16_ss(tmem + kColSg, sdesc_sw128(pq_base + qo, 16, 1024), sdesc_sw128(pk_base + ko, 16, 1024),
+                      id_n64, kk > 0);
+          // inter-chunk readout: (scaled phi(Q)) x S, S as MN-major B
+          mma_bf16_ss(tmem + kColO, sdesc_sw128(q_base + qo, 16, 1024),
+                      sdesc_sw128(sb_base + kk * 2048, D * 128, 1024), id_inter, kk > 0);
+        }
+        // state carry S += Ktilde^T V_cur (both MN-major)
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+          mma_bf16_ss(tmem + kColS, sdesc_sw128(kt_base + kk * 2048, lbo_kt, 1024),
+                      sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
+        mma_commit(sg_done);
+        mma_commit(q_empty);
+        if (!mbar_wait(p_ready, c & 1, wc)) break;
+        tc_fence_after();
+        // O += P_prev V_prev + P_cur V_cur
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16_ss(tmem + kColO, sdesc_sw128(pq_base + kk * 32, 16, 1024),
+                      sdesc_sw128(vp + kk * 2048, C * 128, 1024), id_inter, 1u);
+          mma_bf16_ss(tmem + kColO, sdesc_sw128(pq_base + ROWS * 128 + kk * 32, 16, 1024),
+                      sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_inter, 1u);
+        }
+        mma_commit(o_done);
+        mma_commit(&kv_empty[ps]);
+      }
+      mma_commit(drain);
+    }
+  } else {   // ---------------- rows (threads 0..127)
+    const int r = threadIdx.x;
+    const int i = r >> 1, hl = r & 1;          // token in chunk, head in pair
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float alpha = p.alpha, beta = 1.0f - p.alpha;
+    const float kLog2e = 1.4426950408889634f;
+    const float sscale = kLog2e / sqrtf((float)D);
+    char* const qb = smem + L::Q0;
+    char* const pqb = smem + L::PQ;
+    char* const sbb = smem + L::SB;
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+
+    // entering state of this segment -> TMEM (rows >= D repeat rows 0..D-1)
+    {
+      const float* src = p.ds + (((size_t)seg * p.Hkv + kv) * D + (r % D)) * D;
+#pragma unroll
+      for (int col = 0; col < D; col += 32) {
+        float v[32];
+#pragma unroll
+        for (int u = 0; u < 32; u += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src + col + u);
+          v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
+        }
+        tmem_st32(lane_base + kColS + col, v);
+      }
+      tmem_wait_st();
+    }
+
+    for (int c = 0; c < nch; ++c) {
+      const int ks = (c + 1) % 3;
+      const int t0 = sg.t_begin + c * C;
+      const int nv = min(C, sg.t_end - t0);
+      // (row threads never leave the loop early; see seg_state_kernel)
+      if (c == 0) mbar_wait(&kv_full[0], 0, wc);
+      mbar_wait(&kv_full[ks], ((c + 1) / 3) & 1, wc);
+      mbar_wait(q_full, c & 1, wc);
+
+      // ---- keys: phi(k), gates, running sums, decay-scaled keys
+      float ph[D / 2];
+      key_features<D>(smem + L::K0 + ks * L::KV, smem + L::PK, bsh, r, nv, ph);
+      const float bC = bsh[nv - 1];
+      write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+      const float bi = bsh[i];
+
+      // ---- queries: e_q = exp(q - max) (bf16) and its sum
+      float mq = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < D; e += 8) {
+        float x[8];
+        ld_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mq = fmaxf(mq, x[u]);
+      }
+      float zq = 0.f;
+#pragma unroll
+      for (int e = 0; e < D; e += 8) {
+        float x[8];
+        ld_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          x[u] = __expf(x[u] - mq);
+          zq += x[u];
+        }
+        st_chunk8(pqb, kmajor_off(r, e, ROWS * 128), x);
+      }
+      const float izq = 1.0f / zq;
+
+      // ---- after the window-score MMA has read raw q: scaled phi(q) in its place
+      mbar_wait(ss_done, c & 1, wc);
+      {
+        const float sc = alpha * __expf(bi) * izq;
+#pragma unroll
+        for (int e = 0; e < D; e += 8) {
+          float x[8];
+          ld_chunk8(pqb, kmajor_off(r, e, ROWS * 128), x);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[u] *= sc;
+          st_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
+        }
+      }
+      // ---- state: bf16 copy of S (MN-major B of the readout), then S <- e^{b_C} S
+      {
+        const float dec = __expf(bC);
+#pragma unroll
+        for (int col = 0; col < D; col += 32) {
+          float v[32];
+          tmem_ld32(lane_base + kColS + col, v);
+          tmem_wait_ld();
+          if (r < D) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 8)
+              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), &v[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= dec;
+          tmem_st32(lane_base + kColS + col, v);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(feat);
+
+      // ---- window softmax and the fused probability tile
+      mbar_wait(sg_done, c & 1, wc);
+      tc_fence_after();
+      {
+        float s[128];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float v[32];
+          tmem_ld32(lane_base + kColSs + q4 * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) s[q4 * 32 + u] = v[u];
+        }
+        // previous-chunk key kk is position t0 - 64 + kk: inside the window iff kk > i,
+        // inside the sequence iff kk >= 64 - (t0 - q0)
+        const int prev_lo = max(i + 1, C - (t0 - sg.q0));
+        float m = -INFINITY;
+#pragma unroll
+        for (int kk = 0; kk < 64; ++kk) {
+          if (kk >= prev_lo) m = fmaxf(m, s[kk]);
+          if (kk <= i) m = fmaxf(m, s[64 + kk]);
+        }
+        float l = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 64; ++kk) {
+          s[kk] = kk >= prev_lo ? exp2f((s[kk] - m) * sscale) : 0.f;
+          s[64 + kk] = kk <= i ? exp2f((s[64 + kk] - m) * sscale) : 0.f;
+          l += s[kk] + s[64 + kk];
+        }
+        const float coef = beta / l;
+#pragma unroll
+        for (int kk = 0; kk < 64; ++kk) s[kk] *= coef;
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          float v[32];
+          tmem_ld32(lane_base + kColSg + q2 * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int kk = q2 * 32 + u;
+            const float grm = kk <= i ? alpha * v[u] * izq * __expf(bi - bsh[kk]) : 0.f;
+            s[64 + kk] = s[64 + kk] * coef + grm;
+          }
+        }
+        // P tiles overwrite phi(q): K-major [128 rows][64 keys], previous then current
+#pragma unroll
+        for (int kk = 0; kk < 64; kk += 8) {
+          st_chunk8(pqb, sw128(r, kk >> 3), &s[kk]);
+          st_chunk8(pqb + ROWS * 128, sw128(r, kk >> 3), &s[64 + kk]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+
+      // ---- epilogue: O -> bf16 rows of out
+      const bool live = mbar_wait(o_done, c & 1, wc) && !*abort_flag;
+      tc_fence_after();
+      {
+        const long t = (long)t0 + i;
+        __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
+#pragma unroll
+        for (int col = 0; col < D; col += 32) {
+          float v[32];
+          tmem_ld32(lane_base + kColO + col, v);
+          tmem_wait_ld();
+          if (i < nv && live) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 8) {
+              uint4 w;
+              w.x = pack_bf16(v[u], v[u + 1]);
+              w.y = pack_bf16(v[u + 2], v[u + 3]);
+              w.z = pack_bf16(v[u + 4], v[u + 5]);
+              w.w = pack_bf16(v[u + 6], v[u + 7]);
+              *reinterpret_cast<uint4*>(orow + col + u) = w;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(o_free);
+      named_bar(1, 128);   // bsh is rewritten by the next chunk
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    mbar_wait(drain, 0, WaitCtx{never, nullptr, p.wait_ns});
+    tc_fence_after();
+    tmem_dealloc(tmem, TCOLS);
+  }
+}
+
+// ============================================================== host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+inline thread_local const char* g_msg = "";
+inline const char* last_message() { return g_msg; }
+
+inline bool supports(int d) { return d == 64 || d == 128; }
+
+inline int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Segment length (chunks) and the bound on segments: a segment is one chunk
+// CTA per q-head pair; pick the length that minimises waves x (length + fixed
+// per-segment cost) for one CTA per SM.
+inline Plan make_plan(int B, int Hq, int Hkv, long T, int d, int n_seqs, bool varlen) {
+  Plan pl{};
+  const long NT = varlen ? T : (long)B * T;
+  const long chunks_total = (NT + C - 1) / C + (varlen ? n_seqs : 0);
+  const long chunks_per_seq = varlen ? 0 : (T + C - 1) / C;
+  const int sms = num_sms();
+  const int pairs = Hq / 2;
+  double best = 1e300;
+  int bestL = 1;
+  const long maxL = chunks_total > 0 ? chunks_total : 1;
+  for (long Lc = 1; Lc <= maxL; Lc = Lc < 64 ? Lc + 1 : Lc + Lc / 8) {
+    long nseg = varlen ? (NT + C * Lc - 1) / (C * Lc) + n_seqs : (long)B * ((chunks_per_seq + Lc - 1) / Lc);
+    if (nseg < 1) nseg = 1;
+    const double waves = std::ceil((double)nseg * pairs / sms);
+    const double cost = waves * ((double)Lc + 1.5);
+    if (cost < best) { best = cost; bestL = (int)Lc; }
+  }
+  pl.L = bestL;
+  long nseg = varlen ? (NT + (long)C * bestL - 1) / ((long)C * bestL) + n_seqs
+                     : (long)B * ((chunks_per_seq + bestL - 1) / bestL);
+  if (nseg < 1) nseg = 1;
+  pl.n_seg_max = (int)nseg;
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  size_t off = 256;   // header: error word, segment count
+  pl.off_seqs = off;  off = al(off + sizeof(SeqInfo) * (size_t)n_seqs);
+  pl.off_segs = off;  off = al(off + sizeof(SegInfo) * (size_t)nseg);
+  pl.off_lam = off;   off = al(off + sizeof(float) * (size_t)nseg * Hkv);
+  pl.off_ds = off;    off = al(off + sizeof(float) * (size_t)nseg * Hkv * d * d);
+  pl.total = off;
+  return pl;
+}
+
+inline size_t workspace_bytes(int B, int Hq, int Hkv, long T, int d, int n_seqs) {
+  (void)n_seqs;
+  // The varlen bound is the larger one; use it so one size serves both forms.
+  const Plan a = make_plan(B, Hq, Hkv, T, d, B, false);
+  const Plan b = make_plan(1, Hq, Hkv, (long)B * T, d, n_seqs > 0 ? n_seqs : B, true);
+  return a.total > b.total ? a.total : b.total;
+}
+
+inline bool make_map(CUtensorMap* m, const void* ptr, int d, int H, long NT, int box_h) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)NT};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)C};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launch hooks supplied by the ABI layer (timing events and launch counting).
+struct LaunchHooks {
+  void (*before_main)(cudaStream_t);
+  void (*after_main)(cudaStream_t);
+  void (*count)(int);
+};
+
+inline uint64_t wait_limit_ns() {
+  const char* s = std::getenv("LIGER_WAIT_LIMIT_NS");
+  if (s && *s) {
+    const unsigned long long v = std::strtoull(s, nullptr, 10);
+    if (v > 0) return v;
+  }
+  return kDefaultWaitNs;
+}
+
+template <int D>
+liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk) {
+  const bool varlen = pb.cu != nullptr;
+  const long NT = varlen ? pb.T : (long)pb.B * pb.T;
+  const Plan pl = make_plan(pb.B, pb.Hq, pb.Hkv, pb.T, D, pb.n_seqs, varlen);
+  char* w = static_cast<char*>(ws);
+  DevParams p{};
+  p.seqs = reinterpret_cast<const SeqInfo*>(w + pl.off_seqs);
+  p.segs = reinterpret_cast<const SegInfo*>(w + pl.off_segs);
+  p.n_segs = reinterpret_cast<const int32_t*>(w + 4);
+  p.err = reinterpret_cast<uint32_t*>(w);
+  p.lam = reinterpret_cast<float*>(w + pl.off_lam);
+  p.ds = reinterpret_cast<float*>(w + pl.off_ds);
+  p.out = pb.out;
+  p.final_state = pb.final_state;
+  p.cu = pb.cu;
+  p.T = pb.T;
+  p.NT = NT;
+  p.Hq = pb.Hq;
+  p.Hkv = pb.Hkv;
+  p.n_seqs = pb.n_seqs;
+  p.n_seg_max = pl.n_seg_max;
+  p.L = pl.L;
+  p.alpha = pb.alpha;
+  p.wait_ns = wait_limit_ns();
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, pb.q, D, pb.Hq, NT, 2) || !make_map(&mk, pb.k, D, pb.Hkv, NT, 1) ||
+      !make_map(&mv, pb.v, D, pb.Hkv, NT, 1)) {
+    g_msg = "cuTensorMapEncodeTiled failed (driver entry point missing or unsupported layout)";
+    return LIGER_ERR_CUDA;
+  }
+  cudaError_t e;
+  plan_kernel<<<1, 32, 0, s>>>(p, reinterpret_cast<SeqInfo*>(w + pl.off_seqs),
+                               reinterpret_cast<SegInfo*>(w + pl.off_segs), reinterpret_cast<int32_t*>(w + 4));
+  hk.count(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+
+  auto seg_k = seg_state_kernel<D>;
+  if (cudaFuncSetAttribute(seg_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SegSmem<D>::BYTES) !=
+      cudaSuccess) {
+    g_msg = "cudaFuncSetAttribute(seg_state) failed";
+    cudaGetLastError();
+    return LIGER_ERR_CUDA;
+  }
+  seg_k<<<(unsigned)pl.n_seg_max * pb.Hkv, NTHREADS, SegSmem<D>::BYTES, s>>>(mk, mv, p);
+  hk.count(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+
+  dim3 sgrid((unsigned)(pb.n_seqs * pb.Hkv), (unsigned)((D * D) / 1024));
+  scan_kernel<D><<<sgrid, 256, 0, s>>>(p);
+  hk.count(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+
+  auto chunk_k = chunk_kernel<D>;
+  if (cudaFuncSetAttribute(chunk_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChunkSmem<D>::BYTES) !=
+      cudaSuccess) {
+    g_msg = "cudaFuncSetAttribute(chunk) failed";
+    cudaGetLastError();
+    return LIGER_ERR_CUDA;
+  }
+  hk.before_main(s);
+  chunk_k<<<(unsigned)pl.n_seg_max * (pb.Hq / 2), NTHREADS, ChunkSmem<D>::BYTES, s>>>(mq, mk, mv, p);
+  hk.after_main(s);
+  hk.count(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  return LIGER_OK;
+}
+
+inline liger_status run_prefill(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk) {
+  g_msg = "";
+  return pb.d == 64 ? run_prefill_d<64>(pb, ws, s, hk) : run_prefill_d<128>(pb, ws, s, hk);
+}
 
 }  // namespace tc
 }  // namespace liger
