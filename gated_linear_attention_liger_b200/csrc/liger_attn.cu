@@ -114,6 +114,11 @@ liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n
 
 }  // namespace
 
+namespace liger {
+// Records a failure for liger_last_error() from other translation units of the library.
+void set_last_error(liger_status status, const char* message) { fail(status, "%s", message); }
+}  // namespace liger
+
 extern "C" {
 
 int liger_abi_version(void) { return LIGER_ABI_VERSION; }

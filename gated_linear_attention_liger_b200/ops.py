@@ -35,6 +35,8 @@ SIGNATURES = {
                                 _vp, _vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "liger_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
                                _i, _vp]),
+    "liger_attn_prefill_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                                        _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }

@@ -126,6 +126,35 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
                                void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                int d, int w, float alpha, liger_dtype dt, void* stream);
 
+/*
+ * Prefill without caller-provided scratch (the pages have no counterpart; this
+ * is a deployment convenience).  For callers that cannot allocate device
+ * memory where they run the prefill -- a plugin whose host framework owns all
+ * device allocations and offers it no allocator, a serving loop that reserved
+ * all device memory up front, a latency-critical path that must not take the
+ * implicit synchronisation of cudaMalloc/cudaFree.  Same arguments and results
+ * as liger_attn_prefill without the workspace pair; the scratch is a fixed
+ * array of LIGER_PREFILL_NOALLOC_SCRATCH_BYTES in this library's device image,
+ * which every GPU that loads the library holds until the process exits.
+ *   - Sizes whose liger_attn_prefill_workspace_size() exceeds that maximum are
+ *     rejected with LIGER_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - The function itself allocates nothing: no cudaMalloc, no cudaFree, no
+ *     allocating library routine.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose work may
+ *     overlap on the GPU (different streams, or several host threads) race on
+ *     it: serialise them, or use liger_attn_prefill with separate workspaces.
+ */
+#define LIGER_PREFILL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+liger_status liger_attn_prefill_noalloc(const void* q, const void* k, const void* v, void* out,
+                                        float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
+                                        float alpha, liger_dtype dt, const float* initial_state,
+                                        const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
+                                        int32_t* pos_out, void* stream);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char* liger_last_error(void);
 
