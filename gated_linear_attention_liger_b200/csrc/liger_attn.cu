@@ -107,6 +107,20 @@ liger_status launch_ring(const void* k, const void* v, void* ring, int32_t* pos,
   return cuda_check("prefill_ring launch");
 }
 
+template <typename Tin, int D>
+liger_status launch_decode(const liger::DecodeArgs& a, unsigned blocks, cudaStream_t s) {
+  constexpr size_t smem = liger::decode_smem_bytes<Tin, D>();
+  auto kern = liger::decode_kernel<Tin, D>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(decode)");
+  mark_start(s);
+  kern<<<blocks, liger::kDecodeThreads, smem, s>>>(a);
+  mark_stop(s);
+  ++g_launches;
+  return cuda_check("decode launch");
+}
+
 template <typename Tin>
 liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, cudaStream_t s) {
   return d == 64 ? launch_simt_prefill<Tin, 64>(a, n_seqs, s) : launch_simt_prefill<Tin, 128>(a, n_seqs, s);
@@ -207,17 +221,9 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha};
   const unsigned blocks = (unsigned)((long)B * Hq);
-  mark_start(s);
-  if (dt == LIGER_BF16) {
-    if (d == 64) liger::decode_kernel<__nv_bfloat16, 64><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
-    else liger::decode_kernel<__nv_bfloat16, 128><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
-  } else {
-    if (d == 64) liger::decode_kernel<float, 64><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
-    else liger::decode_kernel<float, 128><<<blocks, liger::kDecodeThreads, 0, s>>>(a);
-  }
-  mark_stop(s);
-  ++g_launches;
-  st = cuda_check("decode launch");
+  if (dt == LIGER_BF16) st = d == 64 ? launch_decode<__nv_bfloat16, 64>(a, blocks, s)
+                                     : launch_decode<__nv_bfloat16, 128>(a, blocks, s);
+  else st = d == 64 ? launch_decode<float, 64>(a, blocks, s) : launch_decode<float, 128>(a, blocks, s);
   if (st != LIGER_OK) return st;
   liger::advance_pos_kernel<<<(B + 255) / 256, 256, 0, s>>>(pos, B);
   ++g_launches;

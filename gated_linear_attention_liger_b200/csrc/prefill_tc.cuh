@@ -17,16 +17,19 @@
 //               launch needs no host synchronisation).
 //   seg_state : per (segment, kv head) the state a segment adds from a zero
 //               start, dS = sum over its chunks, and its total log decay.
-//   scan      : per (sequence, kv head) the state entering every segment and the
-//               final state (written to each q head of the group).
-//   chunk     : per (segment, pair of q heads of one kv head) the fused pass:
-//               TMA stages q/k/v chunks; four warps compute phi, gates and the
-//               window softmax on TMEM rows; one thread issues tcgen05 MMAs:
+//   chunk     : per (segment, pair of q heads of one kv head) the fused pass.
+//               Its prologue sums the earlier segments' dS into the entering
+//               state; after the last chunk it writes the final state.  TMA
+//               stages q/k/v chunks; four "feature" warps compute phi, gates and
+//               the state carry of chunk c+1 while four more warps run the window
+//               softmax and the epilogue of chunk c on TMEM rows; one thread
+//               issues the tcgen05 MMAs:
 //                 Ss = Q [K_prev;K_cur]^T        raw scores of the window band
 //                 Sg = phi(Q) phi(K)^T           recurrent scores
 //                 O  = (alpha e^{b_i}/Z_i e_q) S  inter-chunk readout
 //                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
 //                 O += P_prev V_prev + P_cur V_cur, P_cur = beta*softmax + alpha*decayed Sg
+//               (P is written to TMEM and read from there as the A operand)
 //               and the epilogue stores bf16 rows.
 // Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
 // is exactly the order a TMA box over (d, head, token) produces.
@@ -85,7 +88,7 @@ struct DevParams {
   const SeqInfo* seqs;
   const int32_t* n_segs;
   float* lam;            // [n_seg_max][Hkv]
-  float* ds;             // [n_seg_max][Hkv][D][D]: dS, replaced by the entering state by scan
+  float* ds;             // [n_seg_max][Hkv][D][D]: state each segment adds from a zero start
   uint32_t* err;
   void* out;
   float* final_state;
@@ -100,7 +103,8 @@ struct DevParams {
 
 __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* n_segs) {
   if (threadIdx.x != 0) return;
-  *p.err = 0u;
+  p.err[0] = 0u;
+  p.err[1] = 0u;
   int seg = 0;
   const long span = (long)C * p.L;
   for (int s = 0; s < p.n_seqs; ++s) {
@@ -121,6 +125,15 @@ __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* 
     }
   }
   *n_segs = seg;
+}
+
+// Final state of the sequences that have no token (packed input only): zero.
+// Grid (n_seqs, Hq), 256 threads.
+template <int D>
+__global__ void zero_empty_kernel(DevParams p) {
+  if (p.seqs[blockIdx.x].n_seg != 0) return;
+  float4* dst = reinterpret_cast<float4*>(p.final_state + ((size_t)blockIdx.x * p.Hq + blockIdx.y) * D * D);
+  for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ============================================================== row helpers
@@ -377,54 +390,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// ============================================================== scan kernel
-
-// Grid (n_seqs * Hkv, D*D / 1024), 256 threads x 4 floats.  Replaces dS of each
-// segment by the state entering it and writes the final state to every q head.
-template <int D>
-__global__ void scan_kernel(DevParams p) {
-  const int seq = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
-  const size_t e = ((size_t)blockIdx.y * blockDim.x + threadIdx.x) * 4;
-  if (e >= (size_t)D * D) return;
-  const SeqInfo si = p.seqs[seq];
-  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = si.first_seg; s < si.first_seg + si.n_seg; ++s) {
-    float4* cell = reinterpret_cast<float4*>(p.ds + ((size_t)s * p.Hkv + kv) * D * D + e);
-    const float4 d = *cell;
-    *cell = run;
-    const float g = __expf(p.lam[(size_t)s * p.Hkv + kv]);
-    run = make_float4(fmaf(g, run.x, d.x), fmaf(g, run.y, d.y), fmaf(g, run.z, d.z), fmaf(g, run.w, d.w));
-  }
-  if (p.final_state) {
-    const int G = p.Hq / p.Hkv;
-    for (int h = kv * G; h < (kv + 1) * G; ++h)
-      *reinterpret_cast<float4*>(p.final_state + ((size_t)seq * p.Hq + h) * D * D + e) = run;
-  }
-}
-
 // ============================================================== chunk kernel
 
 template <int D>
 struct ChunkSmem {
-  static constexpr uint32_t QB = ROWS * D * 2;    // q tile (two heads)
+  static constexpr uint32_t QB = ROWS * D * 2;    // q tile (two heads): raw q, then scaled phi(q)
   static constexpr uint32_t KV = C * D * 2;       // one chunk of k or v
-  static constexpr uint32_t PQB = ROWS * D * 2 > 2 * ROWS * 64 * 2 ? ROWS * D * 2 : 2 * ROWS * 64 * 2;
   static constexpr uint32_t Q0 = 0;
-  static constexpr uint32_t K0 = Q0 + QB;         // 3 slots
-  static constexpr uint32_t V0 = K0 + 3 * KV;     // 3 slots
-  static constexpr uint32_t PQ = V0 + 3 * KV;     // phi(q) (unnormalised), later P
-  static constexpr uint32_t PK = PQ + PQB;        // phi(k)
+  static constexpr uint32_t EQ = Q0 + QB;         // e_q = exp(q - max), bf16
+  static constexpr uint32_t K0 = EQ + QB;         // 2 key slots
+  static constexpr uint32_t V0 = K0 + 2 * KV;     // 3 value slots
+  static constexpr uint32_t PK = V0 + 3 * KV;     // phi(k)
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
   static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
   static constexpr uint32_t SMALL = SB + D * D * 2;
-  static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
+  static constexpr uint32_t SMALL_BYTES = 2560;
+  static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
-// TMEM columns of the chunk kernel.
-constexpr uint32_t kColSs = 0, kColSg = 128, kColO = 192;
+// TMEM columns of the chunk kernel (fp32 cells, lane = tile row).
+constexpr uint32_t kColSs = 0;     // window scores, previous keys then current keys (128)
+constexpr uint32_t kColSg = 128;   // recurrent scores (64)
+constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
+constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
+
+constexpr int kChunkThreads = 320;   // warps 0-3 window/epilogue, 4-7 features, 8 TMA, 9 MMA
 
 template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(kChunkThreads, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, DevParams p) {
   using L = ChunkSmem<D>;
@@ -433,21 +426,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   extern __shared__ __align__(1024) char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
-  uint64_t* kv_full = bars;          // [3]
-  uint64_t* kv_empty = bars + 3;     // [3]
-  uint64_t* q_full = bars + 6;
-  uint64_t* q_empty = bars + 7;
-  uint64_t* ss_done = bars + 8;
-  uint64_t* feat = bars + 9;
-  uint64_t* sg_done = bars + 10;
-  uint64_t* p_ready = bars + 11;
-  uint64_t* o_done = bars + 12;
-  uint64_t* o_free = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_full = bars;           // [2]
+  uint64_t* k_empty = bars + 2;      // [2]
+  uint64_t* v_full = bars + 4;       // [3]
+  uint64_t* v_empty = bars + 7;      // [3]
+  uint64_t* q_full = bars + 10;
+  uint64_t* q_empty = bars + 11;
+  uint64_t* ss_done = bars + 12;     // window scores written; raw q read
+  uint64_t* feat = bars + 13;        // features of the chunk ready (128 arrivals)
+  uint64_t* sg_done = bars + 14;     // recurrent scores and state carry done
+  uint64_t* mma2_done = bars + 15;   // + readout done: feature buffers free again
+  uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (128 arrivals)
+  uint64_t* p_ready = bars + 17;     // probability tile in TMEM (128 arrivals)
+  uint64_t* o_done = bars + 18;      // output accumulator complete
+  uint64_t* o_free = bars + 19;      // output read out (128 arrivals)
+  uint64_t* drain = bars + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
-  float* bsh = reinterpret_cast<float*>(bars + 18);   // 64 floats
+  volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
+  float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256);  // [2][64] running log-gate sums
+  float* eneg2 = bsh2 + 128;                                    // [2][64] e^{-b_j} (factored decay)
+  float* izq2 = eneg2 + 128;                                    // [2][128] 1 / sum_d e_q per row
+  float* fast2 = izq2 + 256;                                    // [2] factored decay usable
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -459,10 +459,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
-    mbar_init(ss_done, 1); mbar_init(feat, 128); mbar_init(sg_done, 1);
-    mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128); mbar_init(drain, 1);
+    mbar_init(ss_done, 1); mbar_init(feat, 128); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
+    mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
+    mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
     fence_mbar_init();
@@ -477,20 +479,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.err, p.wait_ns};
 
-  if (warp == 4) {   // ---------------- TMA producer
+  if (warp == 8) {   // ---------------- TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmq);
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
-      auto load_kv = [&](int u) {   // u-th key/value chunk: tokens t_begin + 64 (u - 1)
-        const int slot = u % 3;
-        const int t = sg.t_begin + (u - 1) * C;
-        mbar_arrive_expect_tx(&kv_full[slot], 2 * L::KV);
+      // key / value load u holds tokens t_begin + 64 (u - 1): u = 0 is the chunk before the segment
+      auto load_k = [&](int u) {
+        const int slot = u & 1;
+        mbar_arrive_expect_tx(&k_full[slot], L::KV);
 #pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb) {
-          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &kv_full[slot], kb * 64, kv, t);
-          tma_load_3d(smem + L::V0 + slot * L::KV + kb * C * 128, &tmv, &kv_full[slot], kb * 64, kv, t);
-        }
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &k_full[slot], kb * 64, kv,
+                      sg.t_begin + (u - 1) * C);
+      };
+      auto load_v = [&](int u) {
+        const int slot = u % 3;
+        mbar_arrive_expect_tx(&v_full[slot], L::KV);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(smem + L::V0 + slot * L::KV + kb * C * 128, &tmv, &v_full[slot], kb * 64, kv,
+                      sg.t_begin + (u - 1) * C);
       };
       auto load_q = [&](int c) {
         mbar_arrive_expect_tx(q_full, L::QB);
@@ -498,44 +507,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(smem + L::Q0 + kb * ROWS * 128, &tmq, q_full, kb * 64, h0, sg.t_begin + c * C);
       };
-      int kv_issued = 2, q_issued = 1;
-      load_kv(0);
-      load_kv(1);
+      int k_issued = 2, v_issued = 2, q_issued = 1;
+      load_k(0); load_v(0);
+      load_k(1); load_v(1);
       load_q(0);
       for (int c = 0; c + 1 < nch; ++c) {
         const int u = c + 2;
-        if (u >= 3 && !mbar_wait(&kv_empty[u % 3], (u / 3 - 1) & 1, wc)) break;
-        load_kv(u);
-        kv_issued = u + 1;
-        if (!mbar_wait(q_empty, c & 1, wc)) break;
+        if (!mbar_wait(&k_empty[u & 1], ((u >> 1) - 1) & 1, wc, wsite(1, 1, c))) break;
+        load_k(u);
+        k_issued = u + 1;
+        if (u >= 3 && !mbar_wait(&v_empty[u % 3], (u / 3 - 1) & 1, wc, wsite(1, 2, c))) break;
+        load_v(u);
+        v_issued = u + 1;
+        if (!mbar_wait(q_empty, c & 1, wc, wsite(1, 3, c))) break;
         load_q(c + 1);
         q_issued = c + 2;
       }
-      const WaitCtx drain_wc{never, nullptr, p.wait_ns};
-      for (int u = (kv_issued > 3 ? kv_issued - 3 : 0); u < kv_issued; ++u)
-        mbar_wait(&kv_full[u % 3], (u / 3) & 1, drain_wc);
-      mbar_wait(q_full, (q_issued - 1) & 1, drain_wc);
+      const WaitCtx dw{never, nullptr, p.wait_ns};   // never leave with copies in flight
+      for (int u = (k_issued > 2 ? k_issued - 2 : 0); u < k_issued; ++u) mbar_wait(&k_full[u & 1], (u >> 1) & 1, dw);
+      for (int u = (v_issued > 3 ? v_issued - 3 : 0); u < v_issued; ++u) mbar_wait(&v_full[u % 3], (u / 3) & 1, dw);
+      mbar_wait(q_full, (q_issued - 1) & 1, dw);
     }
-  } else if (warp == 5) {   // ---------------- MMA issuer
+  } else if (warp == 9) {   // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
       const uint32_t id_inter = idesc_bf16(128, D, 0, 1);
       const uint32_t id_state = idesc_bf16(128, D, 1, 1);
-      const uint32_t lbo_kt = D == 128 ? C * 128 : 0;
+      const uint32_t lbo_kt = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
       const uint32_t q_base = smem_u32(smem + L::Q0);
-      const uint32_t pq_base = smem_u32(smem + L::PQ);
+      const uint32_t eq_base = smem_u32(smem + L::EQ);
       const uint32_t pk_base = smem_u32(smem + L::PK);
       const uint32_t kt_base = smem_u32(smem + L::KT);
       const uint32_t sb_base = smem_u32(smem + L::SB);
-      for (int c = 0; c < nch; ++c) {
-        const int ks = (c + 1) % 3, ps = c % 3;
-        const uint32_t kc = smem_u32(smem + L::K0 + ks * L::KV), kp = smem_u32(smem + L::K0 + ps * L::KV);
-        const uint32_t vc = smem_u32(smem + L::V0 + ks * L::KV), vp = smem_u32(smem + L::V0 + ps * L::KV);
-        if (c == 0 && !mbar_wait(&kv_full[0], 0, wc)) break;
-        if (!mbar_wait(&kv_full[ks], ((c + 1) / 3) & 1, wc)) break;
-        if (!mbar_wait(q_full, c & 1, wc)) break;
+      bool ok = true;
+      auto issue_ss = [&](int c) {   // window scores against the previous and the current keys
+        if (c == 0) ok = ok && mbar_wait(&k_full[0], 0, wc, wsite(2, 1, c));
+        ok = ok && mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(2, 2, c));
+        ok = ok && mbar_wait(q_full, c & 1, wc, wsite(2, 3, c));
+        if (c > 0) ok = ok && mbar_wait(s_read, (c - 1) & 1, wc, wsite(2, 4, c));
+        if (!ok) return;
         tc_fence_after();
-        // window scores against the previous and the current chunk of keys
+        const uint32_t kp = smem_u32(smem + L::K0 + (c & 1) * L::KV);
+        const uint32_t kc = smem_u32(smem + L::K0 + ((c + 1) & 1) * L::KV);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
@@ -544,87 +557,129 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16_ss(tmem + kColSs + 64, a, sdesc_sw128(kc + ko, 16, 1024), id_n64, kk > 0);
         }
         mma_commit(ss_done);
-        if (!mbar_wait(feat, c & 1, wc)) break;
-        if (c > 0 && !mbar_wait(o_free, (c - 1) & 1, wc)) break;
+        mma_commit(&k_empty[c & 1]);   // the previous chunk's keys are no longer needed
+      };
+      auto issue_pv = [&](int c) {   // O += P_prev V_prev + P_cur V_cur, P read from TMEM
+        if (c == 0) ok = ok && mbar_wait(&v_full[0], 0, wc, wsite(2, 5, c));
+        ok = ok && mbar_wait(p_ready, c & 1, wc, wsite(2, 6, c));
+        if (!ok) return;
         tc_fence_after();
+        const uint32_t vp = smem_u32(smem + L::V0 + (c % 3) * L::KV);
+        const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk) {
+          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc_sw128(vp + kk * 2048, C * 128, 1024),
+                      id_inter, 1u);
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 + kk * 8, sdesc_sw128(vc + kk * 2048, C * 128, 1024),
+                      id_inter, 1u);
+        }
+        mma_commit(o_done);
+        mma_commit(&v_empty[c % 3]);   // the previous chunk's values are no longer needed
+      };
+      auto issue_sg_state = [&](int c) {
+        ok = ok && mbar_wait(feat, c & 1, wc, wsite(2, 7, c));
+        ok = ok && mbar_wait(&v_full[(c + 1) % 3], ((c + 1) / 3) & 1, wc, wsite(2, 8, c));
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-          // recurrent scores phi(Q) phi(K)^T
-          mma_bf16_ss(tmem + kColSg, sdesc_sw128(pq_base + qo, 16, 1024), sdesc_sw128(pk_base + ko, 16, 1024),
+          mma_bf16_ss(tmem + kColSg, sdesc_sw128(eq_base + qo, 16, 1024), sdesc_sw128(pk_base + ko, 16, 1024),
                       id_n64, kk > 0);
-          // inter-chunk readout: (scaled phi(Q)) x S, S as MN-major B
-          mma_bf16_ss(tmem + kColO, sdesc_sw128(q_base + qo, 16, 1024),
-                      sdesc_sw128(sb_base + kk * 2048, D * 128, 1024), id_inter, kk > 0);
         }
-        // state carry S += Ktilde^T V_cur (both MN-major)
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
           mma_bf16_ss(tmem + kColS, sdesc_sw128(kt_base + kk * 2048, lbo_kt, 1024),
                       sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
         mma_commit(sg_done);
-        mma_commit(q_empty);
-        if (!mbar_wait(p_ready, c & 1, wc)) break;
+      };
+      auto issue_inter = [&](int c) {   // O = (alpha e^{b_i} / Z_i e_q) S, S as MN-major B
+        if (c > 0) ok = ok && mbar_wait(o_free, (c - 1) & 1, wc, wsite(2, 9, c));
+        if (!ok) return;
         tc_fence_after();
-        // O += P_prev V_prev + P_cur V_cur
 #pragma unroll
-        for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16_ss(tmem + kColO, sdesc_sw128(pq_base + kk * 32, 16, 1024),
-                      sdesc_sw128(vp + kk * 2048, C * 128, 1024), id_inter, 1u);
-          mma_bf16_ss(tmem + kColO, sdesc_sw128(pq_base + ROWS * 128 + kk * 32, 16, 1024),
-                      sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_inter, 1u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
+          mma_bf16_ss(tmem + kColO, sdesc_sw128(q_base + qo, 16, 1024),
+                      sdesc_sw128(sb_base + kk * 2048, D * 128, 1024), id_inter, kk > 0);
         }
-        mma_commit(o_done);
-        mma_commit(&kv_empty[ps]);
+        mma_commit(mma2_done);
+        mma_commit(q_empty);
+      };
+      issue_ss(0);
+      issue_sg_state(0);
+      issue_inter(0);
+      for (int c = 1; c < nch && ok; ++c) {
+        issue_ss(c);
+        issue_pv(c - 1);
+        issue_sg_state(c);
+        issue_inter(c);
       }
+      issue_pv(nch - 1);
       mma_commit(drain);
     }
-  } else {   // ---------------- rows (threads 0..127)
-    const int r = threadIdx.x;
-    const int i = r >> 1, hl = r & 1;          // token in chunk, head in pair
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const float alpha = p.alpha, beta = 1.0f - p.alpha;
-    const float kLog2e = 1.4426950408889634f;
-    const float sscale = kLog2e / sqrtf((float)D);
+  } else if (warp >= 4) {   // ---------------- features (threads 0..127 of warps 4-7)
+    // Row threads never leave the loop early: after a timeout every wait returns
+    // at once (the CTA's abort flag is set), so the group still meets at each
+    // named barrier and warp-collective TMEM access stays uniform.
+    const int r = threadIdx.x - 128;
+    const int i = r >> 1;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float alpha = p.alpha;
     char* const qb = smem + L::Q0;
-    char* const pqb = smem + L::PQ;
+    char* const eqb = smem + L::EQ;
     char* const sbb = smem + L::SB;
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 
-    // entering state of this segment -> TMEM (rows >= D repeat rows 0..D-1)
+    // state entering the segment: sum over the earlier segments of the sequence of
+    // their contribution dS, each decayed by the total log gate of the segments after it
     {
-      const float* src = p.ds + (((size_t)seg * p.Hkv + kv) * D + (r % D)) * D;
+      const SeqInfo si = p.seqs[sg.seq];
+      const int row = r % D;
 #pragma unroll
       for (int col = 0; col < D; col += 32) {
-        float v[32];
+        float acc[32];
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src + col + u);
-          v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
+        for (int u = 0; u < 32; ++u) acc[u] = 0.f;
+        float dec = 1.f;
+        for (int s2 = seg - 1; s2 >= si.first_seg; --s2) {
+          const float* src = p.ds + (((size_t)s2 * p.Hkv + kv) * D + row) * D + col;
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src + u);
+            acc[u] = fmaf(dec, x.x, acc[u]);
+            acc[u + 1] = fmaf(dec, x.y, acc[u + 1]);
+            acc[u + 2] = fmaf(dec, x.z, acc[u + 2]);
+            acc[u + 3] = fmaf(dec, x.w, acc[u + 3]);
+          }
+          dec *= __expf(p.lam[(size_t)s2 * p.Hkv + kv]);
         }
-        tmem_st32(lane_base + kColS + col, v);
+        tmem_st32(lane_base + kColS + col, acc);
       }
       tmem_wait_st();
     }
 
     for (int c = 0; c < nch; ++c) {
-      const int ks = (c + 1) % 3;
       const int t0 = sg.t_begin + c * C;
       const int nv = min(C, sg.t_end - t0);
-      // (row threads never leave the loop early; see seg_state_kernel)
-      if (c == 0) mbar_wait(&kv_full[0], 0, wc);
-      mbar_wait(&kv_full[ks], ((c + 1) / 3) & 1, wc);
-      mbar_wait(q_full, c & 1, wc);
+      float* bsh = bsh2 + (c & 1) * 64;
+      mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
+      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 3, c));   // feature buffers and the state are free
+      tc_fence_after();
 
-      // ---- keys: phi(k), gates, running sums, decay-scaled keys
+      // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
       float ph[D / 2];
-      key_features<D>(smem + L::K0 + ks * L::KV, smem + L::PK, bsh, r, nv, ph);
+      key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, bsh, r, nv, ph);
       const float bC = bsh[nv - 1];
       write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+      const bool fast = bC >= -80.f;   // e^{-b_j} <= e^{80} stays finite in fp32
+      if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bsh[i]) : 0.f;
+      if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
       const float bi = bsh[i];
 
-      // ---- queries: e_q = exp(q - max) (bf16) and its sum
+      // queries: e_q = exp(q - max) (bf16) and its sum
       float mq = -INFINITY;
 #pragma unroll
       for (int e = 0; e < D; e += 8) {
@@ -643,24 +698,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           x[u] = __expf(x[u] - mq);
           zq += x[u];
         }
-        st_chunk8(pqb, kmajor_off(r, e, ROWS * 128), x);
+        st_chunk8(eqb, kmajor_off(r, e, ROWS * 128), x);
       }
       const float izq = 1.0f / zq;
+      izq2[(c & 1) * 128 + r] = izq;
 
-      // ---- after the window-score MMA has read raw q: scaled phi(q) in its place
-      mbar_wait(ss_done, c & 1, wc);
+      // after the window-score MMA has read raw q: scaled phi(q) in its place
+      mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
       {
         const float sc = alpha * __expf(bi) * izq;
 #pragma unroll
         for (int e = 0; e < D; e += 8) {
           float x[8];
-          ld_chunk8(pqb, kmajor_off(r, e, ROWS * 128), x);
+          ld_chunk8(eqb, kmajor_off(r, e, ROWS * 128), x);
 #pragma unroll
           for (int u = 0; u < 8; ++u) x[u] *= sc;
           st_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
         }
       }
-      // ---- state: bf16 copy of S (MN-major B of the readout), then S <- e^{b_C} S
+      // state: bf16 copy of S (MN-major B of the readout), then S <- e^{b_C} S
       {
         const float dec = __expf(bC);
 #pragma unroll
@@ -682,10 +738,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
-
-      // ---- window softmax and the fused probability tile
-      mbar_wait(sg_done, c & 1, wc);
+      named_bar(1, 128);   // this group's bsh buffer is rewritten two chunks later only
+    }
+    // final state of the sequence: the carry after the last chunk of its last segment
+    const SeqInfo si = p.seqs[sg.seq];
+    const bool last = seg == si.first_seg + si.n_seg - 1;
+    if (p.final_state && last && mbar_wait(mma2_done, (nch - 1) & 1, wc, wsite(3, 5, nch)) && !*abort_flag) {
       tc_fence_after();
+#pragma unroll
+      for (int col = 0; col < D; col += 32) {
+        float v[32];
+        tmem_ld32(lane_base + kColS + col, v);
+        tmem_wait_ld();
+        if (r < D) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float* dst = p.final_state + (((size_t)sg.seq * p.Hq + h0 + hh) * D + r) * D + col;
+#pragma unroll
+            for (int u = 0; u < 32; u += 4)
+              *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+          }
+        }
+      }
+    }
+  } else {   // ---------------- window softmax and epilogue (threads 0..127, warps 0-3)
+    const int r = threadIdx.x;
+    const int i = r >> 1, hl = r & 1;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float alpha = p.alpha, beta = 1.0f - p.alpha;
+    const float sscale = 1.4426950408889634f / sqrtf((float)D);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+
+    for (int c = 0; c < nch; ++c) {
+      const int t0 = sg.t_begin + c * C;
+      const int nv = min(C, sg.t_end - t0);
+      const float* bsh = bsh2 + (c & 1) * 64;
+      const float* eneg = eneg2 + (c & 1) * 64;
+      mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
+      tc_fence_after();
+      uint32_t pk[64];   // bf16 pairs: previous keys 0..31, current keys 32..63
       {
         float s[128];
 #pragma unroll
@@ -714,32 +805,52 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const float coef = beta / l;
 #pragma unroll
-        for (int kk = 0; kk < 64; ++kk) s[kk] *= coef;
+        for (int kk = 0; kk < 64; kk += 2) pk[kk >> 1] = pack_bf16(s[kk] * coef, s[kk + 1] * coef);
+        // recurrent part of the current-key probabilities: alpha phi(q_i).phi(k_j) e^{b_i - b_j}
+        const float izq = izq2[(c & 1) * 128 + r];
+        const float bi = bsh[i];
+        const bool fast = fast2[c & 1] != 0.f;
+        const float rowc = alpha * izq * (fast ? __expf(bi) : 1.f);
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
           float v[32];
           tmem_ld32(lane_base + kColSg + q2 * 32, v);
           tmem_wait_ld();
+          if (q2 == 1) {   // both score tiles are in registers: their TMEM may be reused
+            tc_fence_before();
+            mbar_arrive(s_read);
+          }
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
+          for (int u = 0; u < 32; u += 2) {
             const int kk = q2 * 32 + u;
-            const float grm = kk <= i ? alpha * v[u] * izq * __expf(bi - bsh[kk]) : 0.f;
-            s[64 + kk] = s[64 + kk] * coef + grm;
+            float g0, g1;
+            if (fast) {
+              g0 = rowc * v[u] * eneg[kk];
+              g1 = rowc * v[u + 1] * eneg[kk + 1];
+            } else {
+              g0 = rowc * v[u] * __expf(bi - bsh[kk]);
+              g1 = rowc * v[u + 1] * __expf(bi - bsh[kk + 1]);
+            }
+            g0 = kk <= i ? g0 : 0.f;
+            g1 = kk + 1 <= i ? g1 : 0.f;
+            pk[32 + (kk >> 1)] = pack_bf16(fmaf(s[64 + kk], coef, g0), fmaf(s[64 + kk + 1], coef, g1));
           }
         }
-        // P tiles overwrite phi(q): K-major [128 rows][64 keys], previous then current
-#pragma unroll
-        for (int kk = 0; kk < 64; kk += 8) {
-          st_chunk8(pqb, sw128(r, kk >> 3), &s[kk]);
-          st_chunk8(pqb + ROWS * 128, sw128(r, kk >> 3), &s[64 + kk]);
-        }
       }
-      fence_proxy_async_smem();
+      // the probability tile goes to TMEM, where the P.V MMA reads it as its A operand
+      {
+        float lo[32], hi[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) { lo[u] = __uint_as_float(pk[u]); hi[u] = __uint_as_float(pk[32 + u]); }
+        tmem_st32(lane_base + kColP, lo);
+        tmem_st32(lane_base + kColP + 32, hi);
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(p_ready);
 
-      // ---- epilogue: O -> bf16 rows of out
-      const bool live = mbar_wait(o_done, c & 1, wc) && !*abort_flag;
+      // epilogue: O -> bf16 rows of out
+      const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
       tc_fence_after();
       {
         const long t = (long)t0 + i;
@@ -764,7 +875,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(o_free);
-      named_bar(1, 128);   // bsh is rewritten by the next chunk
     }
   }
   __syncthreads();
@@ -885,7 +995,7 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   DevParams p{};
   p.seqs = reinterpret_cast<const SeqInfo*>(w + pl.off_seqs);
   p.segs = reinterpret_cast<const SegInfo*>(w + pl.off_segs);
-  p.n_segs = reinterpret_cast<const int32_t*>(w + 4);
+  p.n_segs = reinterpret_cast<const int32_t*>(w + 8);
   p.err = reinterpret_cast<uint32_t*>(w);
   p.lam = reinterpret_cast<float*>(w + pl.off_lam);
   p.ds = reinterpret_cast<float*>(w + pl.off_ds);
@@ -910,7 +1020,7 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   }
   cudaError_t e;
   plan_kernel<<<1, 32, 0, s>>>(p, reinterpret_cast<SeqInfo*>(w + pl.off_seqs),
-                               reinterpret_cast<SegInfo*>(w + pl.off_segs), reinterpret_cast<int32_t*>(w + 4));
+                               reinterpret_cast<SegInfo*>(w + pl.off_segs), reinterpret_cast<int32_t*>(w + 8));
   hk.count(1);
   if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
@@ -925,10 +1035,11 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   hk.count(1);
   if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
-  dim3 sgrid((unsigned)(pb.n_seqs * pb.Hkv), (unsigned)((D * D) / 1024));
-  scan_kernel<D><<<sgrid, 256, 0, s>>>(p);
-  hk.count(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (varlen && pb.final_state) {
+    zero_empty_kernel<D><<<dim3((unsigned)pb.n_seqs, (unsigned)pb.Hq), 256, 0, s>>>(p);
+    hk.count(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  }
 
   auto chunk_k = chunk_kernel<D>;
   if (cudaFuncSetAttribute(chunk_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChunkSmem<D>::BYTES) !=
@@ -938,7 +1049,7 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     return LIGER_ERR_CUDA;
   }
   hk.before_main(s);
-  chunk_k<<<(unsigned)pl.n_seg_max * (pb.Hq / 2), NTHREADS, ChunkSmem<D>::BYTES, s>>>(mq, mk, mv, p);
+  chunk_k<<<(unsigned)pl.n_seg_max * (pb.Hq / 2), kChunkThreads, ChunkSmem<D>::BYTES, s>>>(mq, mk, mv, p);
   hk.after_main(s);
   hk.count(1);
   if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }

@@ -71,8 +71,11 @@ struct WaitCtx {
 };
 
 // Wait for `parity` on `bar`; gives up after limit_ns (or as soon as another
-// role of the CTA has given up), recording the timeout.  Returns false on give-up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+// role of the CTA has given up), recording the timeout in error[0] and, for
+// the first wait to give up anywhere, its call-site code in error[1].
+// Returns false on give-up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          uint32_t site = 0xFFFFu) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -80,10 +83,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (*w.abort) return false;
     if (globaltimer_ns() - t0 > w.limit_ns) {
       *w.abort = 1u;
-      if (w.error) atomicOr(w.error, kErrTimeout);
+      if (w.error) {
+        atomicOr(w.error, kErrTimeout);
+        atomicCAS(w.error + 1, 0u, site);
+      }
       return false;
     }
   }
+}
+
+// Call-site code of a wait: role (1 producer, 2 MMA, 3 features, 4 window), barrier id, chunk.
+__device__ __forceinline__ uint32_t wsite(uint32_t role, uint32_t barrier, int chunk) {
+  return (role << 28) | (barrier << 20) | ((uint32_t)chunk & 0xFFFFFu);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -134,6 +145,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc]: A read from tensor memory, lane = row,
+// two consecutive bf16 K elements per 32-bit column (K-major).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
