@@ -170,25 +170,28 @@ template <int D>
 __device__ __forceinline__ void key_features(const char* kraw, char* phik, float* bsh, int r, int nv,
                                              float (&ph)[D / 2]) {
   constexpr int HALF = D / 2;
+  constexpr float kLog2e = 1.4426950408889634f;
   const int j = r >> 1, h = r & 1;
   float m = -INFINITY, sum = 0.f;
 #pragma unroll
   for (int c = 0; c < HALF / 8; ++c) {
-    float x[8];
-    ld_chunk8(kraw, kmajor_off(j, h * HALF + c * 8, C * 128), x);
+    const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, C * 128));
+    m = fmaxf(m, bf16x8_max(u));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      ph[c * 8 + u] = x[u];
-      m = fmaxf(m, x[u]);
-      sum += x[u];
+    for (int q = 0; q < 4; ++q) {
+      ph[c * 8 + 2 * q] = bf16_lo(w4[q]);
+      ph[c * 8 + 2 * q + 1] = bf16_hi(w4[q]);
+      sum += ph[c * 8 + 2 * q] + ph[c * 8 + 2 * q + 1];
     }
   }
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  const float ml = m * kLog2e;
   float z = 0.f;
 #pragma unroll
   for (int u = 0; u < HALF; ++u) {
-    ph[u] = __expf(ph[u] - m);
+    ph[u] = ex2(fmaf(ph[u], kLog2e, -ml));
     z += ph[u];
   }
   z += __shfl_xor_sync(0xffffffffu, z, 1);
@@ -410,7 +413,7 @@ struct ChunkSmem {
 
 // TMEM columns of the chunk kernel (fp32 cells, lane = tile row).
 constexpr uint32_t kColSs = 0;     // window scores, previous keys then current keys (128)
-constexpr uint32_t kColSg = 128;   // recurrent scores (64)
+constexpr uint32_t kColSg = 128;   // recurrent scores (64); then the recurrent probability tile (32)
 constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
 constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
 
@@ -446,8 +449,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
   float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256);  // [2][64] running log-gate sums
   float* eneg2 = bsh2 + 128;                                    // [2][64] e^{-b_j} (factored decay)
-  float* izq2 = eneg2 + 128;                                    // [2][128] 1 / sum_d e_q per row
-  float* fast2 = izq2 + 256;                                    // [2] factored decay usable
+  float* fast2 = eneg2 + 128;                                   // [2] factored decay usable
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -568,10 +570,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
-          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc_sw128(vp + kk * 2048, C * 128, 1024),
-                      id_inter, 1u);
-          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 + kk * 8, sdesc_sw128(vc + kk * 2048, C * 128, 1024),
-                      id_inter, 1u);
+          const uint64_t bp = sdesc_sw128(vp + kk * 2048, C * 128, 1024);
+          const uint64_t bc = sdesc_sw128(vc + kk * 2048, C * 128, 1024);
+          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, bp, id_inter, 1u);        // window, previous keys
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 + kk * 8, bc, id_inter, 1u);   // window, current keys
+          mma_bf16_ts(tmem + kColO, tmem + kColSg + kk * 8, bc, id_inter, 1u);       // recurrent, current keys
         }
         mma_commit(o_done);
         mma_commit(&v_empty[c % 3]);   // the previous chunk's values are no longer needed
@@ -595,18 +598,21 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                       sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
         mma_commit(sg_done);
       };
-      auto issue_inter = [&](int c) {   // O = (alpha e^{b_i} / Z_i e_q) S, S as MN-major B
+      auto issue_inter = [&](int c) {   // O = (e^{b_i} / Z_i e_q) (alpha S), S as MN-major B
         if (c > 0) ok = ok && mbar_wait(o_free, (c - 1) & 1, wc, wsite(2, 9, c));
         if (!ok) return;
         tc_fence_after();
+        // factored mode: the scaled e_q tile already is the A operand; otherwise it sits in the q buffer
+        const bool fast = fast2[c & 1] != 0.f;
+        const uint32_t a_base = fast ? eq_base : q_base;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColO, sdesc_sw128(q_base + qo, 16, 1024),
+          mma_bf16_ss(tmem + kColO, sdesc_sw128(a_base + qo, 16, 1024),
                       sdesc_sw128(sb_base + kk * 2048, D * 128, 1024), id_inter, kk > 0);
         }
         mma_commit(mma2_done);
-        mma_commit(q_empty);
+        if (!fast) mma_commit(q_empty);   // in factored mode the feature warps released it
       };
       issue_ss(0);
       issue_sg_state(0);
@@ -628,6 +634,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const int i = r >> 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float alpha = p.alpha;
+    constexpr float kLog2e = 1.4426950408889634f;
     char* const qb = smem + L::Q0;
     char* const eqb = smem + L::EQ;
     char* const sbb = smem + L::SB;
@@ -670,53 +677,75 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_after();
 
       // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
-      float ph[D / 2];
-      key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, bsh, r, nv, ph);
-      const float bC = bsh[nv - 1];
-      write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
-      const bool fast = bC >= -80.f;   // e^{-b_j} <= e^{80} stays finite in fp32
+      float bC;
+      {
+        float ph[D / 2];
+        key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, bsh, r, nv, ph);
+        bC = bsh[nv - 1];
+        write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+      }
+      // Factored mode (the chunk's total log gate >= -80): e^{b_i} and e^{-b_j} stay
+      // finite in fp32, so e^{b_i - b_j} can be split between the two operands.
+      const bool fast = bC >= -80.f;
       if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bsh[i]) : 0.f;
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
       const float bi = bsh[i];
 
-      // queries: e_q = exp(q - max) (bf16) and its sum
+      // queries: the raw row into registers, e_q = exp(q - max), Z = sum e_q
+      float e[D];
       float mq = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < D; e += 8) {
-        float x[8];
-        ld_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mq = fmaxf(mq, x[u]);
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8, ROWS * 128));
+        mq = fmaxf(mq, bf16x8_max(u));
+        e[c8 * 8 + 0] = bf16_lo(u.x); e[c8 * 8 + 1] = bf16_hi(u.x);
+        e[c8 * 8 + 2] = bf16_lo(u.y); e[c8 * 8 + 3] = bf16_hi(u.y);
+        e[c8 * 8 + 4] = bf16_lo(u.z); e[c8 * 8 + 5] = bf16_hi(u.z);
+        e[c8 * 8 + 6] = bf16_lo(u.w); e[c8 * 8 + 7] = bf16_hi(u.w);
       }
+      if (fast) {   // raw q now lives in registers: release its buffer once the score MMA read it too
+        named_bar(1, 128);
+        if (r == 0) {
+          mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
+          mbar_arrive(q_empty);
+        }
+      }
+      const float mql = mq * kLog2e;
       float zq = 0.f;
 #pragma unroll
-      for (int e = 0; e < D; e += 8) {
-        float x[8];
-        ld_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          x[u] = __expf(x[u] - mq);
-          zq += x[u];
-        }
-        st_chunk8(eqb, kmajor_off(r, e, ROWS * 128), x);
+      for (int u = 0; u < D; ++u) {
+        e[u] = ex2(fmaf(e[u], kLog2e, -mql));
+        zq += e[u];
       }
       const float izq = 1.0f / zq;
-      izq2[(c & 1) * 128 + r] = izq;
-
-      // after the window-score MMA has read raw q: scaled phi(q) in its place
-      mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-      {
-        const float sc = alpha * __expf(bi) * izq;
+      if (fast) {   // one tile e^{b_i} phi(q_i) serves the recurrent scores and the readout
+        const float sc = __expf(bi) * izq;
 #pragma unroll
-        for (int e = 0; e < D; e += 8) {
+        for (int c8 = 0; c8 < D / 8; ++c8) {
           float x[8];
-          ld_chunk8(eqb, kmajor_off(r, e, ROWS * 128), x);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] *= sc;
-          st_chunk8(qb, kmajor_off(r, e, ROWS * 128), x);
+          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * sc;
+          st_chunk8(eqb, kmajor_off(r, c8 * 8, ROWS * 128), x);
+        }
+      } else {      // phi(q_i) for the scores; e^{b_i} phi(q_i) for the readout in the q buffer
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * izq;
+          st_chunk8(eqb, kmajor_off(r, c8 * 8, ROWS * 128), x);
+        }
+        mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
+        const float sc = __expf(bi) * izq;
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * sc;
+          st_chunk8(qb, kmajor_off(r, c8 * 8, ROWS * 128), x);
         }
       }
-      // state: bf16 copy of S (MN-major B of the readout), then S <- e^{b_C} S
+      // state: bf16 copy of alpha S (MN-major B of the readout), then S <- e^{b_C} S
       {
         const float dec = __expf(bC);
 #pragma unroll
@@ -726,8 +755,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           tmem_wait_ld();
           if (r < D) {
 #pragma unroll
-            for (int u = 0; u < 32; u += 8)
-              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), &v[u]);
+            for (int u = 0; u < 32; u += 8) {
+              float x[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
+              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
+            }
           }
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] *= dec;
@@ -764,6 +797,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   } else {   // ---------------- window softmax and epilogue (threads 0..127, warps 0-3)
     const int r = threadIdx.x;
     const int i = r >> 1, hl = r & 1;
+    const int wq = warp, il = i - 16 * wq;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
@@ -776,74 +810,82 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float* eneg = eneg2 + (c & 1) * 64;
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
       tc_fence_after();
-      uint32_t pk[64];   // bf16 pairs: previous keys 0..31, current keys 32..63
-      {
-        float s[128];
+      const bool fast = fast2[c & 1] != 0.f;
+      // Window band.  Key index x over [previous chunk | current chunk] (0..127): row i
+      // sees x in [i+1, i+64].  This warp's tokens are 16 wq .. 16 wq + 15, so it reads the
+      // 80 columns starting at 16 wq; column j then holds x = 16 wq + j and is live for
+      // j in [il+1, il+64], il = i - 16 wq.
+      float s[80];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float v[32];
-          tmem_ld32(lane_base + kColSs + q4 * 32, v);
-          tmem_wait_ld();
+      for (int q5 = 0; q5 < 5; ++q5) tmem_ld16(lane_base + kColSs + 16 * wq + 16 * q5, s + 16 * q5);
+      tmem_wait_ld();
+      s[0] = -INFINITY;
 #pragma unroll
-          for (int u = 0; u < 32; ++u) s[q4 * 32 + u] = v[u];
-        }
-        // previous-chunk key kk is position t0 - 64 + kk: inside the window iff kk > i,
-        // inside the sequence iff kk >= 64 - (t0 - q0)
-        const int prev_lo = max(i + 1, C - (t0 - sg.q0));
-        float m = -INFINITY;
+      for (int j = 1; j < 16; ++j) s[j] = j <= il ? -INFINITY : s[j];
 #pragma unroll
-        for (int kk = 0; kk < 64; ++kk) {
-          if (kk >= prev_lo) m = fmaxf(m, s[kk]);
-          if (kk <= i) m = fmaxf(m, s[64 + kk]);
-        }
-        float l = 0.f;
+      for (int j = 64; j < 80; ++j) s[j] = j > il + 64 ? -INFINITY : s[j];
+      if (t0 == sg.q0) {   // first chunk of the sequence: the previous chunk's keys are not its own
+        const int lim = 64 - 16 * wq;
 #pragma unroll
-        for (int kk = 0; kk < 64; ++kk) {
-          s[kk] = kk >= prev_lo ? exp2f((s[kk] - m) * sscale) : 0.f;
-          s[64 + kk] = kk <= i ? exp2f((s[64 + kk] - m) * sscale) : 0.f;
-          l += s[kk] + s[64 + kk];
-        }
-        const float coef = beta / l;
+        for (int j = 0; j < 64; ++j) s[j] = j < lim ? -INFINITY : s[j];
+      }
+      float m = s[1];
 #pragma unroll
-        for (int kk = 0; kk < 64; kk += 2) pk[kk >> 1] = pack_bf16(s[kk] * coef, s[kk + 1] * coef);
-        // recurrent part of the current-key probabilities: alpha phi(q_i).phi(k_j) e^{b_i - b_j}
-        const float izq = izq2[(c & 1) * 128 + r];
-        const float bi = bsh[i];
-        const bool fast = fast2[c & 1] != 0.f;
-        const float rowc = alpha * izq * (fast ? __expf(bi) : 1.f);
+      for (int j = 2; j < 80; ++j) m = fmaxf(m, s[j]);
+      const float msc = m * sscale;
+      float l = 0.f;
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-          float v[32];
-          tmem_ld32(lane_base + kColSg + q2 * 32, v);
-          tmem_wait_ld();
-          if (q2 == 1) {   // both score tiles are in registers: their TMEM may be reused
-            tc_fence_before();
-            mbar_arrive(s_read);
-          }
+      for (int j = 0; j < 80; ++j) {
+        s[j] = ex2(fmaf(s[j], sscale, -msc));
+        l += s[j];
+      }
+      const float coef = beta / l;
+      uint32_t pd[40];
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const int kk = q2 * 32 + u;
-            float g0, g1;
-            if (fast) {
-              g0 = rowc * v[u] * eneg[kk];
-              g1 = rowc * v[u + 1] * eneg[kk + 1];
-            } else {
-              g0 = rowc * v[u] * __expf(bi - bsh[kk]);
-              g1 = rowc * v[u + 1] * __expf(bi - bsh[kk + 1]);
-            }
-            g0 = kk <= i ? g0 : 0.f;
-            g1 = kk + 1 <= i ? g1 : 0.f;
-            pk[32 + (kk >> 1)] = pack_bf16(fmaf(s[64 + kk], coef, g0), fmaf(s[64 + kk + 1], coef, g1));
-          }
+      for (int k = 0; k < 40; ++k) pd[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
+
+      // recurrent scores of the current keys kk <= i (this warp needs kk < 16 wq + 16)
+      float g[64];
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        if (bb <= wq) {
+          tmem_ld16(lane_base + kColSg + 16 * bb, g + 16 * bb);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) g[16 * bb + u] = 0.f;
         }
       }
-      // the probability tile goes to TMEM, where the P.V MMA reads it as its A operand
-      {
-        float lo[32], hi[32];
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_read);   // both score tiles are in registers: their TMEM may be reused
+      uint32_t ag[32];
+      if (fast) {   // e^{b_i} is already in the scores: multiply by e^{-b_kk}
 #pragma unroll
-        for (int u = 0; u < 32; ++u) { lo[u] = __uint_as_float(pk[u]); hi[u] = __uint_as_float(pk[32 + u]); }
-        tmem_st32(lane_base + kColP, lo);
-        tmem_st32(lane_base + kColP + 32, hi);
+        for (int k = 0; k < 32; ++k) {
+          const int kk = 2 * k;
+          const float g0 = kk <= i ? alpha * g[kk] * eneg[kk] : 0.f;
+          const float g1 = kk + 1 <= i ? alpha * g[kk + 1] * eneg[kk + 1] : 0.f;
+          ag[k] = pack_bf16(g0, g1);
+        }
+      } else {
+        const float bi = bsh[i];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int kk = 2 * k;
+          const float g0 = kk <= i ? alpha * g[kk] * __expf(bi - bsh[kk]) : 0.f;
+          const float g1 = kk + 1 <= i ? alpha * g[kk + 1] * __expf(bi - bsh[kk + 1]) : 0.f;
+          ag[k] = pack_bf16(g0, g1);
+        }
+      }
+      // probability tiles to TMEM: the window tile over all 128 keys (zeros outside this
+      // warp's band) and the recurrent tile over the current keys (in the score tile's place)
+      {
+        const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 5; ++k) tmem_st8u(lane_base + kColP + 8 * wq + 8 * k, pd + 8 * k);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) tmem_st8u(lane_base + kColP + ((8 * wq + 40 + 8 * k) & 63), zero8);
+        tmem_st32u(lane_base + kColSg, ag);
         tmem_wait_st();
       }
       tc_fence_before();
