@@ -184,6 +184,12 @@ def barrier(world):
         dist.barrier()
 
 
+def weak_scaling_value(tokens_per_rank: int, world: int, max_ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload, the step time
+    is the slowest rank's."""
+    return world * tokens_per_rank / (max_ms_per_step * 1e-3)
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     if world == 1:
         return x
@@ -321,7 +327,7 @@ def run_ours(args, world, rank, local):
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     ms_step = ms_total / args.steps
     k_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ks, ke)), world, dev)
-    value = world * wl.tokens / (ms_step * 1e-3)
+    value = weak_scaling_value(wl.tokens, world, ms_step)
     alg_bytes, alg_flops = prefill_algorithmic(wl)
     achieved = alg_bytes / (k_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -172,28 +172,36 @@ __device__ __forceinline__ void key_features(const char* kraw, char* phik, float
   constexpr int HALF = D / 2;
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r >> 1, h = r & 1;
-  float m = -INFINITY, sum = 0.f;
+  // independent partial maxima and sums keep the dependency chains short
+  float mx[HALF / 8], sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < HALF / 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, C * 128));
-    m = fmaxf(m, bf16x8_max(u));
+    mx[c] = bf16x8_max(u);
     const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       ph[c * 8 + 2 * q] = bf16_lo(w4[q]);
       ph[c * 8 + 2 * q + 1] = bf16_hi(w4[q]);
-      sum += ph[c * 8 + 2 * q] + ph[c * 8 + 2 * q + 1];
+      sm[q] += ph[c * 8 + 2 * q] + ph[c * 8 + 2 * q + 1];
     }
   }
+#pragma unroll
+  for (int c = HALF / 16; c >= 1; c >>= 1)
+#pragma unroll
+    for (int t = 0; t < c; ++t) mx[t] = fmaxf(mx[t], mx[t + c]);
+  float m = mx[0];
+  float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   const float ml = m * kLog2e;
-  float z = 0.f;
+  float zs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int u = 0; u < HALF; ++u) {
     ph[u] = ex2(fmaf(ph[u], kLog2e, -ml));
-    z += ph[u];
+    zs[u & 3] += ph[u];
   }
+  float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
   z += __shfl_xor_sync(0xffffffffu, z, 1);
   const float iz = 1.0f / z;
 #pragma unroll
@@ -394,6 +402,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // ============================================================== chunk kernel
+
+// Rows of the state entering segment `seg` (columns [c0, c0 + NC)): the sum over
+// the earlier segments of the sequence of their contribution dS, each decayed by
+// the total log gate of the segments after it, stored to TMEM.  Three segments'
+// loads are issued before their products are accumulated.
+template <int D, int NC>
+__device__ __forceinline__ void entering_state(const DevParams& p, int seg, int first_seg, int kv, int row,
+                                               uint32_t taddr, int c0) {
+#pragma unroll
+  for (int col = c0; col < c0 + NC; col += 32) {
+    float acc[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) acc[u] = 0.f;
+    float dec = 1.f;
+    for (int s2 = seg - 1; s2 >= first_seg; s2 -= 3) {
+      float4 x[3][8];
+      float g[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const int sk = s2 - k;
+        const bool in = sk >= first_seg;
+        const float* src = p.ds + (((size_t)(in ? sk : s2) * p.Hkv + kv) * D + row) * D + col;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          x[k][u] = in ? *reinterpret_cast<const float4*>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        g[k] = in ? __expf(p.lam[(size_t)sk * p.Hkv + kv]) : 1.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          acc[4 * u] = fmaf(dec, x[k][u].x, acc[4 * u]);
+          acc[4 * u + 1] = fmaf(dec, x[k][u].y, acc[4 * u + 1]);
+          acc[4 * u + 2] = fmaf(dec, x[k][u].z, acc[4 * u + 2]);
+          acc[4 * u + 3] = fmaf(dec, x[k][u].w, acc[4 * u + 3]);
+        }
+        dec *= g[k];
+      }
+    }
+    tmem_st32(taddr + col, acc);
+  }
+  tmem_wait_st();
+}
 
 template <int D>
 struct ChunkSmem {
@@ -639,33 +690,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     char* const eqb = smem + L::EQ;
     char* const sbb = smem + L::SB;
 
-    // state entering the segment: sum over the earlier segments of the sequence of
-    // their contribution dS, each decayed by the total log gate of the segments after it
-    {
-      const SeqInfo si = p.seqs[sg.seq];
-      const int row = r % D;
-#pragma unroll
-      for (int col = 0; col < D; col += 32) {
-        float acc[32];
-#pragma unroll
-        for (int u = 0; u < 32; ++u) acc[u] = 0.f;
-        float dec = 1.f;
-        for (int s2 = seg - 1; s2 >= si.first_seg; --s2) {
-          const float* src = p.ds + (((size_t)s2 * p.Hkv + kv) * D + row) * D + col;
-#pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(src + u);
-            acc[u] = fmaf(dec, x.x, acc[u]);
-            acc[u + 1] = fmaf(dec, x.y, acc[u + 1]);
-            acc[u + 2] = fmaf(dec, x.z, acc[u + 2]);
-            acc[u + 3] = fmaf(dec, x.w, acc[u + 3]);
-          }
-          dec *= __expf(p.lam[(size_t)s2 * p.Hkv + kv]);
-        }
-        tmem_st32(lane_base + kColS + col, acc);
-      }
-      tmem_wait_st();
-    }
+    // state entering the segment, first half of the columns (the window warps do the rest)
+    entering_state<D, D / 2>(p, seg, p.seqs[sg.seq].first_seg, kv, r % D, lane_base + kColS, 0);
+    tc_fence_before();
+    named_bar(2, 256);
+    tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -673,7 +702,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       float* bsh = bsh2 + (c & 1) * 64;
       mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
       mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 3, c));   // feature buffers and the state are free
+      if (c > 0) mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));   // phi(k), keys~ and the state are free
       tc_fence_after();
 
       // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
@@ -691,18 +720,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
       const float bi = bsh[i];
 
-      // queries: the raw row into registers, e_q = exp(q - max), Z = sum e_q
-      float e[D];
-      float mq = -INFINITY;
+      // queries: the raw row into registers (bf16 pairs), e_q = exp(q - max), Z = sum e_q
+      uint32_t ep[D / 2];
+      float mxq[D / 8];
 #pragma unroll
       for (int c8 = 0; c8 < D / 8; ++c8) {
         const uint4 u = *reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8, ROWS * 128));
-        mq = fmaxf(mq, bf16x8_max(u));
-        e[c8 * 8 + 0] = bf16_lo(u.x); e[c8 * 8 + 1] = bf16_hi(u.x);
-        e[c8 * 8 + 2] = bf16_lo(u.y); e[c8 * 8 + 3] = bf16_hi(u.y);
-        e[c8 * 8 + 4] = bf16_lo(u.z); e[c8 * 8 + 5] = bf16_hi(u.z);
-        e[c8 * 8 + 6] = bf16_lo(u.w); e[c8 * 8 + 7] = bf16_hi(u.w);
+        mxq[c8] = bf16x8_max(u);
+        ep[4 * c8] = u.x; ep[4 * c8 + 1] = u.y; ep[4 * c8 + 2] = u.z; ep[4 * c8 + 3] = u.w;
       }
+#pragma unroll
+      for (int w2 = D / 16; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int t = 0; t < w2; ++t) mxq[t] = fmaxf(mxq[t], mxq[t + w2]);
+      const float mq = mxq[0];
       if (fast) {   // raw q now lives in registers: release its buffer once the score MMA read it too
         named_bar(1, 128);
         if (r == 0) {
@@ -711,51 +742,48 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
       }
       const float mql = mq * kLog2e;
-      float zq = 0.f;
+      float zqs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int u = 0; u < D; ++u) {
-        e[u] = ex2(fmaf(e[u], kLog2e, -mql));
-        zq += e[u];
+      for (int k = 0; k < D / 2; ++k) {
+        const float lo = ex2(fmaf(bf16_lo(ep[k]), kLog2e, -mql));
+        const float hi = ex2(fmaf(bf16_hi(ep[k]), kLog2e, -mql));
+        zqs[k & 7] += lo + hi;
+        ep[k] = pack_bf16(lo, hi);
       }
-      const float izq = 1.0f / zq;
+      const float izq = 1.0f / (((zqs[0] + zqs[1]) + (zqs[2] + zqs[3])) + ((zqs[4] + zqs[5]) + (zqs[6] + zqs[7])));
+      // the e_q tile and the state copy are still read by the previous chunk's readout
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));
+      auto store_scaled = [&](char* dst, float sc) {
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          float x[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            x[2 * q] = bf16_lo(ep[4 * c8 + q]) * sc;
+            x[2 * q + 1] = bf16_hi(ep[4 * c8 + q]) * sc;
+          }
+          st_chunk8(dst, kmajor_off(r, c8 * 8, ROWS * 128), x);
+        }
+      };
       if (fast) {   // one tile e^{b_i} phi(q_i) serves the recurrent scores and the readout
-        const float sc = __expf(bi) * izq;
-#pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          float x[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * sc;
-          st_chunk8(eqb, kmajor_off(r, c8 * 8, ROWS * 128), x);
-        }
+        store_scaled(eqb, __expf(bi) * izq);
       } else {      // phi(q_i) for the scores; e^{b_i} phi(q_i) for the readout in the q buffer
-#pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          float x[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * izq;
-          st_chunk8(eqb, kmajor_off(r, c8 * 8, ROWS * 128), x);
-        }
+        store_scaled(eqb, izq);
         mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-        const float sc = __expf(bi) * izq;
-#pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          float x[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] = e[c8 * 8 + u] * sc;
-          st_chunk8(qb, kmajor_off(r, c8 * 8, ROWS * 128), x);
-        }
+        store_scaled(qb, __expf(bi) * izq);
       }
       // state: bf16 copy of alpha S (MN-major B of the readout), then S <- e^{b_C} S
       {
         const float dec = __expf(bC);
 #pragma unroll
-        for (int col = 0; col < D; col += 32) {
-          float v[32];
+        for (int col = 0; col < D; col += 64) {
+          float v[64];
           tmem_ld32(lane_base + kColS + col, v);
+          tmem_ld32(lane_base + kColS + col + 32, v + 32);
           tmem_wait_ld();
           if (r < D) {
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) {
+            for (int u = 0; u < 64; u += 8) {
               float x[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
@@ -763,8 +791,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             }
           }
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= dec;
+          for (int u = 0; u < 64; ++u) v[u] *= dec;
           tmem_st32(lane_base + kColS + col, v);
+          tmem_st32(lane_base + kColS + col + 32, v + 32);
         }
         tmem_wait_st();
       }
@@ -802,6 +831,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    // state entering the segment, second half of the columns (TMEM: the state follows O)
+    entering_state<D, D / 2>(p, seg, p.seqs[sg.seq].first_seg, kv, r % D, lane_base + kColO + D, D / 2);
+    tc_fence_before();
+    named_bar(2, 256);
+    tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -829,17 +863,21 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
         for (int j = 0; j < 64; ++j) s[j] = j < lim ? -INFINITY : s[j];
       }
-      float m = s[1];
+      float mw[8];
 #pragma unroll
-      for (int j = 2; j < 80; ++j) m = fmaxf(m, s[j]);
+      for (int t = 0; t < 8; ++t) mw[t] = fmaxf(s[t], s[t + 8]);
+#pragma unroll
+      for (int j = 16; j < 80; ++j) mw[j & 7] = fmaxf(mw[j & 7], s[j]);
+      const float m = fmaxf(fmaxf(fmaxf(mw[0], mw[1]), fmaxf(mw[2], mw[3])),
+                            fmaxf(fmaxf(mw[4], mw[5]), fmaxf(mw[6], mw[7])));
       const float msc = m * sscale;
-      float l = 0.f;
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 80; ++j) {
         s[j] = ex2(fmaf(s[j], sscale, -msc));
-        l += s[j];
+        ls[j & 7] += s[j];
       }
-      const float coef = beta / l;
+      const float coef = beta / (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
       uint32_t pd[40];
 #pragma unroll
       for (int k = 0; k < 40; ++k) pd[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
