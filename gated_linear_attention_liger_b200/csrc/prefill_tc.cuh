@@ -161,14 +161,32 @@ __device__ __forceinline__ void st_chunk8(char* base, uint32_t off, const float*
   *reinterpret_cast<uint4*>(base + off) = u;
 }
 
+// Running sums of the log gates of one chunk: lane l of every warp of the group
+// holds the sums up to tokens 2l and 2l+1; b_at() fetches token x's sum.
+struct GateSums {
+  float b0, b1;
+  __device__ __forceinline__ float at(int x) const {
+    const float v0 = __shfl_sync(0xffffffffu, b0, x >> 1);
+    const float v1 = __shfl_sync(0xffffffffu, b1, x >> 1);
+    return (x & 1) ? v1 : v0;
+  }
+};
+
+// log sigmoid(m) = -softplus(-m) with the fast exp/log units (no overflow either side).
+__device__ __forceinline__ float log_sigmoid_fast(float m) {
+  const float t = __logf(1.0f + __expf(-fabsf(m)));
+  return fminf(m, 0.f) - t;
+}
+
 // Feature map and gate of one chunk of keys, shared by the seg_state and chunk
 // kernels.  Thread r (0..127) owns half of token j = r >> 1: elements
 // [h * D/2, (h+1) * D/2) with h = r & 1.  Writes phi(k) (bf16) to `phik` (may be
-// null), the log gates to bsh[0..63] (0 past the valid tokens), scans them to
-// running sums in bsh, and returns the thread's phi values in ph.
+// null), the log gates to lg[0..63] (0 past the valid tokens), and returns the
+// thread's phi values in ph and the running sums in gs (every warp scans the 64
+// gates itself); lanes of the group's first warp also store the sums to bsh.
 template <int D>
-__device__ __forceinline__ void key_features(const char* kraw, char* phik, float* bsh, int r, int nv,
-                                             float (&ph)[D / 2]) {
+__device__ __forceinline__ void key_features(const char* kraw, char* phik, float* lg, float* bsh, int r, int nv,
+                                             float (&ph)[D / 2], GateSums& gs) {
   constexpr int HALF = D / 2;
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r >> 1, h = r & 1;
@@ -210,32 +228,35 @@ __device__ __forceinline__ void key_features(const char* kraw, char* phik, float
 #pragma unroll
     for (int c = 0; c < HALF / 8; ++c) st_chunk8(phik, kmajor_off(j, h * HALF + c * 8, C * 128), &ph[c * 8]);
   }
-  if (h == 0) bsh[j] = j < nv ? log_sigmoid(sum / (float)D) : 0.f;
+  if (h == 0) lg[j] = j < nv ? log_sigmoid_fast(sum / (float)D) : 0.f;
   named_bar(1, 128);
-  if (r < 32) {   // inclusive running sum over the 64 tokens, two per lane
-    const float a0 = bsh[2 * r], a1 = bsh[2 * r + 1];
+  {   // inclusive running sum over the 64 tokens, two per lane, in every warp
+    const int lane = r & 31;
+    const float a0 = lg[2 * lane], a1 = lg[2 * lane + 1];
     float s = a0 + a1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float t = __shfl_up_sync(0xffffffffu, s, o);
-      if (r >= o) s += t;
+      if (lane >= o) s += t;
     }
     const float before = s - a0 - a1;
-    __syncwarp();
-    bsh[2 * r] = before + a0;
-    bsh[2 * r + 1] = before + a0 + a1;
+    gs.b0 = before + a0;
+    gs.b1 = before + a0 + a1;
+    if (r < 32 && bsh) {
+      bsh[2 * r] = gs.b0;
+      bsh[2 * r + 1] = gs.b1;
+    }
   }
-  named_bar(1, 128);
 }
 
 // Decay-scaled keys e^{b_C - b_j} phi(k_j) (zero past the valid tokens), written
 // in the same swizzled layout; read by the MMA as the MN-major A operand K^T.
 template <int D>
-__device__ __forceinline__ void write_ktilde(char* kt, const float* bsh, int r, int nv, float bC,
+__device__ __forceinline__ void write_ktilde(char* kt, float bj, int r, int nv, float bC,
                                              const float (&ph)[D / 2]) {
   constexpr int HALF = D / 2;
   const int j = r >> 1, h = r & 1;
-  const float sc = j < nv ? __expf(bC - bsh[j]) : 0.f;
+  const float sc = j < nv ? __expf(bC - bj) : 0.f;
 #pragma unroll
   for (int c = 0; c < HALF / 8; ++c) {
     float x[8];
@@ -270,7 +291,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
-  float* bsh = reinterpret_cast<float*>(bars + 10);   // 64 floats
+  float* lg = reinterpret_cast<float*>(bars + 10);   // 64 floats
 
   const int seg = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
   if (seg >= *p.n_segs) return;
@@ -350,14 +371,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
       mbar_wait(&kv_full[slot], (c >> 1) & 1, wc);
       float ph[D / 2];
-      key_features<D>(smem + L::K0 + slot * L::KV, nullptr, bsh, r, nv, ph);
-      const float bC = bsh[nv - 1];
+      GateSums gs;
+      key_features<D>(smem + L::K0 + slot * L::KV, nullptr, lg, nullptr, r, nv, ph, gs);
+      const float bC = gs.at(nv - 1);
+      const float bj = gs.at(r >> 1);
       lam += bC;
       if (c > 0) {
         mbar_wait(mma_done, (c - 1) & 1, wc);
         tc_fence_after();
       }
-      write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+      write_ktilde<D>(smem + L::KT, bj, r, nv, bC, ph);
       if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
         const float dec = __expf(bC);
 #pragma unroll
@@ -374,7 +397,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
-      named_bar(1, 128);   // bsh is rewritten by the next chunk
+      named_bar(1, 128);   // lg is rewritten by the next chunk
     }
     if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
       tc_fence_after();
@@ -458,7 +481,7 @@ struct ChunkSmem {
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
   static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
   static constexpr uint32_t SMALL = SB + D * D * 2;
-  static constexpr uint32_t SMALL_BYTES = 2560;
+  static constexpr uint32_t SMALL_BYTES = 3072;
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
@@ -500,7 +523,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
   float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256);  // [2][64] running log-gate sums
   float* eneg2 = bsh2 + 128;                                    // [2][64] e^{-b_j} (factored decay)
-  float* fast2 = eneg2 + 128;                                   // [2] factored decay usable
+  float* zq2 = eneg2 + 128;                                     // [2][128] Z = sum_d e_q per row
+  float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
+  float* fast2 = lg + 64;                                       // [2] factored decay usable
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -706,21 +731,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_after();
 
       // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
-      float bC;
+      float bC, bi;
       {
         float ph[D / 2];
-        key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, bsh, r, nv, ph);
-        bC = bsh[nv - 1];
-        write_ktilde<D>(smem + L::KT, bsh, r, nv, bC, ph);
+        GateSums gs;
+        key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, lg, bsh, r, nv, ph, gs);
+        bC = gs.at(nv - 1);
+        bi = gs.at(i);
+        write_ktilde<D>(smem + L::KT, bi, r, nv, bC, ph);   // key token j = r >> 1 = i
       }
       // Factored mode (the chunk's total log gate >= -80): e^{b_i} and e^{-b_j} stay
       // finite in fp32, so e^{b_i - b_j} can be split between the two operands.
       const bool fast = bC >= -80.f;
-      if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bsh[i]) : 0.f;
+      if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bi) : 0.f;
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
-      const float bi = bsh[i];
 
-      // queries: the raw row into registers (bf16 pairs), e_q = exp(q - max), Z = sum e_q
+      // queries: the raw row into registers (bf16 pairs), e_q = exp(q - max) and Z = sum e_q.
+      // The tiles carry e_q unnormalised; the window warps fold Z into P and 1/Z into the output.
       uint32_t ep[D / 2];
       float mxq[D / 8];
 #pragma unroll
@@ -733,7 +760,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       for (int w2 = D / 16; w2 >= 1; w2 >>= 1)
 #pragma unroll
         for (int t = 0; t < w2; ++t) mxq[t] = fmaxf(mxq[t], mxq[t + w2]);
-      const float mq = mxq[0];
+      const float mql = mxq[0] * kLog2e;
       if (fast) {   // raw q now lives in registers: release its buffer once the score MMA read it too
         named_bar(1, 128);
         if (r == 0) {
@@ -741,19 +768,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           mbar_arrive(q_empty);
         }
       }
-      const float mql = mq * kLog2e;
+      // factored mode: pack e^{b_i} e_q (one tile for the recurrent scores and the readout);
+      // otherwise pack e_q for the scores (e^{b_i} e_q for the readout goes to the q buffer)
+      const float ebi = fast ? __expf(bi) : 1.f;
       float zqs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < D / 2; ++k) {
         const float lo = ex2(fmaf(bf16_lo(ep[k]), kLog2e, -mql));
         const float hi = ex2(fmaf(bf16_hi(ep[k]), kLog2e, -mql));
         zqs[k & 7] += lo + hi;
-        ep[k] = pack_bf16(lo, hi);
+        ep[k] = pack_bf16(lo * ebi, hi * ebi);
       }
-      const float izq = 1.0f / (((zqs[0] + zqs[1]) + (zqs[2] + zqs[3])) + ((zqs[4] + zqs[5]) + (zqs[6] + zqs[7])));
+      zq2[(c & 1) * 128 + r] = ((zqs[0] + zqs[1]) + (zqs[2] + zqs[3])) + ((zqs[4] + zqs[5]) + (zqs[6] + zqs[7]));
       // the e_q tile and the state copy are still read by the previous chunk's readout
       if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));
-      auto store_scaled = [&](char* dst, float sc) {
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; ++c8)
+        *reinterpret_cast<uint4*>(eqb + kmajor_off(r, c8 * 8, ROWS * 128)) =
+            make_uint4(ep[4 * c8], ep[4 * c8 + 1], ep[4 * c8 + 2], ep[4 * c8 + 3]);
+      if (!fast) {
+        mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
+        const float sc = __expf(bi);
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
           float x[8];
@@ -762,15 +797,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             x[2 * q] = bf16_lo(ep[4 * c8 + q]) * sc;
             x[2 * q + 1] = bf16_hi(ep[4 * c8 + q]) * sc;
           }
-          st_chunk8(dst, kmajor_off(r, c8 * 8, ROWS * 128), x);
+          st_chunk8(qb, kmajor_off(r, c8 * 8, ROWS * 128), x);
         }
-      };
-      if (fast) {   // one tile e^{b_i} phi(q_i) serves the recurrent scores and the readout
-        store_scaled(eqb, __expf(bi) * izq);
-      } else {      // phi(q_i) for the scores; e^{b_i} phi(q_i) for the readout in the q buffer
-        store_scaled(eqb, izq);
-        mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-        store_scaled(qb, __expf(bi) * izq);
       }
       // state: bf16 copy of alpha S (MN-major B of the readout), then S <- e^{b_C} S
       {
@@ -877,7 +905,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         s[j] = ex2(fmaf(s[j], sscale, -msc));
         ls[j & 7] += s[j];
       }
-      const float coef = beta / (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+      const float zrow = zq2[(c & 1) * 128 + r];   // the tiles carry e_q unnormalised: scale P by Z
+      const float coef = beta * zrow / (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
       uint32_t pd[40];
 #pragma unroll
       for (int k = 0; k < 40; ++k) pd[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
@@ -933,6 +962,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
       tc_fence_after();
       {
+        const float iz = 1.0f / zrow;
         const long t = (long)t0 + i;
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
 #pragma unroll
@@ -944,10 +974,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
             for (int u = 0; u < 32; u += 8) {
               uint4 w;
-              w.x = pack_bf16(v[u], v[u + 1]);
-              w.y = pack_bf16(v[u + 2], v[u + 3]);
-              w.z = pack_bf16(v[u + 4], v[u + 5]);
-              w.w = pack_bf16(v[u + 6], v[u + 7]);
+              w.x = pack_bf16(v[u] * iz, v[u + 1] * iz);
+              w.y = pack_bf16(v[u + 2] * iz, v[u + 3] * iz);
+              w.z = pack_bf16(v[u + 4] * iz, v[u + 5] * iz);
+              w.w = pack_bf16(v[u + 6] * iz, v[u + 7] * iz);
               *reinterpret_cast<uint4*>(orow + col + u) = w;
             }
           }
