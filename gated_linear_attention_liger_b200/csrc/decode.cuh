@@ -36,10 +36,22 @@ struct DecodeArgs {
 
 constexpr int kDecodeThreads = 256;
 
+// Shared-memory ring rows are padded by 16 bytes so that rows sit 4 banks apart.
+template <typename Tin, int D>
+constexpr int ring_row_elems() {
+  return D + 16 / (int)sizeof(Tin);
+}
 template <typename Tin, int D>
 constexpr size_t decode_smem_bytes() {
-  return sizeof(Tin) * 2 * 64 * D;   // window ring keys and values
+  return sizeof(Tin) * 2 * 64 * ring_row_elems<Tin, D>();   // window ring keys and values
 }
+
+// Programmatic dependent launch: let the next kernel in the stream start
+// launching now, and wait for the previous kernel's memory before touching it.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ float4 ld_stream(const float* p) {
   return __ldcs(reinterpret_cast<const float4*>(p));
@@ -57,6 +69,80 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+
+// Copies the window's ring rows (positions p-w+1 .. p-1, slot jj of the window =
+// position p-(w-1)+jj) of one (sequence, kv head) into shared memory (padded rows):
+// a flat loop over (row, 16-byte piece), no integer division in the loop.
+template <typename Tin, int D, int NT>
+__device__ __forceinline__ void ring_to_smem(const Tin* rk, const Tin* rv, Tin* rk_s, Tin* rv_s, int p, int w,
+                                             int tid) {
+  constexpr int CPR = D * (int)sizeof(Tin) / 16;   // a power of two
+  constexpr int RS = ring_row_elems<Tin, D>();
+  const int base = (p + 1) % w;   // slot of window position jj = 0
+  for (int idx = tid; idx < 2 * w * CPR; idx += NT) {
+    const int rowi = idx / CPR, piece = idx % CPR;
+    const int which = rowi >= w ? 1 : 0;
+    const int jj = rowi - which * w;
+    const int j = p - (w - 1) + jj;
+    if (j < 0 || j == p) continue;
+    int slot = base + jj;
+    slot = slot >= w ? slot - w : slot;
+    const char* src = reinterpret_cast<const char*>((which ? rv : rk) + (size_t)slot * D);
+    char* dst = reinterpret_cast<char*>((which ? rv_s : rk_s) + jj * RS);
+    cp_async16(dst + piece * 16, src + piece * 16);
+  }
+}
+
+// Unpack 16 bytes of ring row into floats.
+template <typename Tin> __device__ __forceinline__ void ld16_vals(const Tin* p, float* x);
+template <> __device__ __forceinline__ void ld16_vals<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w4[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+  }
+}
+template <> __device__ __forceinline__ void ld16_vals<float>(const float* p, float* x) {
+  const float4 u = *reinterpret_cast<const float4*>(p);
+  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+}
+
+// Window scores q . k_j / sqrt(d) for the w slots, four threads per slot; thread
+// quarter qq takes the 16-byte pieces qq, qq+4, ... of the row (conflict-free on
+// the padded rows), reduced with two shuffles.  Needs blockDim >= 4 * w.
+template <typename Tin, int D>
+__device__ __forceinline__ void window_scores(const float* qv, const float* ks, const Tin* rk_s, float* sc, int p,
+                                              int w, int tid) {
+  constexpr int EPP = 16 / (int)sizeof(Tin);      // elements per 16-byte piece
+  constexpr int NP = D / EPP;                     // pieces per row
+  constexpr int RS = ring_row_elems<Tin, D>();
+  const int jj = tid >> 2, qq = tid & 3;
+  if (jj < 64) {   // all four lanes of a slot take part in the shuffles
+    const int j = p - (w - 1) + jj;
+    const bool live = jj < w && j >= 0;
+    float acc = 0.f;
+    if (live) {
+#pragma unroll
+      for (int pc = qq; pc < NP; pc += 4) {
+        float x[EPP];
+        if (j == p) {
+#pragma unroll
+          for (int e = 0; e < EPP; ++e) x[e] = ks[pc * EPP + e];
+        } else {
+          ld16_vals<Tin>(rk_s + jj * RS + pc * EPP, x);
+        }
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) acc = fmaf(qv[pc * EPP + e], x[e], acc);
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (qq == 0 && jj < w) sc[jj] = live ? acc * (1.0f / sqrtf((float)D)) : -INFINITY;
+  }
+}
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a) {
   constexpr int NT = kDecodeThreads;
@@ -68,7 +154,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   constexpr int ROWB = D * (int)sizeof(Tin);   // bytes of one ring row
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
-  Tin* rv_s = rk_s + 64 * D;                         // [64][D]
+  Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
   __shared__ __align__(16) float qs[D], ks[D], vs[D], fq[D], fk[D];
   __shared__ float sc[64];
   __shared__ __align__(16) float part[RGN][D];
@@ -80,6 +166,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cq = tid % CQ, rg = tid / CQ;
 
+  pdl_wait();
+  pdl_launch_dependents();
   // 1. the state rows this thread updates: all loads in flight at once
   float* S = a.state + ((size_t)b * Hq + h) * D * D;
   float4 st[RPT];
@@ -91,19 +179,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   Tin* ring = static_cast<Tin*>(a.ring);
   const Tin* rk = ring + (((size_t)b * Hkv + kv) * 2 + 0) * w * D;
   const Tin* rv = ring + (((size_t)b * Hkv + kv) * 2 + 1) * w * D;
-  {
-    constexpr int CPR = ROWB / 16;   // 16-byte pieces per row
-    for (int idx = tid; idx < w * CPR * 2; idx += NT) {
-      const int which = idx / (w * CPR);           // 0 keys, 1 values
-      const int rem = idx % (w * CPR);
-      const int jj = rem / CPR, piece = rem % CPR;
-      const long j = (long)p - (w - 1) + jj;
-      if (j < 0 || j == p) continue;
-      const Tin* src = (which ? rv : rk) + (size_t)(j % w) * D;
-      Tin* dst = (which ? rv_s : rk_s) + jj * D;
-      cp_async16(reinterpret_cast<char*>(dst) + piece * 16, reinterpret_cast<const char*>(src) + piece * 16);
-    }
-  }
+  ring_to_smem<Tin, D, NT>(rk, rv, rk_s, rv_s, p, w, tid);
   const Tin* qrow = static_cast<const Tin*>(a.q) + ((size_t)b * Hq + h) * D;
   const Tin* krow = static_cast<const Tin*>(a.k) + ((size_t)b * Hkv + kv) * D;
   const Tin* vrow = static_cast<const Tin*>(a.v) + ((size_t)b * Hkv + kv) * D;
@@ -116,25 +192,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   __syncthreads();
 
   // 3. window scores from shared memory (slot jj covers position p - (w-1) + jj)
-  const float inv_sqrt_d = 1.0f / sqrtf((float)D);
-  {
-    float qv[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) qv[e] = qs[lane + 32 * e];
-    for (int jj = warp; jj < w; jj += NT / 32) {
-      const long j = (long)p - (w - 1) + jj;
-      float dot = -INFINITY;
-      if (j >= 0) {
-        const Tin* kr = (j == p) ? nullptr : rk_s + jj * D;
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          acc = fmaf(qv[e], kr ? io<Tin>::ld(kr + lane + 32 * e) : ks[lane + 32 * e], acc);
-        dot = warp_sum(acc) * inv_sqrt_d;
-      }
-      if (lane == 0) sc[jj] = dot;
-    }
-  }
+  window_scores<Tin, D>(qs, ks, rk_s, sc, p, w, tid);
   // 4. phi(k) with the gate, and phi(q)
   if (warp == 0) {
     float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
@@ -179,7 +237,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
     for (int jj = grp; jj < w; jj += VG) {
       const long j = (long)p - (w - 1) + jj;
       if (j < 0) continue;
-      const float vx = (j == p) ? vs[e] : io<Tin>::ld(rv_s + jj * D + e);
+      const float vx = (j == p) ? vs[e] : io<Tin>::ld(rv_s + jj * ring_row_elems<Tin, D>() + e);
       acc = fmaf(sc[jj], vx, acc);
     }
     wpart[grp][e] = acc;
@@ -223,8 +281,170 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
 }
 
 __global__ void advance_pos_kernel(int32_t* pos, int B) {
+  pdl_wait();   // every CTA of the decode kernel has read pos
+  pdl_launch_dependents();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) pos[b] += 1;
+}
+
+}  // namespace liger
+
+namespace liger {
+
+// Decode over one state per (sequence, kv head): state [B, Hkv, d, d].  The q
+// heads of a group read the same state -- prefill writes identical copies and
+// a per-head decode keeps them identical -- so one CTA per (sequence, kv head)
+// streams that state once, applies S <- g S + phi(k)^T v once, and forms
+// o_h = alpha phi(q_h) S + (1 - alpha) window_h for each of the G heads.  The
+// fp32 state traffic per step drops by G.
+template <typename Tin, int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(DecodeArgs a) {
+  constexpr int NT = kDecodeThreads;
+  constexpr int CQ = D / 4;
+  constexpr int RGN = NT / CQ;
+  constexpr int RPT = D / RGN;
+  constexpr int EPL = D / 32;
+  constexpr int VG = NT / D;
+  constexpr int ROWB = D * (int)sizeof(Tin);
+  extern __shared__ __align__(16) unsigned char dsm[];
+  Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
+  Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
+  __shared__ __align__(16) float qs[G][D], fq[G][D], ks[D], vs[D], fk[D];
+  __shared__ float sc[G][64];
+  __shared__ __align__(16) float part[RGN][G][D];
+  __shared__ float wpart[VG][G][D];
+  __shared__ float gsh;
+
+  const int Hkv = a.Hkv, w = a.w, Hq = a.Hq;
+  const int b = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cq = tid % CQ, rg = tid / CQ;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  float* S = a.state + ((size_t)b * Hkv + kv) * D * D;
+  float4 st[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) st[r] = ld_stream(S + (size_t)(rg * RPT + r) * D + 4 * cq);
+
+  const int p = max(a.pos[b], 0);
+  Tin* ring = static_cast<Tin*>(a.ring);
+  const Tin* rk = ring + (((size_t)b * Hkv + kv) * 2 + 0) * w * D;
+  const Tin* rv = ring + (((size_t)b * Hkv + kv) * 2 + 1) * w * D;
+  ring_to_smem<Tin, D, NT>(rk, rv, rk_s, rv_s, p, w, tid);
+  const Tin* krow = static_cast<const Tin*>(a.k) + ((size_t)b * Hkv + kv) * D;
+  const Tin* vrow = static_cast<const Tin*>(a.v) + ((size_t)b * Hkv + kv) * D;
+  for (int idx = tid; idx < G * D; idx += NT) {
+    const int hh = idx / D, e = idx % D;
+    qs[hh][e] = io<Tin>::ld(static_cast<const Tin*>(a.q) + ((size_t)b * Hq + kv * G + hh) * D + e);
+  }
+  if (tid < D) {
+    ks[tid] = io<Tin>::ld(krow + tid);
+    vs[tid] = io<Tin>::ld(vrow + tid);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // window scores, head by head
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) window_scores<Tin, D>(qs[hh], ks, rk_s, sc[hh], p, w, tid);
+  // phi(k) with the gate (warp 0), phi(q_h) (warps 1..G)
+  if (warp == 0) {
+    float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { x[j] = ks[lane + 32 * j]; m = fmaxf(m, x[j]); sum += x[j]; }
+    m = warp_max(m);
+    sum = warp_sum(sum);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
+    z = warp_sum(z);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) fk[lane + 32 * j] = x[j] / z;
+    if (lane == 0) gsh = expf(log_sigmoid(sum / (float)D));
+  } else if (warp <= G) {
+    const int hh = warp - 1;
+    float x[EPL], m = -INFINITY, z = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { x[j] = qs[hh][lane + 32 * j]; m = fmaxf(m, x[j]); }
+    m = warp_max(m);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
+    z = warp_sum(z);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) fq[hh][lane + 32 * j] = x[j] / z;
+  }
+  __syncthreads();
+  if (warp < G) {   // window softmax of head `warp`
+    const int hh = warp;
+    const float x0 = lane < w ? sc[hh][lane] : -INFINITY;
+    const float x1 = lane + 32 < w ? sc[hh][lane + 32] : -INFINITY;
+    const float m = warp_max(fmaxf(x0, x1));
+    const float e0 = lane < w ? expf(x0 - m) : 0.f;
+    const float e1 = lane + 32 < w ? expf(x1 - m) : 0.f;
+    const float z = warp_sum(e0 + e1);
+    if (lane < w) sc[hh][lane] = e0 / z;
+    if (lane + 32 < w) sc[hh][lane + 32] = e1 / z;
+  }
+  __syncthreads();
+  {   // window value sums
+    const int e = tid % D, grp = tid / D;
+    float acc[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) acc[hh] = 0.f;
+    for (int jj = grp; jj < w; jj += VG) {
+      const long j = (long)p - (w - 1) + jj;
+      if (j < 0) continue;
+      const float vx = (j == p) ? vs[e] : io<Tin>::ld(rv_s + jj * ring_row_elems<Tin, D>() + e);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) acc[hh] = fmaf(sc[hh][jj], vx, acc[hh]);
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) wpart[grp][hh][e] = acc[hh];
+  }
+  // state update once, readout for every head of the group
+  const float g = gsh;
+  const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
+  float4 acc[G];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int row = rg * RPT + r;
+    const float kr = fk[row];
+    float4 x = st[r];
+    x.x = fmaf(g, x.x, kr * vv.x);
+    x.y = fmaf(g, x.y, kr * vv.y);
+    x.z = fmaf(g, x.z, kr * vv.z);
+    x.w = fmaf(g, x.w, kr * vv.w);
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const float qr = fq[hh][row];
+      acc[hh].x = fmaf(qr, x.x, acc[hh].x);
+      acc[hh].y = fmaf(qr, x.y, acc[hh].y);
+      acc[hh].z = fmaf(qr, x.z, acc[hh].z);
+      acc[hh].w = fmaf(qr, x.w, acc[hh].w);
+    }
+    st_stream(S + (size_t)row * D + 4 * cq, x);
+  }
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = acc[hh];
+  __syncthreads();
+  for (int idx = tid; idx < G * D; idx += NT) {
+    const int hh = idx / D, e = idx % D;
+    float grm = 0.f, swa = 0.f;
+#pragma unroll
+    for (int r = 0; r < RGN; ++r) grm += part[r][hh][e];
+#pragma unroll
+    for (int r = 0; r < VG; ++r) swa += wpart[r][hh][e];
+    Tin* orow = static_cast<Tin*>(a.out) + ((size_t)b * Hq + kv * G + hh) * D;
+    io<Tin>::st(orow + e, a.alpha * grm + (1.0f - a.alpha) * swa);
+  }
+  if (tid < D) {
+    Tin* wk = ring + (((size_t)b * Hkv + kv) * 2 + 0) * w * D + (size_t)(p % w) * D;
+    Tin* wv = ring + (((size_t)b * Hkv + kv) * 2 + 1) * w * D + (size_t)(p % w) * D;
+    wk[tid] = krow[tid];
+    wv[tid] = vrow[tid];
+  }
 }
 
 }  // namespace liger

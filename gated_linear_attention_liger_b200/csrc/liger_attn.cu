@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <string>
+#include <utility>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -35,6 +36,25 @@ void record(cudaEvent_t ev, cudaStream_t s) {
 void mark_start(cudaStream_t s) { if (g_ev_start) record(g_ev_start, s); }
 void mark_stop(cudaStream_t s) { if (g_ev_stop) record(g_ev_stop, s); }
 void count_launches(int n) { g_launches += (uint64_t)n; }
+
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel in the stream drains; it calls griddepcontrol.wait before it
+// touches memory that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 liger_status fail(liger_status s, const char* fmt, ...) {
   char buf[512];
@@ -115,10 +135,36 @@ liger_status launch_decode(const liger::DecodeArgs& a, unsigned blocks, cudaStre
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return cuda_check("cudaFuncSetAttribute(decode)");
   mark_start(s);
-  kern<<<blocks, liger::kDecodeThreads, smem, s>>>(a);
+  if (launch_pdl(kern, dim3(blocks), dim3(liger::kDecodeThreads), smem, s, a) != cudaSuccess)
+    return cuda_check("decode launch");
   mark_stop(s);
   ++g_launches;
   return cuda_check("decode launch");
+}
+
+template <typename Tin, int D, int G>
+liger_status launch_decode_kvshared(const liger::DecodeArgs& a, unsigned blocks, cudaStream_t s) {
+  constexpr size_t smem = liger::decode_smem_bytes<Tin, D>();
+  auto kern = liger::decode_kvshared_kernel<Tin, D, G>;
+  // static + dynamic shared memory can exceed the default 48 KiB: always raise the limit
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(decode_kvshared)");
+  mark_start(s);
+  if (launch_pdl(kern, dim3(blocks), dim3(liger::kDecodeThreads), smem, s, a) != cudaSuccess)
+    return cuda_check("decode_kvshared launch");
+  mark_stop(s);
+  ++g_launches;
+  return cuda_check("decode_kvshared launch");
+}
+
+template <typename Tin, int D>
+liger_status decode_kvshared_g(const liger::DecodeArgs& a, int G, unsigned blocks, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode_kvshared<Tin, D, 1>(a, blocks, s);
+    case 2: return launch_decode_kvshared<Tin, D, 2>(a, blocks, s);
+    case 4: return launch_decode_kvshared<Tin, D, 4>(a, blocks, s);
+    default: return fail(LIGER_ERR_UNSUPPORTED, "shared-state decode supports Hq/Hkv in {1, 2, 4} (got %d)", G);
+  }
 }
 
 template <typename Tin>
@@ -225,7 +271,39 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
                                      : launch_decode<__nv_bfloat16, 128>(a, blocks, s);
   else st = d == 64 ? launch_decode<float, 64>(a, blocks, s) : launch_decode<float, 128>(a, blocks, s);
   if (st != LIGER_OK) return st;
-  liger::advance_pos_kernel<<<(B + 255) / 256, 256, 0, s>>>(pos, B);
+  if (launch_pdl(liger::advance_pos_kernel, dim3((B + 255) / 256), dim3(256), 0, s, pos, B) != cudaSuccess)
+    return cuda_check("advance_pos launch");
+  ++g_launches;
+  return cuda_check("advance_pos launch");
+}
+
+liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void* v, float* state,
+                                        void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                                        int d, int w, float alpha, liger_dtype dt, void* stream) {
+  g_last_error.clear();
+  liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
+  if (st != LIGER_OK) return st;
+  if (B < 1) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 (B=%d)", B);
+  if ((long)B * Hkv > 0x7fffffffL) return fail(LIGER_ERR_UNSUPPORTED, "too many (sequence, kv head) units");
+  if (!q || !k || !v || !state || !swa_ring || !out || !pos)
+    return fail(LIGER_ERR_INVALID_ARG, "all decode pointers must be non-null");
+  const void* ptrs[] = {q, k, v, state, swa_ring, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(pos) & 3u) return fail(LIGER_ERR_INVALID_ARG, "pos must be 4-byte aligned");
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4)
+    return fail(LIGER_ERR_UNSUPPORTED, "shared-state decode supports Hq/Hkv in {1, 2, 4} (got %d)", G);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha};
+  const unsigned blocks = (unsigned)((long)B * Hkv);
+  if (dt == LIGER_BF16) st = d == 64 ? decode_kvshared_g<__nv_bfloat16, 64>(a, G, blocks, s)
+                                     : decode_kvshared_g<__nv_bfloat16, 128>(a, G, blocks, s);
+  else st = d == 64 ? decode_kvshared_g<float, 64>(a, G, blocks, s) : decode_kvshared_g<float, 128>(a, G, blocks, s);
+  if (st != LIGER_OK) return st;
+  if (launch_pdl(liger::advance_pos_kernel, dim3((B + 255) / 256), dim3(256), 0, s, pos, B) != cudaSuccess)
+    return cuda_check("advance_pos launch");
   ++g_launches;
   return cuda_check("advance_pos launch");
 }

@@ -35,6 +35,8 @@ SIGNATURES = {
                                 _vp, _vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "liger_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
                                _i, _vp]),
+    "liger_attn_decode_kvshared": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
+                                        _i, _vp]),
     "liger_attn_prefill_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                         _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "liger_set_timing_events": (None, [_vp, _vp]),
@@ -167,6 +169,26 @@ def decode(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None)
     if out is None:
         out = torch.empty_like(q)
     st = lib.liger_attn_decode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos), B, Hq, Hkv, d, w,
+        float(alpha), _dt(q), _stream_ptr(stream))
+    _check(st)
+    return out
+
+
+def decode_kvshared(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None):
+    """One decode step over one state per (sequence, kv head): state [B, Hkv, d, d] fp32.
+
+    Equivalent to `decode` when the per-head states of each group are equal (as
+    prefill leaves them); moves G = Hq/Hkv times less state per step.
+    """
+    lib = load()
+    _need_cuda(q, k, v, state, ring, pos)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    w = ring.shape[3]
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib.liger_attn_decode_kvshared(
         _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos), B, Hq, Hkv, d, w,
         float(alpha), _dt(q), _stream_ptr(stream))
     _check(st)

@@ -127,6 +127,22 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
                                int d, int w, float alpha, liger_dtype dt, void* stream);
 
 /*
+ * Decode over one state per (sequence, kv head).  Same operation as
+ * liger_attn_decode when the G = Hq/Hkv per-head states of a group are equal,
+ * which holds by construction after liger_attn_prefill (it writes identical
+ * copies) and under liger_attn_decode (identical updates).  The state is then
+ * stored once per group, and each step moves G times less of it.
+ *
+ *   q      [B, Hq, d] dt; k, v [B, Hkv, d] dt; out [B, Hq, d] dt
+ *   state  [B, Hkv, d, d] fp32 (in/out): S <- g S + phi(k)^T v once per group
+ *   swa_ring, pos: as for liger_attn_decode.
+ * Supported: G in {1, 2, 4} (other group sizes return LIGER_ERR_UNSUPPORTED).
+ */
+liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void* v, float* state,
+                                        void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                                        int d, int w, float alpha, liger_dtype dt, void* stream);
+
+/*
  * Prefill without caller-provided scratch (the pages have no counterpart; this
  * is a deployment convenience).  For callers that cannot allocate device
  * memory where they run the prefill -- a plugin whose host framework owns all

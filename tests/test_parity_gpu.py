@@ -238,3 +238,60 @@ def test_full_llama8b_decode(cuda_device):
         assert_close(np64(g_state[b:b + 1, hs]), st, wl.dtype, "state")
         np.testing.assert_array_equal(np64(g_ring[b:b + 1, kv:kv + 1]), rg)
     assert int(g_pos.min()) == wl.T + 200 == int(g_pos.max())
+
+
+# ----------------------------------------------------------------- shared-state decode
+
+@pytest.mark.parametrize("dtype,d,w,T0,G", [
+    (torch.bfloat16, 128, 64, 70, 4),
+    (torch.bfloat16, 64, 64, 0, 2),
+    (torch.bfloat16, 64, 16, 5, 1),
+    (torch.float32, 128, 64, 100, 4),
+])
+def test_decode_kvshared_parity(dtype, d, w, T0, G, cuda_device):
+    """One state per kv head: the oracle runs with that state copied to every q head of
+    the group; outputs, the (shared) state, ring and positions must match."""
+    B, Hkv, steps = 3, 2, 10
+    Hq = Hkv * G
+    wl = inputs.small("deckv", B=B, Hq=Hq, Hkv=Hkv, T=T0 + steps, d=d, dtype=dtype, seed=29)
+    q, k, v = inputs.prefill_inputs(wl)
+    if T0:
+        _, st, rg, ps = oracle.prefill(np64(q[:, :T0]), np64(k[:, :T0]), np64(v[:, :T0]), w=w)
+        kv_state = torch.tensor(st[:, ::G], dtype=torch.float32)   # heads of a group hold equal copies
+    else:
+        kv_state = torch.zeros(B, Hkv, d, d)
+        rg, ps = np.zeros((B, Hkv, 2, w, d)), np.zeros(B, np.int32)
+    st = np.repeat(np64(kv_state), G, axis=1)
+    g_state = kv_state.to(cuda_device)
+    g_ring = torch.tensor(rg).to(dtype)
+    rg = np64(g_ring)
+    g_ring = g_ring.to(cuda_device)
+    g_pos = torch.tensor(ps, dtype=torch.int32, device=cuda_device)
+    for t in range(T0, T0 + steps):
+        qt, kt, vt = q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous()
+        o = ops.decode_kvshared(qt.to(cuda_device), kt.to(cuda_device), vt.to(cuda_device), g_state, g_ring, g_pos)
+        ro, st, rg, ps = oracle.decode(np64(qt), np64(kt), np64(vt), st, rg, ps, w=w)
+        torch.cuda.synchronize()
+        assert_close(np64(o), ro, dtype, f"kv-shared decode out step {t}")
+    assert_close(np64(g_state), st[:, ::G], dtype, "kv-shared state")
+    np.testing.assert_array_equal(np64(g_ring), rg)
+    np.testing.assert_array_equal(g_pos.cpu().numpy(), ps)
+
+
+def test_decode_kvshared_matches_per_head_decode_full_shape(cuda_device):
+    """B=64 at the Llama-3-8B shape after a GPU prefill: 20 steps of the shared-state decode
+    track the per-head decode (same inputs, same starting point)."""
+    wl = inputs.WORKLOADS["llama8b_decode"]
+    G = wl.Hq // wl.Hkv
+    pre = inputs.Workload("pre", "prefill", wl.B, wl.Hq, wl.Hkv, 256, wl.d, wl.dtype, seed=wl.seed)
+    q, k, v = (t.to(cuda_device) for t in inputs.prefill_inputs(pre))
+    _, st, rg, ps = ops.prefill(q, k, v, return_ring=True)
+    st_kv = st[:, ::G].contiguous()
+    rg2, ps2 = rg.clone(), ps.clone()
+    for step in range(20):
+        qt, kt, vt = (t.to(cuda_device) for t in inputs.decode_step_inputs(wl, step))
+        o1 = ops.decode(qt, kt, vt, st, rg, ps)
+        o2 = ops.decode_kvshared(qt, kt, vt, st_kv, rg2, ps2)
+        assert_close(np64(o2), np64(o1), wl.dtype, f"step {step}")
+    assert_close(np64(st_kv), np64(st[:, ::G]), wl.dtype, "state")
+    assert torch.equal(rg, rg2) and torch.equal(ps, ps2)
