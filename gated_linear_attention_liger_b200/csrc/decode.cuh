@@ -151,7 +151,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   constexpr int RPT = D / RGN;       // rows per thread
   constexpr int EPL = D / 32;
   constexpr int VG = NT / D;         // window-sum key groups
-  constexpr int ROWB = D * (int)sizeof(Tin);   // bytes of one ring row
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
   Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
@@ -305,7 +304,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
   constexpr int RPT = D / RGN;
   constexpr int EPL = D / 32;
   constexpr int VG = NT / D;
-  constexpr int ROWB = D * (int)sizeof(Tin);
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
   Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]

@@ -277,6 +277,19 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
   return cuda_check("advance_pos launch");
 }
 
+liger_status liger_attn_prefill_status(const void* workspace, size_t workspace_bytes) {
+  g_last_error.clear();
+  if (!workspace || workspace_bytes < 12) return LIGER_OK;   // no tensor-core pass ran with it
+  uint32_t hdr[3] = {0u, 0u, 0u};
+  const cudaError_t e = cudaMemcpy(hdr, workspace, sizeof hdr, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "reading the workspace header: %s", cudaGetErrorString(e));
+  if (hdr[0] & 1u)
+    return fail(LIGER_ERR_TIMEOUT, "a prefill kernel gave up waiting (site 0x%08x: role %u, barrier %u, chunk %u)",
+                hdr[1], hdr[1] >> 28, (hdr[1] >> 20) & 0xFFu, hdr[1] & 0xFFFFFu);
+  if (hdr[0]) return fail(LIGER_ERR_CUDA, "prefill error word 0x%x", hdr[0]);
+  return LIGER_OK;
+}
+
 liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void* v, float* state,
                                         void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                         int d, int w, float alpha, liger_dtype dt, void* stream) {

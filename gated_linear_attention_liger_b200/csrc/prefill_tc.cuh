@@ -80,23 +80,29 @@ struct PrefillProblem {
 struct Plan {
   int L;            // chunks per segment
   int n_seg_max;    // upper bound on segments
+  int nsub, Ls;     // sub-segments per segment for the state pass, and their length in chunks
   size_t off_seqs, off_segs, off_lam, off_ds, total;
 };
+
+constexpr int kMaxSub = 8;
 
 struct DevParams {
   const SegInfo* segs;
   const SeqInfo* seqs;
   const int32_t* n_segs;
-  float* lam;            // [n_seg_max][Hkv]
-  float* ds;             // [n_seg_max][Hkv][D][D]: state each segment adds from a zero start
+  float* lam;            // [n_seg_max][nsub][Hkv] total log gate of each sub-segment
+  float* ds;             // [n_seg_max][nsub][Hkv][D][D]: state each sub-segment adds from a zero
+                         // start; the scan replaces [s][0] by the state entering segment s
   uint32_t* err;
   void* out;
   float* final_state;
   const int32_t* cu;
   long T, NT;
-  int Hq, Hkv, n_seqs, n_seg_max, L;
+  int Hq, Hkv, n_seqs, n_seg_max, L, nsub, Ls;
   float alpha;
   uint64_t wait_ns;
+  int out_v8;            // out is 32-byte aligned: 256-bit stores
+  int inject_stall;      // test switch: withhold one MMA completion so a wait runs out
 };
 
 // ============================================================== plan kernel
@@ -134,6 +140,46 @@ __global__ void zero_empty_kernel(DevParams p) {
   if (p.seqs[blockIdx.x].n_seg != 0) return;
   float4* dst = reinterpret_cast<float4*>(p.final_state + ((size_t)blockIdx.x * p.Hq + blockIdx.y) * D * D);
   for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// 32 bytes to global memory in one store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+// Per (sequence, kv head): folds the sub-segment contributions in order and
+// stores the state entering each segment in its first sub-segment slot.  Grid
+// (n_seqs * Hkv, D*D / 1024), 256 threads x 4 floats; every load of a segment is
+// issued before its products are accumulated.
+template <int D>
+__global__ void scan_kernel(DevParams p) {
+  const int seq = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  const size_t e = ((size_t)blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (e >= (size_t)D * D) return;
+  const SeqInfo si = p.seqs[seq];
+  const int nsub = p.nsub;
+  float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = si.first_seg; s < si.first_seg + si.n_seg; ++s) {
+    float4 d[kMaxSub];
+    float g[kMaxSub];
+#pragma unroll
+    for (int k = 0; k < kMaxSub; ++k) {
+      if (k < nsub) {
+        const size_t u = (size_t)s * nsub + k;
+        d[k] = *reinterpret_cast<const float4*>(p.ds + (u * p.Hkv + kv) * D * D + e);
+        g[k] = __expf(p.lam[u * p.Hkv + kv]);
+      }
+    }
+    *reinterpret_cast<float4*>(p.ds + ((size_t)s * nsub * p.Hkv + kv) * D * D + e) = run;
+#pragma unroll
+    for (int k = 0; k < kMaxSub; ++k) {
+      if (k < nsub)
+        run = make_float4(fmaf(g[k], run.x, d[k].x), fmaf(g[k], run.y, d[k].y), fmaf(g[k], run.z, d[k].z),
+                          fmaf(g[k], run.w, d[k].w));
+    }
+  }
 }
 
 // ============================================================== row helpers
@@ -276,7 +322,7 @@ struct SegSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, 2)
     seg_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      DevParams p) {
   using L = SegSmem<D>;
@@ -293,10 +339,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
   float* lg = reinterpret_cast<float*>(bars + 10);   // 64 floats
 
-  const int seg = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  const int unit = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
+  const int seg = unit / p.nsub, sub = unit % p.nsub;
   if (seg >= *p.n_segs) return;
-  const SegInfo sg = p.segs[seg];
-  const int nch = (sg.t_end - sg.t_begin + C - 1) / C;
+  const SegInfo sg0 = p.segs[seg];
+  const int nch_seg = (sg0.t_end - sg0.t_begin + C - 1) / C;
+  const int c_lo = sub * p.Ls, c_hi = min(c_lo + p.Ls, nch_seg);
+  float* const ds_out = p.ds + ((size_t)unit * p.Hkv + kv) * D * D;
+  if (c_lo >= c_hi) {   // an empty sub-segment adds nothing
+    for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x)
+      reinterpret_cast<float4*>(ds_out)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (threadIdx.x == 0) p.lam[(size_t)unit * p.Hkv + kv] = 0.f;
+    return;
+  }
+  SegInfo sg = sg0;   // this CTA's tokens
+  sg.t_begin = sg0.t_begin + c_lo * C;
+  sg.t_end = min(sg0.t_end, sg0.t_begin + c_hi * C);
+  const int nch = c_hi - c_lo;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t TCOLS = D < 32 ? 32 : D;
 
@@ -401,7 +460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
       tc_fence_after();
-      float* dst = p.ds + (((size_t)seg * p.Hkv + kv) * D + r) * D;
+      float* dst = ds_out + (size_t)r * D;
 #pragma unroll
       for (int col = 0; col < D; col += 32) {
         float v[32];
@@ -413,7 +472,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             *reinterpret_cast<float4*>(dst + col + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
         }
       }
-      if (r == 0) p.lam[(size_t)seg * p.Hkv + kv] = lam;
+      if (r == 0) p.lam[(size_t)unit * p.Hkv + kv] = lam;
     }
   }
   __syncthreads();
@@ -426,45 +485,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 // ============================================================== chunk kernel
 
-// Rows of the state entering segment `seg` (columns [c0, c0 + NC)): the sum over
-// the earlier segments of the sequence of their contribution dS, each decayed by
-// the total log gate of the segments after it, stored to TMEM.  Three segments'
-// loads are issued before their products are accumulated.
+// Rows of the state entering segment `seg` (columns [c0, c0 + NC)) from the scan's
+// output, stored to TMEM.
 template <int D, int NC>
-__device__ __forceinline__ void entering_state(const DevParams& p, int seg, int first_seg, int kv, int row,
-                                               uint32_t taddr, int c0) {
+__device__ __forceinline__ void entering_state(const DevParams& p, int seg, int kv, int row, uint32_t taddr,
+                                               int c0) {
+  const float* src = p.ds + (((size_t)seg * p.nsub * p.Hkv + kv) * D + row) * D;
 #pragma unroll
   for (int col = c0; col < c0 + NC; col += 32) {
-    float acc[32];
+    float v[32];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) acc[u] = 0.f;
-    float dec = 1.f;
-    for (int s2 = seg - 1; s2 >= first_seg; s2 -= 3) {
-      float4 x[3][8];
-      float g[3];
-#pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        const int sk = s2 - k;
-        const bool in = sk >= first_seg;
-        const float* src = p.ds + (((size_t)(in ? sk : s2) * p.Hkv + kv) * D + row) * D + col;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          x[k][u] = in ? *reinterpret_cast<const float4*>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
-        g[k] = in ? __expf(p.lam[(size_t)sk * p.Hkv + kv]) : 1.f;
-      }
-#pragma unroll
-      for (int k = 0; k < 3; ++k) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          acc[4 * u] = fmaf(dec, x[k][u].x, acc[4 * u]);
-          acc[4 * u + 1] = fmaf(dec, x[k][u].y, acc[4 * u + 1]);
-          acc[4 * u + 2] = fmaf(dec, x[k][u].z, acc[4 * u + 2]);
-          acc[4 * u + 3] = fmaf(dec, x[k][u].w, acc[4 * u + 3]);
-        }
-        dec *= g[k];
-      }
+    for (int u = 0; u < 32; u += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(src + col + u);
+      v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
     }
-    tmem_st32(taddr + col, acc);
+    tmem_st32(taddr + col, v);
   }
   tmem_wait_st();
 }
@@ -518,10 +553,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* o_done = bars + 18;      // output accumulator complete
   uint64_t* o_free = bars + 19;      // output read out (128 arrivals)
   uint64_t* drain = bars + 20;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* keys_ready = bars + 21;  // gates of the chunk known (128 arrivals)
+  uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (128 arrivals)
+  uint64_t* state_done = bars + 23;  // the chunk's state carry done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
-  float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256);  // [2][64] running log-gate sums
+  float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256 + 64);  // [2][64] running log-gate sums
   float* eneg2 = bsh2 + 128;                                    // [2][64] e^{-b_j} (factored decay)
   float* zq2 = eneg2 + 128;                                     // [2][128] Z = sum_d e_q per row
   float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
@@ -541,6 +579,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
     mbar_init(ss_done, 1); mbar_init(feat, 128); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
+    mbar_init(keys_ready, 128); mbar_init(state_ready, 128); mbar_init(state_done, 1);
     mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
     mbar_init(drain, 1);
     *abort_flag = 0u;
@@ -656,11 +695,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mma_commit(&v_empty[c % 3]);   // the previous chunk's values are no longer needed
       };
       auto issue_sg_state = [&](int c) {
+        // recurrent scores as soon as the feature warps are done
         ok = ok && mbar_wait(feat, c & 1, wc, wsite(2, 7, c));
-        ok = ok && mbar_wait(&v_full[(c + 1) % 3], ((c + 1) / 3) & 1, wc, wsite(2, 8, c));
         if (!ok) return;
         tc_fence_after();
-        const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
@@ -668,11 +706,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           mma_bf16_ss(tmem + kColSg, sdesc_sw128(eq_base + qo, 16, 1024), sdesc_sw128(pk_base + ko, 16, 1024),
                       id_n64, kk > 0);
         }
+        // (failure-detection test: withhold the first completion; the waits downstream
+        // then run out, record a timeout and drain)
+        if (!(p.inject_stall && c == 0)) mma_commit(sg_done);
+        // the state carry once the window warps have copied and rescaled S
+        ok = ok && mbar_wait(state_ready, c & 1, wc, wsite(2, 10, c));
+        ok = ok && mbar_wait(&v_full[(c + 1) % 3], ((c + 1) / 3) & 1, wc, wsite(2, 8, c));
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
           mma_bf16_ss(tmem + kColS, sdesc_sw128(kt_base + kk * 2048, lbo_kt, 1024),
                       sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
-        mma_commit(sg_done);
+        mma_commit(state_done);
       };
       auto issue_inter = [&](int c) {   // O = (e^{b_i} / Z_i e_q) (alpha S), S as MN-major B
         if (c > 0) ok = ok && mbar_wait(o_free, (c - 1) & 1, wc, wsite(2, 9, c));
@@ -709,14 +756,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const int r = threadIdx.x - 128;
     const int i = r >> 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const float alpha = p.alpha;
     constexpr float kLog2e = 1.4426950408889634f;
     char* const qb = smem + L::Q0;
     char* const eqb = smem + L::EQ;
-    char* const sbb = smem + L::SB;
 
     // state entering the segment, first half of the columns (the window warps do the rest)
-    entering_state<D, D / 2>(p, seg, p.seqs[sg.seq].first_seg, kv, r % D, lane_base + kColS, 0);
+    entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColS, 0);
     tc_fence_before();
     named_bar(2, 256);
     tc_fence_after();
@@ -727,7 +772,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       float* bsh = bsh2 + (c & 1) * 64;
       mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
       mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
-      if (c > 0) mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));   // phi(k), keys~ and the state are free
+      if (c > 0) {   // phi(k) and keys~ are free once the previous scores and carry are done
+        mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));
+        mbar_wait(state_done, (c - 1) & 1, wc, wsite(3, 7, c));
+      }
       tc_fence_after();
 
       // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
@@ -745,6 +793,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const bool fast = bC >= -80.f;
       if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bi) : 0.f;
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
+      mbar_arrive(keys_ready);   // the window warps may now prepare the state copy of this chunk
 
       // queries: the raw row into registers (bf16 pairs), e_q = exp(q - max) and Z = sum e_q.
       // The tiles carry e_q unnormalised; the window warps fold Z into P and 1/Z into the output.
@@ -800,31 +849,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           st_chunk8(qb, kmajor_off(r, c8 * 8, ROWS * 128), x);
         }
       }
-      // state: bf16 copy of alpha S (MN-major B of the readout), then S <- e^{b_C} S
-      {
-        const float dec = __expf(bC);
-#pragma unroll
-        for (int col = 0; col < D; col += 64) {
-          float v[64];
-          tmem_ld32(lane_base + kColS + col, v);
-          tmem_ld32(lane_base + kColS + col + 32, v + 32);
-          tmem_wait_ld();
-          if (r < D) {
-#pragma unroll
-            for (int u = 0; u < 64; u += 8) {
-              float x[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
-              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 64; ++u) v[u] *= dec;
-          tmem_st32(lane_base + kColS + col, v);
-          tmem_st32(lane_base + kColS + col + 32, v + 32);
-        }
-        tmem_wait_st();
-      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
@@ -860,10 +884,50 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     // state entering the segment, second half of the columns (TMEM: the state follows O)
-    entering_state<D, D / 2>(p, seg, p.seqs[sg.seq].first_seg, kv, r % D, lane_base + kColO + D, D / 2);
+    entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColO + D, D / 2);
     tc_fence_before();
     named_bar(2, 256);
     tc_fence_after();
+    char* const sbb = smem + L::SB;
+    // State for chunk cc: the bf16 copy of alpha S (MN-major B of the readout), then
+    // S <- e^{b_C} S in TMEM before that chunk's carry accumulates onto it.  Needs the
+    // chunk's gates (keys_ready), the previous carry done (sg_done, waited by the caller)
+    // and the previous readout done with the copy (mma2_done).
+    auto prepare_state = [&](int cc) {
+      mbar_wait(keys_ready, cc & 1, wc, wsite(4, 3, cc));
+      if (cc > 0) {
+        mbar_wait(state_done, (cc - 1) & 1, wc, wsite(4, 5, cc));
+        mbar_wait(mma2_done, (cc - 1) & 1, wc, wsite(4, 4, cc));
+      }
+      tc_fence_after();
+      const int nvc = min(C, sg.t_end - (sg.t_begin + cc * C));
+      const float dec = __expf(bsh2[(cc & 1) * 64 + nvc - 1]);
+#pragma unroll
+      for (int col = 0; col < D; col += 64) {
+        float v[64];
+        tmem_ld32(lane_base + kColS + col, v);
+        tmem_ld32(lane_base + kColS + col + 32, v + 32);
+        tmem_wait_ld();
+        if (r < D) {
+#pragma unroll
+          for (int u = 0; u < 64; u += 8) {
+            float x[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
+            st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 64; ++u) v[u] *= dec;
+        tmem_st32(lane_base + kColS + col, v);
+        tmem_st32(lane_base + kColS + col + 32, v + 32);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(state_ready);
+    };
+    prepare_state(0);
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -957,6 +1021,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(p_ready);
+      if (c + 1 < nch) prepare_state(c + 1);   // overlaps this chunk's P.V on the tensor core
 
       // epilogue: O -> bf16 rows of out
       const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
@@ -965,20 +1030,24 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const float iz = 1.0f / zrow;
         const long t = (long)t0 + i;
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
+        float ov[D];
+#pragma unroll
+        for (int col = 0; col < D; col += 32) tmem_ld32(lane_base + kColO + col, ov + col);
+        tmem_wait_ld();
 #pragma unroll
         for (int col = 0; col < D; col += 32) {
-          float v[32];
-          tmem_ld32(lane_base + kColO + col, v);
-          tmem_wait_ld();
+          const float* v = ov + col;
           if (i < nv && live) {
+            uint32_t pw[16];
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) {
-              uint4 w;
-              w.x = pack_bf16(v[u] * iz, v[u + 1] * iz);
-              w.y = pack_bf16(v[u + 2] * iz, v[u + 3] * iz);
-              w.z = pack_bf16(v[u + 4] * iz, v[u + 5] * iz);
-              w.w = pack_bf16(v[u + 6] * iz, v[u + 7] * iz);
-              *reinterpret_cast<uint4*>(orow + col + u) = w;
+            for (int u = 0; u < 16; ++u) pw[u] = pack_bf16(v[2 * u] * iz, v[2 * u + 1] * iz);
+            if (p.out_v8) {   // two full 32-byte sectors per instruction
+#pragma unroll
+              for (int u = 0; u < 16; u += 8) st_global_v8(orow + col + 2 * u, pw + u);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 16; u += 4)
+                *reinterpret_cast<uint4*>(orow + col + 2 * u) = make_uint4(pw[u], pw[u + 1], pw[u + 2], pw[u + 3]);
             }
           }
         }
@@ -1050,12 +1119,17 @@ inline Plan make_plan(int B, int Hq, int Hkv, long T, int d, int n_seqs, bool va
                      : (long)B * ((chunks_per_seq + bestL - 1) / bestL);
   if (nseg < 1) nseg = 1;
   pl.n_seg_max = (int)nseg;
+  // the state pass splits segments so that about two of its CTAs run per SM
+  long nsub = (2L * sms + nseg * Hkv - 1) / (nseg * Hkv);
+  nsub = nsub < 1 ? 1 : (nsub > kMaxSub ? kMaxSub : (nsub > bestL ? bestL : nsub));
+  pl.nsub = (int)nsub;
+  pl.Ls = (int)((bestL + nsub - 1) / nsub);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  size_t off = 256;   // header: error word, segment count
+  size_t off = 256;   // header: error word, first timeout, segment count
   pl.off_seqs = off;  off = al(off + sizeof(SeqInfo) * (size_t)n_seqs);
   pl.off_segs = off;  off = al(off + sizeof(SegInfo) * (size_t)nseg);
-  pl.off_lam = off;   off = al(off + sizeof(float) * (size_t)nseg * Hkv);
-  pl.off_ds = off;    off = al(off + sizeof(float) * (size_t)nseg * Hkv * d * d);
+  pl.off_lam = off;   off = al(off + sizeof(float) * (size_t)nseg * nsub * Hkv);
+  pl.off_ds = off;    off = al(off + sizeof(float) * (size_t)nseg * nsub * Hkv * d * d);
   pl.total = off;
   return pl;
 }
@@ -1119,8 +1193,15 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   p.n_seqs = pb.n_seqs;
   p.n_seg_max = pl.n_seg_max;
   p.L = pl.L;
+  p.nsub = pl.nsub;
+  p.Ls = pl.Ls;
   p.alpha = pb.alpha;
   p.wait_ns = wait_limit_ns();
+  p.out_v8 = (reinterpret_cast<uintptr_t>(pb.out) & 31u) == 0 ? 1 : 0;
+  {
+    const char* st = std::getenv("LIGER_TEST_INJECT_STALL");
+    p.inject_stall = (st && *st && *st != '0') ? 1 : 0;
+  }
 
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, pb.q, D, pb.Hq, NT, 2) || !make_map(&mk, pb.k, D, pb.Hkv, NT, 1) ||
@@ -1141,7 +1222,11 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     cudaGetLastError();
     return LIGER_ERR_CUDA;
   }
-  seg_k<<<(unsigned)pl.n_seg_max * pb.Hkv, NTHREADS, SegSmem<D>::BYTES, s>>>(mk, mv, p);
+  seg_k<<<(unsigned)pl.n_seg_max * pl.nsub * pb.Hkv, NTHREADS, SegSmem<D>::BYTES, s>>>(mk, mv, p);
+  hk.count(1);
+  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+
+  scan_kernel<D><<<dim3((unsigned)(pb.n_seqs * pb.Hkv), (unsigned)(D * D / 1024)), 256, 0, s>>>(p);
   hk.count(1);
   if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 

@@ -39,6 +39,7 @@ SIGNATURES = {
                                         _i, _vp]),
     "liger_attn_prefill_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                         _i, _vp, _vp, _i, _vp, _vp, _vp]),
+    "liger_attn_prefill_status": (_i, [_vp, ctypes.c_size_t]),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }
@@ -193,3 +194,11 @@ def decode_kvshared(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, str
         float(alpha), _dt(q), _stream_ptr(stream))
     _check(st)
     return out
+
+
+def prefill_status(workspace) -> int:
+    """LIGER_OK, or LIGER_ERR_TIMEOUT if the last prefill on this workspace gave up waiting
+    (call after its stream has completed)."""
+    if workspace is None:
+        return LIGER_OK
+    return int(load().liger_attn_prefill_status(_ptr(workspace), workspace.numel() * workspace.element_size()))

@@ -105,6 +105,17 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
                                 void* stream);
 
 /*
+ * Status of the last prefill that used this workspace (tensor-core path):
+ * LIGER_ERR_TIMEOUT if one of its kernels gave up waiting on an internal
+ * barrier (every wait is bounded, by default 2 s; the kernel then drains and
+ * exits, the outputs are unspecified and the CUDA context stays usable),
+ * LIGER_OK otherwise.  Reads the workspace header with a synchronous copy:
+ * call it after the prefill's stream has completed.  (The pages have no
+ * counterpart; this is failure detection.)
+ */
+liger_status liger_attn_prefill_status(const void* workspace, size_t workspace_bytes);
+
+/*
  * Decode: one new token for each of B independent sequences.
  * Source: the same recurrence and hybrid, stepped once; the constant-size
  * state replacing the growing key/value cache is the linear-time,
