@@ -226,54 +226,46 @@ __device__ __forceinline__ float log_sigmoid_fast(float m) {
 
 // Feature map and gate of one chunk of keys, shared by the seg_state and chunk
 // kernels.  Thread r (0..127) owns half of token j = r >> 1: elements
-// [h * D/2, (h+1) * D/2) with h = r & 1.  Writes phi(k) (bf16) to `phik` (may be
-// null), the log gates to lg[0..63] (0 past the valid tokens), and returns the
-// thread's phi values in ph and the running sums in gs (every warp scans the 64
-// gates itself); lanes of the group's first warp also store the sums to bsh.
+// [h * D/2, (h+1) * D/2) with h = r & 1.  Writes e = exp(k - max_d k) (bf16, not
+// yet divided by its sum) to `ebuf` in the key tile's swizzled layout and the log
+// gates to lg[0..63] (0 past the valid tokens); returns 1 / sum_d e, which the
+// callers fold into per-token scalars, and the running sums in gs (every warp
+// scans the 64 gates itself); lanes of the group's first warp also store the sums
+// to bsh.  Each pass is a short loop over 16-byte groups: the role loops of the
+// chunk kernel share one SM sub-partition, and fully unrolled straight-line code
+// for all of them would not stay in the instruction caches.
 template <int D>
-__device__ __forceinline__ void key_features(const char* kraw, char* phik, float* lg, float* bsh, int r, int nv,
-                                             float (&ph)[D / 2], GateSums& gs) {
+__device__ __forceinline__ float key_features(const char* kraw, char* ebuf, float* lg, float* bsh, int r, int nv,
+                                              GateSums& gs) {
   constexpr int HALF = D / 2;
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r >> 1, h = r & 1;
-  // independent partial maxima and sums keep the dependency chains short
-  float mx[HALF / 8], sm[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+  float m = -INFINITY, sa = 0.f, sb = 0.f;
+#pragma unroll 2
   for (int c = 0; c < HALF / 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, C * 128));
-    mx[c] = bf16x8_max(u);
-    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      ph[c * 8 + 2 * q] = bf16_lo(w4[q]);
-      ph[c * 8 + 2 * q + 1] = bf16_hi(w4[q]);
-      sm[q] += ph[c * 8 + 2 * q] + ph[c * 8 + 2 * q + 1];
-    }
+    m = fmaxf(m, bf16x8_max(u));
+    sa += (bf16_lo(u.x) + bf16_hi(u.x)) + (bf16_lo(u.y) + bf16_hi(u.y));
+    sb += (bf16_lo(u.z) + bf16_hi(u.z)) + (bf16_lo(u.w) + bf16_hi(u.w));
   }
-#pragma unroll
-  for (int c = HALF / 16; c >= 1; c >>= 1)
-#pragma unroll
-    for (int t = 0; t < c; ++t) mx[t] = fmaxf(mx[t], mx[t + c]);
-  float m = mx[0];
-  float sum = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+  float sum = sa + sb;
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   const float ml = m * kLog2e;
-  float zs[4] = {0.f, 0.f, 0.f, 0.f};
+  float za = 0.f, zb = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < HALF / 8; ++c) {
+    const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
+    float x[8];
+    ld_chunk8(kraw, off, x);
 #pragma unroll
-  for (int u = 0; u < HALF; ++u) {
-    ph[u] = ex2(fmaf(ph[u], kLog2e, -ml));
-    zs[u & 3] += ph[u];
+    for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
+    za += (x[0] + x[1]) + (x[2] + x[3]);
+    zb += (x[4] + x[5]) + (x[6] + x[7]);
+    st_chunk8(ebuf, off, x);
   }
-  float z = (zs[0] + zs[1]) + (zs[2] + zs[3]);
+  float z = za + zb;
   z += __shfl_xor_sync(0xffffffffu, z, 1);
-  const float iz = 1.0f / z;
-#pragma unroll
-  for (int u = 0; u < HALF; ++u) ph[u] *= iz;
-  if (phik) {
-#pragma unroll
-    for (int c = 0; c < HALF / 8; ++c) st_chunk8(phik, kmajor_off(j, h * HALF + c * 8, C * 128), &ph[c * 8]);
-  }
   if (h == 0) lg[j] = j < nv ? log_sigmoid_fast(sum / (float)D) : 0.f;
   named_bar(1, 128);
   {   // inclusive running sum over the 64 tokens, two per lane, in every warp
@@ -293,22 +285,24 @@ __device__ __forceinline__ void key_features(const char* kraw, char* phik, float
       bsh[2 * r + 1] = gs.b1;
     }
   }
+  return 1.0f / z;
 }
 
-// Decay-scaled keys e^{b_C - b_j} phi(k_j) (zero past the valid tokens), written
-// in the same swizzled layout; read by the MMA as the MN-major A operand K^T.
+// Decay-scaled keys sc * e (sc = e^{b_C - b_j} / z_j, zero past the valid tokens),
+// from this thread's features in `ebuf` to `kt` in the same swizzled layout; read
+// by the MMA as the MN-major A operand K^T.
 template <int D>
-__device__ __forceinline__ void write_ktilde(char* kt, float bj, int r, int nv, float bC,
-                                             const float (&ph)[D / 2]) {
+__device__ __forceinline__ void write_ktilde(const char* ebuf, char* kt, int r, float sc) {
   constexpr int HALF = D / 2;
   const int j = r >> 1, h = r & 1;
-  const float sc = j < nv ? __expf(bC - bj) : 0.f;
-#pragma unroll
+#pragma unroll 2
   for (int c = 0; c < HALF / 8; ++c) {
+    const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
     float x[8];
+    ld_chunk8(ebuf, off, x);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = ph[c * 8 + u] * sc;
-    st_chunk8(kt, kmajor_off(j, h * HALF + c * 8, C * 128), x);
+    for (int q = 0; q < 8; ++q) x[q] *= sc;
+    st_chunk8(kt, off, x);
   }
 }
 
@@ -317,7 +311,7 @@ __device__ __forceinline__ void write_ktilde(char* kt, float bj, int r, int nv, 
 template <int D>
 struct SegSmem {
   static constexpr uint32_t KV = C * D * 2;        // one chunk of k (or v)
-  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 4 * KV, SMALL = 5 * KV;
+  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 4 * KV, E = 5 * KV, SMALL = 6 * KV;
   static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
 };
 
@@ -429,9 +423,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const int slot = c & 1;
       const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
       mbar_wait(&kv_full[slot], (c >> 1) & 1, wc);
-      float ph[D / 2];
       GateSums gs;
-      key_features<D>(smem + L::K0 + slot * L::KV, nullptr, lg, nullptr, r, nv, ph, gs);
+      const float iz = key_features<D>(smem + L::K0 + slot * L::KV, smem + L::E, lg, nullptr, r, nv, gs);
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 1);
       lam += bC;
@@ -439,10 +432,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         mbar_wait(mma_done, (c - 1) & 1, wc);
         tc_fence_after();
       }
-      write_ktilde<D>(smem + L::KT, bj, r, nv, bC, ph);
+      write_ktilde<D>(smem + L::E, smem + L::KT, r, (r >> 1) < nv ? __expf(bC - bj) * iz : 0.f);
       if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
         const float dec = __expf(bC);
-#pragma unroll
+#pragma unroll 1
         for (int col = 0; col < D; col += 32) {
           float v[32];
           tmem_ld32(lane_base + col, v);
@@ -461,7 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
       tc_fence_after();
       float* dst = ds_out + (size_t)r * D;
-#pragma unroll
+#pragma unroll 1
       for (int col = 0; col < D; col += 32) {
         float v[32];
         tmem_ld32(lane_base + col, v);
@@ -516,7 +509,7 @@ struct ChunkSmem {
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
   static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
   static constexpr uint32_t SMALL = SB + D * D * 2;
-  static constexpr uint32_t SMALL_BYTES = 3072;
+  static constexpr uint32_t SMALL_BYTES = 4096;
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
@@ -564,6 +557,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   float* zq2 = eneg2 + 128;                                     // [2][128] Z = sum_d e_q per row
   float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
   float* fast2 = lg + 64;                                       // [2] factored decay usable
+  float* izk2 = fast2 + 2;                                      // [2][64] 1 / z_k per key token
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -771,95 +765,92 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int nv = min(C, sg.t_end - t0);
       float* bsh = bsh2 + (c & 1) * 64;
       mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
-      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
       if (c > 0) {   // phi(k) and keys~ are free once the previous scores and carry are done
         mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));
         mbar_wait(state_done, (c - 1) & 1, wc, wsite(3, 7, c));
       }
       tc_fence_after();
 
-      // keys: phi(k), gates, running sums, decay-scaled keys, e^{-b_j}
-      float bC, bi;
+      // keys: e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running
+      // sums, decay-scaled keys
+      float bC, bi, iz;
       {
-        float ph[D / 2];
         GateSums gs;
-        key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, lg, bsh, r, nv, ph, gs);
+        iz = key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, lg, bsh, r, nv, gs);
         bC = gs.at(nv - 1);
         bi = gs.at(i);
-        write_ktilde<D>(smem + L::KT, bi, r, nv, bC, ph);   // key token j = r >> 1 = i
+        write_ktilde<D>(smem + L::PK, smem + L::KT, r, i < nv ? __expf(bC - bi) * iz : 0.f);   // token r >> 1 = i
       }
       // Factored mode (the chunk's total log gate >= -80): e^{b_i} and e^{-b_j} stay
       // finite in fp32, so e^{b_i - b_j} can be split between the two operands.
       const bool fast = bC >= -80.f;
-      if ((r & 1) == 0) eneg2[(c & 1) * 64 + i] = fast ? __expf(-bi) : 0.f;
+      if ((r & 1) == 0) {
+        eneg2[(c & 1) * 64 + i] = fast ? __expf(-bi) * iz : 0.f;
+        izk2[(c & 1) * 64 + i] = iz;
+      }
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
       mbar_arrive(keys_ready);   // the window warps may now prepare the state copy of this chunk
 
-      // queries: the raw row into registers (bf16 pairs), e_q = exp(q - max) and Z = sum e_q.
-      // The tiles carry e_q unnormalised; the window warps fold Z into P and 1/Z into the output.
-      uint32_t ep[D / 2];
-      float mxq[D / 8];
-#pragma unroll
+      // queries: e_q = exp(q - max) and Z = sum e_q; the tiles carry e_q unnormalised and
+      // the window warps fold Z into P and 1/Z into the output.  The raw row is first
+      // copied into the e_q buffer (free once the previous readout is done), so the q
+      // buffer can take the next chunk's tile while e_q is computed in place.
+      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));
+      float mq = -INFINITY;
+#pragma unroll 4
       for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8, ROWS * 128));
-        mxq[c8] = bf16x8_max(u);
-        ep[4 * c8] = u.x; ep[4 * c8 + 1] = u.y; ep[4 * c8 + 2] = u.z; ep[4 * c8 + 3] = u.w;
+        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
+        const uint4 u = *reinterpret_cast<const uint4*>(qb + off);
+        mq = fmaxf(mq, bf16x8_max(u));
+        *reinterpret_cast<uint4*>(eqb + off) = u;
       }
-#pragma unroll
-      for (int w2 = D / 16; w2 >= 1; w2 >>= 1)
-#pragma unroll
-        for (int t = 0; t < w2; ++t) mxq[t] = fmaxf(mxq[t], mxq[t + w2]);
-      const float mql = mxq[0] * kLog2e;
-      if (fast) {   // raw q now lives in registers: release its buffer once the score MMA read it too
+      const float mql = mq * kLog2e;
+      if (fast) {   // raw q no longer needed here: release it once the score MMA read it too
         named_bar(1, 128);
         if (r == 0) {
           mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
           mbar_arrive(q_empty);
         }
-      }
-      // factored mode: pack e^{b_i} e_q (one tile for the recurrent scores and the readout);
-      // otherwise pack e_q for the scores (e^{b_i} e_q for the readout goes to the q buffer)
-      const float ebi = fast ? __expf(bi) : 1.f;
-      float zqs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < D / 2; ++k) {
-        const float lo = ex2(fmaf(bf16_lo(ep[k]), kLog2e, -mql));
-        const float hi = ex2(fmaf(bf16_hi(ep[k]), kLog2e, -mql));
-        zqs[k & 7] += lo + hi;
-        ep[k] = pack_bf16(lo * ebi, hi * ebi);
-      }
-      zq2[(c & 1) * 128 + r] = ((zqs[0] + zqs[1]) + (zqs[2] + zqs[3])) + ((zqs[4] + zqs[5]) + (zqs[6] + zqs[7]));
-      // the e_q tile and the state copy are still read by the previous chunk's readout
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));
-#pragma unroll
-      for (int c8 = 0; c8 < D / 8; ++c8)
-        *reinterpret_cast<uint4*>(eqb + kmajor_off(r, c8 * 8, ROWS * 128)) =
-            make_uint4(ep[4 * c8], ep[4 * c8 + 1], ep[4 * c8 + 2], ep[4 * c8 + 3]);
-      if (!fast) {
+      } else {      // the q buffer takes e^{b_i} e_q for the readout after the score MMA
         mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-        const float sc = __expf(bi);
-#pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          float x[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            x[2 * q] = bf16_lo(ep[4 * c8 + q]) * sc;
-            x[2 * q + 1] = bf16_hi(ep[4 * c8 + q]) * sc;
-          }
-          st_chunk8(qb, kmajor_off(r, c8 * 8, ROWS * 128), x);
-        }
       }
+      // factored mode: e^{b_i} e_q (one tile for the recurrent scores and the readout);
+      // otherwise e_q for the scores and e^{b_i} e_q in the q buffer for the readout
+      const float ebi = __expf(bi);
+      const float eqs = fast ? ebi : 1.f;
+      float za = 0.f, zb = 0.f;
+#pragma unroll 2
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
+        float x[8];
+        ld_chunk8(eqb, off, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
+        za += (x[0] + x[1]) + (x[2] + x[3]);
+        zb += (x[4] + x[5]) + (x[6] + x[7]);
+        if (!fast) {
+          float y[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) y[q] = x[q] * ebi;
+          st_chunk8(qb, off, y);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] *= eqs;
+        st_chunk8(eqb, off, x);
+      }
+      zq2[(c & 1) * 128 + r] = za + zb;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
-      named_bar(1, 128);   // this group's bsh buffer is rewritten two chunks later only
+      named_bar(1, 128);   // lg is rewritten by the next chunk's keys
     }
     // final state of the sequence: the carry after the last chunk of its last segment
     const SeqInfo si = p.seqs[sg.seq];
     const bool last = seg == si.first_seg + si.n_seg - 1;
     if (p.final_state && last && mbar_wait(mma2_done, (nch - 1) & 1, wc, wsite(3, 5, nch)) && !*abort_flag) {
       tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int col = 0; col < D; col += 32) {
         float v[32];
         tmem_ld32(lane_base + kColS + col, v);
@@ -891,8 +882,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     char* const sbb = smem + L::SB;
     // State for chunk cc: the bf16 copy of alpha S (MN-major B of the readout), then
     // S <- e^{b_C} S in TMEM before that chunk's carry accumulates onto it.  Needs the
-    // chunk's gates (keys_ready), the previous carry done (sg_done, waited by the caller)
-    // and the previous readout done with the copy (mma2_done).
+    // chunk's gates (keys_ready), the previous carry done (state_done) and the previous
+    // readout done with the copy (mma2_done).
     auto prepare_state = [&](int cc) {
       mbar_wait(keys_ready, cc & 1, wc, wsite(4, 3, cc));
       if (cc > 0) {
@@ -902,15 +893,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_after();
       const int nvc = min(C, sg.t_end - (sg.t_begin + cc * C));
       const float dec = __expf(bsh2[(cc & 1) * 64 + nvc - 1]);
-#pragma unroll
-      for (int col = 0; col < D; col += 64) {
-        float v[64];
+#pragma unroll 1
+      for (int col = 0; col < D; col += 32) {
+        float v[32];
         tmem_ld32(lane_base + kColS + col, v);
-        tmem_ld32(lane_base + kColS + col + 32, v + 32);
         tmem_wait_ld();
         if (r < D) {
 #pragma unroll
-          for (int u = 0; u < 64; u += 8) {
+          for (int u = 0; u < 32; u += 8) {
             float x[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
@@ -918,9 +908,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           }
         }
 #pragma unroll
-        for (int u = 0; u < 64; ++u) v[u] *= dec;
+        for (int u = 0; u < 32; ++u) v[u] *= dec;
         tmem_st32(lane_base + kColS + col, v);
-        tmem_st32(lane_base + kColS + col + 32, v + 32);
       }
       tmem_wait_st();
       fence_proxy_async_smem();
@@ -934,91 +923,98 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int nv = min(C, sg.t_end - t0);
       const float* bsh = bsh2 + (c & 1) * 64;
       const float* eneg = eneg2 + (c & 1) * 64;
-      mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
-      tc_fence_after();
-      const bool fast = fast2[c & 1] != 0.f;
+      const float* izk = izk2 + (c & 1) * 64;
       // Window band.  Key index x over [previous chunk | current chunk] (0..127): row i
       // sees x in [i+1, i+64].  This warp's tokens are 16 wq .. 16 wq + 15, so it reads the
       // 80 columns starting at 16 wq; column j then holds x = 16 wq + j and is live for
-      // j in [il+1, il+64], il = i - 16 wq.
-      float s[80];
+      // j in [il+1, il+64], il = i - 16 wq (only x >= 64 in the sequence's first chunk).
+      const int jlo = max(il + 1, t0 == sg.q0 ? 64 - 16 * wq : 0), jhi = il + 64;
+      const uint32_t ss_base = lane_base + kColSs + 16 * wq;
+      mbar_wait(ss_done, c & 1, wc, wsite(4, 6, c));
+      tc_fence_after();
+      float m = -INFINITY;
+#pragma unroll 1
+      for (int q5 = 0; q5 < 5; ++q5) {
+        float s[16];
+        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_wait_ld();
 #pragma unroll
-      for (int q5 = 0; q5 < 5; ++q5) tmem_ld16(lane_base + kColSs + 16 * wq + 16 * q5, s + 16 * q5);
-      tmem_wait_ld();
-      s[0] = -INFINITY;
-#pragma unroll
-      for (int j = 1; j < 16; ++j) s[j] = j <= il ? -INFINITY : s[j];
-#pragma unroll
-      for (int j = 64; j < 80; ++j) s[j] = j > il + 64 ? -INFINITY : s[j];
-      if (t0 == sg.q0) {   // first chunk of the sequence: the previous chunk's keys are not its own
-        const int lim = 64 - 16 * wq;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) s[j] = j < lim ? -INFINITY : s[j];
+        for (int u = 0; u < 16; ++u) {
+          const int j = 16 * q5 + u;
+          if (j >= jlo && j <= jhi) m = fmaxf(m, s[u]);
+        }
       }
-      float mw[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mw[t] = fmaxf(s[t], s[t + 8]);
-#pragma unroll
-      for (int j = 16; j < 80; ++j) mw[j & 7] = fmaxf(mw[j & 7], s[j]);
-      const float m = fmaxf(fmaxf(fmaxf(mw[0], mw[1]), fmaxf(mw[2], mw[3])),
-                            fmaxf(fmaxf(mw[4], mw[5]), fmaxf(mw[6], mw[7])));
       const float msc = m * sscale;
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float la = 0.f, lb = 0.f;   // exps written back over the scores
+#pragma unroll 1
+      for (int q5 = 0; q5 < 5; ++q5) {
+        float s[16];
+        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 80; ++j) {
-        s[j] = ex2(fmaf(s[j], sscale, -msc));
-        ls[j & 7] += s[j];
+        for (int u = 0; u < 16; ++u) {
+          const int j = 16 * q5 + u;
+          s[u] = (j >= jlo && j <= jhi) ? ex2(fmaf(s[u], sscale, -msc)) : 0.f;
+        }
+        la += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+        lb += ((s[8] + s[9]) + (s[10] + s[11])) + ((s[12] + s[13]) + (s[14] + s[15]));
+        tmem_st16(ss_base + 16 * q5, s);
       }
+      tmem_wait_st();
+      // Z of the rows and the recurrent scores come with the feature warps' tiles
+      mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
+      tc_fence_after();
+      const bool fast = fast2[c & 1] != 0.f;
       const float zrow = zq2[(c & 1) * 128 + r];   // the tiles carry e_q unnormalised: scale P by Z
-      const float coef = beta * zrow / (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
-      uint32_t pd[40];
+      const float coef = beta * zrow / (la + lb);
+#pragma unroll 1
+      for (int q5 = 0; q5 < 5; ++q5) {
+        float s[16];
+        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_wait_ld();
+        uint32_t pw[8];
 #pragma unroll
-      for (int k = 0; k < 40; ++k) pd[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
-
-      // recurrent scores of the current keys kk <= i (this warp needs kk < 16 wq + 16)
-      float g[64];
-#pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
-        if (bb <= wq) {
-          tmem_ld16(lane_base + kColSg + 16 * bb, g + 16 * bb);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) g[16 * bb + u] = 0.f;
-        }
+        for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
+        tmem_st8u(lane_base + kColP + 8 * wq + 8 * q5, pw);
       }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_read);   // both score tiles are in registers: their TMEM may be reused
-      uint32_t ag[32];
-      if (fast) {   // e^{b_i} is already in the scores: multiply by e^{-b_kk}
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int kk = 2 * k;
-          const float g0 = kk <= i ? alpha * g[kk] * eneg[kk] : 0.f;
-          const float g1 = kk + 1 <= i ? alpha * g[kk + 1] * eneg[kk + 1] : 0.f;
-          ag[k] = pack_bf16(g0, g1);
-        }
-      } else {
-        const float bi = bsh[i];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int kk = 2 * k;
-          const float g0 = kk <= i ? alpha * g[kk] * __expf(bi - bsh[kk]) : 0.f;
-          const float g1 = kk + 1 <= i ? alpha * g[kk + 1] * __expf(bi - bsh[kk + 1]) : 0.f;
-          ag[k] = pack_bf16(g0, g1);
-        }
-      }
-      // probability tiles to TMEM: the window tile over all 128 keys (zeros outside this
-      // warp's band) and the recurrent tile over the current keys (in the score tile's place)
-      {
+      {   // zeros for the keys outside this warp's band
         const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int k = 0; k < 5; ++k) tmem_st8u(lane_base + kColP + 8 * wq + 8 * k, pd + 8 * k);
-#pragma unroll
         for (int k = 0; k < 3; ++k) tmem_st8u(lane_base + kColP + ((8 * wq + 40 + 8 * k) & 63), zero8);
-        tmem_st32u(lane_base + kColSg, ag);
-        tmem_wait_st();
       }
+      tc_fence_before();
+      mbar_arrive(s_read);   // the window scores are consumed: their TMEM may be reused
+
+      // recurrent probability tile over the current keys kk <= i, written over the
+      // recurrent scores (this warp needs kk < 16 wq + 16; later blocks are zero)
+      const float bi = bsh[i];
+#pragma unroll 1
+      for (int bb = 0; bb < 4; ++bb) {
+        uint32_t ag[8];
+        if (bb <= wq) {
+          float g[16];
+          tmem_ld16(lane_base + kColSg + 16 * bb, g);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int kk = 16 * bb + 2 * k;
+            float g0, g1;
+            if (fast) {   // e^{b_i} is already in the scores: multiply by e^{-b_kk} / z_kk
+              g0 = alpha * g[2 * k] * eneg[kk];
+              g1 = alpha * g[2 * k + 1] * eneg[kk + 1];
+            } else {
+              g0 = alpha * g[2 * k] * (__expf(bi - bsh[kk]) * izk[kk]);
+              g1 = alpha * g[2 * k + 1] * (__expf(bi - bsh[kk + 1]) * izk[kk + 1]);
+            }
+            ag[k] = pack_bf16(kk <= i ? g0 : 0.f, kk + 1 <= i ? g1 : 0.f);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) ag[k] = 0u;
+        }
+        tmem_st8u(lane_base + kColSg + 8 * bb, ag);
+      }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_ready);
       if (c + 1 < nch) prepare_state(c + 1);   // overlaps this chunk's P.V on the tensor core
@@ -1030,20 +1026,19 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         const float iz = 1.0f / zrow;
         const long t = (long)t0 + i;
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
-        float ov[D];
-#pragma unroll
-        for (int col = 0; col < D; col += 32) tmem_ld32(lane_base + kColO + col, ov + col);
-        tmem_wait_ld();
-#pragma unroll
+        const bool store = i < nv && live;
+#pragma unroll 1
         for (int col = 0; col < D; col += 32) {
-          const float* v = ov + col;
-          if (i < nv && live) {
+          float v[32];
+          tmem_ld32(lane_base + kColO + col, v);
+          tmem_wait_ld();
+          if (store) {
             uint32_t pw[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) pw[u] = pack_bf16(v[2 * u] * iz, v[2 * u + 1] * iz);
             if (p.out_v8) {   // two full 32-byte sectors per instruction
-#pragma unroll
-              for (int u = 0; u < 16; u += 8) st_global_v8(orow + col + 2 * u, pw + u);
+              st_global_v8(orow + col, pw);
+              st_global_v8(orow + col + 16, pw + 8);
             } else {
 #pragma unroll
               for (int u = 0; u < 16; u += 4)
