@@ -241,7 +241,7 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r >> 1, h = r & 1;
   float m = -INFINITY, sa = 0.f, sb = 0.f;
-#pragma unroll 2
+#pragma unroll 4
   for (int c = 0; c < HALF / 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, C * 128));
     m = fmaxf(m, bf16x8_max(u));
@@ -253,7 +253,7 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   const float ml = m * kLog2e;
   float za = 0.f, zb = 0.f;
-#pragma unroll 2
+#pragma unroll 4
   for (int c = 0; c < HALF / 8; ++c) {
     const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
     float x[8];
@@ -295,7 +295,7 @@ template <int D>
 __device__ __forceinline__ void write_ktilde(const char* ebuf, char* kt, int r, float sc) {
   constexpr int HALF = D / 2;
   const int j = r >> 1, h = r & 1;
-#pragma unroll 2
+#pragma unroll 4
   for (int c = 0; c < HALF / 8; ++c) {
     const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
     float x[8];
@@ -519,7 +519,7 @@ constexpr uint32_t kColSg = 128;   // recurrent scores (64); then the recurrent 
 constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
 constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
 
-constexpr int kChunkThreads = 320;   // warps 0-3 window/epilogue, 4-7 features, 8 TMA, 9 MMA
+constexpr int kChunkThreads = 448;   // warps 0-3 window/epilogue, 4-7 keys, 8-11 queries, 12 TMA, 13 MMA
 
 template <int D>
 __global__ void __launch_bounds__(kChunkThreads, 1)
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* q_full = bars + 10;
   uint64_t* q_empty = bars + 11;
   uint64_t* ss_done = bars + 12;     // window scores written; raw q read
-  uint64_t* feat = bars + 13;        // features of the chunk ready (128 arrivals)
+  uint64_t* feat = bars + 13;        // key and query tiles of the chunk ready (256 arrivals)
   uint64_t* sg_done = bars + 14;     // recurrent scores and state carry done
   uint64_t* mma2_done = bars + 15;   // + readout done: feature buffers free again
   uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (128 arrivals)
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
-    mbar_init(ss_done, 1); mbar_init(feat, 128); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
+    mbar_init(ss_done, 1); mbar_init(feat, 256); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
     mbar_init(keys_ready, 128); mbar_init(state_ready, 128); mbar_init(state_done, 1);
     mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
     mbar_init(drain, 1);
@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.err, p.wait_ns};
 
-  if (warp == 8) {   // ---------------- TMA producer
+  if (warp == 12) {   // ---------------- TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmq);
       prefetch_tensormap(&tmk);
@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       for (int u = (v_issued > 3 ? v_issued - 3 : 0); u < v_issued; ++u) mbar_wait(&v_full[u % 3], (u / 3) & 1, dw);
       mbar_wait(q_full, (q_issued - 1) & 1, dw);
     }
-  } else if (warp == 9) {   // ---------------- MMA issuer
+  } else if (warp == 13) {   // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
       const uint32_t id_inter = idesc_bf16(128, D, 0, 1);
@@ -743,16 +743,71 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       issue_pv(nch - 1);
       mma_commit(drain);
     }
-  } else if (warp >= 4) {   // ---------------- features (threads 0..127 of warps 4-7)
+  } else if (warp >= 8) {   // ---------------- queries (threads 0..127 of warps 8-11)
+    // e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the window
+    // warps fold Z into P and 1/Z into the output).  Needs no gate: with the decay
+    // factored around the chunk's midpoint the row factor e^{b_i - m} is applied in the
+    // epilogue.  Never leaves the loop early (see the key warps).
+    const int r = threadIdx.x - 256;
+    const int i = r >> 1;
+    constexpr float kLog2e = 1.4426950408889634f;
+    char* const qb = smem + L::Q0;
+    char* const eqb = smem + L::EQ;
+    for (int c = 0; c < nch; ++c) {
+      mbar_wait(q_full, c & 1, wc, wsite(5, 1, c));
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(5, 2, c));   // e_q tile free
+      float mq0 = -INFINITY, mq1 = -INFINITY;
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; c8 += 2) {
+        mq0 = fmaxf(mq0, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8, ROWS * 128))));
+        mq1 = fmaxf(mq1, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8 + 8, ROWS * 128))));
+      }
+      const float mql = fmaxf(mq0, mq1) * kLog2e;
+      float za = 0.f, zb = 0.f;
+#pragma unroll 4
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
+        float x[8];
+        ld_chunk8(qb, off, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
+        za += (x[0] + x[1]) + (x[2] + x[3]);
+        zb += (x[4] + x[5]) + (x[6] + x[7]);
+        st_chunk8(eqb, off, x);
+      }
+      zq2[(c & 1) * 128 + r] = za + zb;
+      // the decay mode of the chunk comes with its keys
+      mbar_wait(keys_ready, c & 1, wc, wsite(5, 3, c));
+      if (fast2[c & 1] != 0.f) {   // raw q no longer needed: release it once the score MMA read it too
+        named_bar(4, 128);
+        if (r == 0) {
+          mbar_wait(ss_done, c & 1, wc, wsite(5, 4, c));
+          mbar_arrive(q_empty);
+        }
+      } else {   // exact decay: the q buffer takes e^{b_i} e_q, the readout's A operand
+        mbar_wait(ss_done, c & 1, wc, wsite(5, 4, c));
+        const float ebi = __expf(bsh2[(c & 1) * 64 + i]);
+#pragma unroll 4
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
+          float x[8];
+          ld_chunk8(eqb, off, x);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) x[q] *= ebi;
+          st_chunk8(qb, off, x);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(feat);
+    }
+  } else if (warp >= 4) {   // ---------------- keys (threads 0..127 of warps 4-7)
     // Row threads never leave the loop early: after a timeout every wait returns
     // at once (the CTA's abort flag is set), so the group still meets at each
     // named barrier and warp-collective TMEM access stays uniform.
     const int r = threadIdx.x - 128;
     const int i = r >> 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    constexpr float kLog2e = 1.4426950408889634f;
-    char* const qb = smem + L::Q0;
-    char* const eqb = smem + L::EQ;
+    char* const sbb = smem + L::SB;
 
     // state entering the segment, first half of the columns (the window warps do the rest)
     entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColS, 0);
@@ -765,14 +820,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int nv = min(C, sg.t_end - t0);
       float* bsh = bsh2 + (c & 1) * 64;
       mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
-      if (c > 0) {   // phi(k) and keys~ are free once the previous scores and carry are done
+      if (c > 0) {   // e_k and keys~ are free once the previous scores and carry are done
         mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));
         mbar_wait(state_done, (c - 1) & 1, wc, wsite(3, 7, c));
       }
       tc_fence_after();
 
-      // keys: e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running
-      // sums, decay-scaled keys
+      // e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running sums,
+      // decay-scaled keys
       float bC, bi, iz;
       {
         GateSums gs;
@@ -781,68 +836,51 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         bi = gs.at(i);
         write_ktilde<D>(smem + L::PK, smem + L::KT, r, i < nv ? __expf(bC - bi) * iz : 0.f);   // token r >> 1 = i
       }
-      // Factored mode (the chunk's total log gate >= -80): e^{b_i} and e^{-b_j} stay
-      // finite in fp32, so e^{b_i - b_j} can be split between the two operands.
+      // Factored mode (the chunk's total log gate >= -80): with m = b_C / 2,
+      // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-40}.
       const bool fast = bC >= -80.f;
       if ((r & 1) == 0) {
-        eneg2[(c & 1) * 64 + i] = fast ? __expf(-bi) * iz : 0.f;
+        eneg2[(c & 1) * 64 + i] = fast ? __expf(0.5f * bC - bi) * iz : 0.f;
         izk2[(c & 1) * 64 + i] = iz;
       }
       if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
-      mbar_arrive(keys_ready);   // the window warps may now prepare the state copy of this chunk
-
-      // queries: e_q = exp(q - max) and Z = sum e_q; the tiles carry e_q unnormalised and
-      // the window warps fold Z into P and 1/Z into the output.  The raw row is first
-      // copied into the e_q buffer (free once the previous readout is done), so the q
-      // buffer can take the next chunk's tile while e_q is computed in place.
-      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));
-      float mq = -INFINITY;
-#pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
-        const uint4 u = *reinterpret_cast<const uint4*>(qb + off);
-        mq = fmaxf(mq, bf16x8_max(u));
-        *reinterpret_cast<uint4*>(eqb + off) = u;
-      }
-      const float mql = mq * kLog2e;
-      if (fast) {   // raw q no longer needed here: release it once the score MMA read it too
-        named_bar(1, 128);
-        if (r == 0) {
-          mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-          mbar_arrive(q_empty);
-        }
-      } else {      // the q buffer takes e^{b_i} e_q for the readout after the score MMA
-        mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-      }
-      // factored mode: e^{b_i} e_q (one tile for the recurrent scores and the readout);
-      // otherwise e_q for the scores and e^{b_i} e_q in the q buffer for the readout
-      const float ebi = __expf(bi);
-      const float eqs = fast ? ebi : 1.f;
-      float za = 0.f, zb = 0.f;
-#pragma unroll 2
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
-        float x[8];
-        ld_chunk8(eqb, off, x);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
-        za += (x[0] + x[1]) + (x[2] + x[3]);
-        zb += (x[4] + x[5]) + (x[6] + x[7]);
-        if (!fast) {
-          float y[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) y[q] = x[q] * ebi;
-          st_chunk8(qb, off, y);
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] *= eqs;
-        st_chunk8(eqb, off, x);
-      }
-      zq2[(c & 1) * 128 + r] = za + zb;
       fence_proxy_async_smem();
       tc_fence_before();
+      mbar_arrive(keys_ready);   // gates known: decay mode, running sums
       mbar_arrive(feat);
+
+      // State for this chunk: the bf16 copy of alpha e^{m} S (MN-major B of the readout;
+      // e^{m} only in factored mode), then S <- e^{b_C} S in TMEM before the chunk's
+      // carry accumulates onto it.  The previous carry is done (state_done, above); the
+      // previous readout must be done with the copy.
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 8, c));
+      tc_fence_after();
+      {
+        const float dec = __expf(bC);
+        const float sbs = fast ? p.alpha * __expf(0.5f * bC) : p.alpha;
+#pragma unroll 1
+        for (int col = 0; col < D; col += 32) {
+          float v[32];
+          tmem_ld32(lane_base + kColS + col, v);
+          tmem_wait_ld();
+          if (r < D) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 8) {
+              float x[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) x[q] = sbs * v[u + q];
+              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] *= dec;
+          tmem_st32(lane_base + kColS + col, v);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(state_ready);
       named_bar(1, 128);   // lg is rewritten by the next chunk's keys
     }
     // final state of the sequence: the carry after the last chunk of its last segment
@@ -879,44 +917,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     tc_fence_before();
     named_bar(2, 256);
     tc_fence_after();
-    char* const sbb = smem + L::SB;
-    // State for chunk cc: the bf16 copy of alpha S (MN-major B of the readout), then
-    // S <- e^{b_C} S in TMEM before that chunk's carry accumulates onto it.  Needs the
-    // chunk's gates (keys_ready), the previous carry done (state_done) and the previous
-    // readout done with the copy (mma2_done).
-    auto prepare_state = [&](int cc) {
-      mbar_wait(keys_ready, cc & 1, wc, wsite(4, 3, cc));
-      if (cc > 0) {
-        mbar_wait(state_done, (cc - 1) & 1, wc, wsite(4, 5, cc));
-        mbar_wait(mma2_done, (cc - 1) & 1, wc, wsite(4, 4, cc));
-      }
-      tc_fence_after();
-      const int nvc = min(C, sg.t_end - (sg.t_begin + cc * C));
-      const float dec = __expf(bsh2[(cc & 1) * 64 + nvc - 1]);
-#pragma unroll 1
-      for (int col = 0; col < D; col += 32) {
-        float v[32];
-        tmem_ld32(lane_base + kColS + col, v);
-        tmem_wait_ld();
-        if (r < D) {
-#pragma unroll
-          for (int u = 0; u < 32; u += 8) {
-            float x[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) x[q] = alpha * v[u + q];
-            st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 32; ++u) v[u] *= dec;
-        tmem_st32(lane_base + kColS + col, v);
-      }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(state_ready);
-    };
-    prepare_state(0);
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -932,17 +932,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const uint32_t ss_base = lane_base + kColSs + 16 * wq;
       mbar_wait(ss_done, c & 1, wc, wsite(4, 6, c));
       tc_fence_after();
+      // Columns 16..63 are inside every row's band except in the sequence's first chunk:
+      // only the outer groups (and that chunk) take the mask.
+      const bool first = t0 == sg.q0;
       float m = -INFINITY;
 #pragma unroll 1
       for (int q5 = 0; q5 < 5; ++q5) {
         float s[16];
         tmem_ld16(ss_base + 16 * q5, s);
         tmem_wait_ld();
+        if (first || q5 == 0 || q5 == 4) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = 16 * q5 + u;
-          if (j >= jlo && j <= jhi) m = fmaxf(m, s[u]);
+          for (int u = 0; u < 16; ++u) {
+            const int j = 16 * q5 + u;
+            s[u] = (j >= jlo && j <= jhi) ? s[u] : -INFINITY;
+          }
         }
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int u = 0; u < w; ++u) s[u] = fmaxf(s[u], s[u + w]);
+        m = fmaxf(m, s[0]);
       }
       const float msc = m * sscale;
       float la = 0.f, lb = 0.f;   // exps written back over the scores
@@ -952,9 +962,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         tmem_ld16(ss_base + 16 * q5, s);
         tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = 16 * q5 + u;
-          s[u] = (j >= jlo && j <= jhi) ? ex2(fmaf(s[u], sscale, -msc)) : 0.f;
+        for (int u = 0; u < 16; ++u) s[u] = ex2(fmaf(s[u], sscale, -msc));
+        if (first || q5 == 0 || q5 == 4) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int j = 16 * q5 + u;
+            s[u] = (j >= jlo && j <= jhi) ? s[u] : 0.f;
+          }
         }
         la += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
         lb += ((s[8] + s[9]) + (s[10] + s[11])) + ((s[12] + s[13]) + (s[14] + s[15]));
@@ -965,8 +979,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
       tc_fence_after();
       const bool fast = fast2[c & 1] != 0.f;
-      const float zrow = zq2[(c & 1) * 128 + r];   // the tiles carry e_q unnormalised: scale P by Z
-      const float coef = beta * zrow / (la + lb);
+      // The tiles carry e_q unnormalised: P is scaled by Z and the output by 1/Z.  In
+      // factored mode P also carries e^{m - b_i} and the output e^{b_i - m}.
+      const float zrow = zq2[(c & 1) * 128 + r];
+      const float bi = bsh[i];
+      const float mrow = fast ? 0.5f * bsh[nv - 1] - bi : 0.f;
+      const float coef = beta * zrow * __expf(mrow) / (la + lb);
+      const float oscale = __expf(-mrow) / zrow;
 #pragma unroll 1
       for (int q5 = 0; q5 < 5; ++q5) {
         float s[16];
@@ -987,7 +1006,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 
       // recurrent probability tile over the current keys kk <= i, written over the
       // recurrent scores (this warp needs kk < 16 wq + 16; later blocks are zero)
-      const float bi = bsh[i];
 #pragma unroll 1
       for (int bb = 0; bb < 4; ++bb) {
         uint32_t ag[8];
@@ -999,7 +1017,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           for (int k = 0; k < 8; ++k) {
             const int kk = 16 * bb + 2 * k;
             float g0, g1;
-            if (fast) {   // e^{b_i} is already in the scores: multiply by e^{-b_kk} / z_kk
+            if (fast) {   // e^{m - b_kk} / z_kk; the row's e^{b_i - m} comes in the epilogue
               g0 = alpha * g[2 * k] * eneg[kk];
               g1 = alpha * g[2 * k + 1] * eneg[kk + 1];
             } else {
@@ -1017,13 +1035,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_ready);
-      if (c + 1 < nch) prepare_state(c + 1);   // overlaps this chunk's P.V on the tensor core
 
       // epilogue: O -> bf16 rows of out
       const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
       tc_fence_after();
       {
-        const float iz = 1.0f / zrow;
+        const float iz = oscale;
         const long t = (long)t0 + i;
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
         const bool store = i < nv && live;

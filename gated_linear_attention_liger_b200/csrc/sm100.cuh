@@ -93,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// Call-site code of a wait: role (1 producer, 2 MMA, 3 features, 4 window), barrier id, chunk.
+// Call-site code of a wait: role (1 producer, 2 MMA, 3 keys, 4 window, 5 queries), barrier id, chunk.
 __device__ __forceinline__ uint32_t wsite(uint32_t role, uint32_t barrier, int chunk) {
   return (role << 28) | (barrier << 20) | ((uint32_t)chunk & 0xFFFFFu);
 }

@@ -33,7 +33,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
         del os.environ["LIGER_WAIT_LIMIT_NS"]
     assert ops.prefill_status(ws) == ops.LIGER_ERR_TIMEOUT
     msg = ops.last_error()
-    assert "gave up waiting" in msg and any(f"role {r}," in msg for r in (2, 3, 4))
+    assert "gave up waiting" in msg and any(f"role {r}," in msg for r in (2, 3, 4, 5))
     # the context is intact: a normal call right after is correct and reports OK
     out, fs = ops.prefill(q, k, v, workspace=ws)
     torch.cuda.synchronize()
