@@ -161,17 +161,23 @@ __global__ void scan_kernel(DevParams p) {
   const SeqInfo si = p.seqs[seq];
   const int nsub = p.nsub;
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = si.first_seg; s < si.first_seg + si.n_seg; ++s) {
-    float4 d[kMaxSub];
-    float g[kMaxSub];
+  // the next segment's contributions are in flight while the current one is folded
+  float4 d[kMaxSub], dn[kMaxSub];
+  float g[kMaxSub], gn[kMaxSub];
+  auto fetch = [&](int s, float4 (&dd)[kMaxSub], float (&gg)[kMaxSub]) {
 #pragma unroll
     for (int k = 0; k < kMaxSub; ++k) {
       if (k < nsub) {
         const size_t u = (size_t)s * nsub + k;
-        d[k] = *reinterpret_cast<const float4*>(p.ds + (u * p.Hkv + kv) * D * D + e);
-        g[k] = __expf(p.lam[u * p.Hkv + kv]);
+        dd[k] = __ldcs(reinterpret_cast<const float4*>(p.ds + (u * p.Hkv + kv) * D * D + e));
+        gg[k] = __expf(p.lam[u * p.Hkv + kv]);
       }
     }
+  };
+  const int s_end = si.first_seg + si.n_seg;
+  if (si.n_seg > 0) fetch(si.first_seg, d, g);
+  for (int s = si.first_seg; s < s_end; ++s) {
+    if (s + 1 < s_end) fetch(s + 1, dn, gn);
     *reinterpret_cast<float4*>(p.ds + ((size_t)s * nsub * p.Hkv + kv) * D * D + e) = run;
 #pragma unroll
     for (int k = 0; k < kMaxSub; ++k) {
@@ -179,6 +185,8 @@ __global__ void scan_kernel(DevParams p) {
         run = make_float4(fmaf(g[k], run.x, d[k].x), fmaf(g[k], run.y, d[k].y), fmaf(g[k], run.z, d[k].z),
                           fmaf(g[k], run.w, d[k].w));
     }
+#pragma unroll
+    for (int k = 0; k < kMaxSub; ++k) { d[k] = dn[k]; g[k] = gn[k]; }
   }
 }
 
@@ -234,7 +242,7 @@ __device__ __forceinline__ float log_sigmoid_fast(float m) {
 // to bsh.  Each pass is a short loop over 16-byte groups: the role loops of the
 // chunk kernel share one SM sub-partition, and fully unrolled straight-line code
 // for all of them would not stay in the instruction caches.
-template <int D>
+template <int D, uint32_t KSTRIDE = C * 128>   // KSTRIDE: byte stride of the raw tile's 64-element blocks
 __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, float* lg, float* bsh, int r, int nv,
                                               GateSums& gs) {
   constexpr int HALF = D / 2;
@@ -243,7 +251,7 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   float m = -INFINITY, sa = 0.f, sb = 0.f;
 #pragma unroll 4
   for (int c = 0; c < HALF / 8; ++c) {
-    const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, C * 128));
+    const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, KSTRIDE));
     m = fmaxf(m, bf16x8_max(u));
     sa += (bf16_lo(u.x) + bf16_hi(u.x)) + (bf16_lo(u.y) + bf16_hi(u.y));
     sb += (bf16_lo(u.z) + bf16_hi(u.z)) + (bf16_lo(u.w) + bf16_hi(u.w));
@@ -255,14 +263,13 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   float za = 0.f, zb = 0.f;
 #pragma unroll 4
   for (int c = 0; c < HALF / 8; ++c) {
-    const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
     float x[8];
-    ld_chunk8(kraw, off, x);
+    ld_chunk8(kraw, kmajor_off(j, h * HALF + c * 8, KSTRIDE), x);
 #pragma unroll
     for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
     za += (x[0] + x[1]) + (x[2] + x[3]);
     zb += (x[4] + x[5]) + (x[6] + x[7]);
-    st_chunk8(ebuf, off, x);
+    st_chunk8(ebuf, kmajor_off(j, h * HALF + c * 8, C * 128), x);
   }
   float z = za + zb;
   z += __shfl_xor_sync(0xffffffffu, z, 1);
@@ -483,16 +490,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 template <int D, int NC>
 __device__ __forceinline__ void entering_state(const DevParams& p, int seg, int kv, int row, uint32_t taddr,
                                                int c0) {
+  static_assert(NC % 16 == 0, "columns come in groups of 16");
   const float* src = p.ds + (((size_t)seg * p.nsub * p.Hkv + kv) * D + row) * D;
+#pragma unroll 1
+  for (int col = c0; col < c0 + NC; col += 16) {
+    float v[16];
 #pragma unroll
-  for (int col = c0; col < c0 + NC; col += 32) {
-    float v[32];
-#pragma unroll
-    for (int u = 0; u < 32; u += 4) {
+    for (int u = 0; u < 16; u += 4) {
       const float4 x = *reinterpret_cast<const float4*>(src + col + u);
       v[u] = x.x; v[u + 1] = x.y; v[u + 2] = x.z; v[u + 3] = x.w;
     }
-    tmem_st32(taddr + col, v);
+    tmem_st16(taddr + col, v);
   }
   tmem_wait_st();
 }
@@ -503,13 +511,13 @@ struct ChunkSmem {
   static constexpr uint32_t KV = C * D * 2;       // one chunk of k or v
   static constexpr uint32_t Q0 = 0;
   static constexpr uint32_t EQ = Q0 + QB;         // e_q = exp(q - max), bf16
-  static constexpr uint32_t K0 = EQ + QB;         // 2 key slots
+  static constexpr uint32_t K0 = EQ + QB;         // 2 key slots, laid out [64-d block][slot][64 rows]
   static constexpr uint32_t V0 = K0 + 2 * KV;     // 3 value slots
   static constexpr uint32_t PK = V0 + 3 * KV;     // phi(k)
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
   static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
   static constexpr uint32_t SMALL = SB + D * D * 2;
-  static constexpr uint32_t SMALL_BYTES = 4096;
+  static constexpr uint32_t SMALL_BYTES = 6144;
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
@@ -519,7 +527,13 @@ constexpr uint32_t kColSg = 128;   // recurrent scores (64); then the recurrent 
 constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
 constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
 
-constexpr int kChunkThreads = 448;   // warps 0-3 window/epilogue, 4-7 keys, 8-11 queries, 12 TMA, 13 MMA
+// Window warps per TMEM lane quarter (1 or 2: two split the columns).
+constexpr int kWinHalves = 1;
+constexpr int kWinThreads = 128 * kWinHalves;
+// warps [0, 4 kWinHalves) window/epilogue, then 4 keys, 4 queries, 1 TMA, 1 MMA
+constexpr int kKeyWarp0 = 4 * kWinHalves, kQueryWarp0 = kKeyWarp0 + 4;
+constexpr int kTmaWarp = kQueryWarp0 + 4, kMmaWarp = kTmaWarp + 1;
+constexpr int kChunkThreads = 32 * (kMmaWarp + 1);
 
 template <int D>
 __global__ void __launch_bounds__(kChunkThreads, 1)
@@ -541,10 +555,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* feat = bars + 13;        // key and query tiles of the chunk ready (256 arrivals)
   uint64_t* sg_done = bars + 14;     // recurrent scores and state carry done
   uint64_t* mma2_done = bars + 15;   // + readout done: feature buffers free again
-  uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (128 arrivals)
-  uint64_t* p_ready = bars + 17;     // probability tile in TMEM (128 arrivals)
+  uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (window threads)
+  uint64_t* p_ready = bars + 17;     // probability tile in TMEM (window threads)
   uint64_t* o_done = bars + 18;      // output accumulator complete
-  uint64_t* o_free = bars + 19;      // output read out (128 arrivals)
+  uint64_t* o_free = bars + 19;      // output read out (window threads)
   uint64_t* drain = bars + 20;
   uint64_t* keys_ready = bars + 21;  // gates of the chunk known (128 arrivals)
   uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (128 arrivals)
@@ -558,6 +572,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
   float* fast2 = lg + 64;                                       // [2] factored decay usable
   float* izk2 = fast2 + 2;                                      // [2][64] 1 / z_k per key token
+  float* rowx = izk2 + 128;                                     // [2][128] row maxima, [2][128] row sums
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -571,10 +586,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-    mbar_init(q_full, 1); mbar_init(q_empty, 1);
+    mbar_init(q_full, 1); mbar_init(q_empty, 2);
     mbar_init(ss_done, 1); mbar_init(feat, 256); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
     mbar_init(keys_ready, 128); mbar_init(state_ready, 128); mbar_init(state_done, 1);
-    mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
+    mbar_init(s_read, kWinThreads); mbar_init(p_ready, kWinThreads); mbar_init(o_done, 1);
+    mbar_init(o_free, kWinThreads);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
@@ -590,7 +606,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.err, p.wait_ns};
 
-  if (warp == 12) {   // ---------------- TMA producer
+  if (warp == kTmaWarp) {   // ---------------- TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmq);
       prefetch_tensormap(&tmk);
@@ -601,7 +617,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mbar_arrive_expect_tx(&k_full[slot], L::KV);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
-          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &k_full[slot], kb * 64, kv,
+          tma_load_3d(smem + L::K0 + slot * (C * 128) + kb * (2 * C * 128), &tmk, &k_full[slot], kb * 64, kv,
                       sg.t_begin + (u - 1) * C);
       };
       auto load_v = [&](int u) {
@@ -639,9 +655,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       for (int u = (v_issued > 3 ? v_issued - 3 : 0); u < v_issued; ++u) mbar_wait(&v_full[u % 3], (u / 3) & 1, dw);
       mbar_wait(q_full, (q_issued - 1) & 1, dw);
     }
-  } else if (warp == 13) {   // ---------------- MMA issuer
+  } else if (warp == kMmaWarp) {   // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_n64 = idesc_bf16(128, 64, 0, 0);
+      const uint32_t id_n128 = idesc_bf16(128, 128, 0, 0);
       const uint32_t id_inter = idesc_bf16(128, D, 0, 1);
       const uint32_t id_state = idesc_bf16(128, D, 1, 1);
       const uint32_t lbo_kt = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
@@ -658,16 +675,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (c > 0) ok = ok && mbar_wait(s_read, (c - 1) & 1, wc, wsite(2, 4, c));
         if (!ok) return;
         tc_fence_after();
-        const uint32_t kp = smem_u32(smem + L::K0 + (c & 1) * L::KV);
-        const uint32_t kc = smem_u32(smem + L::K0 + ((c + 1) & 1) * L::KV);
+        // both key slots as one 128-row operand: score columns [slot 0 | slot 1], that is
+        // [previous | current] for even chunks and [current | previous] for odd ones
+        const uint32_t kb = smem_u32(smem + L::K0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
           const uint64_t a = sdesc_sw128(q_base + (kk >> 2) * (ROWS * 128) + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + kColSs, a, sdesc_sw128(kp + ko, 16, 1024), id_n64, kk > 0);
-          mma_bf16_ss(tmem + kColSs + 64, a, sdesc_sw128(kc + ko, 16, 1024), id_n64, kk > 0);
+          const uint64_t b = sdesc_sw128(kb + (kk >> 2) * (2 * C * 128) + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + kColSs, a, b, id_n128, kk > 0);
         }
         mma_commit(ss_done);
+        mma_commit(q_empty);           // one of the q buffer's two releases (the raw q was read)
         mma_commit(&k_empty[c & 1]);   // the previous chunk's keys are no longer needed
       };
       auto issue_pv = [&](int c) {   // O += P_prev V_prev + P_cur V_cur, P read from TMEM
@@ -729,26 +747,28 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                       sdesc_sw128(sb_base + kk * 2048, D * 128, 1024), id_inter, kk > 0);
         }
         mma_commit(mma2_done);
-        if (!fast) mma_commit(q_empty);   // in factored mode the feature warps released it
+        if (!fast) mma_commit(q_empty);   // exact decay: the readout read e^{b_i} e_q from the q buffer
       };
+      // A chunk's P.V goes out before the next chunk's window scores: the window warps
+      // wait for it, while the next scores are needed only after their epilogue.
       issue_ss(0);
       issue_sg_state(0);
       issue_inter(0);
       for (int c = 1; c < nch && ok; ++c) {
-        issue_ss(c);
         issue_pv(c - 1);
+        issue_ss(c);
         issue_sg_state(c);
         issue_inter(c);
       }
       issue_pv(nch - 1);
       mma_commit(drain);
     }
-  } else if (warp >= 8) {   // ---------------- queries (threads 0..127 of warps 8-11)
+  } else if (warp >= kQueryWarp0) {   // ---------------- queries (128 threads)
     // e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the window
     // warps fold Z into P and 1/Z into the output).  Needs no gate: with the decay
     // factored around the chunk's midpoint the row factor e^{b_i - m} is applied in the
     // epilogue.  Never leaves the loop early (see the key warps).
-    const int r = threadIdx.x - 256;
+    const int r = threadIdx.x - 32 * kQueryWarp0;
     const int i = r >> 1;
     constexpr float kLog2e = 1.4426950408889634f;
     char* const qb = smem + L::Q0;
@@ -776,15 +796,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         st_chunk8(eqb, off, x);
       }
       zq2[(c & 1) * 128 + r] = za + zb;
-      // the decay mode of the chunk comes with its keys
+      // The decay mode of the chunk comes with its keys.  The q buffer is released twice
+      // per chunk: by the score MMA's commit, and by these warps once done with the raw q
+      // (factored mode) or by the readout's commit (exact mode: the buffer then holds
+      // e^{b_i} e_q, the readout's A operand).
       mbar_wait(keys_ready, c & 1, wc, wsite(5, 3, c));
-      if (fast2[c & 1] != 0.f) {   // raw q no longer needed: release it once the score MMA read it too
+      if (fast2[c & 1] != 0.f) {
         named_bar(4, 128);
-        if (r == 0) {
-          mbar_wait(ss_done, c & 1, wc, wsite(5, 4, c));
-          mbar_arrive(q_empty);
-        }
-      } else {   // exact decay: the q buffer takes e^{b_i} e_q, the readout's A operand
+        if (r == 0) mbar_arrive(q_empty);
+      } else {
         mbar_wait(ss_done, c & 1, wc, wsite(5, 4, c));
         const float ebi = __expf(bsh2[(c & 1) * 64 + i]);
 #pragma unroll 4
@@ -800,11 +820,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(feat);
     }
-  } else if (warp >= 4) {   // ---------------- keys (threads 0..127 of warps 4-7)
+  } else if (warp >= kKeyWarp0) {   // ---------------- keys (128 threads)
     // Row threads never leave the loop early: after a timeout every wait returns
     // at once (the CTA's abort flag is set), so the group still meets at each
     // named barrier and warp-collective TMEM access stays uniform.
-    const int r = threadIdx.x - 128;
+    const int r = threadIdx.x - 32 * kKeyWarp0;
     const int i = r >> 1;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     char* const sbb = smem + L::SB;
@@ -812,7 +832,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     // state entering the segment, first half of the columns (the window warps do the rest)
     entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColS, 0);
     tc_fence_before();
-    named_bar(2, 256);
+    named_bar(2, 128 + kWinThreads);
     tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
@@ -831,7 +851,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       float bC, bi, iz;
       {
         GateSums gs;
-        iz = key_features<D>(smem + L::K0 + ((c + 1) & 1) * L::KV, smem + L::PK, lg, bsh, r, nv, gs);
+        iz = key_features<D, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK, lg, bsh, r, nv, gs);
         bC = gs.at(nv - 1);
         bi = gs.at(i);
         write_ktilde<D>(smem + L::PK, smem + L::KT, r, i < nv ? __expf(bC - bi) * iz : 0.f);   // token r >> 1 = i
@@ -904,19 +924,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
       }
     }
-  } else {   // ---------------- window softmax and epilogue (threads 0..127, warps 0-3)
-    const int r = threadIdx.x;
+  } else {   // ---------------- window softmax and epilogue (kWinThreads threads)
+    // kWinHalves warps per TMEM lane quarter: with two, warps wq and wq + 4 share rows
+    // 32 wq .. 32 wq + 31 and split the columns (window groups 0-2 / 3-4, recurrent blocks
+    // by parity after all are loaded, output columns 0..D/2-1 / D/2..D-1); row maxima and
+    // sums are then exchanged through shared memory.
+    const int r = threadIdx.x & 127, sh = threadIdx.x >> 7;
     const int i = r >> 1, hl = r & 1;
-    const int wq = warp, il = i - 16 * wq;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int wq = warp & 3, il = i - 16 * wq;
+    const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    // state entering the segment, second half of the columns (TMEM: the state follows O)
-    entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColO + D, D / 2);
+    // state entering the segment, this thread's share of the second half of the columns
+    // (the key warps load the first half; TMEM: the state follows O)
+    constexpr int kEnt = D / (2 * kWinHalves);
+    entering_state<D, kEnt>(p, seg, kv, r % D, lane_base + kColO + D, D / 2 + sh * kEnt);
     tc_fence_before();
-    named_bar(2, 256);
+    named_bar(2, 128 + kWinThreads);
     tc_fence_after();
+    // this thread's window column groups
+    const int g_lo = kWinHalves == 1 ? 0 : (sh ? 3 : 0), g_hi = kWinHalves == 1 ? 5 : (sh ? 5 : 3);
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -925,11 +953,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float* eneg = eneg2 + (c & 1) * 64;
       const float* izk = izk2 + (c & 1) * 64;
       // Window band.  Key index x over [previous chunk | current chunk] (0..127): row i
-      // sees x in [i+1, i+64].  This warp's tokens are 16 wq .. 16 wq + 15, so it reads the
-      // 80 columns starting at 16 wq; column j then holds x = 16 wq + j and is live for
+      // sees x in [i+1, i+64].  This quarter's tokens are 16 wq .. 16 wq + 15, so it reads
+      // the 80 columns starting at 16 wq; column j then holds x = 16 wq + j and is live for
       // j in [il+1, il+64], il = i - 16 wq (only x >= 64 in the sequence's first chunk).
       const int jlo = max(il + 1, t0 == sg.q0 ? 64 - 16 * wq : 0), jhi = il + 64;
-      const uint32_t ss_base = lane_base + kColSs + 16 * wq;
+      // score column of key x: (x + 64 (c & 1)) mod 128 (the two key slots form one operand)
+      const int ss_rot = 16 * wq + ((c & 1) << 6);
+      auto ss_col = [&](int q5) { return lane_base + kColSs + ((ss_rot + 16 * q5) & 127); };
       mbar_wait(ss_done, c & 1, wc, wsite(4, 6, c));
       tc_fence_after();
       // Columns 16..63 are inside every row's band except in the sequence's first chunk:
@@ -937,9 +967,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const bool first = t0 == sg.q0;
       float m = -INFINITY;
 #pragma unroll 1
-      for (int q5 = 0; q5 < 5; ++q5) {
+      for (int q5 = g_lo; q5 < g_hi; ++q5) {
         float s[16];
-        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_ld16(ss_col(q5), s);
         tmem_wait_ld();
         if (first || q5 == 0 || q5 == 4) {
 #pragma unroll
@@ -954,12 +984,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           for (int u = 0; u < w; ++u) s[u] = fmaxf(s[u], s[u + w]);
         m = fmaxf(m, s[0]);
       }
+      if (kWinHalves == 2) {
+        rowx[sh * 128 + r] = m;
+        named_bar(3, kWinThreads);
+        m = fmaxf(rowx[r], rowx[128 + r]);
+      }
       const float msc = m * sscale;
       float la = 0.f, lb = 0.f;   // exps written back over the scores
 #pragma unroll 1
-      for (int q5 = 0; q5 < 5; ++q5) {
+      for (int q5 = g_lo; q5 < g_hi; ++q5) {
         float s[16];
-        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_ld16(ss_col(q5), s);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u) s[u] = ex2(fmaf(s[u], sscale, -msc));
@@ -972,31 +1007,47 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
         la += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
         lb += ((s[8] + s[9]) + (s[10] + s[11])) + ((s[12] + s[13]) + (s[14] + s[15]));
-        tmem_st16(ss_base + 16 * q5, s);
+        tmem_st16(ss_col(q5), s);
       }
       tmem_wait_st();
-      // Z of the rows and the recurrent scores come with the feature warps' tiles
+      if (kWinHalves == 2) rowx[256 + sh * 128 + r] = la + lb;
+      // Z of the rows and the recurrent scores come with the key and query tiles.  Both
+      // recurrent blocks of this half are read before the barrier: the probability tile is
+      // packed over the scores' first columns, which the other half may still be reading.
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
       tc_fence_after();
+      constexpr int kBlk = 4 / kWinHalves;   // recurrent blocks per thread: bb = kWinHalves t + sh
+      float g[kBlk][16];
+#pragma unroll
+      for (int t = 0; t < kBlk; ++t) {
+        const int bb = kWinHalves * t + sh;
+        if (bb <= wq) tmem_ld16(lane_base + kColSg + 16 * bb, g[t]);
+      }
+      tmem_wait_ld();
+      float lsum = la + lb;
+      if (kWinHalves == 2) {
+        named_bar(3, kWinThreads);
+        lsum = rowx[256 + r] + rowx[384 + r];
+      }
       const bool fast = fast2[c & 1] != 0.f;
       // The tiles carry e_q unnormalised: P is scaled by Z and the output by 1/Z.  In
       // factored mode P also carries e^{m - b_i} and the output e^{b_i - m}.
       const float zrow = zq2[(c & 1) * 128 + r];
       const float bi = bsh[i];
       const float mrow = fast ? 0.5f * bsh[nv - 1] - bi : 0.f;
-      const float coef = beta * zrow * __expf(mrow) / (la + lb);
+      const float coef = beta * zrow * __expf(mrow) / lsum;
       const float oscale = __expf(-mrow) / zrow;
 #pragma unroll 1
-      for (int q5 = 0; q5 < 5; ++q5) {
+      for (int q5 = g_lo; q5 < g_hi; ++q5) {
         float s[16];
-        tmem_ld16(ss_base + 16 * q5, s);
+        tmem_ld16(ss_col(q5), s);
         tmem_wait_ld();
         uint32_t pw[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
         tmem_st8u(lane_base + kColP + 8 * wq + 8 * q5, pw);
       }
-      {   // zeros for the keys outside this warp's band
+      if (sh == kWinHalves - 1) {   // zeros for the keys outside this quarter's band
         const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
         for (int k = 0; k < 3; ++k) tmem_st8u(lane_base + kColP + ((8 * wq + 40 + 8 * k) & 63), zero8);
@@ -1004,25 +1055,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_before();
       mbar_arrive(s_read);   // the window scores are consumed: their TMEM may be reused
 
-      // recurrent probability tile over the current keys kk <= i, written over the
-      // recurrent scores (this warp needs kk < 16 wq + 16; later blocks are zero)
-#pragma unroll 1
-      for (int bb = 0; bb < 4; ++bb) {
+      // recurrent probability tile over the current keys kk <= i, packed over the
+      // recurrent scores (this quarter needs kk < 16 wq + 16; later blocks are zero)
+#pragma unroll
+      for (int t = 0; t < kBlk; ++t) {
+        const int bb = kWinHalves * t + sh;
         uint32_t ag[8];
         if (bb <= wq) {
-          float g[16];
-          tmem_ld16(lane_base + kColSg + 16 * bb, g);
-          tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int kk = 16 * bb + 2 * k;
             float g0, g1;
             if (fast) {   // e^{m - b_kk} / z_kk; the row's e^{b_i - m} comes in the epilogue
-              g0 = alpha * g[2 * k] * eneg[kk];
-              g1 = alpha * g[2 * k + 1] * eneg[kk + 1];
+              g0 = alpha * g[t][2 * k] * eneg[kk];
+              g1 = alpha * g[t][2 * k + 1] * eneg[kk + 1];
             } else {
-              g0 = alpha * g[2 * k] * (__expf(bi - bsh[kk]) * izk[kk]);
-              g1 = alpha * g[2 * k + 1] * (__expf(bi - bsh[kk + 1]) * izk[kk + 1]);
+              g0 = alpha * g[t][2 * k] * (__expf(bi - bsh[kk]) * izk[kk]);
+              g1 = alpha * g[t][2 * k + 1] * (__expf(bi - bsh[kk + 1]) * izk[kk + 1]);
             }
             ag[k] = pack_bf16(kk <= i ? g0 : 0.f, kk + 1 <= i ? g1 : 0.f);
           }
@@ -1036,23 +1085,22 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_before();
       mbar_arrive(p_ready);
 
-      // epilogue: O -> bf16 rows of out
+      // epilogue: O -> bf16 rows of out, this half's columns
       const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
       tc_fence_after();
       {
-        const float iz = oscale;
         const long t = (long)t0 + i;
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
         const bool store = i < nv && live;
 #pragma unroll 1
-        for (int col = 0; col < D; col += 32) {
+        for (int col = sh * (D / kWinHalves); col < (sh + 1) * (D / kWinHalves); col += 32) {
           float v[32];
           tmem_ld32(lane_base + kColO + col, v);
           tmem_wait_ld();
           if (store) {
             uint32_t pw[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) pw[u] = pack_bf16(v[2 * u] * iz, v[2 * u + 1] * iz);
+            for (int u = 0; u < 16; ++u) pw[u] = pack_bf16(v[2 * u] * oscale, v[2 * u + 1] * oscale);
             if (p.out_v8) {   // two full 32-byte sectors per instruction
               st_global_v8(orow + col, pw);
               st_global_v8(orow + col + 16, pw + 8);
@@ -1131,9 +1179,19 @@ inline Plan make_plan(int B, int Hq, int Hkv, long T, int d, int n_seqs, bool va
                      : (long)B * ((chunks_per_seq + bestL - 1) / bestL);
   if (nseg < 1) nseg = 1;
   pl.n_seg_max = (int)nseg;
-  // the state pass splits segments so that about two of its CTAs run per SM
-  long nsub = (2L * sms + nseg * Hkv - 1) / (nseg * Hkv);
-  nsub = nsub < 1 ? 1 : (nsub > kMaxSub ? kMaxSub : (nsub > bestL ? bestL : nsub));
+  // The state pass splits segments into sub-segments; two of its CTAs run per SM.
+  // Minimise waves x sub-segment length (plus a fixed cost per CTA).
+  long nsub = 1;
+  {
+    const long units = nseg * Hkv;
+    double best_s = 1e300;
+    const long max_sub = bestL < kMaxSub ? bestL : kMaxSub;
+    for (long ns = 1; ns <= max_sub; ++ns) {
+      const double waves = std::ceil((double)units * ns / (2.0 * sms));
+      const double cost = waves * (std::ceil((double)bestL / ns) + 0.5);
+      if (cost < best_s - 1e-9) { best_s = cost; nsub = ns; }
+    }
+  }
   pl.nsub = (int)nsub;
   pl.Ls = (int)((bestL + nsub - 1) / nsub);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
