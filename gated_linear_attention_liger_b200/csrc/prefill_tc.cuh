@@ -53,7 +53,7 @@ using namespace liger::sm100;
 
 constexpr int C = 64;             // tokens per chunk
 constexpr int ROWS = 128;         // MMA M: two heads x 64 tokens
-constexpr int NTHREADS = 192;     // warps 0-3 rows, warp 4 TMA, warp 5 MMA
+constexpr int kSegThreads = 320;  // state pass: warps 0-7 rows, warp 8 TMA, warp 9 MMA
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;   // 2 s per wait
 
 struct SegInfo {
@@ -233,48 +233,53 @@ __device__ __forceinline__ float log_sigmoid_fast(float m) {
 }
 
 // Feature map and gate of one chunk of keys, shared by the seg_state and chunk
-// kernels.  Thread r (0..127) owns half of token j = r >> 1: elements
-// [h * D/2, (h+1) * D/2) with h = r & 1.  Writes e = exp(k - max_d k) (bf16, not
-// yet divided by its sum) to `ebuf` in the key tile's swizzled layout and the log
-// gates to lg[0..63] (0 past the valid tokens); returns 1 / sum_d e, which the
-// callers fold into per-token scalars, and the running sums in gs (every warp
-// scans the 64 gates itself); lanes of the group's first warp also store the sums
-// to bsh.  Each pass is a short loop over 16-byte groups: the role loops of the
-// chunk kernel share one SM sub-partition, and fully unrolled straight-line code
-// for all of them would not stay in the instruction caches.
-template <int D, uint32_t KSTRIDE = C * 128>   // KSTRIDE: byte stride of the raw tile's 64-element blocks
+// kernels.  TPT threads (2 or 4, adjacent lanes) share a key token: thread r owns
+// elements [h D/TPT, (h+1) D/TPT) of token j = r / TPT, h = r % TPT, and the group
+// is 64 TPT threads.  Writes e = exp(k - max_d k) (bf16, not yet divided by its sum)
+// to `ebuf` in the key tile's swizzled layout and the log gates to lg[0..63] (0 past
+// the valid tokens); returns 1 / sum_d e, which the callers fold into per-token
+// scalars, and the running sums in gs (every warp scans the 64 gates itself); lanes
+// of the group's first warp also store the sums to bsh.  Each pass is a short loop
+// over 16-byte groups: the role loops of the chunk kernel share one SM
+// sub-partition, and fully unrolled straight-line code for all of them would not
+// stay in the instruction caches.
+template <int D, int TPT = 2, uint32_t KSTRIDE = C * 128>   // KSTRIDE: byte stride of the raw tile's 64-element blocks
 __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, float* lg, float* bsh, int r, int nv,
                                               GateSums& gs) {
-  constexpr int HALF = D / 2;
+  constexpr int PART = D / TPT;
   constexpr float kLog2e = 1.4426950408889634f;
-  const int j = r >> 1, h = r & 1;
+  const int j = r / TPT, h = r % TPT;
   float m = -INFINITY, sa = 0.f, sb = 0.f;
 #pragma unroll 4
-  for (int c = 0; c < HALF / 8; ++c) {
-    const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * HALF + c * 8, KSTRIDE));
+  for (int c = 0; c < PART / 8; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * PART + c * 8, KSTRIDE));
     m = fmaxf(m, bf16x8_max(u));
     sa += (bf16_lo(u.x) + bf16_hi(u.x)) + (bf16_lo(u.y) + bf16_hi(u.y));
     sb += (bf16_lo(u.z) + bf16_hi(u.z)) + (bf16_lo(u.w) + bf16_hi(u.w));
   }
   float sum = sa + sb;
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+#pragma unroll
+  for (int o = 1; o < TPT; o <<= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
   const float ml = m * kLog2e;
   float za = 0.f, zb = 0.f;
 #pragma unroll 4
-  for (int c = 0; c < HALF / 8; ++c) {
+  for (int c = 0; c < PART / 8; ++c) {
     float x[8];
-    ld_chunk8(kraw, kmajor_off(j, h * HALF + c * 8, KSTRIDE), x);
+    ld_chunk8(kraw, kmajor_off(j, h * PART + c * 8, KSTRIDE), x);
 #pragma unroll
     for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
     za += (x[0] + x[1]) + (x[2] + x[3]);
     zb += (x[4] + x[5]) + (x[6] + x[7]);
-    st_chunk8(ebuf, kmajor_off(j, h * HALF + c * 8, C * 128), x);
+    st_chunk8(ebuf, kmajor_off(j, h * PART + c * 8, C * 128), x);
   }
   float z = za + zb;
-  z += __shfl_xor_sync(0xffffffffu, z, 1);
+#pragma unroll
+  for (int o = 1; o < TPT; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   if (h == 0) lg[j] = j < nv ? log_sigmoid_fast(sum / (float)D) : 0.f;
-  named_bar(1, 128);
+  named_bar(1, 64 * TPT);
   {   // inclusive running sum over the 64 tokens, two per lane, in every warp
     const int lane = r & 31;
     const float a0 = lg[2 * lane], a1 = lg[2 * lane + 1];
@@ -296,15 +301,15 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
 }
 
 // Decay-scaled keys sc * e (sc = e^{b_C - b_j} / z_j, zero past the valid tokens),
-// from this thread's features in `ebuf` to `kt` in the same swizzled layout; read
-// by the MMA as the MN-major A operand K^T.
-template <int D>
+// from this thread's features in `ebuf` to `kt` in the same swizzled layout (thread
+// layout as in key_features); read by the MMA as the MN-major A operand K^T.
+template <int D, int TPT = 2>
 __device__ __forceinline__ void write_ktilde(const char* ebuf, char* kt, int r, float sc) {
-  constexpr int HALF = D / 2;
-  const int j = r >> 1, h = r & 1;
+  constexpr int PART = D / TPT;
+  const int j = r / TPT, h = r % TPT;
 #pragma unroll 4
-  for (int c = 0; c < HALF / 8; ++c) {
-    const uint32_t off = kmajor_off(j, h * HALF + c * 8, C * 128);
+  for (int c = 0; c < PART / 8; ++c) {
+    const uint32_t off = kmajor_off(j, h * PART + c * 8, C * 128);
     float x[8];
     ld_chunk8(ebuf, off, x);
 #pragma unroll
@@ -318,27 +323,31 @@ __device__ __forceinline__ void write_ktilde(const char* ebuf, char* kt, int r, 
 template <int D>
 struct SegSmem {
   static constexpr uint32_t KV = C * D * 2;        // one chunk of k (or v)
-  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 4 * KV, E = 5 * KV, SMALL = 6 * KV;
+  // key ring (2 slots, released by the row warps once the features are out), value
+  // ring (3 slots, released by the MMA), decay-scaled keys
+  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 5 * KV, SMALL = 6 * KV;
   static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
 };
 
 template <int D>
-__global__ void __launch_bounds__(NTHREADS, 2)
+__global__ void __launch_bounds__(kSegThreads, 2)
     seg_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      DevParams p) {
   using L = SegSmem<D>;
   extern __shared__ __align__(1024) char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
-  uint64_t* kv_full = bars;        // [2]
-  uint64_t* kv_empty = bars + 2;   // [2]
-  uint64_t* feat = bars + 4;
-  uint64_t* mma_done = bars + 5;
-  uint64_t* drain = bars + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* k_full = bars;         // [2]
+  uint64_t* k_empty = bars + 2;    // [2] (256 arrivals)
+  uint64_t* v_full = bars + 4;     // [3]
+  uint64_t* v_empty = bars + 7;    // [3]
+  uint64_t* feat = bars + 10;
+  uint64_t* mma_done = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
-  float* lg = reinterpret_cast<float*>(bars + 10);   // 64 floats
+  float* lg = reinterpret_cast<float*>(bars + 16);   // 64 floats
 
   const int unit = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
   const int seg = unit / p.nsub, sub = unit % p.nsub;
@@ -361,9 +370,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   constexpr uint32_t TCOLS = D < 32 ? 32 : D;
 
   if (threadIdx.x == 0) {
-    mbar_init(&kv_full[0], 1); mbar_init(&kv_full[1], 1);
-    mbar_init(&kv_empty[0], 1); mbar_init(&kv_empty[1], 1);
-    mbar_init(feat, 128); mbar_init(mma_done, 1); mbar_init(drain, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 256); }
+    for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    mbar_init(feat, 256); mbar_init(mma_done, 1); mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
     fence_mbar_init();
@@ -378,50 +387,57 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.err, p.wait_ns};
 
-  if (warp == 4) {   // ---------------- TMA producer
+  if (warp == 8) {   // ---------------- TMA producer
     if (lane == 0) {
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int c = 0; c < nch; ++c) {
-        const int slot = c & 1;
-        if (c >= 2 && !mbar_wait(&kv_empty[slot], ((c >> 1) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&kv_full[slot], 2 * L::KV);
         const int t = sg.t_begin + c * C;
+        const int ks = c & 1, vs = c % 3;
+        if (c >= 2 && !mbar_wait(&k_empty[ks], ((c >> 1) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&k_full[ks], L::KV);
 #pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb) {
-          tma_load_3d(smem + L::K0 + slot * L::KV + kb * C * 128, &tmk, &kv_full[slot], kb * 64, kv, t);
-          tma_load_3d(smem + L::V0 + slot * L::KV + kb * C * 128, &tmv, &kv_full[slot], kb * 64, kv, t);
-        }
-        issued = c + 1;
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(smem + L::K0 + ks * L::KV + kb * C * 128, &tmk, &k_full[ks], kb * 64, kv, t);
+        k_issued = c + 1;
+        if (c >= 3 && !mbar_wait(&v_empty[vs], (c / 3 - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&v_full[vs], L::KV);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(smem + L::V0 + vs * L::KV + kb * C * 128, &tmv, &v_full[vs], kb * 64, kv, t);
+        v_issued = c + 1;
       }
       // never leave the CTA with copies in flight
-      for (int c = (issued > 2 ? issued - 2 : 0); c < issued; ++c)
-        mbar_wait(&kv_full[c & 1], (c >> 1) & 1, WaitCtx{never, nullptr, p.wait_ns});
+      const WaitCtx dw{never, nullptr, p.wait_ns};
+      for (int c = (k_issued > 2 ? k_issued - 2 : 0); c < k_issued; ++c) mbar_wait(&k_full[c & 1], (c >> 1) & 1, dw);
+      for (int c = (v_issued > 3 ? v_issued - 3 : 0); c < v_issued; ++c) mbar_wait(&v_full[c % 3], (c / 3) & 1, dw);
     }
-  } else if (warp == 5) {   // ---------------- MMA issuer
+  } else if (warp == 9) {   // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, D, 1, 1);
       const uint32_t lbo_a = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
       for (int c = 0; c < nch; ++c) {
-        const int slot = c & 1;
-        if (!mbar_wait(&kv_full[slot], (c >> 1) & 1, wc)) break;
+        const int vs = c % 3;
+        if (!mbar_wait(&v_full[vs], (c / 3) & 1, wc)) break;
         if (!mbar_wait(feat, c & 1, wc)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint64_t a = sdesc_sw128(smem_u32(smem + L::KT) + kk * 2048, lbo_a, 1024);
-          const uint64_t b = sdesc_sw128(smem_u32(smem + L::V0 + slot * L::KV) + kk * 2048, C * 128, 1024);
+          const uint64_t b = sdesc_sw128(smem_u32(smem + L::V0 + vs * L::KV) + kk * 2048, C * 128, 1024);
           mma_bf16_ss(tmem, a, b, idesc, (c > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(mma_done);
-        mma_commit(&kv_empty[slot]);
+        mma_commit(&v_empty[vs]);
       }
       mma_commit(drain);
     }
-  } else {   // ---------------- rows (threads 0..127)
+  } else {   // ---------------- rows (threads 0..255: four per key token; warps w and w + 4
+             // share TMEM lanes 32 (w & 3) .. and split the state's columns)
     const int r = threadIdx.x;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = r & 127, half = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float lam = 0.f;
     // Row threads never leave the loop early: after a timeout every wait returns
     // at once (the CTA's abort flag is set), so all rows still meet at each
@@ -429,21 +445,22 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     for (int c = 0; c < nch; ++c) {
       const int slot = c & 1;
       const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
-      mbar_wait(&kv_full[slot], (c >> 1) & 1, wc);
-      GateSums gs;
-      const float iz = key_features<D>(smem + L::K0 + slot * L::KV, smem + L::E, lg, nullptr, r, nv, gs);
-      const float bC = gs.at(nv - 1);
-      const float bj = gs.at(r >> 1);
-      lam += bC;
-      if (c > 0) {
+      mbar_wait(&k_full[slot], (c >> 1) & 1, wc);
+      if (c > 0) {   // the features go to the keys~ tile: the previous product must be done
         mbar_wait(mma_done, (c - 1) & 1, wc);
         tc_fence_after();
       }
-      write_ktilde<D>(smem + L::E, smem + L::KT, r, (r >> 1) < nv ? __expf(bC - bj) * iz : 0.f);
+      GateSums gs;
+      const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, smem + L::KT, lg, nullptr, r, nv, gs);
+      mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
+      const float bC = gs.at(nv - 1);
+      const float bj = gs.at(r >> 2);
+      lam += bC;
+      write_ktilde<D, 4>(smem + L::KT, smem + L::KT, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
       if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
         const float dec = __expf(bC);
 #pragma unroll 1
-        for (int col = 0; col < D; col += 32) {
+        for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
           float v[32];
           tmem_ld32(lane_base + col, v);
           tmem_wait_ld();
@@ -456,17 +473,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
-      named_bar(1, 128);   // lg is rewritten by the next chunk
+      named_bar(1, 256);   // lg is rewritten by the next chunk
     }
     if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
       tc_fence_after();
-      float* dst = ds_out + (size_t)r * D;
+      float* dst = ds_out + (size_t)row * D;
 #pragma unroll 1
-      for (int col = 0; col < D; col += 32) {
+      for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
         float v[32];
         tmem_ld32(lane_base + col, v);
         tmem_wait_ld();
-        if (r < D) {
+        if (row < D) {
 #pragma unroll
           for (int u = 0; u < 32; u += 4)
             *reinterpret_cast<float4*>(dst + col + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
@@ -851,7 +868,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       float bC, bi, iz;
       {
         GateSums gs;
-        iz = key_features<D, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK, lg, bsh, r, nv, gs);
+        iz = key_features<D, 2, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK, lg, bsh, r, nv, gs);
         bC = gs.at(nv - 1);
         bi = gs.at(i);
         write_ktilde<D>(smem + L::PK, smem + L::KT, r, i < nv ? __expf(bC - bi) * iz : 0.f);   // token r >> 1 = i
@@ -1292,7 +1309,7 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     cudaGetLastError();
     return LIGER_ERR_CUDA;
   }
-  seg_k<<<(unsigned)pl.n_seg_max * pl.nsub * pb.Hkv, NTHREADS, SegSmem<D>::BYTES, s>>>(mk, mv, p);
+  seg_k<<<(unsigned)pl.n_seg_max * pl.nsub * pb.Hkv, kSegThreads, SegSmem<D>::BYTES, s>>>(mk, mv, p);
   hk.count(1);
   if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
