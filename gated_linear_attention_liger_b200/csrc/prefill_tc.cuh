@@ -324,8 +324,8 @@ template <int D>
 struct SegSmem {
   static constexpr uint32_t KV = C * D * 2;        // one chunk of k (or v)
   // key ring (2 slots, released by the row warps once the features are out), value
-  // ring (3 slots, released by the MMA), decay-scaled keys
-  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 5 * KV, SMALL = 6 * KV;
+  // ring (2 slots, released by the MMA), decay-scaled keys (2 slots)
+  static constexpr uint32_t K0 = 0, V0 = 2 * KV, KT = 4 * KV, SMALL = 6 * KV;
   static constexpr uint32_t BYTES = SMALL + 1024 + 1024;   // + alignment slack
 };
 
@@ -339,8 +339,8 @@ __global__ void __launch_bounds__(kSegThreads, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
   uint64_t* k_full = bars;         // [2]
   uint64_t* k_empty = bars + 2;    // [2] (256 arrivals)
-  uint64_t* v_full = bars + 4;     // [3]
-  uint64_t* v_empty = bars + 7;    // [3]
+  uint64_t* v_full = bars + 4;     // [2]
+  uint64_t* v_empty = bars + 7;    // [2]
   uint64_t* feat = bars + 10;
   uint64_t* mma_done = bars + 11;
   uint64_t* drain = bars + 12;
@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 256); }
-    for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(feat, 256); mbar_init(mma_done, 1); mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
@@ -394,14 +394,14 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       int k_issued = 0, v_issued = 0;
       for (int c = 0; c < nch; ++c) {
         const int t = sg.t_begin + c * C;
-        const int ks = c & 1, vs = c % 3;
+        const int ks = c & 1, vs = c & 1;
         if (c >= 2 && !mbar_wait(&k_empty[ks], ((c >> 1) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&k_full[ks], L::KV);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(smem + L::K0 + ks * L::KV + kb * C * 128, &tmk, &k_full[ks], kb * 64, kv, t);
         k_issued = c + 1;
-        if (c >= 3 && !mbar_wait(&v_empty[vs], (c / 3 - 1) & 1, wc)) break;
+        if (c >= 2 && !mbar_wait(&v_empty[vs], ((c >> 1) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&v_full[vs], L::KV);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
@@ -411,20 +411,20 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       // never leave the CTA with copies in flight
       const WaitCtx dw{never, nullptr, p.wait_ns};
       for (int c = (k_issued > 2 ? k_issued - 2 : 0); c < k_issued; ++c) mbar_wait(&k_full[c & 1], (c >> 1) & 1, dw);
-      for (int c = (v_issued > 3 ? v_issued - 3 : 0); c < v_issued; ++c) mbar_wait(&v_full[c % 3], (c / 3) & 1, dw);
+      for (int c = (v_issued > 2 ? v_issued - 2 : 0); c < v_issued; ++c) mbar_wait(&v_full[c & 1], (c >> 1) & 1, dw);
     }
   } else if (warp == 9) {   // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, D, 1, 1);
       const uint32_t lbo_a = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
       for (int c = 0; c < nch; ++c) {
-        const int vs = c % 3;
-        if (!mbar_wait(&v_full[vs], (c / 3) & 1, wc)) break;
+        const int vs = c & 1;
+        if (!mbar_wait(&v_full[vs], (c >> 1) & 1, wc)) break;
         if (!mbar_wait(feat, c & 1, wc)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk) {
-          const uint64_t a = sdesc_sw128(smem_u32(smem + L::KT) + kk * 2048, lbo_a, 1024);
+          const uint64_t a = sdesc_sw128(smem_u32(smem + L::KT + (c & 1) * L::KV) + kk * 2048, lbo_a, 1024);
           const uint64_t b = sdesc_sw128(smem_u32(smem + L::V0 + vs * L::KV) + kk * 2048, C * 128, 1024);
           mma_bf16_ss(tmem, a, b, idesc, (c > 0 || kk > 0) ? 1u : 0u);
         }
@@ -446,17 +446,18 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       const int slot = c & 1;
       const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
       mbar_wait(&k_full[slot], (c >> 1) & 1, wc);
-      if (c > 0) {   // the features go to the keys~ tile: the previous product must be done
-        mbar_wait(mma_done, (c - 1) & 1, wc);
-        tc_fence_after();
-      }
+      char* const kt = smem + L::KT + slot * L::KV;   // read by the product two chunks back: long done
       GateSums gs;
-      const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, smem + L::KT, lg, nullptr, r, nv, gs);
+      const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, kt, lg, nullptr, r, nv, gs);
       mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 2);
       lam += bC;
-      write_ktilde<D, 4>(smem + L::KT, smem + L::KT, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
+      write_ktilde<D, 4>(kt, kt, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
+      if (c > 0) {   // the previous product must be done with S before it is rescaled
+        mbar_wait(mma_done, (c - 1) & 1, wc);
+        tc_fence_after();
+      }
       if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
         const float dec = __expf(bC);
 #pragma unroll 1
