@@ -4,11 +4,13 @@
 Workload (Llama-3-8B attention shape, synthetic seeded N(0,1) data):
   prefill: B=2, T=8192, Hq=32, Hkv=8, d=128, bf16, w=64, alpha=0.5, fp32 final state
   decode:  B=64, Hq=32, Hkv=8, d=128 after a 1024-token prefill; steps captured in a CUDA graph
+  shared-state decode (one state per kv head): B=256, same shape
 
 One step = one prefill call over the whole batch (the headline `value`,
-tokens/s); the decode loop is timed in the same run and reported under
-"decode".  Inputs are larger than L2 (q, k, v 201 MB; decode states 268 MB),
-so no L2 flush is needed between iterations.  Multi-GPU: one process per GPU,
+tokens/s); the decode loops are timed in the same run and reported under
+"decode" and "decode_kvshared".  Inputs are larger than L2 (q, k, v 201 MB;
+decode states 268 MB per head at B=64 and 134 MB per kv head at B=256), so no
+L2 flush is needed between iterations.  Multi-GPU: one process per GPU,
 every rank runs the same per-GPU workload (weak scaling, no collective on the
 data path); times are the max over ranks.
 
@@ -36,6 +38,7 @@ from gated_linear_attention_liger_b200 import inputs  # noqa: E402
 METRIC = "prefill tokens/s & decode tokens/s (8B attn shape), % of roofline"
 PREFILL = inputs.WORKLOADS["llama8b_prefill"]
 DECODE = inputs.WORKLOADS["llama8b_decode"]
+DECODE_KV = inputs.WORKLOADS["llama8b_decode_kvshared"]
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -262,13 +265,15 @@ def run_reference(args, world, rank):
 
 
 def workload_config():
-    p, d = PREFILL, DECODE
+    p, d, dk = PREFILL, DECODE, DECODE_KV
     return {"workload": "llama8b_prefill (+ llama8b_decode)",
             "prefill": {"B": p.B, "T": p.T, "Hq": p.Hq, "Hkv": p.Hkv, "d": p.d, "w": p.w,
                         "alpha": p.alpha},
             "decode": {"B": d.B, "prefix": d.T, "Hq": d.Hq, "Hkv": d.Hkv, "d": d.d, "w": d.w,
                        "alpha": d.alpha},
-            "l2": "inputs larger than L2 (prefill q+k+v 201 MB, decode states 268 MB > 126 MB)"}
+            "decode_kvshared": {"B": dk.B, "prefix": dk.T},
+            "l2": "inputs larger than L2 (prefill q+k+v 201 MB; decode states 268 MB per head at B=64, "
+                  "134 MB per kv head at B=256; L2 126 MB)"}
 
 
 # ----------------------------------------------------------------- GPU arm
@@ -400,7 +405,7 @@ def run_ours(args, world, rank, local):
 
 def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
     from gated_linear_attention_liger_b200 import ops
-    wl = DECODE
+    wl = DECODE_KV if kvshared else DECODE
     n_graph = args.decode_steps
     # state, ring and pos from a seeded 1024-token prefill through the library
     pre = inputs.Workload("decode_prefix", "prefill", wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.dtype,
@@ -476,12 +481,14 @@ def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
     alg = decode_algorithmic(wl, kvshared)
     achieved = alg / (kms * 1e-3) / 1e9
     del graph, tgraph
-    name = "decode tokens/s (8B attn shape, B=64" + (", one state per kv head)" if kvshared else ")")
+    name = f"decode tokens/s (8B attn shape, B={wl.B}" + (", one state per kv head)" if kvshared else ")")
     return {"metric": name, "value": world * wl.B / (ms_step * 1e-3),
             "unit": "tokens/s", "ms_per_step": ms_step, "graph_steps": n_graph, "replays": reps,
             "gpu_launches": per_graph_launches * reps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": measured_traffic("decode_kernel<bf16,128>"),
+                         "frac": achieved / pk["hbm_gbs"],
+                         "traffic": measured_traffic("decode_kvshared_kernel<bf16,128,4>" if kvshared
+                                                     else "decode_kernel<bf16,128>"),
                          "kernel": "decode state stream" + (" (kv-shared)" if kvshared else ""), "kernel_ms": kms,
                          "kernel_timing": "events in graph" if kernel_events else "graph step average",
                          "algorithmic_bytes": alg, "peak_source": pk["source"]}}

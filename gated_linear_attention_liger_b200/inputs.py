@@ -65,6 +65,10 @@ WORKLOADS = {
     # Llama-3-8B decode: 64 sequences after a 1024-token prefill, 1000 steps
     "llama8b_decode": Workload("llama8b_decode", "decode", 64, 32, 8, 1024, 128, torch.bfloat16,
                                seed=1004, steps=1000),
+    # the same with one state per kv head: 256 sequences, so that the fp32 states
+    # (134 MB) exceed the 126 MB L2 as the per-head states (268 MB at 64) do
+    "llama8b_decode_kvshared": Workload("llama8b_decode_kvshared", "decode", 256, 32, 8, 1024, 128,
+                                        torch.bfloat16, seed=1006, steps=1000),
     # 32K packed as 4 sequences, keys biased per kv head by N(0, 0.5^2)
     "long_varlen": Workload("long_varlen", "prefill", 1, 32, 8, 32768, 128, torch.bfloat16,
                             seed=1005, seqlens=(4096, 8192, 8192, 12288), key_bias_std=0.5),
