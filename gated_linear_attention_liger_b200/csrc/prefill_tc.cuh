@@ -548,9 +548,9 @@ constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows 
 // Window warps per TMEM lane quarter (1 or 2: two split the columns).
 constexpr int kWinHalves = 1;
 constexpr int kWinThreads = 128 * kWinHalves;
-// warps [0, 4 kWinHalves) window/epilogue, then 4 keys, 4 queries, 1 TMA, 1 MMA
-constexpr int kKeyWarp0 = 4 * kWinHalves, kQueryWarp0 = kKeyWarp0 + 4;
-constexpr int kTmaWarp = kQueryWarp0 + 4, kMmaWarp = kTmaWarp + 1;
+// warps [0, 4 kWinHalves) window/epilogue, then 8 features, 1 TMA, 1 MMA
+constexpr int kFeatWarp0 = 4 * kWinHalves;
+constexpr int kTmaWarp = kFeatWarp0 + 8, kMmaWarp = kTmaWarp + 1;
 constexpr int kChunkThreads = 32 * (kMmaWarp + 1);
 
 template <int D>
@@ -578,8 +578,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* o_done = bars + 18;      // output accumulator complete
   uint64_t* o_free = bars + 19;      // output read out (window threads)
   uint64_t* drain = bars + 20;
-  uint64_t* keys_ready = bars + 21;  // gates of the chunk known (128 arrivals)
-  uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (128 arrivals)
+  uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (256 arrivals)
   uint64_t* state_done = bars + 23;  // the chunk's state carry done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -606,7 +605,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     for (int i = 0; i < 3; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(q_full, 1); mbar_init(q_empty, 2);
     mbar_init(ss_done, 1); mbar_init(feat, 256); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
-    mbar_init(keys_ready, 128); mbar_init(state_ready, 128); mbar_init(state_done, 1);
+    mbar_init(state_ready, 256); mbar_init(state_done, 1);
     mbar_init(s_read, kWinThreads); mbar_init(p_ready, kWinThreads); mbar_init(o_done, 1);
     mbar_init(o_free, kWinThreads);
     mbar_init(drain, 1);
@@ -781,76 +780,25 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       issue_pv(nch - 1);
       mma_commit(drain);
     }
-  } else if (warp >= kQueryWarp0) {   // ---------------- queries (128 threads)
-    // e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the window
-    // warps fold Z into P and 1/Z into the output).  Needs no gate: with the decay
-    // factored around the chunk's midpoint the row factor e^{b_i - m} is applied in the
-    // epilogue.  Never leaves the loop early (see the key warps).
-    const int r = threadIdx.x - 32 * kQueryWarp0;
-    const int i = r >> 1;
+  } else if (warp >= kFeatWarp0) {   // ---------------- features (256 threads)
+    // One group does the chunk's key features (four threads per key token), then its
+    // query features (two threads per row), then the state copy (two warps per TMEM
+    // lane quarter, half the columns each).  Never leaves the loop early: after a
+    // timeout every wait returns at once (the CTA's abort flag is set), so the group
+    // still meets at each named barrier and warp-collective TMEM access stays uniform.
+    const int t = threadIdx.x - 32 * kFeatWarp0;
+    const int half = t >> 7, lrow = t & 127;   // state-column half, TMEM lane (state row)
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     constexpr float kLog2e = 1.4426950408889634f;
     char* const qb = smem + L::Q0;
     char* const eqb = smem + L::EQ;
-    for (int c = 0; c < nch; ++c) {
-      mbar_wait(q_full, c & 1, wc, wsite(5, 1, c));
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(5, 2, c));   // e_q tile free
-      float mq0 = -INFINITY, mq1 = -INFINITY;
-#pragma unroll
-      for (int c8 = 0; c8 < D / 8; c8 += 2) {
-        mq0 = fmaxf(mq0, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8, ROWS * 128))));
-        mq1 = fmaxf(mq1, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(r, c8 * 8 + 8, ROWS * 128))));
-      }
-      const float mql = fmaxf(mq0, mq1) * kLog2e;
-      float za = 0.f, zb = 0.f;
-#pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
-        const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
-        float x[8];
-        ld_chunk8(qb, off, x);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
-        za += (x[0] + x[1]) + (x[2] + x[3]);
-        zb += (x[4] + x[5]) + (x[6] + x[7]);
-        st_chunk8(eqb, off, x);
-      }
-      zq2[(c & 1) * 128 + r] = za + zb;
-      // The decay mode of the chunk comes with its keys.  The q buffer is released twice
-      // per chunk: by the score MMA's commit, and by these warps once done with the raw q
-      // (factored mode) or by the readout's commit (exact mode: the buffer then holds
-      // e^{b_i} e_q, the readout's A operand).
-      mbar_wait(keys_ready, c & 1, wc, wsite(5, 3, c));
-      if (fast2[c & 1] != 0.f) {
-        named_bar(4, 128);
-        if (r == 0) mbar_arrive(q_empty);
-      } else {
-        mbar_wait(ss_done, c & 1, wc, wsite(5, 4, c));
-        const float ebi = __expf(bsh2[(c & 1) * 64 + i]);
-#pragma unroll 4
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint32_t off = kmajor_off(r, c8 * 8, ROWS * 128);
-          float x[8];
-          ld_chunk8(eqb, off, x);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) x[q] *= ebi;
-          st_chunk8(qb, off, x);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(feat);
-    }
-  } else if (warp >= kKeyWarp0) {   // ---------------- keys (128 threads)
-    // Row threads never leave the loop early: after a timeout every wait returns
-    // at once (the CTA's abort flag is set), so the group still meets at each
-    // named barrier and warp-collective TMEM access stays uniform.
-    const int r = threadIdx.x - 32 * kKeyWarp0;
-    const int i = r >> 1;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     char* const sbb = smem + L::SB;
 
-    // state entering the segment, first half of the columns (the window warps do the rest)
-    entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColS, 0);
+    // state entering the segment: this warp's quarter of the first half of the columns
+    // (the window warps load the second half)
+    entering_state<D, D / 4>(p, seg, kv, lrow % D, lane_base + kColS, half * (D / 4));
     tc_fence_before();
-    named_bar(2, 128 + kWinThreads);
+    named_bar(2, 256 + kWinThreads);
     tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
@@ -864,50 +812,93 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       tc_fence_after();
 
-      // e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running sums,
+      // keys: e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running sums,
       // decay-scaled keys
-      float bC, bi, iz;
-      {
-        GateSums gs;
-        iz = key_features<D, 2, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK, lg, bsh, r, nv, gs);
-        bC = gs.at(nv - 1);
-        bi = gs.at(i);
-        write_ktilde<D>(smem + L::PK, smem + L::KT, r, i < nv ? __expf(bC - bi) * iz : 0.f);   // token r >> 1 = i
-      }
+      const int j = t >> 2;
+      GateSums gs;
+      const float iz = key_features<D, 4, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK,
+                                                        lg, bsh, t, nv, gs);
+      const float bC = gs.at(nv - 1);
+      const float bj = gs.at(j);
+      write_ktilde<D, 4>(smem + L::PK, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
       // Factored mode (the chunk's total log gate >= -80): with m = b_C / 2,
       // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-40}.
       const bool fast = bC >= -80.f;
-      if ((r & 1) == 0) {
-        eneg2[(c & 1) * 64 + i] = fast ? __expf(0.5f * bC - bi) * iz : 0.f;
-        izk2[(c & 1) * 64 + i] = iz;
+      if ((t & 3) == 0) {
+        eneg2[(c & 1) * 64 + j] = fast ? __expf(0.5f * bC - bj) * iz : 0.f;
+        izk2[(c & 1) * 64 + j] = iz;
       }
-      if (r == 0) fast2[c & 1] = fast ? 1.f : 0.f;
+      if (t == 0) fast2[c & 1] = fast ? 1.f : 0.f;
+
+      // queries: e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the
+      // window warps fold Z into P and 1/Z into the output); two threads per row
+      const int row = t >> 1, qh = t & 1;
+      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));   // e_q tile and state copy free
+      float mq = -INFINITY;
+#pragma unroll
+      for (int c8 = 0; c8 < D / 16; ++c8)
+        mq = fmaxf(mq, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(row, qh * (D / 2) + c8 * 8,
+                                                                                     ROWS * 128))));
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
+      const float mql = mq * kLog2e;
+      float za = 0.f, zb = 0.f;
+#pragma unroll 4
+      for (int c8 = 0; c8 < D / 16; ++c8) {
+        const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
+        float x[8];
+        ld_chunk8(qb, off, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
+        za += (x[0] + x[1]) + (x[2] + x[3]);
+        zb += (x[4] + x[5]) + (x[6] + x[7]);
+        st_chunk8(eqb, off, x);
+      }
+      float zq = za + zb;
+      zq += __shfl_xor_sync(0xffffffffu, zq, 1);
+      if (qh == 0) zq2[(c & 1) * 128 + row] = zq;
+      // The q buffer is released twice per chunk: by the score MMA's commit, and by this
+      // group once done with the raw q (factored mode) or by the readout's commit (exact
+      // mode: the buffer then holds e^{b_i} e_q, the readout's A operand).
+      if (fast) {
+        named_bar(1, 256);
+        if (t == 0) mbar_arrive(q_empty);
+      } else {
+        mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
+        const float ebi = __expf(gs.at(row >> 1));
+#pragma unroll 4
+        for (int c8 = 0; c8 < D / 16; ++c8) {
+          const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
+          float x[8];
+          ld_chunk8(eqb, off, x);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) x[q] *= ebi;
+          st_chunk8(qb, off, x);
+        }
+      }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(keys_ready);   // gates known: decay mode, running sums
       mbar_arrive(feat);
 
       // State for this chunk: the bf16 copy of alpha e^{m} S (MN-major B of the readout;
-      // e^{m} only in factored mode), then S <- e^{b_C} S in TMEM before the chunk's
-      // carry accumulates onto it.  The previous carry is done (state_done, above); the
-      // previous readout must be done with the copy.
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 8, c));
+      // e^{m} only in factored mode), then S <- e^{b_C} S in TMEM before the chunk's carry
+      // accumulates onto it (the previous carry and readout are done, above).
       tc_fence_after();
       {
         const float dec = __expf(bC);
         const float sbs = fast ? p.alpha * __expf(0.5f * bC) : p.alpha;
 #pragma unroll 1
-        for (int col = 0; col < D; col += 32) {
+        for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
           float v[32];
           tmem_ld32(lane_base + kColS + col, v);
           tmem_wait_ld();
-          if (r < D) {
+          if (lrow < D) {
 #pragma unroll
             for (int u = 0; u < 32; u += 8) {
               float x[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) x[q] = sbs * v[u + q];
-              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(r, ((col + u) & 63) >> 3), x);
+              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(lrow, ((col + u) & 63) >> 3), x);
             }
           }
 #pragma unroll
@@ -919,7 +910,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(state_ready);
-      named_bar(1, 128);   // lg is rewritten by the next chunk's keys
+      named_bar(1, 256);   // lg is rewritten by the next chunk's keys
     }
     // final state of the sequence: the carry after the last chunk of its last segment
     const SeqInfo si = p.seqs[sg.seq];
@@ -927,14 +918,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     if (p.final_state && last && mbar_wait(mma2_done, (nch - 1) & 1, wc, wsite(3, 5, nch)) && !*abort_flag) {
       tc_fence_after();
 #pragma unroll 1
-      for (int col = 0; col < D; col += 32) {
+      for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
         float v[32];
         tmem_ld32(lane_base + kColS + col, v);
         tmem_wait_ld();
-        if (r < D) {
+        if (lrow < D) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            float* dst = p.final_state + (((size_t)sg.seq * p.Hq + h0 + hh) * D + r) * D + col;
+            float* dst = p.final_state + (((size_t)sg.seq * p.Hq + h0 + hh) * D + lrow) * D + col;
 #pragma unroll
             for (int u = 0; u < 32; u += 4)
               *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
@@ -955,11 +946,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     // state entering the segment, this thread's share of the second half of the columns
-    // (the key warps load the first half; TMEM: the state follows O)
+    // (the feature warps load the first half; TMEM: the state follows O)
     constexpr int kEnt = D / (2 * kWinHalves);
     entering_state<D, kEnt>(p, seg, kv, r % D, lane_base + kColO + D, D / 2 + sh * kEnt);
     tc_fence_before();
-    named_bar(2, 128 + kWinThreads);
+    named_bar(2, 256 + kWinThreads);
     tc_fence_after();
     // this thread's window column groups
     const int g_lo = kWinHalves == 1 ? 0 : (sh ? 3 : 0), g_hi = kWinHalves == 1 ? 5 : (sh ? 5 : 3);
