@@ -3,11 +3,12 @@
 // One CTA per (sequence, q head).  Per step the dominant traffic is reading
 // and writing that head's d x d fp32 state.  Each thread owns a 4-column slab
 // of RPT key rows and issues all of its 128-bit streaming loads first; in the
-// same breath the CTA copies the window ring's keys and values (the valid
-// slots only) into shared memory with cp.async, so every later step of the
-// window branch reads shared memory and no warp waits on a chain of dependent
-// global loads.  Then S <- g S + phi(k)^T v is applied to the registers,
-// phi(q) S is accumulated, and the rows stream back.  The new key/value is
+// same breath the CTA starts copying the window ring's keys and values (the
+// valid slots only) into shared memory with cp.async.  S <- g S + phi(k)^T v is
+// applied to the registers and phi(q) S accumulated as soon as the rows land,
+// and the rows stream back before the window branch runs on the shared-memory
+// ring: the CTA's state traffic is done early, and its window work overlaps the
+// other CTAs' streams.  The new key/value is
 // taken from the step's inputs; the group's first q head writes it to slot
 // pos mod w, a slot no other CTA of the step reads.  The position counter is
 // advanced by a second one-thread-per-sequence kernel so that no CTA can see
@@ -64,9 +65,6 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
                    static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
                "l"(gsrc)
                : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 
@@ -143,6 +141,73 @@ __device__ __forceinline__ void window_scores(const float* qv, const float* ks, 
   }
 }
 
+// Window softmax and value sums for NH heads.  sc[h][0..w) holds the scores (-inf
+// for positions before the sequence start).  Every warp reduces the maxima and sums
+// itself (no single-warp phase, no extra barrier).  Thread layout: 16-byte column
+// piece cp = tid % NPC, slot group sg = tid / NPC, slots sg, sg + NSG, ...; each thread
+// accumulates p_h(slot) v(slot) over its pieces, the slot groups of a warp are added
+// with shuffles, and each warp writes wsum[warp][h][...]; the caller adds the NW
+// partial sums.
+template <typename Tin, int D, int NT, int NH>
+struct WindowValues {
+  static constexpr int EPP = 16 / (int)sizeof(Tin);   // elements per 16-byte piece
+  static constexpr int NPC = D / EPP;                 // pieces per row
+  static_assert(NPC <= 32 && 32 % NPC == 0, "a warp holds whole slot groups");
+  static constexpr int NSG = NT / NPC;                // slot groups
+  static constexpr int NW = NT / 32;                  // warps (partial sums)
+  __device__ __forceinline__ static void run(const float (*sc)[64], const Tin* rv_s, const float* vs,
+                                             float (*wsum)[NH][D], int p, int w, int tid, int lane) {
+    float mh[NH], izh[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      const float x0 = lane < w ? sc[h][lane] : -INFINITY;
+      const float x1 = lane + 32 < w ? sc[h][lane + 32] : -INFINITY;
+      const float m = warp_max(fmaxf(x0, x1));
+      const float z = warp_sum((lane < w ? expf(x0 - m) : 0.f) + (lane + 32 < w ? expf(x1 - m) : 0.f));
+      mh[h] = m;
+      izh[h] = 1.0f / z;
+    }
+    constexpr int RS = ring_row_elems<Tin, D>();
+    const int cp = tid % NPC, sg = tid / NPC;
+    float acc[NH][EPP];
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+#pragma unroll
+      for (int e = 0; e < EPP; ++e) acc[h][e] = 0.f;
+    for (int jj = sg; jj < w; jj += NSG) {
+      const int j = p - (w - 1) + jj;
+      if (j < 0) continue;
+      float x[EPP];
+      if (j == p) {
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) x[e] = vs[cp * EPP + e];
+      } else {
+        ld16_vals<Tin>(rv_s + jj * RS + cp * EPP, x);
+      }
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        const float ph = expf(sc[h][jj] - mh[h]) * izh[h];
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) acc[h][e] = fmaf(ph, x[e], acc[h][e]);
+      }
+    }
+#pragma unroll
+    for (int o = NPC; o < 32; o <<= 1)
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
+    if (lane < NPC) {
+#pragma unroll
+      for (int h = 0; h < NH; ++h)
+#pragma unroll
+        for (int e = 0; e < EPP; e += 4)
+          *reinterpret_cast<float4*>(&wsum[tid >> 5][h][cp * EPP + e]) =
+              make_float4(acc[h][e], acc[h][e + 1], acc[h][e + 2], acc[h][e + 3]);
+    }
+  }
+};
+
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a) {
   constexpr int NT = kDecodeThreads;
@@ -150,14 +215,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   constexpr int RGN = NT / CQ;       // row groups
   constexpr int RPT = D / RGN;       // rows per thread
   constexpr int EPL = D / 32;
-  constexpr int VG = NT / D;         // window-sum key groups
+  using WV = WindowValues<Tin, D, NT, 1>;
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
   Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
   __shared__ __align__(16) float qs[D], ks[D], vs[D], fq[D], fk[D];
-  __shared__ float sc[64];
+  __shared__ float sc[1][64];
   __shared__ __align__(16) float part[RGN][D];
-  __shared__ float wpart[VG][D];
+  __shared__ __align__(16) float wsum[WV::NW][1][D];
   __shared__ float gsh;
 
   const int Hq = a.Hq, Hkv = a.Hkv, w = a.w, G = Hq / Hkv;
@@ -173,12 +238,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
 #pragma unroll
   for (int r = 0; r < RPT; ++r) st[r] = ld_stream(S + (size_t)(rg * RPT + r) * D + 4 * cq);
 
-  // 2. the window's ring slots (positions p-w+1 .. p-1) into shared memory
+  // 2. the window's ring slots (positions p-w+1 .. p-1) start towards shared memory;
+  //    they are waited for only after the state has streamed back
   const int p = max(a.pos[b], 0);   // a negative position is read as 0
   Tin* ring = static_cast<Tin*>(a.ring);
   const Tin* rk = ring + (((size_t)b * Hkv + kv) * 2 + 0) * w * D;
   const Tin* rv = ring + (((size_t)b * Hkv + kv) * 2 + 1) * w * D;
   ring_to_smem<Tin, D, NT>(rk, rv, rk_s, rv_s, p, w, tid);
+  asm volatile("cp.async.commit_group;" ::: "memory");
   const Tin* qrow = static_cast<const Tin*>(a.q) + ((size_t)b * Hq + h) * D;
   const Tin* krow = static_cast<const Tin*>(a.k) + ((size_t)b * Hkv + kv) * D;
   const Tin* vrow = static_cast<const Tin*>(a.v) + ((size_t)b * Hkv + kv) * D;
@@ -187,12 +254,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
     ks[tid] = io<Tin>::ld(krow + tid);
     vs[tid] = io<Tin>::ld(vrow + tid);
   }
-  cp_async_wait_all();
   __syncthreads();
 
-  // 3. window scores from shared memory (slot jj covers position p - (w-1) + jj)
-  window_scores<Tin, D>(qs, ks, rk_s, sc, p, w, tid);
-  // 4. phi(k) with the gate, and phi(q)
+  // 3. phi(k) with the gate, and phi(q)
   if (warp == 0) {
     float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
 #pragma unroll
@@ -217,57 +281,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
     for (int j = 0; j < EPL; ++j) fq[lane + 32 * j] = x[j] / z;
   }
   __syncthreads();
-  // 5. window softmax
-  if (warp == 0) {
-    const float x0 = lane < w ? sc[lane] : -INFINITY;
-    const float x1 = lane + 32 < w ? sc[lane + 32] : -INFINITY;
-    const float m = warp_max(fmaxf(x0, x1));
-    const float e0 = lane < w ? expf(x0 - m) : 0.f;
-    const float e1 = lane + 32 < w ? expf(x1 - m) : 0.f;
-    const float z = warp_sum(e0 + e1);
-    if (lane < w) sc[lane] = e0 / z;
-    if (lane + 32 < w) sc[lane + 32] = e1 / z;
-  }
-  __syncthreads();
-  // 6. window value sum, split over VG key groups
+
+  // 4. state update and readout on the streamed rows: the state goes back to memory
+  //    before the window branch is computed
   {
-    const int e = tid % D, grp = tid / D;
-    float acc = 0.f;
-    for (int jj = grp; jj < w; jj += VG) {
-      const long j = (long)p - (w - 1) + jj;
-      if (j < 0) continue;
-      const float vx = (j == p) ? vs[e] : io<Tin>::ld(rv_s + jj * ring_row_elems<Tin, D>() + e);
-      acc = fmaf(sc[jj], vx, acc);
-    }
-    wpart[grp][e] = acc;
-  }
-  // 7. state update and readout on the streamed rows
-  const float g = gsh;
-  const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float g = gsh;
+    const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    const int row = rg * RPT + r;
-    const float kr = fk[row], qr = fq[row];
-    float4 x = st[r];
-    x.x = fmaf(g, x.x, kr * vv.x);
-    x.y = fmaf(g, x.y, kr * vv.y);
-    x.z = fmaf(g, x.z, kr * vv.z);
-    x.w = fmaf(g, x.w, kr * vv.w);
-    acc.x = fmaf(qr, x.x, acc.x);
-    acc.y = fmaf(qr, x.y, acc.y);
-    acc.z = fmaf(qr, x.z, acc.z);
-    acc.w = fmaf(qr, x.w, acc.w);
-    st_stream(S + (size_t)row * D + 4 * cq, x);
+    for (int r = 0; r < RPT; ++r) {
+      const int row = rg * RPT + r;
+      const float kr = fk[row], qr = fq[row];
+      float4 x = st[r];
+      x.x = fmaf(g, x.x, kr * vv.x);
+      x.y = fmaf(g, x.y, kr * vv.y);
+      x.z = fmaf(g, x.z, kr * vv.z);
+      x.w = fmaf(g, x.w, kr * vv.w);
+      acc.x = fmaf(qr, x.x, acc.x);
+      acc.y = fmaf(qr, x.y, acc.y);
+      acc.z = fmaf(qr, x.z, acc.z);
+      acc.w = fmaf(qr, x.w, acc.w);
+      st_stream(S + (size_t)row * D + 4 * cq, x);
+    }
+    *reinterpret_cast<float4*>(&part[rg][4 * cq]) = acc;
   }
-  *reinterpret_cast<float4*>(&part[rg][4 * cq]) = acc;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  // 5. window scores from shared memory (slot jj covers position p - (w-1) + jj)
+  window_scores<Tin, D>(qs, ks, rk_s, sc[0], p, w, tid);
+  __syncthreads();
+  // 6. window softmax and value sums
+  WV::run(sc, rv_s, vs, wsum, p, w, tid, lane);
   __syncthreads();
   if (tid < D) {
     float grm = 0.f, swa = 0.f;
 #pragma unroll
     for (int r = 0; r < RGN; ++r) grm += part[r][tid];
 #pragma unroll
-    for (int r = 0; r < VG; ++r) swa += wpart[r][tid];
+    for (int r = 0; r < WV::NW; ++r) swa += wsum[r][0][tid];
     Tin* orow = static_cast<Tin*>(a.out) + ((size_t)b * Hq + h) * D;
     io<Tin>::st(orow + tid, a.alpha * grm + (1.0f - a.alpha) * swa);
     if (h % G == 0) {
@@ -303,14 +355,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
   constexpr int RGN = NT / CQ;
   constexpr int RPT = D / RGN;
   constexpr int EPL = D / 32;
-  constexpr int VG = NT / D;
+  using WV = WindowValues<Tin, D, NT, G>;
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
   Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
   __shared__ __align__(16) float qs[G][D], fq[G][D], ks[D], vs[D], fk[D];
   __shared__ float sc[G][64];
   __shared__ __align__(16) float part[RGN][G][D];
-  __shared__ float wpart[VG][G][D];
+  __shared__ __align__(16) float wsum[WV::NW][G][D];
   __shared__ float gsh;
 
   const int Hkv = a.Hkv, w = a.w, Hq = a.Hq;
@@ -325,11 +377,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
 #pragma unroll
   for (int r = 0; r < RPT; ++r) st[r] = ld_stream(S + (size_t)(rg * RPT + r) * D + 4 * cq);
 
+  // the ring rows start towards shared memory; waited for after the state has streamed back
   const int p = max(a.pos[b], 0);
   Tin* ring = static_cast<Tin*>(a.ring);
   const Tin* rk = ring + (((size_t)b * Hkv + kv) * 2 + 0) * w * D;
   const Tin* rv = ring + (((size_t)b * Hkv + kv) * 2 + 1) * w * D;
   ring_to_smem<Tin, D, NT>(rk, rv, rk_s, rv_s, p, w, tid);
+  asm volatile("cp.async.commit_group;" ::: "memory");
   const Tin* krow = static_cast<const Tin*>(a.k) + ((size_t)b * Hkv + kv) * D;
   const Tin* vrow = static_cast<const Tin*>(a.v) + ((size_t)b * Hkv + kv) * D;
   for (int idx = tid; idx < G * D; idx += NT) {
@@ -340,12 +394,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
     ks[tid] = io<Tin>::ld(krow + tid);
     vs[tid] = io<Tin>::ld(vrow + tid);
   }
-  cp_async_wait_all();
   __syncthreads();
 
-  // window scores, head by head
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) window_scores<Tin, D>(qs[hh], ks, rk_s, sc[hh], p, w, tid);
   // phi(k) with the gate (warp 0), phi(q_h) (warps 1..G)
   if (warp == 0) {
     float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
@@ -372,60 +422,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
     for (int j = 0; j < EPL; ++j) fq[hh][lane + 32 * j] = x[j] / z;
   }
   __syncthreads();
-  if (warp < G) {   // window softmax of head `warp`
-    const int hh = warp;
-    const float x0 = lane < w ? sc[hh][lane] : -INFINITY;
-    const float x1 = lane + 32 < w ? sc[hh][lane + 32] : -INFINITY;
-    const float m = warp_max(fmaxf(x0, x1));
-    const float e0 = lane < w ? expf(x0 - m) : 0.f;
-    const float e1 = lane + 32 < w ? expf(x1 - m) : 0.f;
-    const float z = warp_sum(e0 + e1);
-    if (lane < w) sc[hh][lane] = e0 / z;
-    if (lane + 32 < w) sc[hh][lane + 32] = e1 / z;
+
+  // state update once, readout for every head of the group; the state goes back to
+  // memory before the window branch is computed
+  {
+    const float g = gsh;
+    const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
+    float4 acc[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const int row = rg * RPT + r;
+      const float kr = fk[row];
+      float4 x = st[r];
+      x.x = fmaf(g, x.x, kr * vv.x);
+      x.y = fmaf(g, x.y, kr * vv.y);
+      x.z = fmaf(g, x.z, kr * vv.z);
+      x.w = fmaf(g, x.w, kr * vv.w);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float qr = fq[hh][row];
+        acc[hh].x = fmaf(qr, x.x, acc[hh].x);
+        acc[hh].y = fmaf(qr, x.y, acc[hh].y);
+        acc[hh].z = fmaf(qr, x.z, acc[hh].z);
+        acc[hh].w = fmaf(qr, x.w, acc[hh].w);
+      }
+      st_stream(S + (size_t)row * D + 4 * cq, x);
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = acc[hh];
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  {   // window value sums
-    const int e = tid % D, grp = tid / D;
-    float acc[G];
+
+  // window scores, head by head
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) acc[hh] = 0.f;
-    for (int jj = grp; jj < w; jj += VG) {
-      const long j = (long)p - (w - 1) + jj;
-      if (j < 0) continue;
-      const float vx = (j == p) ? vs[e] : io<Tin>::ld(rv_s + jj * ring_row_elems<Tin, D>() + e);
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) acc[hh] = fmaf(sc[hh][jj], vx, acc[hh]);
-    }
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) wpart[grp][hh][e] = acc[hh];
-  }
-  // state update once, readout for every head of the group
-  const float g = gsh;
-  const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
-  float4 acc[G];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    const int row = rg * RPT + r;
-    const float kr = fk[row];
-    float4 x = st[r];
-    x.x = fmaf(g, x.x, kr * vv.x);
-    x.y = fmaf(g, x.y, kr * vv.y);
-    x.z = fmaf(g, x.z, kr * vv.z);
-    x.w = fmaf(g, x.w, kr * vv.w);
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      const float qr = fq[hh][row];
-      acc[hh].x = fmaf(qr, x.x, acc[hh].x);
-      acc[hh].y = fmaf(qr, x.y, acc[hh].y);
-      acc[hh].z = fmaf(qr, x.z, acc[hh].z);
-      acc[hh].w = fmaf(qr, x.w, acc[hh].w);
-    }
-    st_stream(S + (size_t)row * D + 4 * cq, x);
-  }
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = acc[hh];
+  for (int hh = 0; hh < G; ++hh) window_scores<Tin, D>(qs[hh], ks, rk_s, sc[hh], p, w, tid);
+  __syncthreads();
+  WV::run(sc, rv_s, vs, wsum, p, w, tid, lane);   // window softmax and value sums
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += NT) {
     const int hh = idx / D, e = idx % D;
@@ -433,7 +468,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
 #pragma unroll
     for (int r = 0; r < RGN; ++r) grm += part[r][hh][e];
 #pragma unroll
-    for (int r = 0; r < VG; ++r) swa += wpart[r][hh][e];
+    for (int r = 0; r < WV::NW; ++r) swa += wsum[r][hh][e];
     Tin* orow = static_cast<Tin*>(a.out) + ((size_t)b * Hq + kv * G + hh) * D;
     io<Tin>::st(orow + e, a.alpha * grm + (1.0f - a.alpha) * swa);
   }
