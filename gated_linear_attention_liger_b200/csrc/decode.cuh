@@ -107,12 +107,14 @@ template <> __device__ __forceinline__ void ld16_vals<float>(const float* p, flo
   x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
 }
 
-// Window scores q . k_j / sqrt(d) for the w slots, four threads per slot; thread
-// quarter qq takes the 16-byte pieces qq, qq+4, ... of the row (conflict-free on
-// the padded rows), reduced with two shuffles.  Needs blockDim >= 4 * w.
-template <typename Tin, int D>
-__device__ __forceinline__ void window_scores(const float* qv, const float* ks, const Tin* rk_s, float* sc, int p,
-                                              int w, int tid) {
+// Window scores q_h . k_j / sqrt(d) of NH heads for the w slots, four threads per
+// slot; thread quarter qq takes the 16-byte pieces qq, qq+4, ... of the row
+// (conflict-free on the padded rows), loads each key piece once for all heads and
+// reduces with two shuffles.  qv[h] is head h's query row (fp32, 16-byte aligned).
+// Needs blockDim >= 4 * w.
+template <typename Tin, int D, int NH>
+__device__ __forceinline__ void window_scores(const float (*qv)[D], const float* ks, const Tin* rk_s,
+                                              float (*sc)[64], int p, int w, int tid) {
   constexpr int EPP = 16 / (int)sizeof(Tin);      // elements per 16-byte piece
   constexpr int NP = D / EPP;                     // pieces per row
   constexpr int RS = ring_row_elems<Tin, D>();
@@ -120,24 +122,42 @@ __device__ __forceinline__ void window_scores(const float* qv, const float* ks, 
   if (jj < 64) {   // all four lanes of a slot take part in the shuffles
     const int j = p - (w - 1) + jj;
     const bool live = jj < w && j >= 0;
-    float acc = 0.f;
+    float acc[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) acc[h] = 0.f;
     if (live) {
 #pragma unroll
       for (int pc = qq; pc < NP; pc += 4) {
         float x[EPP];
         if (j == p) {
 #pragma unroll
-          for (int e = 0; e < EPP; ++e) x[e] = ks[pc * EPP + e];
+          for (int e = 0; e < EPP; e += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(ks + pc * EPP + e);
+            x[e] = t.x; x[e + 1] = t.y; x[e + 2] = t.z; x[e + 3] = t.w;
+          }
         } else {
           ld16_vals<Tin>(rk_s + jj * RS + pc * EPP, x);
         }
 #pragma unroll
-        for (int e = 0; e < EPP; ++e) acc = fmaf(qv[pc * EPP + e], x[e], acc);
+        for (int h = 0; h < NH; ++h) {
+#pragma unroll
+          for (int e = 0; e < EPP; e += 4) {
+            const float4 qf = *reinterpret_cast<const float4*>(&qv[h][pc * EPP + e]);
+            acc[h] = fmaf(qf.x, x[e], acc[h]);
+            acc[h] = fmaf(qf.y, x[e + 1], acc[h]);
+            acc[h] = fmaf(qf.z, x[e + 2], acc[h]);
+            acc[h] = fmaf(qf.w, x[e + 3], acc[h]);
+          }
+        }
       }
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (qq == 0 && jj < w) sc[jj] = live ? acc * (1.0f / sqrtf((float)D)) : -INFINITY;
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      float t = acc[h];
+      t += __shfl_xor_sync(0xffffffffu, t, 1);
+      t += __shfl_xor_sync(0xffffffffu, t, 2);
+      if (qq == 0 && jj < w) sc[h][jj] = live ? t * (1.0f / sqrtf((float)D)) : -INFINITY;
+    }
   }
 }
 
@@ -309,7 +329,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   __syncthreads();
 
   // 5. window scores from shared memory (slot jj covers position p - (w-1) + jj)
-  window_scores<Tin, D>(qs, ks, rk_s, sc[0], p, w, tid);
+  window_scores<Tin, D, 1>(reinterpret_cast<const float(*)[D]>(qs), ks, rk_s, sc, p, w, tid);
   __syncthreads();
   // 6. window softmax and value sums
   WV::run(sc, rv_s, vs, wsum, p, w, tid, lane);
@@ -457,8 +477,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
   __syncthreads();
 
   // window scores, head by head
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) window_scores<Tin, D>(qs[hh], ks, rk_s, sc[hh], p, w, tid);
+  window_scores<Tin, D, G>(qs, ks, rk_s, sc, p, w, tid);
   __syncthreads();
   WV::run(sc, rv_s, vs, wsum, p, w, tid, lane);   // window softmax and value sums
   __syncthreads();
