@@ -108,6 +108,7 @@ struct DevParams {
 // ============================================================== plan kernel
 
 __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* n_segs) {
+  griddep_wait_and_release();   // the previous call's kernels are done with the workspace
   if (threadIdx.x != 0) return;
   p.err[0] = 0u;
   p.err[1] = 0u;
@@ -137,6 +138,7 @@ __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* 
 // Grid (n_seqs, Hq), 256 threads.
 template <int D>
 __global__ void zero_empty_kernel(DevParams p) {
+  griddep_wait_and_release();
   if (p.seqs[blockIdx.x].n_seg != 0) return;
   float4* dst = reinterpret_cast<float4*>(p.final_state + ((size_t)blockIdx.x * p.Hq + blockIdx.y) * D * D);
   for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -155,6 +157,7 @@ __device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
 // issued before its products are accumulated.
 template <int D>
 __global__ void scan_kernel(DevParams p) {
+  griddep_wait_and_release();
   const int seq = blockIdx.x / p.Hkv, kv = blockIdx.x % p.Hkv;
   const size_t e = ((size_t)blockIdx.y * blockDim.x + threadIdx.x) * 4;
   if (e >= (size_t)D * D) return;
@@ -333,6 +336,7 @@ template <int D>
 __global__ void __launch_bounds__(kSegThreads, 2)
     seg_state_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      DevParams p) {
+  griddep_wait_and_release();
   using L = SegSmem<D>;
   extern __shared__ __align__(1024) char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -557,6 +561,7 @@ template <int D>
 __global__ void __launch_bounds__(kChunkThreads, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, DevParams p) {
+  griddep_wait_and_release();
   using L = ChunkSmem<D>;
   constexpr uint32_t kColS = kColO + D;
   constexpr uint32_t TCOLS = 512;
@@ -1249,6 +1254,25 @@ inline uint64_t wait_limit_ns() {
   return kDefaultWaitNs;
 }
 
+// Launch with programmatic stream serialisation: the grid may be scheduled while
+// the previous grid in the stream drains; every prefill kernel starts with
+// griddep_wait_and_release, so nothing is read before its producer has finished.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 template <int D>
 liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk) {
   const bool varlen = pb.cu != nullptr;
@@ -1289,10 +1313,10 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     return LIGER_ERR_CUDA;
   }
   cudaError_t e;
-  plan_kernel<<<1, 32, 0, s>>>(p, reinterpret_cast<SeqInfo*>(w + pl.off_seqs),
-                               reinterpret_cast<SegInfo*>(w + pl.off_segs), reinterpret_cast<int32_t*>(w + 8));
+  e = launch_chained(plan_kernel, dim3(1), dim3(32), 0, s, p, reinterpret_cast<SeqInfo*>(w + pl.off_seqs),
+                     reinterpret_cast<SegInfo*>(w + pl.off_segs), reinterpret_cast<int32_t*>(w + 8));
   hk.count(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
   auto seg_k = seg_state_kernel<D>;
   if (cudaFuncSetAttribute(seg_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SegSmem<D>::BYTES) !=
@@ -1301,18 +1325,20 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     cudaGetLastError();
     return LIGER_ERR_CUDA;
   }
-  seg_k<<<(unsigned)pl.n_seg_max * pl.nsub * pb.Hkv, kSegThreads, SegSmem<D>::BYTES, s>>>(mk, mv, p);
+  e = launch_chained(seg_k, dim3((unsigned)pl.n_seg_max * pl.nsub * pb.Hkv), dim3(kSegThreads), SegSmem<D>::BYTES,
+                     s, mk, mv, p);
   hk.count(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
-  scan_kernel<D><<<dim3((unsigned)(pb.n_seqs * pb.Hkv), (unsigned)(D * D / 1024)), 256, 0, s>>>(p);
+  e = launch_chained(scan_kernel<D>, dim3((unsigned)(pb.n_seqs * pb.Hkv), (unsigned)(D * D / 1024)), dim3(256), 0,
+                     s, p);
   hk.count(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
 
   if (varlen && pb.final_state) {
-    zero_empty_kernel<D><<<dim3((unsigned)pb.n_seqs, (unsigned)pb.Hq), 256, 0, s>>>(p);
+    e = launch_chained(zero_empty_kernel<D>, dim3((unsigned)pb.n_seqs, (unsigned)pb.Hq), dim3(256), 0, s, p);
     hk.count(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+    if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
   }
 
   auto chunk_k = chunk_kernel<D>;
@@ -1323,10 +1349,11 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
     return LIGER_ERR_CUDA;
   }
   hk.before_main(s);
-  chunk_k<<<(unsigned)pl.n_seg_max * (pb.Hq / 2), kChunkThreads, ChunkSmem<D>::BYTES, s>>>(mq, mk, mv, p);
+  e = launch_chained(chunk_k, dim3((unsigned)pl.n_seg_max * (pb.Hq / 2)), dim3(kChunkThreads), ChunkSmem<D>::BYTES,
+                     s, mq, mk, mv, p);
   hk.after_main(s);
   hk.count(1);
-  if ((e = cudaGetLastError()) != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
   return LIGER_OK;
 }
 

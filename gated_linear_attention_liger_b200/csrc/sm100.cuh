@@ -285,6 +285,12 @@ __device__ __forceinline__ float bf16x8_max(uint4 u) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Programmatic dependent launch: wait until the previous grid in the stream has
+// completed and its memory is visible, then let the next grid start launching.
+__device__ __forceinline__ void griddep_wait_and_release() {
+  asm volatile("griddepcontrol.wait;\n\tgriddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over a subset of warps (id 1..15).
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
