@@ -153,8 +153,7 @@ __device__ __forceinline__ void st_global_v8(void* ptr, const uint32_t* v) {
 
 // Per (sequence, kv head): folds the sub-segment contributions in order and
 // stores the state entering each segment in its first sub-segment slot.  Grid
-// (n_seqs * Hkv, D*D / 1024), 256 threads x 4 floats; every load of a segment is
-// issued before its products are accumulated.
+// (n_seqs * Hkv, D*D / 1024), 256 threads x 4 floats.
 template <int D>
 __global__ void scan_kernel(DevParams p) {
   griddep_wait_and_release();
@@ -163,33 +162,33 @@ __global__ void scan_kernel(DevParams p) {
   if (e >= (size_t)D * D) return;
   const SeqInfo si = p.seqs[seq];
   const int nsub = p.nsub;
+  // The sequence's sub-segment contributions in order, sixteen loads in flight at a
+  // time; the state entering a segment is stored over its first sub-segment's slot
+  // (after that slot has been read).
+  constexpr int kBatch = 16;
+  const int n_units = si.n_seg * nsub;
+  const size_t u0 = (size_t)si.first_seg * nsub;
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
-  // the next segment's contributions are in flight while the current one is folded
-  float4 d[kMaxSub], dn[kMaxSub];
-  float g[kMaxSub], gn[kMaxSub];
-  auto fetch = [&](int s, float4 (&dd)[kMaxSub], float (&gg)[kMaxSub]) {
+  for (int base = 0; base < n_units; base += kBatch) {
+    float4 d[kBatch];
+    float g[kBatch];
 #pragma unroll
-    for (int k = 0; k < kMaxSub; ++k) {
-      if (k < nsub) {
-        const size_t u = (size_t)s * nsub + k;
-        dd[k] = __ldcs(reinterpret_cast<const float4*>(p.ds + (u * p.Hkv + kv) * D * D + e));
-        gg[k] = __expf(p.lam[u * p.Hkv + kv]);
+    for (int k = 0; k < kBatch; ++k) {
+      if (base + k < n_units) {
+        const size_t u = u0 + base + k;
+        d[k] = __ldcs(reinterpret_cast<const float4*>(p.ds + (u * p.Hkv + kv) * D * D + e));
+        g[k] = __expf(p.lam[u * p.Hkv + kv]);
       }
     }
-  };
-  const int s_end = si.first_seg + si.n_seg;
-  if (si.n_seg > 0) fetch(si.first_seg, d, g);
-  for (int s = si.first_seg; s < s_end; ++s) {
-    if (s + 1 < s_end) fetch(s + 1, dn, gn);
-    *reinterpret_cast<float4*>(p.ds + ((size_t)s * nsub * p.Hkv + kv) * D * D + e) = run;
+    int rr = base % nsub;   // sub-segment index of unit base + k
 #pragma unroll
-    for (int k = 0; k < kMaxSub; ++k) {
-      if (k < nsub)
+    for (int k = 0; k < kBatch; ++k, rr = rr + 1 == nsub ? 0 : rr + 1) {
+      if (base + k < n_units) {
+        if (rr == 0) *reinterpret_cast<float4*>(p.ds + ((u0 + base + k) * p.Hkv + kv) * D * D + e) = run;
         run = make_float4(fmaf(g[k], run.x, d[k].x), fmaf(g[k], run.y, d[k].y), fmaf(g[k], run.z, d[k].z),
                           fmaf(g[k], run.w, d[k].w));
+      }
     }
-#pragma unroll
-    for (int k = 0; k < kMaxSub; ++k) { d[k] = dn[k]; g[k] = gn[k]; }
   }
 }
 
