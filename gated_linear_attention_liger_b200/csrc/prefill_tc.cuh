@@ -12,25 +12,31 @@
 // Every exponent is a difference of running sums taken later-minus-earlier,
 // so it is <= 0 and cannot overflow however small the gates are.
 //
-// Work split (one GPU):
+// Work split (one GPU), launches chained with programmatic dependent launch:
 //   plan      : segment table from the sequence offsets (device side, so the
 //               launch needs no host synchronisation).
-//   seg_state : per (segment, kv head) the state a segment adds from a zero
-//               start, dS = sum over its chunks, and its total log decay.
+//   seg_state : per (sub-segment, kv head) the state it adds from a zero start,
+//               dS = sum over its chunks, and its total log decay.
+//   scan      : per (sequence, kv head) the state entering each segment, folded
+//               from the sub-segment contributions in order.
 //   chunk     : per (segment, pair of q heads of one kv head) the fused pass.
-//               Its prologue sums the earlier segments' dS into the entering
-//               state; after the last chunk it writes the final state.  TMA
-//               stages q/k/v chunks; four "feature" warps compute phi, gates and
-//               the state carry of chunk c+1 while four more warps run the window
-//               softmax and the epilogue of chunk c on TMEM rows; one thread
-//               issues the tcgen05 MMAs:
-//                 Ss = Q [K_prev;K_cur]^T        raw scores of the window band
-//                 Sg = phi(Q) phi(K)^T           recurrent scores
-//                 O  = (alpha e^{b_i}/Z_i e_q) S  inter-chunk readout
+//               Its prologue loads the entering state into TMEM; after the last
+//               chunk of a sequence it writes the final state.  TMA stages q/k/v
+//               chunks; an 8-warp feature group computes the key features,
+//               gates and decay-scaled keys, then e_q, then the bf16 state copy
+//               for the readout; four window warps run the window softmax, the
+//               recurrent probability tile and the epilogue on TMEM rows; one
+//               thread issues the tcgen05 MMAs:
+//                 Ss = Q [K_slot0 | K_slot1]^T   raw scores of the window band
+//                 Sg = e_Q e_K^T                 recurrent scores
+//                 O  = e_Q (alpha e^m S)         inter-chunk readout
 //                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
-//                 O += P_prev V_prev + P_cur V_cur, P_cur = beta*softmax + alpha*decayed Sg
-//               (P is written to TMEM and read from there as the A operand)
-//               and the epilogue stores bf16 rows.
+//                 O += P_prev V_prev + P_cur V_cur + A_grm V_cur
+//               (P and A_grm are written to TMEM and read from there as the A
+//               operand); e_Q, e_K are the unnormalised exponentials, their sums
+//               and the factored decay e^{b_i - m} e^{m - b_j} (m = b_C / 2) are
+//               folded into per-row and per-key scalars, and the epilogue stores
+//               bf16 rows.
 // Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
 // is exactly the order a TMA box over (d, head, token) produces.
 #pragma once
