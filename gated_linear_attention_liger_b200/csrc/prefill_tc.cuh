@@ -544,21 +544,18 @@ struct ChunkSmem {
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
   static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
   static constexpr uint32_t SMALL = SB + D * D * 2;
-  static constexpr uint32_t SMALL_BYTES = 6144;
+  static constexpr uint32_t SMALL_BYTES = 4096;
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
 // TMEM columns of the chunk kernel (fp32 cells, lane = tile row).
 constexpr uint32_t kColSs = 0;     // window scores, previous keys then current keys (128)
-constexpr uint32_t kColSg = 128;   // recurrent scores (64); then the recurrent probability tile (32)
+constexpr uint32_t kColSg = 128;   // recurrent scores (64)
 constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
 constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
 
-// Window warps per TMEM lane quarter (1 or 2: two split the columns).
-constexpr int kWinHalves = 1;
-constexpr int kWinThreads = 128 * kWinHalves;
-// warps [0, 4 kWinHalves) window/epilogue, then 8 features, 1 TMA, 1 MMA
-constexpr int kFeatWarp0 = 4 * kWinHalves;
+// warps 0-3 window/epilogue, 4-11 features, 12 TMA, 13 MMA
+constexpr int kFeatWarp0 = 4;
 constexpr int kTmaWarp = kFeatWarp0 + 8, kMmaWarp = kTmaWarp + 1;
 constexpr int kChunkThreads = 32 * (kMmaWarp + 1);
 
@@ -583,10 +580,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* feat = bars + 13;        // key and query tiles of the chunk ready (256 arrivals)
   uint64_t* sg_done = bars + 14;     // recurrent scores and state carry done
   uint64_t* mma2_done = bars + 15;   // + readout done: feature buffers free again
-  uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (window threads)
-  uint64_t* p_ready = bars + 17;     // probability tile in TMEM (window threads)
+  uint64_t* s_read = bars + 16;      // score tiles read out of TMEM (128 arrivals)
+  uint64_t* p_ready = bars + 17;     // probability tile in TMEM (128 arrivals)
   uint64_t* o_done = bars + 18;      // output accumulator complete
-  uint64_t* o_free = bars + 19;      // output read out (window threads)
+  uint64_t* o_free = bars + 19;      // output read out (128 arrivals)
   uint64_t* drain = bars + 20;
   uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (256 arrivals)
   uint64_t* state_done = bars + 23;  // the chunk's state carry done
@@ -599,7 +596,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
   float* fast2 = lg + 64;                                       // [2] factored decay usable
   float* izk2 = fast2 + 2;                                      // [2][64] 1 / z_k per key token
-  float* rowx = izk2 + 128;                                     // [2][128] row maxima, [2][128] row sums
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -616,8 +612,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     mbar_init(q_full, 1); mbar_init(q_empty, 2);
     mbar_init(ss_done, 1); mbar_init(feat, 256); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
     mbar_init(state_ready, 256); mbar_init(state_done, 1);
-    mbar_init(s_read, kWinThreads); mbar_init(p_ready, kWinThreads); mbar_init(o_done, 1);
-    mbar_init(o_free, kWinThreads);
+    mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
@@ -715,7 +710,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mma_commit(q_empty);           // one of the q buffer's two releases (the raw q was read)
         mma_commit(&k_empty[c & 1]);   // the previous chunk's keys are no longer needed
       };
-      auto issue_pv = [&](int c) {   // O += P_prev V_prev + P_cur V_cur, P read from TMEM
+      auto issue_pv = [&](int c) {   // O += P_prev V_prev + P_cur V_cur, P read from TMEM (P_cur holds the recurrent tile too)
         if (c == 0) ok = ok && mbar_wait(&v_full[0], 0, wc, wsite(2, 5, c));
         ok = ok && mbar_wait(p_ready, c & 1, wc, wsite(2, 6, c));
         if (!ok) return;
@@ -726,9 +721,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint64_t bp = sdesc_sw128(vp + kk * 2048, C * 128, 1024);
           const uint64_t bc = sdesc_sw128(vc + kk * 2048, C * 128, 1024);
-          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, bp, id_inter, 1u);        // window, previous keys
-          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 + kk * 8, bc, id_inter, 1u);   // window, current keys
-          mma_bf16_ts(tmem + kColO, tmem + kColSg + kk * 8, bc, id_inter, 1u);       // recurrent, current keys
+          mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, bp, id_inter, 1u);        // previous keys
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 + kk * 8, bc, id_inter, 1u);   // current keys (window + recurrent)
         }
         mma_commit(o_done);
         mma_commit(&v_empty[c % 3]);   // the previous chunk's values are no longer needed
@@ -808,7 +802,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     // (the window warps load the second half)
     entering_state<D, D / 4>(p, seg, kv, lrow % D, lane_base + kColS, half * (D / 4));
     tc_fence_before();
-    named_bar(2, 256 + kWinThreads);
+    named_bar(2, 256 + 128);
     tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
@@ -943,27 +937,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
       }
     }
-  } else {   // ---------------- window softmax and epilogue (kWinThreads threads)
-    // kWinHalves warps per TMEM lane quarter: with two, warps wq and wq + 4 share rows
-    // 32 wq .. 32 wq + 31 and split the columns (window groups 0-2 / 3-4, recurrent blocks
-    // by parity after all are loaded, output columns 0..D/2-1 / D/2..D-1); row maxima and
-    // sums are then exchanged through shared memory.
-    const int r = threadIdx.x & 127, sh = threadIdx.x >> 7;
+  } else {   // ---------------- window softmax and epilogue (128 threads, warps 0-3)
+    const int r = threadIdx.x;
     const int i = r >> 1, hl = r & 1;
-    const int wq = warp & 3, il = i - 16 * wq;
+    const int wq = warp, il = i - 16 * wq;
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-    // state entering the segment, this thread's share of the second half of the columns
-    // (the feature warps load the first half; TMEM: the state follows O)
-    constexpr int kEnt = D / (2 * kWinHalves);
-    entering_state<D, kEnt>(p, seg, kv, r % D, lane_base + kColO + D, D / 2 + sh * kEnt);
+    // state entering the segment, second half of the columns (the feature warps load the
+    // first half; TMEM: the state follows O)
+    entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColO + D, D / 2);
     tc_fence_before();
-    named_bar(2, 256 + kWinThreads);
+    named_bar(2, 256 + 128);
     tc_fence_after();
-    // this thread's window column groups
-    const int g_lo = kWinHalves == 1 ? 0 : (sh ? 3 : 0), g_hi = kWinHalves == 1 ? 5 : (sh ? 5 : 3);
 
     for (int c = 0; c < nch; ++c) {
       const int t0 = sg.t_begin + c * C;
@@ -986,7 +973,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const bool first = t0 == sg.q0;
       float m = -INFINITY;
 #pragma unroll 1
-      for (int q5 = g_lo; q5 < g_hi; ++q5) {
+      for (int q5 = 0; q5 < 5; ++q5) {
         float s[16];
         tmem_ld16(ss_col(q5), s);
         tmem_wait_ld();
@@ -1003,15 +990,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           for (int u = 0; u < w; ++u) s[u] = fmaxf(s[u], s[u + w]);
         m = fmaxf(m, s[0]);
       }
-      if (kWinHalves == 2) {
-        rowx[sh * 128 + r] = m;
-        named_bar(3, kWinThreads);
-        m = fmaxf(rowx[r], rowx[128 + r]);
-      }
       const float msc = m * sscale;
       float la = 0.f, lb = 0.f;   // exps written back over the scores
 #pragma unroll 1
-      for (int q5 = g_lo; q5 < g_hi; ++q5) {
+      for (int q5 = 0; q5 < 5; ++q5) {
         float s[16];
         tmem_ld16(ss_col(q5), s);
         tmem_wait_ld();
@@ -1029,82 +1011,56 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         tmem_st16(ss_col(q5), s);
       }
       tmem_wait_st();
-      if (kWinHalves == 2) rowx[256 + sh * 128 + r] = la + lb;
-      // Z of the rows and the recurrent scores come with the key and query tiles.  Both
-      // recurrent blocks of this half are read before the barrier: the probability tile is
-      // packed over the scores' first columns, which the other half may still be reading.
+      // Z of the rows and the recurrent scores come with the feature tiles
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
       tc_fence_after();
-      constexpr int kBlk = 4 / kWinHalves;   // recurrent blocks per thread: bb = kWinHalves t + sh
-      float g[kBlk][16];
-#pragma unroll
-      for (int t = 0; t < kBlk; ++t) {
-        const int bb = kWinHalves * t + sh;
-        if (bb <= wq) tmem_ld16(lane_base + kColSg + 16 * bb, g[t]);
-      }
-      tmem_wait_ld();
-      float lsum = la + lb;
-      if (kWinHalves == 2) {
-        named_bar(3, kWinThreads);
-        lsum = rowx[256 + r] + rowx[384 + r];
-      }
       const bool fast = fast2[c & 1] != 0.f;
       // The tiles carry e_q unnormalised: P is scaled by Z and the output by 1/Z.  In
       // factored mode P also carries e^{m - b_i} and the output e^{b_i - m}.
       const float zrow = zq2[(c & 1) * 128 + r];
       const float bi = bsh[i];
       const float mrow = fast ? 0.5f * bsh[nv - 1] - bi : 0.f;
-      const float coef = beta * zrow * __expf(mrow) / lsum;
+      const float coef = beta * zrow * __expf(mrow) / (la + lb);
       const float oscale = __expf(-mrow) / zrow;
+      // Probability tile over [previous | current] keys.  The recurrent tile covers the
+      // same current keys (kk <= i) and multiplies the same values, so it is added to the
+      // window tile's current half here: one P V product per half.  Group q5 holds the
+      // current keys kk = 16 bb + u with bb = q5 + wq - 4 when bb >= 0.
 #pragma unroll 1
-      for (int q5 = g_lo; q5 < g_hi; ++q5) {
-        float s[16];
+      for (int q5 = 0; q5 < 5; ++q5) {
+        const int bb = q5 + wq - 4;
+        float s[16], g[16];
         tmem_ld16(ss_col(q5), s);
+        if (bb >= 0) tmem_ld16(lane_base + kColSg + 16 * bb, g);
         tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) s[u] *= coef;
+        if (bb >= 0) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int kk = 16 * bb + u;
+            float gv = fast ? alpha * g[u] * eneg[kk]   // e^{m - b_kk} / z_kk; the row's e^{b_i - m} in the epilogue
+                            : alpha * g[u] * (__expf(bi - bsh[kk]) * izk[kk]);
+            if (bb == wq) gv = kk <= i ? gv : 0.f;       // the diagonal block is causal
+            s[u] += gv;
+          }
+        }
         uint32_t pw[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(s[2 * k] * coef, s[2 * k + 1] * coef);
+        for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
         tmem_st8u(lane_base + kColP + 8 * wq + 8 * q5, pw);
       }
-      if (sh == kWinHalves - 1) {   // zeros for the keys outside this quarter's band
+      {   // zeros for the keys outside this quarter's band
         const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
         for (int k = 0; k < 3; ++k) tmem_st8u(lane_base + kColP + ((8 * wq + 40 + 8 * k) & 63), zero8);
       }
-      tc_fence_before();
-      mbar_arrive(s_read);   // the window scores are consumed: their TMEM may be reused
-
-      // recurrent probability tile over the current keys kk <= i, packed over the
-      // recurrent scores (this quarter needs kk < 16 wq + 16; later blocks are zero)
-#pragma unroll
-      for (int t = 0; t < kBlk; ++t) {
-        const int bb = kWinHalves * t + sh;
-        uint32_t ag[8];
-        if (bb <= wq) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int kk = 16 * bb + 2 * k;
-            float g0, g1;
-            if (fast) {   // e^{m - b_kk} / z_kk; the row's e^{b_i - m} comes in the epilogue
-              g0 = alpha * g[t][2 * k] * eneg[kk];
-              g1 = alpha * g[t][2 * k + 1] * eneg[kk + 1];
-            } else {
-              g0 = alpha * g[t][2 * k] * (__expf(bi - bsh[kk]) * izk[kk]);
-              g1 = alpha * g[t][2 * k + 1] * (__expf(bi - bsh[kk + 1]) * izk[kk + 1]);
-            }
-            ag[k] = pack_bf16(kk <= i ? g0 : 0.f, kk + 1 <= i ? g1 : 0.f);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) ag[k] = 0u;
-        }
-        tmem_st8u(lane_base + kColSg + 8 * bb, ag);
-      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive(s_read);    // the scores are consumed: their TMEM may be reused
+      mbar_arrive(p_ready);   // the probability tile is in TMEM
 
-      // epilogue: O -> bf16 rows of out, this half's columns
+      // epilogue: O -> bf16 rows of out
       const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
       tc_fence_after();
       {
@@ -1112,7 +1068,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
         const bool store = i < nv && live;
 #pragma unroll 1
-        for (int col = sh * (D / kWinHalves); col < (sh + 1) * (D / kWinHalves); col += 32) {
+        for (int col = 0; col < D; col += 32) {
           float v[32];
           tmem_ld32(lane_base + kColO + col, v);
           tmem_wait_ld();
