@@ -240,6 +240,11 @@ __device__ __forceinline__ float log_sigmoid_fast(float m) {
   return fminf(m, 0.f) - t;
 }
 
+// Largest log2 spread max - shift of a row whose exponentials are taken against a
+// shift other than its maximum: values stay below 2^24, leaving fp32 and bf16 headroom
+// for the per-row and per-key factors applied later.
+constexpr float kShiftSpan = 24.f;
+
 // Feature map and gate of one chunk of keys, shared by the seg_state and chunk
 // kernels.  TPT threads (2 or 4, adjacent lanes) share a key token: thread r owns
 // elements [h D/TPT, (h+1) D/TPT) of token j = r / TPT, h = r % TPT, and the group
@@ -257,35 +262,60 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   constexpr int PART = D / TPT;
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r / TPT, h = r % TPT;
-  float m = -INFINITY, sa = 0.f, sb = 0.f;
+  // One pass: raw sum (for the gate), maximum, and e = exp(k - k_0) with k_0 the
+  // token's first element.  Any shift leaves the normalised features unchanged; the
+  // maximum is needed only when the token's spread would leave too little fp32
+  // headroom, and then the exponentials are redone against it.
+  const float sl = bf16_lo(*reinterpret_cast<const uint32_t*>(kraw + kmajor_off(j, 0, KSTRIDE))) * kLog2e;
+  float m = -INFINITY, sa = 0.f, sb = 0.f, za = 0.f, zb = 0.f;
 #pragma unroll 4
   for (int c = 0; c < PART / 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * PART + c * 8, KSTRIDE));
     m = fmaxf(m, bf16x8_max(u));
-    sa += (bf16_lo(u.x) + bf16_hi(u.x)) + (bf16_lo(u.y) + bf16_hi(u.y));
-    sb += (bf16_lo(u.z) + bf16_hi(u.z)) + (bf16_lo(u.w) + bf16_hi(u.w));
-  }
-  float sum = sa + sb;
-#pragma unroll
-  for (int o = 1; o < TPT; o <<= 1) {
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  }
-  const float ml = m * kLog2e;
-  float za = 0.f, zb = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < PART / 8; ++c) {
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
     float x[8];
-    ld_chunk8(kraw, kmajor_off(j, h * PART + c * 8, KSTRIDE), x);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
+    for (int q = 0; q < 4; ++q) { x[2 * q] = bf16_lo(w4[q]); x[2 * q + 1] = bf16_hi(w4[q]); }
+    sa += (x[0] + x[1]) + (x[2] + x[3]);
+    sb += (x[4] + x[5]) + (x[6] + x[7]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sl));
     za += (x[0] + x[1]) + (x[2] + x[3]);
     zb += (x[4] + x[5]) + (x[6] + x[7]);
     st_chunk8(ebuf, kmajor_off(j, h * PART + c * 8, C * 128), x);
   }
-  float z = za + zb;
+  float sum = sa + sb, z = za + zb;
 #pragma unroll
-  for (int o = 1; o < TPT; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  for (int o = 1; o < TPT; o <<= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    z += __shfl_xor_sync(0xffffffffu, z, o);
+  }
+  // The redo is decided per token (the same on all its lanes) but entered by the whole
+  // warp, so that the shuffles below always see every lane.
+  const bool redo = m * kLog2e - sl > kShiftSpan;
+  if (__any_sync(0xffffffffu, redo)) {
+    float zr = 0.f;
+    if (redo) {
+      const float ml = m * kLog2e;
+      za = 0.f;
+      zb = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < PART / 8; ++c) {
+        float x[8];
+        ld_chunk8(kraw, kmajor_off(j, h * PART + c * 8, KSTRIDE), x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
+        za += (x[0] + x[1]) + (x[2] + x[3]);
+        zb += (x[4] + x[5]) + (x[6] + x[7]);
+        st_chunk8(ebuf, kmajor_off(j, h * PART + c * 8, C * 128), x);
+      }
+      zr = za + zb;
+    }
+#pragma unroll
+    for (int o = 1; o < TPT; o <<= 1) zr += __shfl_xor_sync(0xffffffffu, zr, o);
+    if (redo) z = zr;
+  }
   if (h == 0) lg[j] = j < nv ? log_sigmoid_fast(sum / (float)D) : 0.f;
   named_bar(1, 64 * TPT);
   {   // inclusive running sum over the 64 tokens, two per lane, in every warp
@@ -839,27 +869,54 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int row = t >> 1, qh = t & 1;
       mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
       if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));   // e_q tile and state copy free
-      float mq = -INFINITY;
-#pragma unroll
-      for (int c8 = 0; c8 < D / 16; ++c8)
-        mq = fmaxf(mq, bf16x8_max(*reinterpret_cast<const uint4*>(qb + kmajor_off(row, qh * (D / 2) + c8 * 8,
-                                                                                     ROWS * 128))));
-      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
-      const float mql = mq * kLog2e;
-      float za = 0.f, zb = 0.f;
+      // one pass: e_q = exp(q - q_0) with q_0 the row's first element (the tiles carry e_q
+      // unnormalised, so the shift cancels against Z), redone against the row maximum if
+      // the spread is too large (see kShiftSpan)
+      const float sl = bf16_lo(*reinterpret_cast<const uint32_t*>(qb + kmajor_off(row, 0, ROWS * 128))) * kLog2e;
+      float mq = -INFINITY, za = 0.f, zb = 0.f;
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 16; ++c8) {
         const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
+        const uint4 u = *reinterpret_cast<const uint4*>(qb + off);
+        mq = fmaxf(mq, bf16x8_max(u));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
         float x[8];
-        ld_chunk8(qb, off, x);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
+        for (int q = 0; q < 4; ++q) { x[2 * q] = bf16_lo(w4[q]); x[2 * q + 1] = bf16_hi(w4[q]); }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sl));
         za += (x[0] + x[1]) + (x[2] + x[3]);
         zb += (x[4] + x[5]) + (x[6] + x[7]);
         st_chunk8(eqb, off, x);
       }
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
       float zq = za + zb;
       zq += __shfl_xor_sync(0xffffffffu, zq, 1);
+      // decided per row (the same on both of its threads), entered by the whole warp so
+      // that the shuffle sees every lane
+      const bool redo = mq * kLog2e - sl > kShiftSpan;
+      if (__any_sync(0xffffffffu, redo)) {
+        float zr = 0.f;
+        if (redo) {
+          const float mql = mq * kLog2e;
+          za = 0.f;
+          zb = 0.f;
+#pragma unroll 1
+          for (int c8 = 0; c8 < D / 16; ++c8) {
+            const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
+            float x[8];
+            ld_chunk8(qb, off, x);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
+            za += (x[0] + x[1]) + (x[2] + x[3]);
+            zb += (x[4] + x[5]) + (x[6] + x[7]);
+            st_chunk8(eqb, off, x);
+          }
+          zr = za + zb;
+        }
+        zr += __shfl_xor_sync(0xffffffffu, zr, 1);
+        if (redo) zq = zr;
+      }
       if (qh == 0) zq2[(c & 1) * 128 + row] = zq;
       // The q buffer is released twice per chunk: by the score MMA's commit, and by this
       // group once done with the raw q (factored mode) or by the readout's commit (exact

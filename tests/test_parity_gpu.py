@@ -85,6 +85,24 @@ def test_prefill_general_kernel_parity(case, cuda_device):
     assert_close(np64(fs), rfs, dtype, "final_state")
 
 
+def test_prefill_wide_feature_spread(cuda_device):
+    """Rows whose first element lies far below their maximum: the feature passes
+    take their exponentials against the row's first element and must fall back
+    to the row maximum (queries and keys, both heads of a tile, several chunks)."""
+    wl = inputs.small("wide_spread", B=1, Hq=4, Hkv=2, T=200, d=128, dtype=torch.bfloat16, seed=77)
+    q, k, v = inputs.prefill_inputs(wl)
+    q[:, ::3, :, 0] = -40.0          # spread 40 (about 58 in log2) on every third token
+    q[:, 1::7, :, 0] = 25.0          # first element is the maximum: no fallback
+    k[:, ::5, :, 0] = -40.0
+    k[:, 2::11, :, 0] = -12.0        # spread about 15 in log2: shifted pass kept
+    dev = cuda_device
+    out, fs = ops.prefill(q.to(dev), k.to(dev), v.to(dev))
+    torch.cuda.synchronize()
+    ro, rfs, _, _ = oracle.prefill(np64(q), np64(k), np64(v))
+    assert_close(np64(out), ro, torch.bfloat16, "out")
+    assert_close(np64(fs), rfs, torch.bfloat16, "final_state")
+
+
 def test_prefill_empty_batch(cuda_device):
     q = torch.zeros(2, 0, 4, 64, dtype=torch.bfloat16, device=cuda_device)
     k = torch.zeros(2, 0, 2, 64, dtype=torch.bfloat16, device=cuda_device)
