@@ -248,17 +248,18 @@ constexpr float kShiftSpan = 24.f;
 // Feature map and gate of one chunk of keys, shared by the seg_state and chunk
 // kernels.  TPT threads (2 or 4, adjacent lanes) share a key token: thread r owns
 // elements [h D/TPT, (h+1) D/TPT) of token j = r / TPT, h = r % TPT, and the group
-// is 64 TPT threads.  Writes e = exp(k - max_d k) (bf16, not yet divided by its sum)
-// to `ebuf` in the key tile's swizzled layout and the log gates to lg[0..63] (0 past
-// the valid tokens); returns 1 / sum_d e, which the callers fold into per-token
-// scalars, and the running sums in gs (every warp scans the 64 gates itself); lanes
-// of the group's first warp also store the sums to bsh.  Each pass is a short loop
-// over 16-byte groups: the role loops of the chunk kernel share one SM
-// sub-partition, and fully unrolled straight-line code for all of them would not
-// stay in the instruction caches.
+// is 64 TPT threads.  Computes e = exp(k - shift) (bf16, not yet divided by its sum;
+// the shift cancels once the sum is divided out), keeps this thread's values packed
+// in ek and writes them to `ebuf` (if not null) in the key tile's swizzled layout;
+// writes the log gates to lg[0..63] (0 past the valid tokens); returns 1 / sum_d e,
+// which the callers fold into per-token scalars, and the running sums in gs (every
+// warp scans the 64 gates itself); lanes of the group's first warp also store the
+// sums to bsh.  The loops run over 16-byte groups and stay short: the role loops of
+// the chunk kernel share one SM sub-partition, and long straight-line code for all
+// of them would not stay in the instruction caches.
 template <int D, int TPT = 2, uint32_t KSTRIDE = C * 128>   // KSTRIDE: byte stride of the raw tile's 64-element blocks
 __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, float* lg, float* bsh, int r, int nv,
-                                              GateSums& gs) {
+                                              GateSums& gs, uint32_t (&ek)[D / TPT / 2]) {
   constexpr int PART = D / TPT;
   constexpr float kLog2e = 1.4426950408889634f;
   const int j = r / TPT, h = r % TPT;
@@ -268,7 +269,7 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   // headroom, and then the exponentials are redone against it.
   const float sl = bf16_lo(*reinterpret_cast<const uint32_t*>(kraw + kmajor_off(j, 0, KSTRIDE))) * kLog2e;
   float m = -INFINITY, sa = 0.f, sb = 0.f, za = 0.f, zb = 0.f;
-#pragma unroll 4
+#pragma unroll
   for (int c = 0; c < PART / 8; ++c) {
     const uint4 u = *reinterpret_cast<const uint4*>(kraw + kmajor_off(j, h * PART + c * 8, KSTRIDE));
     m = fmaxf(m, bf16x8_max(u));
@@ -282,7 +283,11 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
     for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sl));
     za += (x[0] + x[1]) + (x[2] + x[3]);
     zb += (x[4] + x[5]) + (x[6] + x[7]);
-    st_chunk8(ebuf, kmajor_off(j, h * PART + c * 8, C * 128), x);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ek[4 * c + q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+    if (ebuf)
+      *reinterpret_cast<uint4*>(ebuf + kmajor_off(j, h * PART + c * 8, C * 128)) =
+          make_uint4(ek[4 * c], ek[4 * c + 1], ek[4 * c + 2], ek[4 * c + 3]);
   }
   float sum = sa + sb, z = za + zb;
 #pragma unroll
@@ -300,7 +305,7 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
       const float ml = m * kLog2e;
       za = 0.f;
       zb = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < PART / 8; ++c) {
         float x[8];
         ld_chunk8(kraw, kmajor_off(j, h * PART + c * 8, KSTRIDE), x);
@@ -308,7 +313,11 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
         for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -ml));
         za += (x[0] + x[1]) + (x[2] + x[3]);
         zb += (x[4] + x[5]) + (x[6] + x[7]);
-        st_chunk8(ebuf, kmajor_off(j, h * PART + c * 8, C * 128), x);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ek[4 * c + q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+        if (ebuf)
+          *reinterpret_cast<uint4*>(ebuf + kmajor_off(j, h * PART + c * 8, C * 128)) =
+              make_uint4(ek[4 * c], ek[4 * c + 1], ek[4 * c + 2], ek[4 * c + 3]);
       }
       zr = za + zb;
     }
@@ -338,21 +347,23 @@ __device__ __forceinline__ float key_features(const char* kraw, char* ebuf, floa
   return 1.0f / z;
 }
 
-// Decay-scaled keys sc * e (sc = e^{b_C - b_j} / z_j, zero past the valid tokens),
-// from this thread's features in `ebuf` to `kt` in the same swizzled layout (thread
-// layout as in key_features); read by the MMA as the MN-major A operand K^T.
+// Decay-scaled keys sc * e (sc = e^{b_C - b_j} / z_j, zero past the valid tokens), from
+// this thread's packed features ek (as key_features stored them) to `kt` in the key
+// tile's swizzled layout (thread layout as in key_features); read by the MMA as the
+// MN-major A operand K^T.
 template <int D, int TPT = 2>
-__device__ __forceinline__ void write_ktilde(const char* ebuf, char* kt, int r, float sc) {
+__device__ __forceinline__ void write_ktilde(const uint32_t (&ek)[D / TPT / 2], char* kt, int r, float sc) {
   constexpr int PART = D / TPT;
   const int j = r / TPT, h = r % TPT;
-#pragma unroll 4
-  for (int c = 0; c < PART / 8; ++c) {
-    const uint32_t off = kmajor_off(j, h * PART + c * 8, C * 128);
-    float x[8];
-    ld_chunk8(ebuf, off, x);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] *= sc;
-    st_chunk8(kt, off, x);
+  for (int c = 0; c < PART / 8; ++c) {
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      x[2 * q] = bf16_lo(ek[4 * c + q]) * sc;
+      x[2 * q + 1] = bf16_hi(ek[4 * c + q]) * sc;
+    }
+    st_chunk8(kt, kmajor_off(j, h * PART + c * 8, C * 128), x);
   }
 }
 
@@ -487,12 +498,13 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       mbar_wait(&k_full[slot], (c >> 1) & 1, wc);
       char* const kt = smem + L::KT + slot * L::KV;   // read by the product two chunks back: long done
       GateSums gs;
-      const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, kt, lg, nullptr, r, nv, gs);
+      uint32_t ek[D / 8];
+      const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, nullptr, lg, nullptr, r, nv, gs, ek);
       mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 2);
       lam += bC;
-      write_ktilde<D, 4>(kt, kt, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
+      write_ktilde<D, 4>(ek, kt, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
       if (c > 0) {   // the previous product must be done with S before it is rescaled
         mbar_wait(mma_done, (c - 1) & 1, wc);
         tc_fence_after();
@@ -850,11 +862,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       // decay-scaled keys
       const int j = t >> 2;
       GateSums gs;
+      uint32_t ek[D / 8];
       const float iz = key_features<D, 4, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK,
-                                                        lg, bsh, t, nv, gs);
+                                                        lg, bsh, t, nv, gs, ek);
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(j);
-      write_ktilde<D, 4>(smem + L::PK, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
+      write_ktilde<D, 4>(ek, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
       // Factored mode (the chunk's total log gate >= -80): with m = b_C / 2,
       // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-40}.
       const bool fast = bC >= -80.f;
