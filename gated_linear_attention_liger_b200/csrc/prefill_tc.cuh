@@ -392,8 +392,8 @@ __global__ void __launch_bounds__(kSegThreads, 2)
   uint64_t* v_full = bars + 4;     // [2]
   uint64_t* v_empty = bars + 7;    // [2]
   uint64_t* feat = bars + 10;
-  uint64_t* mma_done = bars + 11;
-  uint64_t* drain = bars + 12;
+  uint64_t* mma_done = bars + 11;  // [2], per keys~ slot
+  uint64_t* drain = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;          // stays 0: drain waits ignore aborts
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 256); }
     for (int i = 0; i < 2; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-    mbar_init(feat, 256); mbar_init(mma_done, 1); mbar_init(drain, 1);
+    mbar_init(feat, 256); mbar_init(&mma_done[0], 1); mbar_init(&mma_done[1], 1); mbar_init(drain, 1);
     *abort_flag = 0u;
     *never = 0u;
     fence_mbar_init();
@@ -442,8 +442,8 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
       int k_issued = 0, v_issued = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int t = sg.t_begin + c * C;
+      for (int c = 0; c < nch; ++c) {   // step c handles chunk nch - 1 - c (last to first)
+        const int t = sg.t_begin + (nch - 1 - c) * C;
         const int ks = c & 1, vs = c & 1;
         if (c >= 2 && !mbar_wait(&k_empty[ks], ((c >> 1) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&k_full[ks], L::KV);
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
           const uint64_t b = sdesc_sw128(smem_u32(smem + L::V0 + vs * L::KV) + kk * 2048, C * 128, 1024);
           mma_bf16_ss(tmem, a, b, idesc, (c > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(mma_done);
+        mma_commit(&mma_done[c & 1]);
         mma_commit(&v_empty[vs]);
       }
       mma_commit(drain);
@@ -488,46 +488,37 @@ __global__ void __launch_bounds__(kSegThreads, 2)
     const int r = threadIdx.x;
     const int row = r & 127, half = warp >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    // The chunks are taken last to first, so the decay from a chunk to the end of the
+    // sub-segment (lam, the sum of the later chunks' totals) is known when it is
+    // processed: its keys~ carry it, e^{lam + b_C - b_j} phi(k_j) (exponent <= 0), and
+    // the products accumulate onto dS with no rescale in between.
     float lam = 0.f;
     // Row threads never leave the loop early: after a timeout every wait returns
     // at once (the CTA's abort flag is set), so all rows still meet at each
     // named barrier and warp-collective TMEM access stays uniform.
     for (int c = 0; c < nch; ++c) {
       const int slot = c & 1;
-      const int nv = min(C, sg.t_end - (sg.t_begin + c * C));
+      const int cc = nch - 1 - c;
+      const int nv = min(C, sg.t_end - (sg.t_begin + cc * C));
       mbar_wait(&k_full[slot], (c >> 1) & 1, wc);
-      char* const kt = smem + L::KT + slot * L::KV;   // read by the product two chunks back: long done
       GateSums gs;
       uint32_t ek[D / 8];
       const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, nullptr, lg, nullptr, r, nv, gs, ek);
       mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 2);
-      lam += bC;
-      write_ktilde<D, 4>(ek, kt, r, (r >> 2) < nv ? __expf(bC - bj) * iz : 0.f);
-      if (c > 0) {   // the previous product must be done with S before it is rescaled
-        mbar_wait(mma_done, (c - 1) & 1, wc);
+      if (c >= 2) {   // the product two steps back is done with this keys~ slot
+        mbar_wait(&mma_done[slot], ((c >> 1) - 1) & 1, wc);
         tc_fence_after();
       }
-      if (c > 0) {   // S <- e^{b_C} S before this chunk's product accumulates onto it
-        const float dec = __expf(bC);
-#pragma unroll 1
-        for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
-          float v[32];
-          tmem_ld32(lane_base + col, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= dec;
-          tmem_st32(lane_base + col, v);
-        }
-        tmem_wait_st();
-      }
+      write_ktilde<D, 4>(ek, smem + L::KT + slot * L::KV, r, (r >> 2) < nv ? __expf(lam + bC - bj) * iz : 0.f);
+      lam += bC;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(feat);
       named_bar(1, 256);   // lg is rewritten by the next chunk
     }
-    if (nch > 0 && mbar_wait(mma_done, (nch - 1) & 1, wc) && !*abort_flag) {
+    if (nch > 0 && mbar_wait(&mma_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, wc) && !*abort_flag) {
       tc_fence_after();
       float* dst = ds_out + (size_t)row * D;
 #pragma unroll 1
