@@ -28,14 +28,15 @@
 //               recurrent probability tile and the epilogue on TMEM rows; one
 //               thread issues the tcgen05 MMAs:
 //                 Ss = Q [K_slot0 | K_slot1]^T   raw scores of the window band
-//                 Sg = e_Q e_K^T                 recurrent scores
+//                 Sg = e_Q (e^{b_C-b_j} phi(K))^T recurrent scores (e_Q e_K^T when the
+//                                                decay does not factor)
 //                 O  = e_Q (alpha e^m S)         inter-chunk readout
 //                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
 //                 O += P_prev V_prev + P_cur V_cur + A_grm V_cur
 //               (P and A_grm are written to TMEM and read from there as the A
 //               operand); e_Q, e_K are the unnormalised exponentials, their sums
 //               and the factored decay e^{b_i - m} e^{m - b_j} (m = b_C / 2) are
-//               folded into per-row and per-key scalars, and the epilogue stores
+//               folded into per-row and per-chunk scalars, and the epilogue stores
 //               bf16 rows.
 // Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
 // is exactly the order a TMA box over (d, head, token) produces.
@@ -624,8 +625,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
   float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256 + 64);  // [2][64] running log-gate sums
-  float* eneg2 = bsh2 + 128;                                    // [2][64] e^{-b_j} (factored decay)
-  float* zq2 = eneg2 + 128;                                     // [2][128] Z = sum_d e_q per row
+  float* zq2 = bsh2 + 128;                                     // [2][128] Z = sum_d e_q per row
   float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
   float* fast2 = lg + 64;                                       // [2] factored decay usable
   float* izk2 = fast2 + 2;                                      // [2][64] 1 / z_k per key token
@@ -765,11 +765,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         ok = ok && mbar_wait(feat, c & 1, wc, wsite(2, 7, c));
         if (!ok) return;
         tc_fence_after();
+        // factored mode: the scores against the decay-scaled keys; otherwise against e_k
+        const uint32_t kf_base = fast2[c & 1] != 0.f ? kt_base : pk_base;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
           const uint32_t ko = (kk >> 2) * (C * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColSg, sdesc_sw128(eq_base + qo, 16, 1024), sdesc_sw128(pk_base + ko, 16, 1024),
+          mma_bf16_ss(tmem + kColSg, sdesc_sw128(eq_base + qo, 16, 1024), sdesc_sw128(kf_base + ko, 16, 1024),
                       id_n64, kk > 0);
         }
         // (failure-detection test: withhold the first completion; the waits downstream
@@ -854,18 +856,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int j = t >> 2;
       GateSums gs;
       uint32_t ek[D / 8];
-      const float iz = key_features<D, 4, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), smem + L::PK,
+      const float iz = key_features<D, 4, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), nullptr,
                                                         lg, bsh, t, nv, gs, ek);
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(j);
       write_ktilde<D, 4>(ek, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
-      // Factored mode (the chunk's total log gate >= -80): with m = b_C / 2,
-      // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-40}.
-      const bool fast = bC >= -80.f;
-      if ((t & 3) == 0) {
-        eneg2[(c & 1) * 64 + j] = fast ? __expf(0.5f * bC - bj) * iz : 0.f;
-        izk2[(c & 1) * 64 + j] = iz;
+      // Factored mode (the chunk's total log gate >= -60): with m = b_C / 2,
+      // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-30}.  The
+      // recurrent scores then come from the decay-scaled keys, since
+      // e^{m - b_j} / z_j = e^{-m} (e^{b_C - b_j} / z_j) leaves one scalar per chunk.  A key
+      // feature below 2^-126 e^{b_j - b_C} is flushed in that tile; the bound keeps the
+      // resulting error of a score under 2^-126 e^{60} ~ 1e-12.  Otherwise the scores come
+      // from e_k, written only then.
+      const bool fast = bC >= -60.f;
+      if (!fast) {   // the same decision for the whole CTA
+        const int h = t & 3;
+#pragma unroll
+        for (int c8 = 0; c8 < D / 32; ++c8)
+          *reinterpret_cast<uint4*>(smem + L::PK + kmajor_off(j, h * (D / 4) + c8 * 8, C * 128)) =
+              make_uint4(ek[4 * c8], ek[4 * c8 + 1], ek[4 * c8 + 2], ek[4 * c8 + 3]);
       }
+      if ((t & 3) == 0) izk2[(c & 1) * 64 + j] = iz;
       if (t == 0) fast2[c & 1] = fast ? 1.f : 0.f;
 
       // queries: e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the
@@ -1017,7 +1028,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int t0 = sg.t_begin + c * C;
       const int nv = min(C, sg.t_end - t0);
       const float* bsh = bsh2 + (c & 1) * 64;
-      const float* eneg = eneg2 + (c & 1) * 64;
       const float* izk = izk2 + (c & 1) * 64;
       // Window band.  Key index x over [previous chunk | current chunk] (0..127): row i
       // sees x in [i+1, i+64].  This quarter's tokens are 16 wq .. 16 wq + 15, so it reads
@@ -1083,6 +1093,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float mrow = fast ? 0.5f * bsh[nv - 1] - bi : 0.f;
       const float coef = beta * zrow * __expf(mrow) / (la + lb);
       const float oscale = __expf(-mrow) / zrow;
+      const float gscale = fast ? alpha * __expf(-0.5f * bsh[nv - 1]) : 0.f;   // alpha e^{-m}
       // Probability tile over [previous | current] keys.  The recurrent tile covers the
       // same current keys (kk <= i) and multiplies the same values, so it is added to the
       // window tile's current half here: one P V product per half.  Group q5 holds the
@@ -1100,7 +1111,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const int kk = 16 * bb + u;
-            float gv = fast ? alpha * g[u] * eneg[kk]   // e^{m - b_kk} / z_kk; the row's e^{b_i - m} in the epilogue
+            float gv = fast ? g[u] * gscale   // scores against e^{b_C - b_kk} / z_kk e_k; e^{b_i - m} in the epilogue
                             : alpha * g[u] * (__expf(bi - bsh[kk]) * izk[kk]);
             if (bb == wq) gv = kk <= i ? gv : 0.f;       // the diagonal block is causal
             s[u] += gv;

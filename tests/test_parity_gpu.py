@@ -103,6 +103,26 @@ def test_prefill_wide_feature_spread(cuda_device):
     assert_close(np64(fs), rfs, torch.bfloat16, "final_state")
 
 
+def test_prefill_sharp_gate_drops(cuda_device):
+    """Gates near 1 except one token per chunk whose gate is about e^-50, e^-70 or e^-55:
+    chunk log-gate totals of about -53, -73 and -58 put chunks on both sides of the
+    kernel's switch between factored and exact decay, with the in-chunk decay from keys
+    before the drop to the chunk's end far below the decay between the rows and keys
+    that meet in the recurrent scores."""
+    wl = inputs.small("sharp_drops", B=1, Hq=4, Hkv=2, T=260, d=128, dtype=torch.bfloat16, seed=91)
+    q, k, v = inputs.prefill_inputs(wl)
+    k += 3.0                          # sigmoid(mean k) ~ 0.95: log gate ~ -0.05 per token
+    k[:, 30] = -50.0
+    k[:, 100] = -70.0
+    k[:, 150] = -55.0
+    dev = cuda_device
+    out, fs = ops.prefill(q.to(dev), k.to(dev), v.to(dev))
+    torch.cuda.synchronize()
+    ro, rfs, _, _ = oracle.prefill(np64(q), np64(k), np64(v))
+    assert_close(np64(out), ro, torch.bfloat16, "out")
+    assert_close(np64(fs), rfs, torch.bfloat16, "final_state")
+
+
 def test_prefill_empty_batch(cuda_device):
     q = torch.zeros(2, 0, 4, 64, dtype=torch.bfloat16, device=cuda_device)
     k = torch.zeros(2, 0, 2, 64, dtype=torch.bfloat16, device=cuda_device)
