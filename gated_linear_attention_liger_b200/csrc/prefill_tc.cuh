@@ -30,14 +30,15 @@
 //                 Ss = Q [K_slot0 | K_slot1]^T   raw scores of the window band
 //                 Sg = e_Q (e^{b_C-b_j} phi(K))^T recurrent scores (e_Q e_K^T when the
 //                                                decay does not factor)
-//                 O  = e_Q (alpha e^m S)         inter-chunk readout
+//                 O  = e_Q (e^{b_C} S)           inter-chunk readout (e^{b_i} e_Q and S
+//                                                when the decay does not factor)
 //                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
 //                 O += P_prev V_prev + P_cur V_cur + A_grm V_cur
 //               (P and A_grm are written to TMEM and read from there as the A
-//               operand); e_Q, e_K are the unnormalised exponentials, their sums
-//               and the factored decay e^{b_i - m} e^{m - b_j} (m = b_C / 2) are
-//               folded into per-row and per-chunk scalars, and the epilogue stores
-//               bf16 rows.
+//               operand); e_Q (which also carries alpha) and e_K are unnormalised
+//               exponentials, their sums and the row factor e^{b_i - b_C} of the
+//               decay are folded into per-row scalars, and the epilogue stores bf16
+//               rows.
 // Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
 // is exactly the order a TMA box over (d, head, token) produces.
 #pragma once
@@ -619,7 +620,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* o_done = bars + 18;      // output accumulator complete
   uint64_t* o_free = bars + 19;      // output read out (128 arrivals)
   uint64_t* drain = bars + 20;
-  uint64_t* state_ready = bars + 22; // alpha S copied, S rescaled (256 arrivals)
+  uint64_t* state_ready = bars + 22; // state copied, S rescaled (256 arrivals)
   uint64_t* state_done = bars + 23;  // the chunk's state carry done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -789,7 +790,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
                       sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
         mma_commit(state_done);
       };
-      auto issue_inter = [&](int c) {   // O = (e^{b_i} / Z_i e_q) (alpha S), S as MN-major B
+      auto issue_inter = [&](int c) {   // O = e_q' (e^{b_C} S) or (e^{b_i} e_q') S, the state as MN-major B
         if (c > 0) ok = ok && mbar_wait(o_free, (c - 1) & 1, wc, wsite(2, 9, c));
         if (!ok) return;
         tc_fence_after();
@@ -832,6 +833,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     char* const qb = smem + L::Q0;
     char* const eqb = smem + L::EQ;
     char* const sbb = smem + L::SB;
+    // The e_q tile carries the branch weight: e_q' = a e_q with a = alpha, taken into the
+    // exponent (2^{log2 a}), so that the readout's state copy needs no multiply.  Z is summed
+    // from the same scaled values and divided by a, so any rounding of log2 a cancels.  A
+    // weight below 2^-20 (0 included) stays on the copy instead (a = 1), which keeps the
+    // scaled scores far above fp32's smallest normal.
+    const float qa = p.alpha >= 0x1p-20f ? p.alpha : 1.f;
+    const float lqa = log2f(qa), iqa = 1.f / qa;
+    const float copy_scale = p.alpha / qa;   // 1, or alpha when it stays on the copy
 
     // state entering the segment: this warp's quarter of the first half of the columns
     // (the window warps load the second half)
@@ -861,13 +870,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(j);
       write_ktilde<D, 4>(ek, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
-      // Factored mode (the chunk's total log gate >= -60): with m = b_C / 2,
-      // e^{b_i - b_j} = e^{b_i - m} e^{m - b_j} and both factors lie within e^{+-30}.  The
-      // recurrent scores then come from the decay-scaled keys, since
-      // e^{m - b_j} / z_j = e^{-m} (e^{b_C - b_j} / z_j) leaves one scalar per chunk.  A key
-      // feature below 2^-126 e^{b_j - b_C} is flushed in that tile; the bound keeps the
-      // resulting error of a score under 2^-126 e^{60} ~ 1e-12.  Otherwise the scores come
-      // from e_k, written only then.
+      // Factored mode (the chunk's total log gate b_C >= -60): e^{b_i - b_j} =
+      // e^{b_i - b_C} e^{b_C - b_j}, both factors within e^{+-60}.  The key factor is the one
+      // the decay-scaled keys carry, so the recurrent scores are taken against that tile and
+      // need no per-key scalar; the row factor goes to the epilogue, and the readout uses
+      // e^{b_C} S, which is the rescaled state.  A key feature below 2^-126 e^{b_j - b_C} is
+      // flushed in the tile; the bound keeps the resulting error of a score under
+      // 2^-126 e^{60} ~ 1e-12.  Otherwise the scores come from e_k, written only then.
       const bool fast = bC >= -60.f;
       if (!fast) {   // the same decision for the whole CTA
         const int h = t & 3;
@@ -888,6 +897,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       // unnormalised, so the shift cancels against Z), redone against the row maximum if
       // the spread is too large (see kShiftSpan)
       const float sl = bf16_lo(*reinterpret_cast<const uint32_t*>(qb + kmajor_off(row, 0, ROWS * 128))) * kLog2e;
+      const float sla = sl - lqa;
       float mq = -INFINITY, za = 0.f, zb = 0.f;
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 16; ++c8) {
@@ -899,7 +909,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) { x[2 * q] = bf16_lo(w4[q]); x[2 * q + 1] = bf16_hi(w4[q]); }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sl));
+        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sla));
         za += (x[0] + x[1]) + (x[2] + x[3]);
         zb += (x[4] + x[5]) + (x[6] + x[7]);
         st_chunk8(eqb, off, x);
@@ -913,7 +923,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if (__any_sync(0xffffffffu, redo)) {
         float zr = 0.f;
         if (redo) {
-          const float mql = mq * kLog2e;
+          const float mql = mq * kLog2e - lqa;
           za = 0.f;
           zb = 0.f;
 #pragma unroll 1
@@ -932,7 +942,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         zr += __shfl_xor_sync(0xffffffffu, zr, 1);
         if (redo) zq = zr;
       }
-      if (qh == 0) zq2[(c & 1) * 128 + row] = zq;
+      if (qh == 0) zq2[(c & 1) * 128 + row] = zq * iqa;
       // The q buffer is released twice per chunk: by the score MMA's commit, and by this
       // group once done with the raw q (factored mode) or by the readout's commit (exact
       // mode: the buffer then holds e^{b_i} e_q, the readout's A operand).
@@ -956,30 +966,49 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_before();
       mbar_arrive(feat);
 
-      // State for this chunk: the bf16 copy of alpha e^{m} S (MN-major B of the readout;
-      // e^{m} only in factored mode), then S <- e^{b_C} S in TMEM before the chunk's carry
-      // accumulates onto it (the previous carry and readout are done, above).
+      // State for this chunk: the bf16 copy of the readout's state (MN-major B operand),
+      // then S <- e^{b_C} S in TMEM before the chunk's carry accumulates onto it (the
+      // previous carry and readout are done, above).  Factored mode reads out e^{b_C} S,
+      // the rescaled state itself; exact mode reads out S (its q buffer holds e^{b_i} e_q).
+      // Either copy carries the part of alpha that the e_q tile does not.
       tc_fence_after();
       {
         const float dec = __expf(bC);
-        const float sbs = fast ? p.alpha * __expf(0.5f * bC) : p.alpha;
+        if (fast && copy_scale == 1.f) {   // the same for the whole CTA
 #pragma unroll 1
-        for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
-          float v[32];
-          tmem_ld32(lane_base + kColS + col, v);
-          tmem_wait_ld();
-          if (lrow < D) {
+          for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
+            float v[32];
+            tmem_ld32(lane_base + kColS + col, v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) {
-              float x[8];
+            for (int u = 0; u < 32; ++u) v[u] *= dec;
+            if (lrow < D) {
 #pragma unroll
-              for (int q = 0; q < 8; ++q) x[q] = sbs * v[u + q];
-              st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(lrow, ((col + u) & 63) >> 3), x);
+              for (int u = 0; u < 32; u += 8)
+                st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(lrow, ((col + u) & 63) >> 3), v + u);
             }
+            tmem_st32(lane_base + kColS + col, v);
           }
+        } else {
+          const float sc = fast ? copy_scale * dec : copy_scale;
+#pragma unroll 1
+          for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 16) {
+            float v[16];
+            tmem_ld16(lane_base + kColS + col, v);
+            tmem_wait_ld();
+            if (lrow < D) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] *= dec;
-          tmem_st32(lane_base + kColS + col, v);
+              for (int u = 0; u < 16; u += 8) {
+                float x[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) x[q] = sc * v[u + q];
+                st_chunk8(sbb, (uint32_t)((col + u) >> 6) * (D * 128) + sw128(lrow, ((col + u) & 63) >> 3), x);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] *= dec;
+            tmem_st16(lane_base + kColS + col, v);
+          }
         }
       }
       tmem_wait_st();
@@ -1015,6 +1044,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const int wq = warp, il = i - 16 * wq;
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
+    // the part of alpha that the e_q tile (and so the recurrent scores) does not carry
+    const float gscale = alpha / (alpha >= 0x1p-20f ? alpha : 1.f);
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     // state entering the segment, second half of the columns (the feature warps load the
@@ -1087,13 +1118,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_after();
       const bool fast = fast2[c & 1] != 0.f;
       // The tiles carry e_q unnormalised: P is scaled by Z and the output by 1/Z.  In
-      // factored mode P also carries e^{m - b_i} and the output e^{b_i - m}.
+      // factored mode P also carries e^{b_C - b_i} and the output e^{b_i - b_C}.
       const float zrow = zq2[(c & 1) * 128 + r];
       const float bi = bsh[i];
-      const float mrow = fast ? 0.5f * bsh[nv - 1] - bi : 0.f;
+      const float mrow = fast ? bsh[nv - 1] - bi : 0.f;
       const float coef = beta * zrow * __expf(mrow) / (la + lb);
       const float oscale = __expf(-mrow) / zrow;
-      const float gscale = fast ? alpha * __expf(-0.5f * bsh[nv - 1]) : 0.f;   // alpha e^{-m}
       // Probability tile over [previous | current] keys.  The recurrent tile covers the
       // same current keys (kk <= i) and multiplies the same values, so it is added to the
       // window tile's current half here: one P V product per half.  Group q5 holds the
@@ -1111,8 +1141,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const int kk = 16 * bb + u;
-            float gv = fast ? g[u] * gscale   // scores against e^{b_C - b_kk} / z_kk e_k; e^{b_i - m} in the epilogue
-                            : alpha * g[u] * (__expf(bi - bsh[kk]) * izk[kk]);
+            // factored: the scores already carry e^{b_C - b_kk} / z_kk; exact: e_q e_k scores
+            float gv = fast ? g[u] * gscale : g[u] * (gscale * __expf(bi - bsh[kk]) * izk[kk]);
             if (bb == wq) gv = kk <= i ? gv : 0.f;       // the diagonal block is causal
             s[u] += gv;
           }
