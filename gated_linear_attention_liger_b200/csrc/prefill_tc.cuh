@@ -170,10 +170,10 @@ __global__ void scan_kernel(DevParams p) {
   if (e >= (size_t)D * D) return;
   const SeqInfo si = p.seqs[seq];
   const int nsub = p.nsub;
-  // The sequence's sub-segment contributions in order, sixteen loads in flight at a
+  // The sequence's sub-segment contributions in order, 20 loads in flight at a
   // time; the state entering a segment is stored over its first sub-segment's slot
   // (after that slot has been read).
-  constexpr int kBatch = 16;
+  constexpr int kBatch = 20;
   const int n_units = si.n_seg * nsub;
   const size_t u0 = (size_t)si.first_seg * nsub;
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
