@@ -1,5 +1,6 @@
 /*
- * oracle.c -- plain, slow, fp64 CPU oracle of the Liger Attention forward pass.
+ * oracle.c -- plain, slow, fp64 CPU oracle of the Liger Attention forward pass
+ * (prefill and decode) and of the prefill's gradient.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * CPU-baseline leg of the benchmark may load this library.  The product
@@ -31,6 +32,10 @@
  *   - varlen: state and window restart at each sequence start.
  *   - initial_state seeds the recurrence only; the window starts at the first
  *     token of the call.
+ *
+ * The gradient has no formula on the pages (the linearisation fine-tune they
+ * describe trains through this layer): it is the reverse-mode derivative of the
+ * same token-by-token evaluation, written out step by step.
  *
  * Everything is evaluated token by token, exactly in the order of the
  * recurrence, in double precision.  Work is split over POSIX threads by
@@ -190,6 +195,213 @@ int oracle_prefill(const double* q, const double* k, const double* v, int B, int
     jobs[i].unit_begin = (int)((long)units * i / nthreads);
     jobs[i].unit_end = (int)((long)units * (i + 1) / nthreads);
     pthread_create(&th[i], NULL, prefill_worker, &jobs[i]);
+  }
+  for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+  free(jobs); free(th);
+  return 0;
+}
+
+/* ---- prefill backward ---------------------------------------------------- */
+
+/* log sigmoid(m), overflow-free on both sides (the same form as the gate). */
+static double log_sigmoid(double m) {
+  if (m >= 0.0) return -log1p(exp(-m));
+  return m - log1p(exp(m));
+}
+
+typedef struct {
+  const double *q, *k, *v, *s0, *dout, *dfs;
+  const int* cu;
+  int Hq, Hkv, T, d, w, gate_off;
+  double alpha;
+  double *dq, *dk, *dv, *ds0;
+  int unit_begin, unit_end;  /* units are (seq, kv head) pairs */
+} backward_job;
+
+/* One q head of one sequence: a forward sweep that keeps every state, then the
+ * reverse sweep.  dq of the head is written; dk and dv of its kv head are
+ * accumulated (the caller runs the heads of one kv head one after another). */
+static void backward_head(const backward_job* J, long t0, long t1, int seq, int h) {
+  const int d = J->d, Hq = J->Hq, Hkv = J->Hkv, w = J->w;
+  const int G = Hq / Hkv, kv = h / G;
+  const long len = t1 - t0;
+  const long dd = (long)d * d;
+  const double alpha = J->alpha, beta = 1.0 - J->alpha;
+  const double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+  /* Ss[i] = state after i tokens of the sequence (Ss[0] = initial state) */
+  double* Ss = (double*)malloc(sizeof(double) * dd * (len + 1));
+  double* dS = (double*)malloc(sizeof(double) * dd);
+  double* pk = (double*)malloc(sizeof(double) * d);
+  double* pq = (double*)malloc(sizeof(double) * d);
+  double* dpk = (double*)malloc(sizeof(double) * d);
+  double* dpq = (double*)malloc(sizeof(double) * d);
+  double* p = (double*)malloc(sizeof(double) * w);
+  double* dp = (double*)malloc(sizeof(double) * w);
+  if (J->s0) memcpy(Ss, J->s0 + ((long)seq * Hq + h) * dd, sizeof(double) * dd);
+  else memset(Ss, 0, sizeof(double) * dd);
+  for (long t = t0; t < t1; ++t) {
+    const double* kt = J->k + (t * Hkv + kv) * d;
+    const double* vt = J->v + (t * Hkv + kv) * d;
+    const double g = J->gate_off ? 1.0 : exp(oracle_log_gate(kt, d));
+    oracle_feature_map(kt, d, pk);
+    const double* prev = Ss + (t - t0) * dd;
+    double* cur = Ss + (t - t0 + 1) * dd;
+    for (int r = 0; r < d; ++r)
+      for (int c = 0; c < d; ++c) cur[r * d + c] = g * prev[r * d + c] + pk[r] * vt[c];
+  }
+
+  /* gradient of the final state comes from the loss's second term */
+  if (J->dfs) memcpy(dS, J->dfs + ((long)seq * Hq + h) * dd, sizeof(double) * dd);
+  else memset(dS, 0, sizeof(double) * dd);
+  for (long t = t1 - 1; t >= t0; --t) {
+    const double* qt = J->q + (t * Hq + h) * d;
+    const double* kt = J->k + (t * Hkv + kv) * d;
+    const double* vt = J->v + (t * Hkv + kv) * d;
+    const double* dot = J->dout + (t * Hq + h) * d;
+    double* dqt = J->dq + (t * Hq + h) * d;
+    double* dkt = J->dk + (t * Hkv + kv) * d;
+    double* dvt = J->dv + (t * Hkv + kv) * d;
+    const double* cur = Ss + (t - t0 + 1) * dd;
+    const double* prev = Ss + (t - t0) * dd;
+    oracle_feature_map(kt, d, pk);
+    oracle_feature_map(qt, d, pq);
+
+    /* read-out: out_t += alpha * phi(q_t) S_t */
+    for (int r = 0; r < d; ++r) {
+      double a = 0.0;
+      for (int c = 0; c < d; ++c) a += cur[r * d + c] * dot[c];
+      dpq[r] = alpha * a;
+    }
+    for (int r = 0; r < d; ++r)
+      for (int c = 0; c < d; ++c) dS[r * d + c] += alpha * pq[r] * dot[c];
+
+    /* update: S_t = g_t S_{t-1} + phi(k_t)^T v_t */
+    for (int r = 0; r < d; ++r) {
+      double a = 0.0;
+      for (int c = 0; c < d; ++c) a += dS[r * d + c] * vt[c];
+      dpk[r] = a;
+    }
+    for (int c = 0; c < d; ++c) {
+      double a = 0.0;
+      for (int r = 0; r < d; ++r) a += pk[r] * dS[r * d + c];
+      dvt[c] += a;
+    }
+    double dg = 0.0;
+    for (long e = 0; e < dd; ++e) dg += dS[e] * prev[e];
+    double m = 0.0;
+    for (int i = 0; i < d; ++i) m += kt[i];
+    m /= (double)d;
+    const double g = J->gate_off ? 1.0 : exp(log_sigmoid(m));
+    for (long e = 0; e < dd; ++e) dS[e] *= g;   /* now the gradient of S_{t-1} */
+
+    /* softmax feature maps: dx = phi (dphi - <dphi, phi>) */
+    double a = 0.0, b = 0.0;
+    for (int r = 0; r < d; ++r) { a += dpq[r] * pq[r]; b += dpk[r] * pk[r]; }
+    for (int r = 0; r < d; ++r) {
+      dqt[r] += pq[r] * (dpq[r] - a);
+      dkt[r] += pk[r] * (dpk[r] - b);
+    }
+    /* gate: g = sigmoid(mean k), dg/dm = sigmoid(m) sigmoid(-m) */
+    if (!J->gate_off) {
+      const double gm = dg * exp(log_sigmoid(m) + log_sigmoid(-m)) / (double)d;
+      for (int i = 0; i < d; ++i) dkt[i] += gm;
+    }
+
+    /* window branch: out_t += beta * sum_j p_j v_j, p = softmax_j(q_t.k_j / sqrt d) */
+    long j0 = t - w + 1;
+    if (j0 < t0) j0 = t0;
+    double mx = -INFINITY;
+    for (long j = j0; j <= t; ++j) {
+      const double* kj = J->k + (j * Hkv + kv) * d;
+      double s = 0.0;
+      for (int i = 0; i < d; ++i) s += qt[i] * kj[i];
+      s *= inv_sqrt_d;
+      p[j - j0] = s;
+      if (s > mx) mx = s;
+    }
+    double l = 0.0;
+    for (long j = j0; j <= t; ++j) { p[j - j0] = exp(p[j - j0] - mx); l += p[j - j0]; }
+    for (long j = j0; j <= t; ++j) p[j - j0] /= l;
+    double pdp = 0.0;
+    for (long j = j0; j <= t; ++j) {
+      const double* vj = J->v + (j * Hkv + kv) * d;
+      double s = 0.0;
+      for (int c = 0; c < d; ++c) s += dot[c] * vj[c];
+      dp[j - j0] = beta * s;
+      pdp += p[j - j0] * dp[j - j0];
+    }
+    for (long j = j0; j <= t; ++j) {
+      const double* kj = J->k + (j * Hkv + kv) * d;
+      double* dkj = J->dk + (j * Hkv + kv) * d;
+      double* dvj = J->dv + (j * Hkv + kv) * d;
+      const double pj = p[j - j0];
+      const double dsj = pj * (dp[j - j0] - pdp) * inv_sqrt_d;
+      for (int i = 0; i < d; ++i) {
+        dqt[i] += dsj * kj[i];
+        dkj[i] += dsj * qt[i];
+        dvj[i] += beta * pj * dot[i];
+      }
+    }
+  }
+  if (J->ds0) memcpy(J->ds0 + ((long)seq * Hq + h) * dd, dS, sizeof(double) * dd);
+  free(Ss); free(dS); free(pk); free(pq); free(dpk); free(dpq); free(p); free(dp);
+}
+
+static void* backward_worker(void* arg) {
+  const backward_job* J = (const backward_job*)arg;
+  const int G = J->Hq / J->Hkv;
+  for (int u = J->unit_begin; u < J->unit_end; ++u) {
+    const int seq = u / J->Hkv, kv = u % J->Hkv;
+    long t0, t1;
+    if (J->cu) { t0 = J->cu[seq]; t1 = J->cu[seq + 1]; }
+    else { t0 = (long)seq * J->T; t1 = t0 + J->T; }
+    for (int h = kv * G; h < (kv + 1) * G; ++h) backward_head(J, t0, t1, seq, h);
+  }
+  return NULL;
+}
+
+/*
+ * Gradients of the prefill with respect to q, k, v and the initial state, for
+ * the loss  L = sum(d_out * out) + sum(d_final_state * final_state).
+ * The pages give no backward pass (their linearisation fine-tune needs one);
+ * this is reverse-mode differentiation of the token-by-token evaluation above.
+ *   d_out [B, T, Hq, d]; d_final_state [n_seqs, Hq, d, d] or NULL (zero).
+ *   dq [B, T, Hq, d], dk and dv [B, T, Hkv, d]: written (zeroed first).
+ *   d_initial_state [n_seqs, Hq, d, d] or NULL.
+ * Layouts, cu_seqlens, w, alpha and gate_off as in oracle_prefill.  Memory:
+ * every state of a sequence is kept, len * d * d doubles per (sequence, head)
+ * in flight.  Returns 0, or -1 on a bad argument.
+ */
+int oracle_prefill_backward(const double* q, const double* k, const double* v, int B, int Hq,
+                            int Hkv, int T, int d, int w, double alpha,
+                            const double* initial_state, const int* cu_seqlens, int n_seqs,
+                            const double* d_out, const double* d_final_state, double* dq,
+                            double* dk, double* dv, double* d_initial_state, int gate_off,
+                            int nthreads) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || d < 1 || w < 1 || !d_out) return -1;
+  if (cu_seqlens) {
+    if (B != 1 || n_seqs < 1 || cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return -1;
+    for (int i = 0; i < n_seqs; ++i)
+      if (cu_seqlens[i + 1] < cu_seqlens[i]) return -1;
+  } else {
+    n_seqs = B;
+  }
+  memset(dq, 0, sizeof(double) * (size_t)B * T * Hq * d);
+  memset(dk, 0, sizeof(double) * (size_t)B * T * Hkv * d);
+  memset(dv, 0, sizeof(double) * (size_t)B * T * Hkv * d);
+  const int units = n_seqs * Hkv;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > units) nthreads = units;
+  backward_job base = {q, k, v, initial_state, d_out, d_final_state, cu_seqlens, Hq, Hkv, T, d,
+                       w, gate_off, alpha, dq, dk, dv, d_initial_state, 0, 0};
+  backward_job* jobs = (backward_job*)malloc(sizeof(backward_job) * nthreads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
+  for (int i = 0; i < nthreads; ++i) {
+    jobs[i] = base;
+    jobs[i].unit_begin = (int)((long)units * i / nthreads);
+    jobs[i].unit_end = (int)((long)units * (i + 1) / nthreads);
+    pthread_create(&th[i], NULL, backward_worker, &jobs[i]);
   }
   for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
   free(jobs); free(th);

@@ -1,4 +1,5 @@
-"""Python front end of the fp64 CPU oracle (``oracle.c``).
+"""Python front end of the fp64 CPU oracle (``oracle.c``): the prefill, its gradient, and
+the decode step.
 
 TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
 CPU-baseline leg are the only callers.  The product path never imports this
@@ -52,6 +53,11 @@ def _load():
             lib.oracle_decode.argtypes = [
                 _dp, _dp, _dp, _dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int]
+            lib.oracle_prefill_backward.restype = ctypes.c_int
+            lib.oracle_prefill_backward.argtypes = [
+                _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, _dp, _ip, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp,
+                ctypes.c_int, ctypes.c_int]
             lib.oracle_feature_map.restype = None
             lib.oracle_feature_map.argtypes = [_dp, ctypes.c_int, _dp]
             lib.oracle_log_gate.restype = ctypes.c_double
@@ -134,6 +140,44 @@ def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_
     if rc != 0:
         raise ValueError("oracle_prefill rejected its arguments")
     return out, fs, ring, pos
+
+
+def prefill_backward(q, k, v, d_out, w=64, alpha=0.5, initial_state=None, cu_seqlens=None,
+                     d_final_state=None, gate_off=False, nthreads=None):
+    """Gradients of L = sum(d_out * out) + sum(d_final_state * final_state) of the prefill.
+
+    Returns (dq, dk, dv, d_initial_state) with the shapes of q, k, v and [n, Hq, d, d]; the
+    last is the gradient with respect to the initial state (a zero state when none is given).
+    Arguments as in ``prefill``; d_out has the shape of out, d_final_state [n, Hq, d, d] or None.
+    """
+    lib = _load()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(d_out)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != (B, T, Hkv, d) or dout.shape != q.shape:
+        raise ValueError("prefill_backward: inconsistent shapes")
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        n = cu.shape[0] - 1
+    else:
+        cu = None
+        n = B
+    s0 = None if initial_state is None else _f64(initial_state)
+    dfs = None if d_final_state is None else _f64(d_final_state)
+    for name, a in (("initial_state", s0), ("d_final_state", dfs)):
+        if a is not None and a.shape != (n, Hq, d, d):
+            raise ValueError(f"prefill_backward: {name} must be [n, Hq, d, d]")
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    ds0 = np.zeros((n, Hq, d, d))
+    rc = lib.oracle_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, T, d, w, float(alpha), _ptr(s0), _ptr(cu, _ip), n,
+        _ptr(dout), _ptr(dfs), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds0), int(bool(gate_off)),
+        nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_prefill_backward rejected its arguments")
+    return dq, dk, dv, ds0
 
 
 def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthreads=None):
