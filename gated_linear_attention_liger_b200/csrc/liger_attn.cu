@@ -5,6 +5,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -74,6 +75,15 @@ liger_status cuda_check(const char* where) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A named NVTX range over one entry point, for profilers that attach to NVTX
+// (ncu --nvtx, Nsight Systems); with none attached the calls return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Which prefill kernel serves a call.
 enum class PrefillPath { kSimt, kTensorCore };
@@ -206,6 +216,7 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
                                 const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
                                 int32_t* pos_out, void* workspace, size_t workspace_bytes,
                                 void* stream) {
+  const NvtxRange range("liger_attn_prefill");
   g_last_error.clear();
   liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
   if (st != LIGER_OK) return st;
@@ -252,6 +263,7 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
 liger_status liger_attn_decode(const void* q, const void* k, const void* v, float* state,
                                void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                int d, int w, float alpha, liger_dtype dt, void* stream) {
+  const NvtxRange range("liger_attn_decode");
   g_last_error.clear();
   liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
   if (st != LIGER_OK) return st;
@@ -293,6 +305,7 @@ liger_status liger_attn_prefill_status(const void* workspace, size_t workspace_b
 liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void* v, float* state,
                                         void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                         int d, int w, float alpha, liger_dtype dt, void* stream) {
+  const NvtxRange range("liger_attn_decode_kvshared");
   g_last_error.clear();
   liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
   if (st != LIGER_OK) return st;
