@@ -211,6 +211,18 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_prefill_sample(target_s: float):
     """Times the fp64 oracle on a bounded sample of the prefill workload and returns
     (workload tokens/s, seconds, sample description, threads).  The sample is the first T_s
@@ -258,7 +270,7 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1))", "config": workload_config(),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthr, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -421,7 +433,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
         tps, secs, desc, nthr = oracle_prefill_sample(args.cpu_seconds)
         cpu = {"value": tps, "unit": "tokens/s", "cores": nthr, "kind": "oracle", "sample": desc,
-               "seconds": secs}
+               "seconds": secs, "cpu_model": cpu_model()}
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,

@@ -34,6 +34,7 @@ def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
     assert abs(line["ms_per_step"] - wl.tokens / line["value"] * 1e3) <= 1e-9 * line["ms_per_step"]
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert isinstance(cb["cpu_model"], str) and cb["cpu_model"]
     assert f"all {wl.B} sequences x {wl.Hq} q heads" in cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
