@@ -20,8 +20,10 @@ so that, with G = alpha dO V^T masked to j <= i and E the masked decay matrix,
 
 and d log g_t is the sum of d b_i over i >= t in the chunk; the gate then gives
 dk_t += d log g_t sigmoid(-m_t) / d.  The window branch's backward is the band-masked
-softmax attention backward.  This model evaluates those equations in numpy for one head and
-must reproduce the oracle's token-by-token gradient.
+softmax attention backward.  This model evaluates those equations in numpy for one head, in
+the three passes planned for the kernels (states entering the chunks; their gradients from the
+last chunk back; then every chunk on its own, in shuffled order), and must reproduce the
+oracle's token-by-token gradient.
 """
 import numpy as np
 import pytest
@@ -38,30 +40,40 @@ def log_sigmoid(m):
     return np.where(m >= 0, -np.log1p(np.exp(-np.abs(m))), m - np.log1p(np.exp(-np.abs(m))))
 
 
-def chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C):
-    """One head, one sequence: q, k, v, dout [T, d]; s0, dfs [d, d].  Returns dq, dk, dv, ds0."""
+def chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C, order_seed=None):
+    """One head, one sequence: q, k, v, dout [T, d]; s0, dfs [d, d].  Returns dq, dk, dv, ds0.
+
+    Three passes: (1) h_c, the state entering each chunk; (2) dh_c, the gradient of the state
+    entering each chunk, from the last chunk back; (3) each chunk's gradients from h_c and
+    dh_{c+1} alone, in any order (order_seed shuffles it)."""
     T, d = q.shape
     beta = 1.0 - alpha
     pq, pk = softmax_rows(q), softmax_rows(k)
     m = k.mean(axis=1)
     lg = log_sigmoid(m)
     starts = list(range(0, T, C))
-    states = [s0]                      # state entering each chunk
-    for c0 in starts:
-        n = min(C, T - c0)
-        b = np.cumsum(lg[c0:c0 + n])
-        S = states[-1]
-        states.append(np.exp(b[-1]) * S + (np.exp(b[-1] - b)[:, None] * pk[c0:c0 + n]).T @ v[c0:c0 + n])
+    spans = [slice(c0, min(c0 + C, T)) for c0 in starts]
+    bs = [np.cumsum(lg[sl]) for sl in spans]
+    # pass 1: h[c] enters chunk c, h[len] is the final state
+    h = [s0]
+    for sl, b in zip(spans, bs):
+        h.append(np.exp(b[-1]) * h[-1] + (np.exp(b[-1] - b)[:, None] * pk[sl]).T @ v[sl])
+    # pass 2: dh[c] is the gradient of h[c]; it needs only e^{b_C} and (e^{b} phi Q)^T (alpha dO)
+    dh = [None] * len(spans) + [dfs]
+    for ci in range(len(spans) - 1, -1, -1):
+        sl, b = spans[ci], bs[ci]
+        dh[ci] = np.exp(b[-1]) * dh[ci + 1] + (np.exp(b)[:, None] * pq[sl]).T @ (alpha * dout[sl])
+    # pass 3: per chunk, independent of the others
     dpq, dpk = np.zeros_like(q), np.zeros_like(k)
     dv = np.zeros_like(v)
     dlg = np.zeros(T)
-    dS = dfs.copy()
-    for ci in range(len(starts) - 1, -1, -1):
-        c0 = starts[ci]
-        n = min(C, T - c0)
-        sl = slice(c0, c0 + n)
-        S, Sn = states[ci], states[ci + 1]
-        b = np.cumsum(lg[sl])
+    order = list(range(len(spans)))
+    if order_seed is not None:
+        np.random.default_rng(order_seed).shuffle(order)
+    for ci in order:
+        sl, b = spans[ci], bs[ci]
+        n = b.shape[0]
+        S, Sn, dS = h[ci], h[ci + 1], dh[ci + 1]
         bC = b[-1]
         Pq, Pk, V, dO = pq[sl], pk[sl], v[sl], alpha * dout[sl]
         mask = np.tril(np.ones((n, n), dtype=bool))
@@ -76,7 +88,6 @@ def chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C):
               - ekey * np.sum((Pk @ dS) * V, axis=1))
         db[-1] += np.sum(dS * Sn)
         dlg[sl] = np.cumsum(db[::-1])[::-1]
-        dS = np.exp(bC) * dS + (eb[:, None] * Pq).T @ dO
     dq = pq * (dpq - np.sum(dpq * pq, axis=1, keepdims=True))
     dk = pk * (dpk - np.sum(dpk * pk, axis=1, keepdims=True))
     dk += (dlg * np.exp(log_sigmoid(-m)) / d)[:, None]
@@ -92,7 +103,7 @@ def chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C):
     dq += dsc @ k
     dk += dsc.T @ q
     dv += P.T @ dOs
-    return dq, dk, dv, dS
+    return dq, dk, dv, dh[0]
 
 
 @pytest.mark.parametrize("T,C,w,alpha,kb", [(23, 4, 5, 0.5, 0.0), (16, 8, 3, 0.8, 0.0),
@@ -106,7 +117,7 @@ def test_chunk_equations_reproduce_the_oracle_gradient(T, C, w, alpha, kb):
     s0 = 0.3 * rng.normal(size=(d, d))
     dout = rng.normal(size=(T, d))
     dfs = rng.normal(size=(d, d))
-    got = chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C)
+    got = chunked_backward(q, k, v, s0, dout, dfs, w, alpha, C, order_seed=T)
     ref = oracle.prefill_backward(q[None, :, None], k[None, :, None], v[None, :, None], dout[None, :, None],
                                   w=w, alpha=alpha, initial_state=s0[None, None], d_final_state=dfs[None, None])
     for name, a, r in zip(("dq", "dk", "dv", "d_initial_state"), got,
