@@ -210,6 +210,30 @@ size_t liger_attn_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, i
   return liger::tc::workspace_bytes(B, Hq, Hkv, (long)T, d, n);
 }
 
+liger_status liger_attn_prefill_plan(int B, int Hq, int Hkv, int T, int d, int n_seqs, int packed,
+                                     int* chunks_per_segment, int* max_segments,
+                                     int* state_subsegments, int* sm_count, size_t* plan_bytes) {
+  g_last_error.clear();
+  if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv)
+    return fail(LIGER_ERR_INVALID_ARG, "need B >= 1, T >= 0, Hq >= 1, Hkv >= 1, Hq %% Hkv == 0");
+  if (packed) {
+    if (B != 1 || n_seqs < 1)
+      return fail(LIGER_ERR_INVALID_ARG, "packed input needs B == 1 and n_seqs >= 1 (B=%d n_seqs=%d)", B, n_seqs);
+  } else if (n_seqs != B) {
+    return fail(LIGER_ERR_INVALID_ARG, "without packing n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
+  }
+  if (!liger::tc::supports(d) || (Hq / Hkv) % 2)
+    return fail(LIGER_ERR_UNSUPPORTED, "the general kernel takes these sizes (d=%d, Hq/Hkv=%d); it needs no plan",
+                d, Hq / Hkv);
+  const liger::tc::Plan pl = liger::tc::make_plan(B, Hq, Hkv, (long)T, d, n_seqs, packed != 0);
+  if (chunks_per_segment) *chunks_per_segment = pl.L;
+  if (max_segments) *max_segments = pl.n_seg_max;
+  if (state_subsegments) *state_subsegments = pl.nsub;
+  if (sm_count) *sm_count = liger::tc::num_sms();
+  if (plan_bytes) *plan_bytes = pl.total;
+  return LIGER_OK;
+}
+
 liger_status liger_attn_prefill(const void* q, const void* k, const void* v, void* out,
                                 float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
                                 float alpha, liger_dtype dt, const float* initial_state,

@@ -40,6 +40,8 @@ SIGNATURES = {
     "liger_attn_prefill_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                         _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "liger_attn_prefill_status": (_i, [_vp, ctypes.c_size_t]),
+    "liger_attn_prefill_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                     ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_size_t)]),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }
@@ -116,6 +118,19 @@ def _need_cuda(*ts):
 def prefill_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:
     return int(load().liger_attn_prefill_workspace_size(
         B, Hq, Hkv, T, d, n_seqs, LIGER_BF16 if dtype == torch.bfloat16 else LIGER_FP32))
+
+
+def prefill_plan(B, Hq, Hkv, T, d, n_seqs=None, packed: bool = False) -> dict:
+    """The tensor-core prefill's launch plan for these sizes (host only; see the header)."""
+    lib = load()
+    vals = [_i(), _i(), _i(), _i()]
+    nbytes = ctypes.c_size_t()
+    n = B if n_seqs is None else n_seqs
+    st = lib.liger_attn_prefill_plan(B, Hq, Hkv, T, d, n, int(bool(packed)), *(ctypes.byref(x) for x in vals),
+                                     ctypes.byref(nbytes))
+    _check(st)
+    return {"chunks_per_segment": vals[0].value, "max_segments": vals[1].value,
+            "state_subsegments": vals[2].value, "sm_count": vals[3].value, "plan_bytes": nbytes.value}
 
 
 def prefill(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seqlens=None,

@@ -71,6 +71,32 @@ size_t liger_attn_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, i
                                          liger_dtype dt);
 
 /*
+ * The launch plan the tensor-core prefill (bf16, d in {64, 128}, even
+ * Hq/Hkv, w = 64, no initial state) uses for these sizes.  Host only: no
+ * device work; the planner reads the current device's SM count, or assumes
+ * 148 when no device is present.  (The pages have no counterpart: the
+ * sequence split is this implementation's way of filling the GPU.)
+ *   B, Hq, Hkv, T, d, n_seqs  as for liger_attn_prefill; packed != 0 describes
+ *                a call with cu_seqlens (then B == 1 and n_seqs >= 1),
+ *                otherwise n_seqs must equal B.
+ *   chunks_per_segment  (out, nullable) segment length in 64-token chunks: one
+ *                chunk-kernel CTA per (segment, q-head pair); the length
+ *                minimises waves x (length + 1.5) at one CTA per SM.
+ *   max_segments        (out, nullable) the bound on segments the workspace holds.
+ *   state_subsegments   (out, nullable) sub-segments per segment in the state
+ *                pass (two CTAs per SM; minimises waves x (sub-length + 0.5)).
+ *   sm_count            (out, nullable) the SM count the plan assumed.
+ *   plan_bytes          (out, nullable) device workspace this plan uses (at most
+ *                liger_attn_prefill_workspace_size for the same sizes).
+ * Returns LIGER_ERR_INVALID_ARG for sizes the prefill rejects, and
+ * LIGER_ERR_UNSUPPORTED for sizes the tensor-core path does not take (the
+ * general kernel needs no plan); outputs are then left untouched.
+ */
+liger_status liger_attn_prefill_plan(int B, int Hq, int Hkv, int T, int d, int n_seqs, int packed,
+                                     int* chunks_per_segment, int* max_segments,
+                                     int* state_subsegments, int* sm_count, size_t* plan_bytes);
+
+/*
  * Prefill: runs the recurrence and the window over whole sequences.
  * Sources: the recurrence and the hybrid above (Paper-Notes page, sections
  * 统一的门控线性循环框架 and Liger Attention); the parallel-in-chunk,
