@@ -82,10 +82,11 @@ def prefill_algorithmic(wl=PREFILL):
 
 
 def decode_algorithmic(wl=DECODE, kvshared=False):
-    """Bytes of one decode step: state read + write, window ring read, q/k/v read, out write."""
+    """Bytes of one decode step: state read + write, window ring read, the new key and value
+    written into the ring, q/k/v read, out write."""
     esz = 2
     state = wl.B * (wl.Hkv if kvshared else wl.Hq) * wl.d * wl.d * 4 * 2
-    ring = wl.B * wl.Hkv * 2 * wl.w * wl.d * esz
+    ring = wl.B * wl.Hkv * 2 * wl.w * wl.d * esz + wl.B * wl.Hkv * 2 * wl.d * esz
     io = wl.B * (2 * wl.Hq + 2 * wl.Hkv) * wl.d * esz
     return state + ring + io
 

@@ -57,3 +57,15 @@ def test_oracle_sample_covers_whole_small_workload():
         bench.PREFILL = old
     assert tps > 0 and secs >= 0.2 and nthr >= 1
     assert f"first {wl.T} of {wl.T} tokens" in desc
+
+
+def test_algorithmic_work_matches_the_stated_figures():
+    """The roofline numerators: 339.7 MB and 47.4 GFLOP per Llama-3-8B prefill call, 286.8 MB per
+    decode step at B = 64 (state 268.4, ring 16.8, q/k/v/out and the ring slot 1.6)."""
+    b, f = bench.prefill_algorithmic()
+    assert abs(b / 1e6 - 339.7) < 0.05 and abs(f / 1e9 - 47.4) < 0.05
+    assert abs(bench.decode_algorithmic() / 1e6 - 286.8) < 0.05
+    shared = bench.decode_algorithmic(bench.DECODE_KV, kvshared=True)
+    wl = bench.DECODE_KV
+    assert shared == (wl.B * wl.Hkv * wl.d * wl.d * 8 + wl.B * wl.Hkv * 2 * (wl.w + 1) * wl.d * 2
+                      + wl.B * (2 * wl.Hq + 2 * wl.Hkv) * wl.d * 2)
