@@ -888,8 +888,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       if ((t & 3) == 0) izk2[(c & 1) * 64 + j] = iz;
       if (t == 0) fast2[c & 1] = fast ? 1.f : 0.f;
 
-      // queries: e_q = exp(q - max_d q) per row (bf16, not divided by Z = sum_d e_q: the
-      // window warps fold Z into P and 1/Z into the output); two threads per row
+      // queries: e_q' = a exp(q - q_0) per row (bf16, with the branch weight a above; not
+      // divided by Z = sum_d e_q: the window warps fold Z into P and 1/Z into the output);
+      // two threads per row
       const int row = t >> 1, qh = t & 1;
       mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
       if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));   // e_q tile and state copy free
