@@ -572,12 +572,12 @@ struct ChunkSmem {
   static constexpr uint32_t QB = ROWS * D * 2;    // q tile (two heads): raw q, then scaled phi(q)
   static constexpr uint32_t KV = C * D * 2;       // one chunk of k or v
   static constexpr uint32_t Q0 = 0;
-  static constexpr uint32_t EQ = Q0 + QB;         // e_q = exp(q - max), bf16
+  static constexpr uint32_t EQ = Q0 + QB;         // e_q' = alpha exp(q - q_0), bf16
   static constexpr uint32_t K0 = EQ + QB;         // 2 key slots, laid out [64-d block][slot][64 rows]
   static constexpr uint32_t V0 = K0 + 2 * KV;     // 3 value slots
-  static constexpr uint32_t PK = V0 + 3 * KV;     // phi(k)
+  static constexpr uint32_t PK = V0 + 3 * KV;     // e_k, unnormalised (exact-decay chunks only)
   static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
-  static constexpr uint32_t SB = KT + KV;         // bf16 copy of the entering state
+  static constexpr uint32_t SB = KT + KV;         // bf16 copy of the readout's state
   static constexpr uint32_t SMALL = SB + D * D * 2;
   static constexpr uint32_t SMALL_BYTES = 4096;
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
