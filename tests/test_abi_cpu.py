@@ -113,3 +113,36 @@ def test_workspace_size_is_zero_for_rejected_sizes(lib):
     assert lib.liger_attn_prefill_workspace_size(0, 32, 8, 128, 128, 0, 0) == 0
     assert lib.liger_attn_prefill_workspace_size(1, 3, 2, 128, 128, 1, 0) == 0
     assert lib.liger_attn_prefill_workspace_size(1, 4, 2, 128, 128, 1, 1) == 0  # fp32 needs none
+
+
+def test_binding_refuses_host_tensors(lib):
+    """No CPU fallback: host tensors are an error, not a slow path."""
+    import torch
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.prefill(q, kv, kv)
+    with pytest.raises(ValueError, match="CUDA"):
+        ops.decode(q[:, 0], kv[:, 0], kv[:, 0], torch.zeros(1, 2, 64, 64), torch.zeros(1, 1, 2, 64, 64),
+                   torch.zeros(1, dtype=torch.int32))
+
+
+def test_missing_library_raises():
+    saved = ops._lib
+    ops._lib = None
+    try:
+        with pytest.raises(FileNotFoundError, match="no CPU fallback"):
+            ops.load(os.path.join(os.path.dirname(HEADER), "no_such_library.so"))
+    finally:
+        ops._lib = saved
+
+
+def test_package_never_imports_the_oracle():
+    """The oracle is test infrastructure: no module or source of the package refers to it."""
+    pkg = os.path.join(os.path.dirname(os.path.dirname(HEADER)), "gated_linear_attention_liger_b200")
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(root, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), f
+                assert "liboracle" not in text and "oracle_prefill" not in text, f
