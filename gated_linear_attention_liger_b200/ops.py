@@ -110,9 +110,27 @@ def _stream_ptr(stream) -> ctypes.c_void_p:
 
 
 def _need_cuda(*ts):
+    ref = None
     for t in ts:
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
+        if ref is None:
+            ref = t.device
+        elif t.device != ref:
+            raise ValueError(f"tensors must be on one device ({ref} and {t.device})")
+
+
+def _expect(t, name, shape, dtype):
+    """The library sees only pointers: shapes and dtypes are checked here, so that a wrong
+    output buffer is an error instead of an out-of-bounds write."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
 def prefill_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:
@@ -143,10 +161,22 @@ def prefill(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seq
     cu_seqlens: int32 CUDA tensor of n+1 offsets (B must be 1).
     """
     lib = load()
-    _need_cuda(q, k, v, initial_state, cu_seqlens)
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, T, Hq, d] and k, v [B, T, Hkv, d]")
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
+    _expect(k, "k", (B, T, Hkv, d), q.dtype)
+    _expect(v, "v", (B, T, Hkv, d), q.dtype)
+    if cu_seqlens is not None and (cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2
+                                   or cu_seqlens.dtype != torch.int32):
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of n + 1 offsets")
     n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    _expect(initial_state, "initial_state", (n, Hq, d, d), torch.float32)
+    _expect(out, "out", (B, T, Hq, d), q.dtype)
+    _expect(final_state, "final_state", (n, Hq, d, d), torch.float32)
+    _expect(ring, "ring", (n, Hkv, 2, w, d), q.dtype)
+    _expect(pos, "pos", (n,), torch.int32)
+    _need_cuda(q, k, v, initial_state, cu_seqlens, out, final_state, ring, pos, workspace)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -171,6 +201,22 @@ def prefill(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seq
     return out, final_state
 
 
+def _check_decode(q, k, v, state, ring, pos, out, per_head: bool):
+    if q.dim() != 3 or k.dim() != 3 or ring.dim() != 5:
+        raise ValueError("q must be [B, Hq, d], k and v [B, Hkv, d], ring [B, Hkv, 2, w, d]")
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    w = ring.shape[3]
+    _expect(k, "k", (B, Hkv, d), q.dtype)
+    _expect(v, "v", (B, Hkv, d), q.dtype)
+    _expect(state, "state", (B, Hq if per_head else Hkv, d, d), torch.float32)
+    _expect(ring, "ring", (B, Hkv, 2, w, d), q.dtype)
+    _expect(pos, "pos", (B,), torch.int32)
+    _expect(out, "out", (B, Hq, d), q.dtype)
+    _need_cuda(q, k, v, state, ring, pos, out)
+    return B, Hq, Hkv, d, w
+
+
 def decode(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None):
     """One Liger Attention decode step; updates state, ring and pos in place.
 
@@ -178,10 +224,7 @@ def decode(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None)
     [B, Hkv, 2, w, d]; pos [B] int32.  Returns out [B, Hq, d].
     """
     lib = load()
-    _need_cuda(q, k, v, state, ring, pos)
-    B, Hq, d = q.shape
-    Hkv = k.shape[1]
-    w = ring.shape[3]
+    B, Hq, Hkv, d, w = _check_decode(q, k, v, state, ring, pos, out, per_head=True)
     if out is None:
         out = torch.empty_like(q)
     st = lib.liger_attn_decode(
@@ -198,10 +241,7 @@ def decode_kvshared(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, str
     prefill leaves them); moves G = Hq/Hkv times less state per step.
     """
     lib = load()
-    _need_cuda(q, k, v, state, ring, pos)
-    B, Hq, d = q.shape
-    Hkv = k.shape[1]
-    w = ring.shape[3]
+    B, Hq, Hkv, d, w = _check_decode(q, k, v, state, ring, pos, out, per_head=False)
     if out is None:
         out = torch.empty_like(q)
     st = lib.liger_attn_decode_kvshared(

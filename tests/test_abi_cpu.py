@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from gated_linear_attention_liger_b200 import build as libbuild
 from gated_linear_attention_liger_b200 import ops
@@ -123,8 +124,8 @@ def test_binding_refuses_host_tensors(lib):
     with pytest.raises(ValueError, match="CUDA"):
         ops.prefill(q, kv, kv)
     with pytest.raises(ValueError, match="CUDA"):
-        ops.decode(q[:, 0], kv[:, 0], kv[:, 0], torch.zeros(1, 2, 64, 64), torch.zeros(1, 1, 2, 64, 64),
-                   torch.zeros(1, dtype=torch.int32))
+        ops.decode(q[:, 0], kv[:, 0], kv[:, 0], torch.zeros(1, 2, 64, 64),
+                   torch.zeros(1, 1, 2, 64, 64, dtype=torch.bfloat16), torch.zeros(1, dtype=torch.int32))
 
 
 def test_missing_library_raises():
@@ -146,3 +147,74 @@ def test_package_never_imports_the_oracle():
                 text = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), f
                 assert "liboracle" not in text and "oracle_prefill" not in text, f
+
+
+def _t(*shape, dtype=torch.bfloat16):
+    return torch.zeros(*shape, dtype=dtype)
+
+
+def test_binding_checks_shapes_before_the_library_sees_pointers(lib):
+    """A wrong output buffer must be an error, not an out-of-bounds write on the device."""
+    q, kv = _t(2, 70, 4, 64), _t(2, 70, 2, 64)
+    bad = [
+        dict(k=_t(2, 70, 3, 64)),                                    # Hq % Hkv aside, k != v shape
+        dict(out=_t(2, 70, 4, 32)),
+        dict(out=_t(2, 70, 4, 64, dtype=torch.float32)),
+        dict(final_state=_t(2, 4, 64, 64, dtype=torch.bfloat16)),
+        dict(final_state=_t(1, 4, 64, 64, dtype=torch.float32)),
+        dict(ring=_t(2, 2, 2, 32, 64), return_ring=True),
+        dict(pos=_t(2, dtype=torch.int64), return_ring=True),
+        dict(initial_state=_t(2, 4, 64, 64)),
+    ]
+    for kw in bad:
+        args = dict(k=kv, v=kv)
+        args.update(kw)
+        with pytest.raises(ValueError, match="shape|must be"):
+            ops.prefill(q, args.pop("k"), args.pop("v"), **args)
+    qd, kd = _t(3, 8, 128), _t(3, 2, 128)
+    ring, pos = _t(3, 2, 2, 64, 128), _t(3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="state must have shape"):
+        ops.decode(qd, kd, kd, _t(3, 2, 128, 128, dtype=torch.float32), ring, pos)   # per-head needs Hq
+    with pytest.raises(ValueError, match="state must have shape"):
+        ops.decode_kvshared(qd, kd, kd, _t(3, 8, 128, 128, dtype=torch.float32), ring, pos)
+    with pytest.raises(ValueError, match="pos must be"):
+        ops.decode(qd, kd, kd, _t(3, 8, 128, 128, dtype=torch.float32), ring, _t(3, dtype=torch.int64))
+    with pytest.raises(ValueError, match="out must have shape"):
+        ops.decode(qd, kd, kd, _t(3, 8, 128, 128, dtype=torch.float32), ring, pos, out=_t(3, 2, 128))
+
+
+@pytest.mark.parametrize("call", [
+    # the argument shapes the GPU tests, the smoke check and the benchmark pass: valid, so the
+    # only complaint on a host without tensors on a device is the device check
+    dict(kind="prefill", q=(2, 8192, 32, 128), kv=(2, 8192, 8, 128), out=True, fs=2, ws=True),
+    dict(kind="prefill", q=(1, 270, 4, 128), kv=(1, 270, 1, 128), cu=6, ring=5, pos=5),
+    dict(kind="prefill", q=(2, 0, 4, 64), kv=(2, 0, 2, 64), s0=2, ring=2, pos=2),
+    dict(kind="prefill", q=(1, 150, 4, 128), kv=(1, 150, 2, 128), dtype=torch.float32, s0=1),
+    dict(kind="decode", q=(3, 8, 64), kv=(3, 2, 64), state=8, w=16),
+    dict(kind="decode", q=(64, 32, 128), kv=(64, 8, 128), state=32, w=64, out=True),
+    dict(kind="decode_kvshared", q=(256, 32, 128), kv=(256, 8, 128), state=8, w=64, out=True),
+])
+def test_valid_call_shapes_reach_the_device_check(lib, call):
+    dt = call.get("dtype", torch.bfloat16)
+    q, kv = _t(*call["q"], dtype=dt), _t(*call["kv"], dtype=dt)
+    with pytest.raises(ValueError, match="CUDA"):
+        if call["kind"] == "prefill":
+            B, T, Hq, d = call["q"]
+            Hkv = call["kv"][2]
+            n = call.get("cu", B + 1) - 1 if "cu" in call else B
+            ops.prefill(
+                q, kv, kv,
+                out=_t(B, T, Hq, d, dtype=dt) if call.get("out") else None,
+                final_state=_t(n, Hq, d, d, dtype=torch.float32) if call.get("fs") else None,
+                initial_state=_t(n, Hq, d, d, dtype=torch.float32) if call.get("s0") else None,
+                cu_seqlens=_t(n + 1, dtype=torch.int32) if "cu" in call else None,
+                ring=_t(n, Hkv, 2, 64, d, dtype=dt) if call.get("ring") else None,
+                pos=_t(n, dtype=torch.int32) if call.get("pos") else None,
+                return_ring=bool(call.get("ring")),
+                workspace=_t(16, dtype=torch.uint8) if call.get("ws") else None)
+        else:
+            B, Hq, d = call["q"]
+            Hkv = call["kv"][1]
+            fn = ops.decode if call["kind"] == "decode" else ops.decode_kvshared
+            fn(q, kv, kv, _t(B, call["state"], d, d, dtype=torch.float32), _t(B, Hkv, 2, call["w"], d, dtype=dt),
+               _t(B, dtype=torch.int32), out=_t(B, Hq, d, dtype=dt) if call.get("out") else None)
