@@ -3,16 +3,21 @@
 
 Workload (Llama-3-8B attention shape, synthetic seeded N(0,1) data):
   prefill: B=2, T=8192, Hq=32, Hkv=8, d=128, bf16, w=64, alpha=0.5, fp32 final state
-  decode:  B=64, Hq=32, Hkv=8, d=128 after a 1024-token prefill; steps captured in a CUDA graph
+  decode:  B=64, Hq=32, Hkv=8, d=128 after a 1024-token prefill; 1000 steps captured in a CUDA graph
   shared-state decode (one state per kv head): B=256, same shape
+The Llama-3.2-1B prefill (B=4, T=2048, d=64) and the long packed prefill (4 sequences,
+32768 tokens, d=128) are timed the same way and reported under "llama1b_prefill" and
+"long_varlen".
 
 One step = one prefill call over the whole batch (the headline `value`,
 tokens/s); the decode loops are timed in the same run and reported under
-"decode" and "decode_kvshared".  Inputs are larger than L2 (q, k, v 201 MB;
-decode states 268 MB per head at B=64 and 134 MB per kv head at B=256), so no
-L2 flush is needed between iterations.  Multi-GPU: one process per GPU,
-every rank runs the same per-GPU workload (weak scaling, no collective on the
-data path); times are the max over ranks.
+"decode" and "decode_kvshared".  The 8B and long prefill inputs and the decode
+states are larger than L2 (q, k, v 201 MB; decode states 268 MB per head at
+B=64 and 134 MB per kv head at B=256), so no L2 flush is needed between their
+iterations; the 1B prefill's 86 MB would fit, so an L2-sized buffer is written
+between its timed calls (outside the events that time the chunk pass).
+Multi-GPU: one process per GPU, every rank runs the same per-GPU workload (weak
+scaling, no collective on the data path); times are the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -37,6 +42,8 @@ from gated_linear_attention_liger_b200 import inputs  # noqa: E402
 
 METRIC = "prefill tokens/s & decode tokens/s (8B attn shape), % of roofline"
 PREFILL = inputs.WORKLOADS["llama8b_prefill"]
+PREFILL_1B = inputs.WORKLOADS["llama1b_prefill"]
+PREFILL_LONG = inputs.WORKLOADS["long_varlen"]
 DECODE = inputs.WORKLOADS["llama8b_decode"]
 DECODE_KV = inputs.WORKLOADS["llama8b_decode_kvshared"]
 L2_BYTES = 126 * 2 ** 20
@@ -79,6 +86,25 @@ def prefill_algorithmic(wl=PREFILL):
     flops = tok * (wl.Hq * 2 * wl.d ** 2 + wl.Hq * 4 * wl.d * (C + 1) / 2 + wl.Hkv * 2 * wl.d ** 2
                    + wl.Hq * 4 * wl.w * wl.d)
     return bytes_, flops
+
+
+def exact_decay_chunks(wl, k, threshold=-60.0):
+    """(chunk, kv head) pairs whose total log gate lies below `threshold`: the prefill's chunk
+    pass evaluates their decay without factoring it at the chunk end (a slower mode).  Chunks
+    are 64-token blocks counted from each sequence start.  A statistic of the input for the
+    report, computed here in numpy from the gate's definition (sigmoid of the key's mean)."""
+    kk = k.float().numpy().astype(np.float64)   # [B, T, Hkv, d]
+    cu = wl.cu_seqlens
+    seqs = [kk[0, a:b] for a, b in zip(cu[:-1], cu[1:])] if cu else [kk[b] for b in range(wl.B)]
+    total = exact = 0
+    for ks in seqs:
+        m = ks.mean(-1)                                                   # [len, Hkv]
+        lg = np.minimum(m, 0.0) - np.log1p(np.exp(-np.abs(m)))            # log sigmoid(m)
+        for c0 in range(0, ks.shape[0], 64):
+            bc = lg[c0:c0 + 64].sum(0)
+            total += bc.size
+            exact += int((bc < threshold).sum())
+    return exact, total
 
 
 def decode_algorithmic(wl=DECODE, kvshared=False):
@@ -312,57 +338,12 @@ def run_ours(args, world, rank, local):
 
     # ---------------- prefill
     wl = PREFILL
-    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
-    out = torch.empty_like(q)
-    fs = torch.empty(wl.n_seqs, wl.Hq, wl.d, wl.d, device=dev, dtype=torch.float32)
-    ws_n = ops.prefill_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.n_seqs)
-    ws = torch.empty(max(ws_n, 1), device=dev, dtype=torch.uint8)
-
-    def prefill_call():
-        ops.prefill(q, k, v, alpha=wl.alpha, w=wl.w, out=out, final_state=fs, workspace=ws,
-                    stream=stream)
-
-    torch.cuda.synchronize()
-    for _ in range(args.warmup):
-        prefill_call()
-    ks = timing_events(args.steps, stream)
-    ke = timing_events(args.steps, stream)
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    stream.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    launches0 = ops.kernel_launches()
-    w0 = time.perf_counter()
-    t_start.record(stream)
-    for i in range(args.steps):
-        prefill_call()
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    windows.append((w0, time.perf_counter()))
-    barrier(world)
-    prefill_launches = ops.kernel_launches() - launches0
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-    ms_step = ms_total / args.steps
-    # the chunk kernel's own time, from events around it in a second pass (the events
-    # serialise its launch, so the step time above is taken without them)
-    w1 = time.perf_counter()
-    for i in range(args.steps):
-        ops.set_timing_events(ks[i], ke[i])
-        prefill_call()
-    ops.set_timing_events(None, None)
-    torch.cuda.synchronize()
-    windows.append((w1, time.perf_counter()))
-    barrier(world)
-    k_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ks, ke)), world, dev)
-    value = weak_scaling_value(wl.tokens, world, ms_step)
-    alg_bytes, alg_flops = prefill_algorithmic(wl)
-    achieved = alg_bytes / (k_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                "kernel": "prefill chunk pass", "kernel_ms": k_ms,
-                "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
-                "tensor_frac": alg_flops / (k_ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
-                "peak_source": pk["source"], "frac_of": f"{pk['source']} HBM copy bandwidth"}
+    res8 = time_prefill(wl, args, world, dev, stream, pk, windows)
+    q, k, v, out, fs, ws = res8.pop("_tensors")
+    value = weak_scaling_value(wl.tokens, world, res8["ms_per_step"])
+    ms_step = res8["ms_per_step"]
+    prefill_launches = res8["gpu_launches"]
+    roofline = res8["roofline"]
     roofline["traffic"] = measured_traffic("chunk_kernel<128>")
 
     # ---------------- e2e: host buffers, copies inside the timed region
@@ -424,6 +405,15 @@ def run_ours(args, world, rank, local):
         del hq, hk, hv, ho, hfs, bufs
     del q, k, v, out, ws
 
+    # ---------------- the other prefill workloads (1B shape, long packed sequences)
+    others = {}
+    if args.only is None or args.only == "prefill":
+        for owl, flush in ((PREFILL_1B, True), (PREFILL_LONG, False)):
+            r = time_prefill(owl, args, world, dev, stream, pk, windows, flush_l2=flush)
+            r.pop("_tensors")
+            r["roofline"]["traffic"] = measured_traffic(f"chunk_kernel<{owl.d}>@{owl.name}")
+            others[owl.name] = r
+
     # ---------------- decode
     dec = None if args.only == "prefill" else run_decode(args, world, dev, stream, pk, windows)
     dec_kv = None if args.only == "prefill" else run_decode(args, world, dev, stream, pk, windows, kvshared=True)
@@ -441,10 +431,104 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1), Llama-3-8B attention shapes)",
-            "config": workload_config(), "roofline": roofline, "decode": dec, "decode_kvshared": dec_kv, "e2e": e2e,
+            "config": workload_config(), "roofline": roofline, "prefill_call": res8["call"],
+            "llama1b_prefill": others.get("llama1b_prefill"), "long_varlen": others.get("long_varlen"),
+            "decode": dec, "decode_kvshared": dec_kv, "e2e": e2e,
             "gpu_launches": prefill_launches, "clocks": clocks, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+
+
+def time_prefill(wl, args, world, dev, stream, pk, windows, flush_l2=False):
+    """Times `args.steps` prefill calls of workload `wl` (after `args.warmup` untimed ones) and,
+    in a second pass, the chunk kernel alone with CUDA events the library records around it on
+    the call's stream.  With flush_l2, a buffer larger than L2 is written before every call
+    (between the step events, so the step time then includes it: the kernel time does not)."""
+    from gated_linear_attention_liger_b200 import ops
+    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
+    cu = None if wl.cu_seqlens is None else torch.tensor(wl.cu_seqlens, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    fs = torch.empty(wl.n_seqs, wl.Hq, wl.d, wl.d, device=dev, dtype=torch.float32)
+    ws_n = ops.prefill_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.n_seqs)
+    ws = torch.empty(max(ws_n, 1), device=dev, dtype=torch.uint8)
+    flush = torch.empty(2 * L2_BYTES // 4, device=dev, dtype=torch.float32) if flush_l2 else None
+
+    def call():
+        if flush is not None:
+            with torch.cuda.stream(stream):
+                flush.fill_(1.0)
+        ops.prefill(q, k, v, alpha=wl.alpha, w=wl.w, cu_seqlens=cu, out=out, final_state=fs, workspace=ws,
+                    stream=stream)
+
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        call()
+    ks = timing_events(args.steps, stream)
+    ke = timing_events(args.steps, stream)
+    cs = timing_events(args.steps, stream)
+    ce = timing_events(args.steps, stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = ops.kernel_launches()
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        if flush is not None:   # time each call alone, without the flush in front of it
+            with torch.cuda.stream(stream):
+                flush.fill_(1.0)
+            cs[i].record(stream)
+            ops.prefill(q, k, v, alpha=wl.alpha, w=wl.w, cu_seqlens=cu, out=out, final_state=fs, workspace=ws,
+                        stream=stream)
+            ce[i].record(stream)
+        else:
+            call()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    launches = ops.kernel_launches() - launches0
+    if flush is not None:
+        ms_step = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(cs, ce)), world, dev)
+    else:
+        ms_step = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
+    # the chunk kernel's own time, from events around it in a second pass (the events
+    # serialise its launch, so the step time above is taken without them)
+    w1 = time.perf_counter()
+    for i in range(args.steps):
+        ops.set_timing_events(ks[i], ke[i])
+        call()
+    ops.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    windows.append((w1, time.perf_counter()))
+    barrier(world)
+    k_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ks, ke)), world, dev)
+    alg_bytes, alg_flops = prefill_algorithmic(wl)
+    achieved = alg_bytes / (k_ms * 1e-3) / 1e9
+    res = {
+        "metric": f"prefill tokens/s ({wl.name})", "value": weak_scaling_value(wl.tokens, world, ms_step),
+        "unit": "tokens/s", "ms_per_step": ms_step, "gpu_launches": launches,
+        "workload": {"B": wl.B, "T": wl.T, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "w": wl.w,
+                     "alpha": wl.alpha, "seqlens": list(wl.seqlens) or None,
+                     "l2": "L2-sized buffer written before each timed call" if flush_l2 else
+                           "inputs larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "prefill chunk pass", "kernel_ms": k_ms,
+                     "algorithmic_bytes": alg_bytes, "algorithmic_flops": alg_flops,
+                     "tensor_frac": alg_flops / (k_ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
+                     "peak_source": pk["source"], "frac_of": f"{pk['source']} HBM copy bandwidth"},
+        # the whole call (every kernel of it) against the same roofline
+        "call": {"ms": ms_step, "achieved": alg_bytes / (ms_step * 1e-3) / 1e9,
+                 "frac": alg_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"]},
+    }
+    if wl.key_bias_std or wl.cu_seqlens:
+        ex, tot = exact_decay_chunks(wl, k.cpu())
+        res["exact_decay_chunks"] = {"count": ex, "of": tot,
+                                     "note": "(chunk, kv head) pairs with total log gate < -60"}
+    res["_tensors"] = (q, k, v, out, fs, ws)
+    return res
 
 
 def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
@@ -494,12 +578,12 @@ def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
     except Exception:
         kernel_events = False
 
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, min(args.warmup, 3))):
         graph.replay()
     torch.cuda.synchronize()
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = max(1, args.steps // 10)
+    reps = 2
     w0 = time.perf_counter()
     k_ms = []
     with torch.cuda.stream(stream):
@@ -525,8 +609,47 @@ def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
     alg = decode_algorithmic(wl, kvshared)
     achieved = alg / (kms * 1e-3) / 1e9
     del graph, tgraph
+
+    # end to end through the public call: every step's q, k, v copied in from pinned host
+    # memory and its output copied back, on copy streams that overlap the compute stream
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (dq, dk, dv))
+        ho = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(n_graph)]
+        ev_c = [torch.cuda.Event() for _ in range(n_graph)]
+        torch.cuda.synchronize()
+        barrier(world)
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(s_in)
+        stream.wait_event(ea)
+        with torch.cuda.stream(s_in):
+            for s_ in range(n_graph):
+                dq[s_].copy_(hq[s_], non_blocking=True)
+                dk[s_].copy_(hk[s_], non_blocking=True)
+                dv[s_].copy_(hv[s_], non_blocking=True)
+                ev_in[s_].record(s_in)
+        for s_ in range(n_graph):
+            stream.wait_event(ev_in[s_])
+            step_fn(dq[s_], dk[s_], dv[s_], state, ring, pos, alpha=wl.alpha, out=dout[s_], stream=stream)
+            ev_c[s_].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[s_])
+                ho[s_].copy_(dout[s_], non_blocking=True)
+        s_out.wait_event(ev_c[-1])
+        eb.record(s_out)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(ea.elapsed_time(eb) / n_graph, world, dev)
+        e2e = {"value": world * wl.B / (e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e_ms,
+               "steps": n_graph,
+               "h2d_bytes_per_step": sum(t[0].numel() * t.element_size() for t in (hq, hk, hv)),
+               "d2h_bytes_per_step": ho[0].numel() * ho.element_size(),
+               "pipeline": "per step: q, k, v copied in, one decode call, out copied back; copies on "
+                           "two streams beside the compute stream; states stay on the device"}
+        del hq, hk, hv, ho
     name = f"decode tokens/s (8B attn shape, B={wl.B}" + (", one state per kv head)" if kvshared else ")")
-    return {"metric": name, "value": world * wl.B / (ms_step * 1e-3),
+    return {"metric": name, "value": world * wl.B / (ms_step * 1e-3), "e2e": e2e,
             "unit": "tokens/s", "ms_per_step": ms_step, "graph_steps": n_graph, "replays": reps,
             "gpu_launches": per_graph_launches * reps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -544,7 +667,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-steps", type=int, default=200, help="decode steps per captured graph")
+    ap.add_argument("--decode-steps", type=int, default=1000, help="decode steps per captured graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU baseline")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling); the JSON line is then partial")

@@ -7,6 +7,25 @@
 
 namespace liger {
 
+// Diagnostic options, read from the environment once, when the library is
+// loaded (later changes to the environment have no effect):
+//   LIGER_PREFILL_PATH=general   every prefill takes the general (CUDA-core) kernel
+//   LIGER_WAIT_LIMIT_NS=<n>      give-up time of each bounded wait in the
+//                                tensor-core prefill (default 2 s)
+//   LIGER_TEST_INJECT_STALL=<n>  the first n tensor-core prefill calls of the
+//                                process withhold one MMA completion, so that a
+//                                bounded wait runs out (exercises failure
+//                                detection without a fault); later calls run
+//                                normally
+struct Options {
+  bool force_general_prefill;
+  unsigned long long wait_limit_ns;   // 0: the kernel's default
+  long inject_stall_calls;
+};
+const Options& options();
+// True for the first options().inject_stall_calls calls (thread-safe).
+bool take_injected_stall();
+
 // Storage type <-> fp32.
 template <typename T> struct io;
 template <> struct io<float> {

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -90,8 +91,7 @@ enum class PrefillPath { kSimt, kTensorCore };
 
 PrefillPath choose_prefill_path(long ntok, int Hq, int Hkv, int d, int w, liger_dtype dt,
                                 const float* initial_state) {
-  const char* force = std::getenv("LIGER_PREFILL_PATH");
-  if (force && std::strcmp(force, "simt") == 0) return PrefillPath::kSimt;
+  if (liger::options().force_general_prefill) return PrefillPath::kSimt;
   if (ntok > 0 && dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && initial_state == nullptr &&
       liger::tc::supports(d))
     return PrefillPath::kTensorCore;
@@ -185,8 +185,40 @@ liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n
 }  // namespace
 
 namespace liger {
+
+namespace {
+Options read_options() {
+  Options o{};
+  const char* path = std::getenv("LIGER_PREFILL_PATH");
+  o.force_general_prefill = path && (std::strcmp(path, "general") == 0 || std::strcmp(path, "simt") == 0);
+  const char* lim = std::getenv("LIGER_WAIT_LIMIT_NS");
+  o.wait_limit_ns = (lim && *lim) ? std::strtoull(lim, nullptr, 10) : 0ull;
+  const char* stall = std::getenv("LIGER_TEST_INJECT_STALL");
+  o.inject_stall_calls = (stall && *stall) ? std::strtol(stall, nullptr, 10) : 0;
+  return o;
+}
+// Initialised when the library is loaded; never re-read.
+const Options g_options = read_options();
+std::atomic<long> g_stalls_taken{0};
+}  // namespace
+
+const Options& options() { return g_options; }
+
+bool take_injected_stall() {
+  if (g_options.inject_stall_calls <= 0) return false;
+  return g_stalls_taken.fetch_add(1) < g_options.inject_stall_calls;
+}
+
 // Records a failure for liger_last_error() from other translation units of the library.
 void set_last_error(liger_status status, const char* message) { fail(status, "%s", message); }
+
+// Whether a prefill with these arguments runs on the tensor-core path, the only one that
+// uses the workspace.
+bool prefill_uses_workspace(int B, int Hq, int Hkv, int T, int d, int w, liger_dtype dt,
+                            const float* initial_state) {
+  if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return false;
+  return choose_prefill_path((long)B * T, Hq, Hkv, d, w, dt, initial_state) == PrefillPath::kTensorCore;
+}
 }  // namespace liger
 
 extern "C" {

@@ -47,7 +47,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -1310,12 +1309,8 @@ struct LaunchHooks {
 };
 
 inline uint64_t wait_limit_ns() {
-  const char* s = std::getenv("LIGER_WAIT_LIMIT_NS");
-  if (s && *s) {
-    const unsigned long long v = std::strtoull(s, nullptr, 10);
-    if (v > 0) return v;
-  }
-  return kDefaultWaitNs;
+  const unsigned long long v = options().wait_limit_ns;
+  return v > 0 ? (uint64_t)v : kDefaultWaitNs;
 }
 
 // Launch with programmatic stream serialisation: the grid may be scheduled while
@@ -1365,10 +1360,7 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   p.alpha = pb.alpha;
   p.wait_ns = wait_limit_ns();
   p.out_v8 = (reinterpret_cast<uintptr_t>(pb.out) & 31u) == 0 ? 1 : 0;
-  {
-    const char* st = std::getenv("LIGER_TEST_INJECT_STALL");
-    p.inject_stall = (st && *st && *st != '0') ? 1 : 0;
-  }
+  p.inject_stall = take_injected_stall() ? 1 : 0;
 
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, pb.q, D, pb.Hq, NT, 2) || !make_map(&mk, pb.k, D, pb.Hkv, NT, 1) ||

@@ -40,6 +40,7 @@ SIGNATURES = {
     "liger_attn_prefill_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
                                         _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "liger_attn_prefill_status": (_i, [_vp, ctypes.c_size_t]),
+    "liger_attn_prefill_noalloc_status": (_i, []),
     "liger_attn_prefill_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                                      ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_size_t)]),
     "liger_set_timing_events": (None, [_vp, _vp]),

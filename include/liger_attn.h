@@ -189,11 +189,14 @@ liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void
  * as liger_attn_prefill without the workspace pair; the scratch is a fixed
  * array of LIGER_PREFILL_NOALLOC_SCRATCH_BYTES in this library's device image,
  * which every GPU that loads the library holds until the process exits.
- *   - Sizes whose liger_attn_prefill_workspace_size() exceeds that maximum are
- *     rejected with LIGER_ERR_UNSUPPORTED before anything is launched.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *   - Calls that take the tensor-core path (the only one that uses scratch)
+ *     and whose liger_attn_prefill_workspace_size() exceeds that maximum are
+ *     rejected with LIGER_ERR_UNSUPPORTED before anything is launched; calls
+ *     served by the general kernel have no size limit here.
+ *   - The first call in a device's context looks up the array's device address
+ *     (with that device current) and caches it, tagged with the context, so a
+ *     context created again after cudaDeviceReset gets a fresh lookup; make
+ *     that first call before any stream capture.
  *   - The function itself allocates nothing: no cudaMalloc, no cudaFree, no
  *     allocating library routine.
  *   - All calls on a device share the one array, which keeps the last call's
@@ -207,6 +210,29 @@ liger_status liger_attn_prefill_noalloc(const void* q, const void* k, const void
                                         float alpha, liger_dtype dt, const float* initial_state,
                                         const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
                                         int32_t* pos_out, void* stream);
+
+/*
+ * Status of the last liger_attn_prefill_noalloc call on the current device, as
+ * liger_attn_prefill_status reports it for a workspace: LIGER_ERR_TIMEOUT
+ * (with the site in liger_last_error()) if one of its kernels gave up on a
+ * bounded wait, LIGER_OK otherwise.  Reads the scratch header with a
+ * synchronous copy: call it after that call's stream has completed.  (No
+ * counterpart on the pages; failure detection.)
+ */
+liger_status liger_attn_prefill_noalloc_status(void);
+
+/*
+ * Diagnostic options (no counterpart on the pages), read from the environment
+ * once, when the library is loaded; later changes have no effect:
+ *   LIGER_PREFILL_PATH=general   every prefill takes the general (CUDA-core) kernel
+ *   LIGER_WAIT_LIMIT_NS=<n>      give-up time of each bounded wait (default 2 s)
+ *   LIGER_TEST_INJECT_STALL=<n>  the first n tensor-core prefill calls of the
+ *                                process withhold one internal completion, so
+ *                                that a bounded wait runs out and the call
+ *                                reports LIGER_ERR_TIMEOUT (for testing failure
+ *                                detection without a GPU fault); later calls
+ *                                run normally
+ */
 
 /* Message of the last failure on the calling thread ("" if none). */
 const char* liger_last_error(void);

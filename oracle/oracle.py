@@ -180,6 +180,33 @@ def prefill_backward(q, k, v, d_out, w=64, alpha=0.5, initial_state=None, cu_seq
     return dq, dk, dv, ds0
 
 
+def decode_inplace(q, k, v, state, ring, pos, alpha=0.5, gate_off=False, nthreads=None):
+    """One decode step that updates state, ring and pos in place and returns out.
+
+    state [B, Hq, d, d] and ring [B, Hkv, 2, w, d] must be C-contiguous float64 arrays and pos a
+    C-contiguous int32 array [B] (they are handed to the C routine as they are, with no copy:
+    for long runs at large B, where copying the state every step would dominate).
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    for name, a, dt in (("state", state, np.float64), ("ring", ring, np.float64), ("pos", pos, np.int32)):
+        if not isinstance(a, np.ndarray) or a.dtype != dt or not a.flags["C_CONTIGUOUS"]:
+            raise ValueError(f"decode_inplace: {name} must be a C-contiguous {np.dtype(dt).name} array")
+    w = ring.shape[3]
+    if k.shape != (B, Hkv, d) or v.shape != (B, Hkv, d) or state.shape != (B, Hq, d, d) \
+            or ring.shape != (B, Hkv, 2, w, d) or pos.shape != (B,):
+        raise ValueError("decode_inplace: inconsistent shapes")
+    out = np.zeros_like(q)
+    rc = lib.oracle_decode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos, _ip), B, Hq, Hkv, d, w,
+        float(alpha), int(bool(gate_off)), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_decode rejected its arguments")
+    return out
+
+
 def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthreads=None):
     """One decode step.  Returns (out, new_state, new_ring, new_pos); inputs are not modified.
 

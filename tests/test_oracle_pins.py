@@ -301,3 +301,23 @@ def test_golden_small_case():
     np.testing.assert_allclose(out, np.array(g["out"]), rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(fs, np.array(g["final_state"]), rtol=1e-12, atol=1e-15)
     assert pos.tolist() == g["pos"]
+
+
+def test_decode_inplace_steps_equal_a_longer_prefill():
+    """The in-place decode front end (no copies; used for long full-size runs) continues a prefill
+    exactly as a longer prefill does, and updates its arrays in place."""
+    B, Hq, Hkv, T1, T2, d, w = 2, 4, 2, 9, 5, 8, 4
+    q, k, v = rand(B, T1 + T2, Hq, d), rand(B, T1 + T2, Hkv, d), rand(B, T1 + T2, Hkv, d)
+    full, fs_full, ring_full, pos_full = oracle.prefill(q, k, v, w=w)
+    _, st, rg, ps = oracle.prefill(q[:, :T1], k[:, :T1], v[:, :T1], w=w)
+    st, rg, ps = np.ascontiguousarray(st), np.ascontiguousarray(rg), np.ascontiguousarray(ps.astype(np.int32))
+    ids = (id(st), id(rg), id(ps))
+    for t in range(T1, T1 + T2):
+        o = oracle.decode_inplace(q[:, t], k[:, t], v[:, t], st, rg, ps)
+        np.testing.assert_allclose(o, full[:, t], rtol=1e-12, atol=1e-14)
+    assert (id(st), id(rg), id(ps)) == ids
+    np.testing.assert_allclose(st, fs_full, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(rg, ring_full)
+    np.testing.assert_array_equal(ps, pos_full)
+    with pytest.raises(ValueError):
+        oracle.decode_inplace(q[:, 0], k[:, 0], v[:, 0], st.astype(np.float32), rg, ps)

@@ -1,12 +1,12 @@
 """CUDA path vs the fp64 oracle, element by element, on seeded inputs.
 
-Small cases compare every output; the full workload sizes run the CUDA
-kernels in the same launch configuration the benchmark times and compare
-sampled (batch row, kv-head group) units that the oracle recomputes from
-scratch.  Tolerances: bf16 max-abs 2e-2 and rel-L2 5e-3, fp32 1e-4 for both;
-the window ring and positions are copies and must match bit for bit.
+Small cases and the full workload sizes alike compare every output: the full
+sizes run the CUDA kernels in the same launch configuration the benchmark times,
+and the oracle recomputes the whole workload (every sequence, head, token and
+final-state element; for decode every sequence over all 1000 steps).
+Tolerances: bf16 max-abs 2e-2 and rel-L2 5e-3, fp32 1e-4 for both; the window
+ring and positions are copies and must match bit for bit.
 """
-import os
 import zlib
 
 import numpy as np
@@ -15,7 +15,8 @@ import torch
 
 from gated_linear_attention_liger_b200 import inputs, ops
 from oracle import oracle
-from tests.parity_util import assert_close, np64, oracle_group
+from tests import child_scenarios
+from tests.parity_util import assert_close, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +39,7 @@ SMALL = [
 ]
 
 
-def run_small(case, device, path=None):
+def run_small(case, device):
     name, B, Hq, Hkv, T, d, dtype, w, alpha, seqlens, kb, with_s0 = case
     wl = inputs.small(name, B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, dtype=dtype, seed=zlib.crc32(name.encode()) % 10000,
                       seqlens=seqlens, key_bias_std=kb)
@@ -46,22 +47,12 @@ def run_small(case, device, path=None):
     cu = wl.cu_seqlens
     n = wl.n_seqs
     s0 = inputs.random_state(n, Hq, d, seed=5, scale=0.05) if with_s0 else None
-    old = os.environ.get("LIGER_PREFILL_PATH")
-    if path:
-        os.environ["LIGER_PREFILL_PATH"] = path
-    try:
-        out, fs, ring, pos = ops.prefill(
-            q.to(device), k.to(device), v.to(device), alpha=alpha, w=w,
-            initial_state=None if s0 is None else s0.to(device),
-            cu_seqlens=None if cu is None else torch.tensor(cu, dtype=torch.int32, device=device),
-            return_ring=True)
-        torch.cuda.synchronize()
-    finally:
-        if path:
-            if old is None:
-                os.environ.pop("LIGER_PREFILL_PATH")
-            else:
-                os.environ["LIGER_PREFILL_PATH"] = old
+    out, fs, ring, pos = ops.prefill(
+        q.to(device), k.to(device), v.to(device), alpha=alpha, w=w,
+        initial_state=None if s0 is None else s0.to(device),
+        cu_seqlens=None if cu is None else torch.tensor(cu, dtype=torch.int32, device=device),
+        return_ring=True)
+    torch.cuda.synchronize()
     ref = oracle.prefill(np64(q), np64(k), np64(v), w=w, alpha=alpha, cu_seqlens=cu,
                          initial_state=None if s0 is None else np64(s0))
     return (out, fs, ring, pos), ref, dtype
@@ -76,13 +67,11 @@ def test_prefill_small_parity(case, cuda_device):
     np.testing.assert_array_equal(pos.cpu().numpy(), rpos)
 
 
-@pytest.mark.parametrize("case", [c for c in SMALL if c[6] == torch.bfloat16][:6],
-                         ids=[c[0] for c in SMALL if c[6] == torch.bfloat16][:6])
-def test_prefill_general_kernel_parity(case, cuda_device):
-    """The general (CUDA-core) prefill kernel, forced for bf16 inputs."""
-    (out, fs, ring, pos), (ro, rfs, rring, rpos), dtype = run_small(case, cuda_device, path="simt")
-    assert_close(np64(out), ro, dtype, "out")
-    assert_close(np64(fs), rfs, dtype, "final_state")
+def test_prefill_general_kernel_parity(cuda_device):
+    """The general (CUDA-core) prefill kernel, forced for bf16 inputs (the first six bf16
+    small cases), in a child process whose library was loaded with LIGER_PREFILL_PATH=general."""
+    out = child_scenarios.run("general_parity", child_scenarios.GENERAL_ENV)
+    assert out.count("general kernel ok") == 6
 
 
 def test_prefill_wide_feature_spread(cuda_device):
@@ -145,7 +134,9 @@ def test_prefill_is_deterministic(cuda_device):
 
 # ----------------------------------------------------------------- full sizes
 
-def _full_prefill_check(name, units, device):
+def _full_prefill_check(name, device):
+    """The whole workload on the GPU and in the oracle; every output, final-state, ring and
+    position element compared."""
     wl = inputs.WORKLOADS[name]
     q, k, v = inputs.prefill_inputs(wl)
     cu = wl.cu_seqlens
@@ -153,30 +144,38 @@ def _full_prefill_check(name, units, device):
     out, fs, ring, pos = ops.prefill(q.to(device), k.to(device), v.to(device), alpha=wl.alpha, w=wl.w,
                                      cu_seqlens=cu_t, return_ring=True)
     torch.cuda.synchronize()
-    out, fs = out.cpu(), fs.cpu()
+    ro, rfs, rring, rpos = oracle.prefill(np64(q), np64(k), np64(v), w=wl.w, alpha=wl.alpha, cu_seqlens=cu)
+    assert_close(np64(out), ro, wl.dtype, f"{name} out")
+    assert_close(np64(fs), rfs, wl.dtype, f"{name} final_state")
+    np.testing.assert_array_equal(np64(ring), rring)
+    np.testing.assert_array_equal(pos.cpu().numpy(), rpos)
+    # every sequence and head on its own as well: a wrong offset for one unit cannot hide
+    # inside the whole-tensor norm
     G = wl.Hq // wl.Hkv
-    for b, kv in units:
-        ro, rfs, rring, rpos = oracle_group(q, k, v, b, kv, G, w=wl.w, alpha=wl.alpha, cu=cu)
-        hs = slice(kv * G, (kv + 1) * G)
-        assert_close(np64(out[b:b + 1, :, hs]), ro, wl.dtype, f"{name} out b={b} kv={kv}")
-        fsel = fs[:, hs] if cu is not None else fs[b:b + 1, hs]
-        assert_close(np64(fsel), rfs, wl.dtype, f"{name} final_state b={b} kv={kv}")
-        rsel = ring[:, kv:kv + 1] if cu is not None else ring[b:b + 1, kv:kv + 1]
-        np.testing.assert_array_equal(np64(rsel), rring)
-    exp_pos = np.diff(cu) if cu is not None else np.full(wl.B, wl.T)
-    np.testing.assert_array_equal(pos.cpu().numpy(), exp_pos)
+    n = wl.n_seqs
+    bounds = cu if cu is not None else None
+    for s_ in range(n):
+        for kv in range(wl.Hkv):
+            hs = slice(kv * G, (kv + 1) * G)
+            if bounds is not None:
+                got, ref = np64(out[0, bounds[s_]:bounds[s_ + 1], hs]), ro[0, bounds[s_]:bounds[s_ + 1], hs]
+            else:
+                got, ref = np64(out[s_, :, hs]), ro[s_, :, hs]
+            if ref.size:
+                assert_close(got, ref, wl.dtype, f"{name} out seq={s_} kv={kv}")
+            assert_close(np64(fs[s_, hs]), rfs[s_, hs], wl.dtype, f"{name} final_state seq={s_} kv={kv}")
 
 
 def test_full_llama1b_prefill(cuda_device):
-    _full_prefill_check("llama1b_prefill", [(0, 0), (3, 7), (1, 4)], cuda_device)
+    _full_prefill_check("llama1b_prefill", cuda_device)
 
 
 def test_full_llama8b_prefill(cuda_device):
-    _full_prefill_check("llama8b_prefill", [(0, 2), (1, 7)], cuda_device)
+    _full_prefill_check("llama8b_prefill", cuda_device)
 
 
 def test_full_long_varlen_prefill(cuda_device):
-    _full_prefill_check("long_varlen", [(0, 5)], cuda_device)
+    _full_prefill_check("long_varlen", cuda_device)
 
 
 def test_full_tiny_fp32(cuda_device):
@@ -243,39 +242,48 @@ def test_prefill_then_decode_matches_longer_prefill(cuda_device):
 
 
 def test_full_llama8b_decode(cuda_device):
-    """B=64 decode at the full shape after a 1024-token prefix; sampled sequences
-    carry an oracle-built state and ring, 200 steps compared step by step."""
+    """The Llama-3-8B decode workload in full: B=64 sequences whose state and ring come from a
+    seeded 1024-token prefill, then 1000 steps.  The GPU prefill of the prefix is compared with
+    the oracle's; both decodes then start from the oracle's prefix (state rounded to fp32, ring
+    to bf16) and every output of every sequence and step is compared, then the final states,
+    ring and positions."""
     wl = inputs.WORKLOADS["llama8b_decode"]
-    B, Hq, Hkv, d, w, G = wl.B, wl.Hq, wl.Hkv, wl.d, wl.w, wl.Hq // wl.Hkv
-    units = [(5, 1), (63, 6)]
-    state = torch.zeros(B, Hq, d, d, dtype=torch.float32)
-    ring = torch.zeros(B, Hkv, 2, w, d, dtype=wl.dtype)
-    pos = torch.full((B,), wl.T, dtype=torch.int32)
-    ref = {}
-    pre = inputs.Workload("pre", "prefill", 1, G, 1, wl.T, d, wl.dtype, seed=wl.seed)
-    for b, kv in units:
-        q, k, v = inputs.prefill_inputs(pre, seed=wl.seed + 97 * b + kv)
-        _, st, rg, ps = oracle.prefill(np64(q), np64(k), np64(v), w=w)
-        hs = slice(kv * G, (kv + 1) * G)
-        state[b, hs] = torch.tensor(st[0], dtype=torch.float32)
-        ring[b, kv] = torch.tensor(rg[0]).to(wl.dtype)
-        ref[(b, kv)] = [np64(state[b:b + 1, hs]), np64(ring[b:b + 1, kv:kv + 1]), np.array([wl.T], np.int32)]
-    g_state, g_ring, g_pos = state.to(cuda_device), ring.to(cuda_device), pos.to(cuda_device)
-    for step in range(200):
-        q, k, v = inputs.decode_step_inputs(wl, step)
-        o = ops.decode(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), g_state, g_ring, g_pos)
-        o = o.cpu()
-        for (b, kv), (st, rg, ps) in ref.items():
-            hs = slice(kv * G, (kv + 1) * G)
-            ro, st, rg, ps = oracle.decode(np64(q[b:b + 1, hs]), np64(k[b:b + 1, kv:kv + 1]),
-                                           np64(v[b:b + 1, kv:kv + 1]), st, rg, ps, w=w)
-            ref[(b, kv)] = [st, rg, ps]
-            assert_close(np64(o[b:b + 1, hs]), ro, wl.dtype, f"decode step {step} b={b} kv={kv}")
-    for (b, kv), (st, rg, ps) in ref.items():
-        hs = slice(kv * G, (kv + 1) * G)
-        assert_close(np64(g_state[b:b + 1, hs]), st, wl.dtype, "state")
-        np.testing.assert_array_equal(np64(g_ring[b:b + 1, kv:kv + 1]), rg)
-    assert int(g_pos.min()) == wl.T + 200 == int(g_pos.max())
+    B, Hq, Hkv, d, w = wl.B, wl.Hq, wl.Hkv, wl.d, wl.w
+    steps = wl.steps
+    dev = cuda_device
+    pre = inputs.Workload("decode_prefix", "prefill", B, Hq, Hkv, wl.T, d, wl.dtype, seed=wl.seed)
+    q, k, v = inputs.prefill_inputs(pre)
+    _, g_st, g_rg, g_ps = ops.prefill(q.to(dev), k.to(dev), v.to(dev), alpha=wl.alpha, w=w, return_ring=True)
+    _, rst, rrg, rps = oracle.prefill(np64(q), np64(k), np64(v), w=w, alpha=wl.alpha)
+    torch.cuda.synchronize()
+    assert_close(np64(g_st), rst, wl.dtype, "prefix final state")
+    np.testing.assert_array_equal(np64(g_rg), rrg)
+    np.testing.assert_array_equal(g_ps.cpu().numpy(), rps)
+    del q, k, v, g_st, g_rg
+    # the common starting point
+    state = torch.tensor(rst, dtype=torch.float32)
+    ring = torch.tensor(rrg).to(wl.dtype)
+    o_st = np.ascontiguousarray(np64(state))
+    o_rg = np.ascontiguousarray(np64(ring))
+    o_ps = np.ascontiguousarray(rps.astype(np.int32))
+    g_state, g_ring = state.to(dev), ring.to(dev)
+    g_pos = torch.tensor(rps, dtype=torch.int32, device=dev)
+    del state, ring, rst, rrg
+    block = 50
+    for s0 in range(0, steps, block):
+        step_in = [inputs.decode_step_inputs(wl, s) for s in range(s0, min(steps, s0 + block))]
+        outs = []
+        for qt, kt, vt in step_in:
+            outs.append(ops.decode(qt.to(dev), kt.to(dev), vt.to(dev), g_state, g_ring, g_pos, alpha=wl.alpha))
+        outs = torch.stack(outs).cpu()
+        for i, (qt, kt, vt) in enumerate(step_in):
+            ro = oracle.decode_inplace(np64(qt), np64(kt), np64(vt), o_st, o_rg, o_ps, alpha=wl.alpha)
+            assert_close(np64(outs[i]), ro, wl.dtype, f"decode step {s0 + i}")
+    torch.cuda.synchronize()
+    assert_close(np64(g_state), o_st, wl.dtype, "state after the steps")
+    np.testing.assert_array_equal(np64(g_ring), o_rg)
+    np.testing.assert_array_equal(g_pos.cpu().numpy(), o_ps)
+    assert int(g_pos.min()) == wl.T + steps == int(g_pos.max())
 
 
 # ----------------------------------------------------------------- shared-state decode
