@@ -414,9 +414,20 @@ def run_ours(args, world, rank, local):
             r["roofline"]["traffic"] = measured_traffic(f"chunk_kernel<{owl.d}>@{owl.name}")
             others[owl.name] = r
 
+    # ---------------- the prefill's gradient (the fine-tune's backward pass)
+    bwd = None
+    if args.only is None or args.only in ("prefill", "backward"):
+        bwd = time_backward(PREFILL, args, world, dev, stream, pk, windows)
+
+    # ---------------- the hybrid's standard attention layer (causal softmax attention)
+    full = None
+    if args.only is None or args.only in ("prefill", "full"):
+        full = time_full_attention(PREFILL, args, world, dev, stream, pk, windows)
+
     # ---------------- decode
-    dec = None if args.only == "prefill" else run_decode(args, world, dev, stream, pk, windows)
-    dec_kv = None if args.only == "prefill" else run_decode(args, world, dev, stream, pk, windows, kvshared=True)
+    dec = None if args.only in ("prefill", "full", "backward") else run_decode(args, world, dev, stream, pk, windows)
+    dec_kv = (None if args.only in ("prefill", "full", "backward")
+              else run_decode(args, world, dev, stream, pk, windows, kvshared=True))
 
     sampler.stop()
     clocks = sampler.summary(windows)
@@ -433,6 +444,7 @@ def run_ours(args, world, rank, local):
             "data": "synthetic (seeded N(0,1), Llama-3-8B attention shapes)",
             "config": workload_config(), "roofline": roofline, "prefill_call": res8["call"],
             "llama1b_prefill": others.get("llama1b_prefill"), "long_varlen": others.get("long_varlen"),
+            "full_attention": full, "backward": bwd,
             "decode": dec, "decode_kvshared": dec_kv, "e2e": e2e,
             "gpu_launches": prefill_launches, "clocks": clocks, "cpu_baseline": cpu,
         }
@@ -529,6 +541,120 @@ def time_prefill(wl, args, world, dev, stream, pk, windows, flush_l2=False):
                                      "note": "(chunk, kv head) pairs with total log gate < -60"}
     res["_tensors"] = (q, k, v, out, fs, ws)
     return res
+
+
+def backward_algorithmic(wl):
+    """Algorithmic bytes and flops of one backward call: read q, k, v and d_out, write dq, dk, dv
+    once; flops per token of the window branch (10 w d per q head: scores, dO.v, and the three
+    gradient products over the band), the recurrent branch's causal intra-chunk products
+    (5 d (C+1) per q head) and its state products (4 d^2 per q head, 6 d^2 per kv head)."""
+    tok = wl.B * wl.T
+    esz = 2
+    bytes_ = tok * (3 * wl.Hq + 4 * wl.Hkv) * wl.d * esz
+    C = 64
+    flops = tok * (wl.Hq * (10 * wl.w * wl.d + 5 * wl.d * (C + 1) + 4 * wl.d ** 2) + wl.Hkv * 6 * wl.d ** 2)
+    return bytes_, flops
+
+
+def time_backward(wl, args, world, dev, stream, pk, windows):
+    """Times the gradient of the prefill (bf16, d_out given, no final-state gradient) with the
+    library's events around its two per-chunk gradient kernels, and the whole call."""
+    from gated_linear_attention_liger_b200 import ops
+    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
+    gen = torch.Generator().manual_seed(23)
+    dout = torch.randn(q.shape, generator=gen).to(q.dtype).to(dev)
+    ws = torch.empty(ops.prefill_backward_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.n_seqs), device=dev,
+                     dtype=torch.uint8)
+
+    def call():
+        ops.prefill_backward(q, k, v, dout, alpha=wl.alpha, workspace=ws, stream=stream)
+
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        call()
+    n = max(3, min(args.steps, 10))
+    ks, ke = timing_events(n, stream), timing_events(n, stream)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    a.record(stream)
+    for i in range(n):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    for i in range(n):
+        ops.set_timing_events(ks[i], ke[i])
+        call()
+    ops.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    status = ops.prefill_status(ws)
+    ms = max_over_ranks(a.elapsed_time(b) / n, world, dev)
+    k_ms = max_over_ranks(statistics.mean(x.elapsed_time(y) for x, y in zip(ks, ke)), world, dev)
+    alg_bytes, alg_flops = backward_algorithmic(wl)
+    t_bw, t_tc = alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (pk["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_bw >= t_tc else "tensor"
+    achieved = alg_bytes / (ms * 1e-3) / 1e9 if bound == "hbm" else alg_flops / (ms * 1e-3) / 1e12
+    peak = pk["hbm_gbs"] if bound == "hbm" else pk["bf16_tflops"]
+    del q, k, v, dout, ws
+    return {"metric": "prefill backward tokens/s (8B attn shape)", "value": world * wl.tokens / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": n, "status": ops.STATUS_NAMES.get(status, status),
+            "gradient_kernels_ms": k_ms,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "kernel": "whole backward call", "algorithmic_bytes": alg_bytes,
+                         "algorithmic_flops": alg_flops,
+                         "tensor_frac": alg_flops / (ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
+                         "peak_source": pk["source"]}}
+
+
+def full_attention_flops(wl):
+    """Algorithmic flops of causal softmax attention: Q K^T and P V over the causal half of the
+    T x T score matrix (diagonal included), 2 flops per multiply-add."""
+    pairs = wl.T * (wl.T + 1) / 2
+    return wl.B * wl.Hq * pairs * wl.d * 4
+
+
+def time_full_attention(wl, args, world, dev, stream, pk, windows):
+    """Times the causal attention layer (the inter-layer hybrid's standard attention) on the
+    workload's q, k, v: kernel time from the library's events, tensor-bound roofline."""
+    from gated_linear_attention_liger_b200 import ops
+    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
+    out = torch.empty_like(q)
+
+    def call():
+        ops.full_causal_attention(q, k, v, out=out, stream=stream)
+
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        call()
+    n = max(3, min(args.steps, 10))
+    ks, ke = timing_events(n, stream), timing_events(n, stream)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for i in range(n):
+        ops.set_timing_events(ks[i], ke[i])
+        call()
+    ops.set_timing_events(None, None)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    status = ops.full_causal_status()
+    k_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(ks, ke)), world, dev)
+    flops = full_attention_flops(wl)
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    del q, k, v, out
+    return {"metric": "causal attention tokens/s (8B attn shape)", "value": world * wl.tokens / (k_ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": k_ms, "steps": n, "status": ops.STATUS_NAMES.get(status, status),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": None, "kernel": "causal attention",
+                         "kernel_ms": k_ms, "algorithmic_flops": flops, "peak_source": pk["source"],
+                         "frac_of": f"{pk['source']} cuBLAS bf16 burst"}}
 
 
 def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
@@ -669,7 +795,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000, help="decode steps per captured graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU baseline")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "full", "backward"], default=None,
                     help="run one part only (for profiling); the JSON line is then partial")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

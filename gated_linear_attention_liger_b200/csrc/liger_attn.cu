@@ -18,6 +18,8 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "full_attn.cuh"
+#include "prefill_bwd.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
 
@@ -92,8 +94,8 @@ enum class PrefillPath { kSimt, kTensorCore };
 PrefillPath choose_prefill_path(long ntok, int Hq, int Hkv, int d, int w, liger_dtype dt,
                                 const float* initial_state) {
   if (liger::options().force_general_prefill) return PrefillPath::kSimt;
-  if (ntok > 0 && dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && initial_state == nullptr &&
-      liger::tc::supports(d))
+  (void)initial_state;   // taken by both paths
+  if (ntok > 0 && dt == LIGER_BF16 && w == 64 && (Hq / Hkv) % 2 == 0 && liger::tc::supports(d))
     return PrefillPath::kTensorCore;
   return PrefillPath::kSimt;
 }
@@ -180,6 +182,25 @@ liger_status decode_kvshared_g(const liger::DecodeArgs& a, int G, unsigned block
 template <typename Tin>
 liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, cudaStream_t s) {
   return d == 64 ? launch_simt_prefill<Tin, 64>(a, n_seqs, s) : launch_simt_prefill<Tin, 128>(a, n_seqs, s);
+}
+
+// Error word of the causal-attention kernel (bit 0: a bounded wait gave up; word 1: the
+// first site), one per device; read and cleared by liger_attn_full_causal_status().
+__device__ uint32_t g_full_attn_err[2];
+
+template <int D>
+liger_status launch_full_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const liger::fa::Params& prm, int Hq, int n_seqs, cudaStream_t s) {
+  auto kern = liger::fa::full_attn_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)liger::fa::Smem<D>::BYTES) !=
+      cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(full_attn)");
+  const dim3 grid((unsigned)prm.n_qblk, (unsigned)Hq, (unsigned)n_seqs);
+  mark_start(s);
+  kern<<<grid, liger::fa::kThreads, liger::fa::Smem<D>::BYTES, s>>>(mq, mk, mv, prm);
+  mark_stop(s);
+  ++g_launches;
+  return cuda_check("full_attn launch");
 }
 
 }  // namespace
@@ -284,7 +305,8 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
     return fail(LIGER_ERR_INVALID_ARG, "without cu_seqlens n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
   }
   const long ntok = (long)B * T;
-  if ((long)T * B * Hq > (1L << 40) / d) return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
+  if ((long)T * B * Hq > (1L << 40) / d || (long)T * B > 0x7fffffffL - 1024)   // 32-bit token indices
+    return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
   if (ntok > 0 && (!q || !k || !v || !out))
     return fail(LIGER_ERR_INVALID_ARG, "q, k, v and out must be non-null");
   const void* ptrs[] = {q, k, v, out, final_state, initial_state, swa_ring_out, workspace};
@@ -301,12 +323,27 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
     const size_t need = liger::tc::workspace_bytes(B, Hq, Hkv, (long)T, d, n_seqs);
     if (need > workspace_bytes || (need && !workspace))
       return fail(LIGER_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, workspace_bytes);
-    liger::tc::PrefillProblem pb{q, k, v, out, final_state, cu_seqlens, B, Hq, Hkv, (long)T, d, n_seqs, alpha};
+    liger::tc::PrefillProblem pb{q, k, v, out, final_state, initial_state, cu_seqlens, B, Hq, Hkv, (long)T, d,
+                                 n_seqs, alpha};
     const liger::tc::LaunchHooks hooks{mark_start, mark_stop, count_launches};
-    st = liger::tc::run_prefill(pb, workspace, s, hooks);
+    const uint32_t* s0_flags = nullptr;
+    st = liger::tc::run_prefill(pb, workspace, s, hooks, &s0_flags);
     if (st != LIGER_OK) return fail(st, "%s", liger::tc::last_message());
+    if (initial_state) {
+      // Groups whose q heads start from different initial states: the general kernel
+      // recomputes those (sequence, kv head) units; its other CTAs return at once.
+      liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha,
+                               s0_flags};
+      const auto hooks_off = std::make_pair(g_ev_start, g_ev_stop);
+      g_ev_start = g_ev_stop = nullptr;   // the timing events bracket the chunk pass only
+      st = prefill_simt_dispatch<__nv_bfloat16>(a, d, n_seqs, s);
+      g_ev_start = hooks_off.first;
+      g_ev_stop = hooks_off.second;
+      if (st != LIGER_OK) return st;
+    }
   } else {
-    liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha};
+    liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha,
+                             nullptr};
     st = dt == LIGER_BF16 ? prefill_simt_dispatch<__nv_bfloat16>(a, d, n_seqs, s)
                           : prefill_simt_dispatch<float>(a, d, n_seqs, s);
     if (st != LIGER_OK) return st;
@@ -355,6 +392,137 @@ liger_status liger_attn_prefill_status(const void* workspace, size_t workspace_b
     return fail(LIGER_ERR_TIMEOUT, "a prefill kernel gave up waiting (site 0x%08x: role %u, barrier %u, chunk %u)",
                 hdr[1], hdr[1] >> 28, (hdr[1] >> 20) & 0xFFu, hdr[1] & 0xFFFFFu);
   if (hdr[0]) return fail(LIGER_ERR_CUDA, "prefill error word 0x%x", hdr[0]);
+  return LIGER_OK;
+}
+
+size_t liger_attn_prefill_backward_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                                  liger_dtype dt) {
+  if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return 0;
+  if (dt != LIGER_BF16 || (d != 64 && d != 128) || (Hq / Hkv) % 2) return 0;
+  return liger::bwd::bwd_workspace_bytes(B, Hq, Hkv, (long)T, d, n_seqs > 0 ? n_seqs : B);
+}
+
+liger_status liger_attn_prefill_backward(const void* q, const void* k, const void* v, const void* d_out,
+                                         const float* d_final_state, const float* initial_state, int B, int Hq,
+                                         int Hkv, int T, int d, int w, float alpha, liger_dtype dt,
+                                         const int32_t* cu_seqlens, int n_seqs, void* dq, void* dk, void* dv,
+                                         float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  const NvtxRange range("liger_attn_prefill_backward");
+  g_last_error.clear();
+  liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
+  if (st != LIGER_OK) return st;
+  if (B < 1 || T < 0) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 and T >= 0 (B=%d T=%d)", B, T);
+  if (cu_seqlens) {
+    if (B != 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (B=%d)", B);
+    if (n_seqs < 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires n_seqs >= 1 (n_seqs=%d)", n_seqs);
+  } else if (n_seqs != B) {
+    return fail(LIGER_ERR_INVALID_ARG, "without cu_seqlens n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
+  }
+  if (dt != LIGER_BF16 || w != 64 || (Hq / Hkv) % 2)
+    return fail(LIGER_ERR_UNSUPPORTED, "the backward takes bf16, w = 64 and an even Hq/Hkv (dt=%d w=%d G=%d)",
+                (int)dt, w, Hq / Hkv);
+  if ((long)T * B * Hq > (1L << 40) / d || (long)T * B > 0x7fffffffL - 1024)
+    return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
+  const long ntok = (long)B * T;
+  if (ntok > 0 && (!q || !k || !v || !d_out || !dq || !dk || !dv))
+    return fail(LIGER_ERR_INVALID_ARG, "q, k, v, d_out, dq, dk and dv must be non-null");
+  const void* ptrs[] = {q, k, v, d_out, d_final_state, initial_state, dq, dk, dv, d_initial_state, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ntok == 0) {   // no tokens: the state passes through unchanged
+    if (d_initial_state) {
+      const size_t bytes = (size_t)n_seqs * Hkv * d * d * 4;
+      if (!d_final_state) {
+        if (cudaMemsetAsync(d_initial_state, 0, bytes, s) != cudaSuccess) return cuda_check("cudaMemsetAsync");
+      } else {
+        return fail(LIGER_ERR_UNSUPPORTED, "an empty backward with d_final_state: sum the group's heads instead");
+      }
+    }
+    return LIGER_OK;
+  }
+  const size_t need = liger::bwd::bwd_workspace_bytes(B, Hq, Hkv, (long)T, d, n_seqs);
+  if (need > workspace_bytes || !workspace)
+    return fail(LIGER_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, workspace_bytes);
+  liger::bwd::BwdProblem pb{q, k, v, d_out, d_final_state, initial_state, dq, dk, dv, d_initial_state, cu_seqlens,
+                            B, Hq, Hkv, (long)T, d, n_seqs, alpha};
+  const liger::tc::LaunchHooks hooks{mark_start, mark_stop, count_launches};
+  st = liger::bwd::run_backward(pb, workspace, s, hooks);
+  if (st != LIGER_OK) return fail(st, "%s", liger::tc::last_message());
+  return LIGER_OK;
+}
+
+liger_status liger_attn_full_causal(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                    int Hkv, int T, int d, liger_dtype dt, const int32_t* cu_seqlens, int n_seqs,
+                                    int max_seqlen, void* stream) {
+  const NvtxRange range("liger_attn_full_causal");
+  g_last_error.clear();
+  if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0)
+    return fail(LIGER_ERR_INVALID_ARG, "need Hq >= 1, Hkv >= 1 and Hq %% Hkv == 0 (Hq=%d Hkv=%d)", Hq, Hkv);
+  if (B < 1 || T < 0) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 and T >= 0 (B=%d T=%d)", B, T);
+  if (dt != LIGER_BF16 && dt != LIGER_FP32) return fail(LIGER_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (dt != LIGER_BF16) return fail(LIGER_ERR_UNSUPPORTED, "causal attention takes bf16 inputs");
+  if (d != 64 && d != 128) return fail(LIGER_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
+  if (cu_seqlens) {
+    if (B != 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (B=%d)", B);
+    if (n_seqs < 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires n_seqs >= 1 (n_seqs=%d)", n_seqs);
+    if (max_seqlen < 0 || max_seqlen > T)
+      return fail(LIGER_ERR_INVALID_ARG, "max_seqlen must lie in [0, T] (max_seqlen=%d T=%d)", max_seqlen, T);
+    if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)
+      return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+  } else if (n_seqs != B) {
+    return fail(LIGER_ERR_INVALID_ARG, "without cu_seqlens n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
+  }
+  const long NT = (long)B * T;
+  if (NT == 0) return LIGER_OK;
+  if (NT * Hq > (1L << 40) / d || NT > 0x7fffffffL - 1024)   // TMA token coordinates are 32-bit
+    return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
+  if (!q || !k || !v || !out) return fail(LIGER_ERR_INVALID_ARG, "q, k, v and out must be non-null");
+  const void* ptrs[] = {q, k, v, out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const long longest = cu_seqlens ? (long)max_seqlen : (long)T;
+  const long n_qblk = (longest + liger::fa::BM - 1) / liger::fa::BM;
+  if (n_qblk == 0) return LIGER_OK;
+  if (n_qblk > 0x7fffffffL || (long)n_seqs > 65535 || Hq > 65535)
+    return fail(LIGER_ERR_UNSUPPORTED, "grid too large");
+  CUtensorMap mq, mk, mv;
+  const auto enc = reinterpret_cast<liger::fa::EncodeTiledFn>(liger::tc::encode_fn());
+  if (!liger::fa::make_map(enc, &mq, q, d, Hq, NT) || !liger::fa::make_map(enc, &mk, k, d, Hkv, NT) ||
+      !liger::fa::make_map(enc, &mv, v, d, Hkv, NT))
+    return fail(LIGER_ERR_CUDA, "cuTensorMapEncodeTiled failed for the causal attention");
+  void* err = nullptr;
+  const cudaError_t ge = cudaGetSymbolAddress(&err, g_full_attn_err);
+  if (ge != cudaSuccess) return fail(LIGER_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(ge));
+  liger::fa::Params prm{};
+  prm.out = out;
+  prm.cu = cu_seqlens;
+  prm.T = T;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.n_qblk = (int)n_qblk;
+  prm.err = static_cast<uint32_t*>(err);
+  prm.wait_ns = liger::tc::wait_limit_ns();
+  prm.scale_log2 = 1.4426950408889634f / std::sqrt((float)d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_full_attn<64>(mq, mk, mv, prm, Hq, n_seqs, s)
+                 : launch_full_attn<128>(mq, mk, mv, prm, Hq, n_seqs, s);
+}
+
+liger_status liger_attn_full_causal_status(void) {
+  g_last_error.clear();
+  uint32_t hdr[2] = {0u, 0u};
+  cudaError_t e = cudaMemcpyFromSymbol(hdr, g_full_attn_err, sizeof hdr);
+  if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "reading the causal attention's error word: %s", cudaGetErrorString(e));
+  const uint32_t zero[2] = {0u, 0u};
+  e = cudaMemcpyToSymbol(g_full_attn_err, zero, sizeof zero);
+  if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "clearing the causal attention's error word: %s", cudaGetErrorString(e));
+  if (hdr[0] & 1u)
+    return fail(LIGER_ERR_TIMEOUT, "a causal attention kernel gave up waiting (site 0x%08x: role %u, barrier %u, block %u)",
+                hdr[1], hdr[1] >> 28, (hdr[1] >> 20) & 0xFFu, hdr[1] & 0xFFFFFu);
   return LIGER_OK;
 }
 

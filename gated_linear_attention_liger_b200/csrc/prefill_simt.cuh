@@ -29,6 +29,8 @@ struct SimtPrefillArgs {
   int Hq, Hkv, w;
   long T;                    // tokens per sequence (no offsets) / packed total
   float alpha;
+  const uint32_t* only_flagged;   // [n][Hkv] or null: when set, a CTA works only if its
+                                  // (sequence, kv head) flag is set, and returns at once otherwise
 };
 
 constexpr int kSimtThreads = 256;
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
   Tin* __restrict__ out = static_cast<Tin*>(a.out);
   const int Hq = a.Hq, Hkv = a.Hkv, w = a.w;
   const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, kv = h / (Hq / Hkv);
+  if (a.only_flagged && a.only_flagged[(size_t)seq * Hkv + kv] == 0u) return;
   const long T_total = a.cu ? a.T : (long)gridDim.x / Hq * a.T;
   long tb, te;
   seq_range(a.cu, seq, a.T, T_total, &tb, &te);

@@ -76,6 +76,7 @@ struct PrefillProblem {
   const void* v;
   void* out;
   float* final_state;
+  const float* s0;       // initial state [n, Hq, D, D] or null
   const int32_t* cu;
   int B, Hq, Hkv;
   long T;
@@ -88,8 +89,13 @@ struct Plan {
   int L;            // chunks per segment
   int n_seg_max;    // upper bound on segments
   int nsub, Ls;     // sub-segments per segment for the state pass, and their length in chunks
-  size_t off_seqs, off_segs, off_lam, off_ds, total;
+  size_t off_seqs, off_segs, off_lam, off_ds, off_kimg, off_bimg, off_flags, total;
 };
+
+// Largest total log gate of a chunk for which its decay is factored at the chunk end
+// (both factors then lie within e^{+-60}); the state pass and the chunk pass take the
+// same decision from the same stored sum.
+constexpr float kFactorFloor = -60.f;
 
 constexpr int kMaxSub = 8;
 
@@ -100,9 +106,17 @@ struct DevParams {
   float* lam;            // [n_seg_max][nsub][Hkv] total log gate of each sub-segment
   float* ds;             // [n_seg_max][nsub][Hkv][D][D]: state each sub-segment adds from a zero
                          // start; the scan replaces [s][0] by the state entering segment s
+  char* kimg;            // [n_seg_max * L][Hkv]: per chunk, the chunk pass's key tile as a
+                         // shared-memory image (C x D bf16, 128-byte swizzle, K-major blocks):
+                         // e^{b_C - b_j} phi(k_j) when the decay factors (b_C >= -60), else phi(k_j)
+  float* bimg;           // [n_seg_max * L][Hkv][C]: per chunk, the running log-gate sums b_j
+                         // (constant past the chunk's last valid token)
   uint32_t* err;
   void* out;
   float* final_state;
+  const float* s0;       // [n][Hq][D][D] initial states or null: the scan starts each group from
+                         // its first head's copy
+  uint32_t* s0_flags;    // [n][Hkv]: set when the G copies of a group's initial state differ
   const int32_t* cu;
   long T, NT;
   int Hq, Hkv, n_seqs, n_seg_max, L, nsub, Ls;
@@ -116,6 +130,8 @@ struct DevParams {
 
 __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* n_segs) {
   griddep_wait_and_release();   // the previous call's kernels are done with the workspace
+  if (p.s0)
+    for (int i = threadIdx.x; i < p.n_seqs * p.Hkv; i += blockDim.x) p.s0_flags[i] = 0u;
   if (threadIdx.x != 0) return;
   p.err[0] = 0u;
   p.err[1] = 0u;
@@ -141,14 +157,16 @@ __global__ void plan_kernel(DevParams p, SeqInfo* seqs, SegInfo* segs, int32_t* 
   *n_segs = seg;
 }
 
-// Final state of the sequences that have no token (packed input only): zero.
-// Grid (n_seqs, Hq), 256 threads.
+// Final state of the sequences that have no token (packed input only): the initial
+// state of that head, or zero.  Grid (n_seqs, Hq), 256 threads.
 template <int D>
 __global__ void zero_empty_kernel(DevParams p) {
   griddep_wait_and_release();
   if (p.seqs[blockIdx.x].n_seg != 0) return;
-  float4* dst = reinterpret_cast<float4*>(p.final_state + ((size_t)blockIdx.x * p.Hq + blockIdx.y) * D * D);
-  for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t off = ((size_t)blockIdx.x * p.Hq + blockIdx.y) * D * D;
+  float4* dst = reinterpret_cast<float4*>(p.final_state + off);
+  const float4* src = p.s0 ? reinterpret_cast<const float4*>(p.s0 + off) : nullptr;
+  for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) dst[e] = src ? src[e] : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // 32 bytes to global memory in one store (the address must be 32-byte aligned).
@@ -176,6 +194,21 @@ __global__ void scan_kernel(DevParams p) {
   const int n_units = si.n_seg * nsub;
   const size_t u0 = (size_t)si.first_seg * nsub;
   float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.s0) {
+    // The recurrence is linear in its start: every head of the group runs from the group's
+    // first copy of the initial state.  When another head's copy differs, the group is
+    // flagged and recomputed by the general kernel after the chunk pass.
+    const int G = p.Hq / p.Hkv;
+    const float* s0g = p.s0 + ((size_t)seq * p.Hq + (size_t)kv * G) * D * D + e;
+    run = *reinterpret_cast<const float4*>(s0g);
+    bool differ = false;
+    for (int g = 1; g < G; ++g) {
+      const float4 o = *reinterpret_cast<const float4*>(s0g + (size_t)g * D * D);
+      differ |= __float_as_uint(o.x) != __float_as_uint(run.x) || __float_as_uint(o.y) != __float_as_uint(run.y) ||
+                __float_as_uint(o.z) != __float_as_uint(run.z) || __float_as_uint(o.w) != __float_as_uint(run.w);
+    }
+    if (differ) atomicOr(p.s0_flags + (size_t)seq * p.Hkv + kv, 1u);
+  }
   for (int base = 0; base < n_units; base += kBatch) {
     float4 d[kBatch];
     float g[kBatch];
@@ -508,11 +541,23 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 2);
+      const bool live = (r >> 2) < nv;
+      // The chunk pass's key tile for this chunk (written once, read by its q-head
+      // pairs): factored at the chunk end when the chunk's decay allows, else phi(k).
+      {
+        const size_t ci = (size_t)(seg * p.L + sub * p.Ls + cc) * p.Hkv + kv;
+        const float sc = live ? (bC >= kFactorFloor ? __expf(bC - bj) * iz : iz) : 0.f;
+        write_ktilde<D, 4>(ek, p.kimg + ci * L::KV, r, sc);
+        if (r < 32) {
+          p.bimg[ci * C + 2 * r] = gs.b0;
+          p.bimg[ci * C + 2 * r + 1] = gs.b1;
+        }
+      }
       if (c >= 2) {   // the product two steps back is done with this keys~ slot
         mbar_wait(&mma_done[slot], ((c >> 1) - 1) & 1, wc);
         tc_fence_after();
       }
-      write_ktilde<D, 4>(ek, smem + L::KT + slot * L::KV, r, (r >> 2) < nv ? __expf(lam + bC - bj) * iz : 0.f);
+      write_ktilde<D, 4>(ek, smem + L::KT + slot * L::KV, r, live ? __expf(lam + bC - bj) * iz : 0.f);
       lam += bC;
       fence_proxy_async_smem();
       tc_fence_before();
@@ -574,11 +619,11 @@ struct ChunkSmem {
   static constexpr uint32_t EQ = Q0 + QB;         // e_q' = alpha exp(q - q_0), bf16
   static constexpr uint32_t K0 = EQ + QB;         // 2 key slots, laid out [64-d block][slot][64 rows]
   static constexpr uint32_t V0 = K0 + 2 * KV;     // 3 value slots
-  static constexpr uint32_t PK = V0 + 3 * KV;     // e_k, unnormalised (exact-decay chunks only)
-  static constexpr uint32_t KT = PK + KV;         // decay-scaled phi(k)
-  static constexpr uint32_t SB = KT + KV;         // bf16 copy of the readout's state
+  static constexpr uint32_t KI = V0 + 3 * KV;     // 2 slots of the state pass's key-tile images
+  static constexpr uint32_t SB = KI + 2 * KV;     // bf16 copy of the readout's state
   static constexpr uint32_t SMALL = SB + D * D * 2;
   static constexpr uint32_t SMALL_BYTES = 4096;
+  static constexpr uint32_t BI = SMALL + 3072;    // 2 slots of the chunks' running log-gate sums
   static constexpr uint32_t BYTES = SMALL + SMALL_BYTES + 1024;   // + alignment slack
 };
 
@@ -621,14 +666,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   uint64_t* drain = bars + 20;
   uint64_t* state_ready = bars + 22; // state copied, S rescaled (256 arrivals)
   uint64_t* state_done = bars + 23;  // the chunk's state carry done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* kimg_full = bars + 24;   // [2] key-tile image and gate sums landed
+  uint64_t* kimg_empty = bars + 26;  // [2] the chunk's products are done with the image slot
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 30);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   volatile uint32_t* never = tmem_slot + 2;                     // stays 0: drain waits ignore aborts
   float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256 + 64);  // [2][64] running log-gate sums
   float* zq2 = bsh2 + 128;                                     // [2][128] Z = sum_d e_q per row
-  float* lg = zq2 + 256;                                        // [64] log gates of the current chunk
-  float* fast2 = lg + 64;                                       // [2] factored decay usable
-  float* izk2 = fast2 + 2;                                      // [2][64] 1 / z_k per key token
+  float* fast2 = zq2 + 256;                                     // [2] factored decay usable
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -647,6 +692,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     mbar_init(state_ready, 256); mbar_init(state_done, 1);
     mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
     mbar_init(drain, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&kimg_full[i], 1); mbar_init(&kimg_empty[i], 1); }
     *abort_flag = 0u;
     *never = 0u;
     fence_mbar_init();
@@ -689,12 +735,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(smem + L::Q0 + kb * ROWS * 128, &tmq, q_full, kb * 64, h0, sg.t_begin + c * C);
       };
-      int k_issued = 2, v_issued = 2, q_issued = 1;
+      auto load_img = [&](int c) {   // the state pass's key tile and gate sums of chunk c
+        const int slot = c & 1;
+        const size_t ci = (size_t)(seg * p.L + c) * p.Hkv + kv;
+        mbar_arrive_expect_tx(&kimg_full[slot], L::KV + C * 4);
+        bulk_load(smem + L::KI + slot * L::KV, p.kimg + ci * L::KV, L::KV, &kimg_full[slot]);
+        bulk_load(smem + L::BI + slot * (C * 4), p.bimg + ci * C, C * 4, &kimg_full[slot]);
+      };
+      int k_issued = 2, v_issued = 2, q_issued = 1, i_issued = 1;
+      load_img(0);
       load_k(0); load_v(0);
       load_k(1); load_v(1);
       load_q(0);
       for (int c = 0; c + 1 < nch; ++c) {
         const int u = c + 2;
+        if (c >= 1 && !mbar_wait(&kimg_empty[(c + 1) & 1], (((c + 1) >> 1) - 1) & 1, wc, wsite(1, 4, c))) break;
+        load_img(c + 1);
+        i_issued = c + 2;
         if (!mbar_wait(&k_empty[u & 1], ((u >> 1) - 1) & 1, wc, wsite(1, 1, c))) break;
         load_k(u);
         k_issued = u + 1;
@@ -709,6 +766,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       for (int u = (k_issued > 2 ? k_issued - 2 : 0); u < k_issued; ++u) mbar_wait(&k_full[u & 1], (u >> 1) & 1, dw);
       for (int u = (v_issued > 3 ? v_issued - 3 : 0); u < v_issued; ++u) mbar_wait(&v_full[u % 3], (u / 3) & 1, dw);
       mbar_wait(q_full, (q_issued - 1) & 1, dw);
+      for (int c = (i_issued > 2 ? i_issued - 2 : 0); c < i_issued; ++c) mbar_wait(&kimg_full[c & 1], (c >> 1) & 1, dw);
     }
   } else if (warp == kMmaWarp) {   // ---------------- MMA issuer
     if (lane == 0) {
@@ -719,8 +777,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const uint32_t lbo_kt = D == 128 ? C * 128 : 0;   // d = 64: both M halves read the same block
       const uint32_t q_base = smem_u32(smem + L::Q0);
       const uint32_t eq_base = smem_u32(smem + L::EQ);
-      const uint32_t pk_base = smem_u32(smem + L::PK);
-      const uint32_t kt_base = smem_u32(smem + L::KT);
+      const uint32_t ki_base = smem_u32(smem + L::KI);
       const uint32_t sb_base = smem_u32(smem + L::SB);
       bool ok = true;
       auto issue_ss = [&](int c) {   // window scores against the previous and the current keys
@@ -762,11 +819,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       };
       auto issue_sg_state = [&](int c) {
         // recurrent scores as soon as the feature warps are done
+        ok = ok && mbar_wait(&kimg_full[c & 1], (c >> 1) & 1, wc, wsite(2, 11, c));
         ok = ok && mbar_wait(feat, c & 1, wc, wsite(2, 7, c));
         if (!ok) return;
         tc_fence_after();
-        // factored mode: the scores against the decay-scaled keys; otherwise against e_k
-        const uint32_t kf_base = fast2[c & 1] != 0.f ? kt_base : pk_base;
+        // the image holds the decay-scaled keys (factored mode) or phi(k) (exact mode)
+        const uint32_t kf_base = ki_base + (c & 1) * L::KV;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * (ROWS * 128) + (kk & 3) * 32;
@@ -783,11 +841,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (!ok) return;
         tc_fence_after();
         const uint32_t vc = smem_u32(smem + L::V0 + ((c + 1) % 3) * L::KV);
+        // (exact mode: the feature warps have scaled the image to the decay-scaled keys by now)
 #pragma unroll
         for (int kk = 0; kk < C / 16; ++kk)
-          mma_bf16_ss(tmem + kColS, sdesc_sw128(kt_base + kk * 2048, lbo_kt, 1024),
+          mma_bf16_ss(tmem + kColS, sdesc_sw128(kf_base + kk * 2048, lbo_kt, 1024),
                       sdesc_sw128(vc + kk * 2048, C * 128, 1024), id_state, 1u);
         mma_commit(state_done);
+        mma_commit(&kimg_empty[c & 1]);   // the image slot may take chunk c + 2
       };
       auto issue_inter = [&](int c) {   // O = e_q' (e^{b_C} S) or (e^{b_i} e_q') S, the state as MN-major B
         if (c > 0) ok = ok && mbar_wait(o_free, (c - 1) & 1, wc, wsite(2, 9, c));
@@ -806,7 +866,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (!fast) mma_commit(q_empty);   // exact decay: the readout read e^{b_i} e_q from the q buffer
       };
       // A chunk's P.V goes out before the next chunk's window scores: the window warps
-      // wait for it, while the next scores are needed only after their epilogue.
+      // wait for it, while the next scores are needed only after their epilogue.  This
+      // order also guards the recurrent scores' TMEM: the window warps release the score
+      // columns (s_read) before they read the recurrent scores of the same chunk, and the
+      // next chunk's Sg is issued only after this chunk's P.V, which waits for p_ready.
       issue_ss(0);
       issue_sg_state(0);
       issue_inter(0);
@@ -820,11 +883,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mma_commit(drain);
     }
   } else if (warp >= kFeatWarp0) {   // ---------------- features (256 threads)
-    // One group does the chunk's key features (four threads per key token), then its
-    // query features (two threads per row), then the state copy (two warps per TMEM
-    // lane quarter, half the columns each).  Never leaves the loop early: after a
-    // timeout every wait returns at once (the CTA's abort flag is set), so the group
-    // still meets at each named barrier and warp-collective TMEM access stays uniform.
+    // Per chunk: the query features (two threads per row), then the state copy (two warps
+    // per TMEM lane quarter, half the columns each).  The key features come ready from the
+    // state pass (the image slots).  Never leaves the loop early: after a timeout every wait
+    // returns at once (the CTA's abort flag is set), so the group still meets at each named
+    // barrier and warp-collective TMEM access stays uniform.
     const int t = threadIdx.x - 32 * kFeatWarp0;
     const int half = t >> 7, lrow = t & 127;   // state-column half, TMEM lane (state row)
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -849,83 +912,67 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     tc_fence_after();
 
     for (int c = 0; c < nch; ++c) {
-      const int t0 = sg.t_begin + c * C;
-      const int nv = min(C, sg.t_end - t0);
+      const int slot = c & 1;
       float* bsh = bsh2 + (c & 1) * 64;
-      mbar_wait(&k_full[(c + 1) & 1], ((c + 1) >> 1) & 1, wc, wsite(3, 1, c));
-      if (c > 0) {   // e_k and keys~ are free once the previous scores and carry are done
-        mbar_wait(sg_done, (c - 1) & 1, wc, wsite(3, 3, c));
-        mbar_wait(state_done, (c - 1) & 1, wc, wsite(3, 7, c));
-      }
+      const float* bimg = reinterpret_cast<const float*>(smem + L::BI + slot * (C * 4));
+      mbar_wait(&kimg_full[slot], (c >> 1) & 1, wc, wsite(3, 1, c));
+      const int row = t >> 1, qh = t & 1;
+      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
+      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));   // e_q tile, state copy, row buffers free
       tc_fence_after();
-
-      // keys: e_k (unnormalised; 1/z_k goes into per-token scalars), gates, running sums,
-      // decay-scaled keys
-      const int j = t >> 2;
-      GateSums gs;
-      uint32_t ek[D / 8];
-      const float iz = key_features<D, 4, 2 * C * 128>(smem + L::K0 + ((c + 1) & 1) * (C * 128), nullptr,
-                                                        lg, bsh, t, nv, gs, ek);
-      const float bC = gs.at(nv - 1);
-      const float bj = gs.at(j);
-      write_ktilde<D, 4>(ek, smem + L::KT, t, j < nv ? __expf(bC - bj) * iz : 0.f);
       // Factored mode (the chunk's total log gate b_C >= -60): e^{b_i - b_j} =
       // e^{b_i - b_C} e^{b_C - b_j}, both factors within e^{+-60}.  The key factor is the one
-      // the decay-scaled keys carry, so the recurrent scores are taken against that tile and
-      // need no per-key scalar; the row factor goes to the epilogue, and the readout uses
-      // e^{b_C} S, which is the rescaled state.  A key feature below 2^-126 e^{b_j - b_C} is
-      // flushed in the tile; the bound keeps the resulting error of a score under
-      // 2^-126 e^{60} ~ 1e-12.  Otherwise the scores come from e_k, written only then.
-      const bool fast = bC >= -60.f;
-      if (!fast) {   // the same decision for the whole CTA
-        const int h = t & 3;
-#pragma unroll
-        for (int c8 = 0; c8 < D / 32; ++c8)
-          *reinterpret_cast<uint4*>(smem + L::PK + kmajor_off(j, h * (D / 4) + c8 * 8, C * 128)) =
-              make_uint4(ek[4 * c8], ek[4 * c8 + 1], ek[4 * c8 + 2], ek[4 * c8 + 3]);
-      }
-      if ((t & 3) == 0) izk2[(c & 1) * 64 + j] = iz;
+      // the image's decay-scaled keys carry, so the recurrent scores need no per-key scalar;
+      // the row factor goes to the epilogue, and the readout uses e^{b_C} S, which is the
+      // rescaled state.  Otherwise the image holds phi(k) and the window warps apply the
+      // decay per element.
+      const float bC = bimg[C - 1];
+      const bool fast = bC >= kFactorFloor;   // the same decision for the whole CTA
+      if (t < C) bsh[t] = bimg[t];
       if (t == 0) fast2[c & 1] = fast ? 1.f : 0.f;
 
       // queries: e_q' = a exp(q - q_0) per row (bf16, with the branch weight a above; not
       // divided by Z = sum_d e_q: the window warps fold Z into P and 1/Z into the output);
-      // two threads per row
-      const int row = t >> 1, qh = t & 1;
-      mbar_wait(q_full, c & 1, wc, wsite(3, 2, c));
-      if (c > 0) mbar_wait(mma2_done, (c - 1) & 1, wc, wsite(3, 6, c));   // e_q tile and state copy free
-      // one pass: e_q = exp(q - q_0) with q_0 the row's first element (the tiles carry e_q
-      // unnormalised, so the shift cancels against Z), redone against the row maximum if
-      // the spread is too large (see kShiftSpan)
+      // two threads per row.  One pass against the row's first element q_0 (the tiles carry
+      // e_q unnormalised, so the shift cancels against Z); a row whose Z exceeds 2^24 (every
+      // row with an element more than kShiftSpan above q_0, in log2) is redone against its
+      // maximum.
       const float sl = bf16_lo(*reinterpret_cast<const uint32_t*>(qb + kmajor_off(row, 0, ROWS * 128))) * kLog2e;
-      const float sla = sl - lqa;
-      float mq = -INFINITY, za = 0.f, zb = 0.f;
+      const float2 nsla = make_float2(lqa - sl, lqa - sl), l2e = make_float2(kLog2e, kLog2e);
+      float2 zacc = make_float2(0.f, 0.f);
 #pragma unroll 4
       for (int c8 = 0; c8 < D / 16; ++c8) {
         const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
         const uint4 u = *reinterpret_cast<const uint4*>(qb + off);
-        mq = fmaxf(mq, bf16x8_max(u));
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-        float x[8];
+        float2 x[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) { x[2 * q] = bf16_lo(w4[q]); x[2 * q + 1] = bf16_hi(w4[q]); }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -sla));
-        za += (x[0] + x[1]) + (x[2] + x[3]);
-        zb += (x[4] + x[5]) + (x[6] + x[7]);
-        st_chunk8(eqb, off, x);
+        for (int q = 0; q < 4; ++q) {
+          x[q] = ffma2(make_float2(bf16_lo(w4[q]), bf16_hi(w4[q])), l2e, nsla);
+          x[q].x = ex2(x[q].x);
+          x[q].y = ex2(x[q].y);
+        }
+        zacc = fadd2(zacc, fadd2(fadd2(x[0], x[1]), fadd2(x[2], x[3])));
+        *reinterpret_cast<uint4*>(eqb + off) = make_uint4(pack_bf16(x[0].x, x[0].y), pack_bf16(x[1].x, x[1].y),
+                                                          pack_bf16(x[2].x, x[2].y), pack_bf16(x[3].x, x[3].y));
       }
-      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
-      float zq = za + zb;
+      float zq = zacc.x + zacc.y;
       zq += __shfl_xor_sync(0xffffffffu, zq, 1);
       // decided per row (the same on both of its threads), entered by the whole warp so
-      // that the shuffle sees every lane
-      const bool redo = mq * kLog2e - sl > kShiftSpan;
+      // that the shuffles see every lane
+      const bool redo = !(zq * iqa <= 0x1p24f);
       if (__any_sync(0xffffffffu, redo)) {
+        float mq = -INFINITY;
+        if (redo) {
+#pragma unroll 1
+          for (int c8 = 0; c8 < D / 16; ++c8)
+            mq = fmaxf(mq, bf16x8_max(*reinterpret_cast<const uint4*>(
+                               qb + kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128))));
+        }
+        mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 1));
         float zr = 0.f;
         if (redo) {
           const float mql = mq * kLog2e - lqa;
-          za = 0.f;
-          zb = 0.f;
 #pragma unroll 1
           for (int c8 = 0; c8 < D / 16; ++c8) {
             const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
@@ -933,11 +980,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             ld_chunk8(qb, off, x);
 #pragma unroll
             for (int q = 0; q < 8; ++q) x[q] = ex2(fmaf(x[q], kLog2e, -mql));
-            za += (x[0] + x[1]) + (x[2] + x[3]);
-            zb += (x[4] + x[5]) + (x[6] + x[7]);
+            zr += ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
             st_chunk8(eqb, off, x);
           }
-          zr = za + zb;
         }
         zr += __shfl_xor_sync(0xffffffffu, zr, 1);
         if (redo) zq = zr;
@@ -951,7 +996,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (t == 0) mbar_arrive(q_empty);
       } else {
         mbar_wait(ss_done, c & 1, wc, wsite(3, 4, c));
-        const float ebi = __expf(gs.at(row >> 1));
+        const float ebi = __expf(bimg[row >> 1]);
 #pragma unroll 4
         for (int c8 = 0; c8 < D / 16; ++c8) {
           const uint32_t off = kmajor_off(row, qh * (D / 2) + c8 * 8, ROWS * 128);
@@ -966,14 +1011,34 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       tc_fence_before();
       mbar_arrive(feat);
 
+      if (!fast) {
+        // exact mode: once the recurrent scores have read phi(k) from the image, scale it in
+        // place to the decay-scaled keys e^{b_C - b_j} phi(k_j) the state carry needs
+        mbar_wait(sg_done, c & 1, wc, wsite(3, 3, c));
+        const int j = t >> 2, h = t & 3;
+        const float sc = __expf(bC - bimg[j]);
+        char* const ki = smem + L::KI + slot * L::KV;
+#pragma unroll
+        for (int c8 = 0; c8 < D / 32; ++c8) {
+          const uint32_t off = kmajor_off(j, h * (D / 4) + c8 * 8, C * 128);
+          float x[8];
+          ld_chunk8(ki, off, x);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) x[q] *= sc;
+          st_chunk8(ki, off, x);
+        }
+      }
+
       // State for this chunk: the bf16 copy of the readout's state (MN-major B operand),
       // then S <- e^{b_C} S in TMEM before the chunk's carry accumulates onto it (the
-      // previous carry and readout are done, above).  Factored mode reads out e^{b_C} S,
-      // the rescaled state itself; exact mode reads out S (its q buffer holds e^{b_i} e_q).
+      // previous carry and readout are done).  Factored mode reads out e^{b_C} S, the
+      // rescaled state itself; exact mode reads out S (its q buffer holds e^{b_i} e_q).
       // Either copy carries the part of alpha that the e_q tile does not.
+      if (c > 0) mbar_wait(state_done, (c - 1) & 1, wc, wsite(3, 7, c));
       tc_fence_after();
       {
         const float dec = __expf(bC);
+        const float2 dec2 = make_float2(dec, dec);
         if (fast && copy_scale == 1.f) {   // the same for the whole CTA
 #pragma unroll 1
           for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
@@ -981,7 +1046,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
             tmem_ld32(lane_base + kColS + col, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) v[u] *= dec;
+            for (int u = 0; u < 32; u += 2) {
+              const float2 y = fmul2(make_float2(v[u], v[u + 1]), dec2);
+              v[u] = y.x;
+              v[u + 1] = y.y;
+            }
             if (lrow < D) {
 #pragma unroll
               for (int u = 0; u < 32; u += 8)
@@ -1015,7 +1084,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(state_ready);
-      named_bar(1, 256);   // lg is rewritten by the next chunk's keys
     }
     // final state of the sequence: the carry after the last chunk of its last segment
     const SeqInfo si = p.seqs[sg.seq];
@@ -1059,7 +1127,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int t0 = sg.t_begin + c * C;
       const int nv = min(C, sg.t_end - t0);
       const float* bsh = bsh2 + (c & 1) * 64;
-      const float* izk = izk2 + (c & 1) * 64;
       // Window band.  Key index x over [previous chunk | current chunk] (0..127): row i
       // sees x in [i+1, i+64].  This quarter's tokens are 16 wq .. 16 wq + 15, so it reads
       // the 80 columns starting at 16 wq; column j then holds x = 16 wq + j and is live for
@@ -1067,52 +1134,42 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int jlo = max(il + 1, t0 == sg.q0 ? 64 - 16 * wq : 0), jhi = il + 64;
       // score column of key x: (x + 64 (c & 1)) mod 128 (the two key slots form one operand)
       const int ss_rot = 16 * wq + ((c & 1) << 6);
-      auto ss_col = [&](int q5) { return lane_base + kColSs + ((ss_rot + 16 * q5) & 127); };
       mbar_wait(ss_done, c & 1, wc, wsite(4, 6, c));
       tc_fence_after();
+      // The row's 80 scores, loaded once and kept in registers.
+      float s[80];
+#pragma unroll
+      for (int q5 = 0; q5 < 5; ++q5) tmem_ld16(lane_base + kColSs + ((ss_rot + 16 * q5) & 127), s + 16 * q5);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_read);   // the score columns are in registers: their TMEM may be reused
       // Columns 16..63 are inside every row's band except in the sequence's first chunk:
-      // only the outer groups (and that chunk) take the mask.
+      // only the outer groups (and that chunk) take the mask, as -inf, whose exponential is 0.
       const bool first = t0 == sg.q0;
+#pragma unroll
+      for (int q5 = 0; q5 < 5; ++q5) {
+        if (first || q5 == 0 || q5 == 4) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int j = 16 * q5 + u;
+            s[16 * q5 + u] = (j >= jlo && j <= jhi) ? s[16 * q5 + u] : -INFINITY;
+          }
+        }
+      }
       float m = -INFINITY;
-#pragma unroll 1
-      for (int q5 = 0; q5 < 5; ++q5) {
-        float s[16];
-        tmem_ld16(ss_col(q5), s);
-        tmem_wait_ld();
-        if (first || q5 == 0 || q5 == 4) {
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int j = 16 * q5 + u;
-            s[u] = (j >= jlo && j <= jhi) ? s[u] : -INFINITY;
-          }
-        }
+      for (int u = 0; u < 80; u += 2) m = fmax3(m, s[u], s[u + 1]);
+      const float2 sc2 = make_float2(sscale, sscale), nmsc = make_float2(-m * sscale, -m * sscale);
+      float2 lsum = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-          for (int u = 0; u < w; ++u) s[u] = fmaxf(s[u], s[u + w]);
-        m = fmaxf(m, s[0]);
+      for (int u = 0; u < 80; u += 2) {
+        float2 y = ffma2(make_float2(s[u], s[u + 1]), sc2, nmsc);
+        y.x = ex2(y.x);
+        y.y = ex2(y.y);
+        s[u] = y.x;
+        s[u + 1] = y.y;
+        lsum = fadd2(lsum, y);
       }
-      const float msc = m * sscale;
-      float la = 0.f, lb = 0.f;   // exps written back over the scores
-#pragma unroll 1
-      for (int q5 = 0; q5 < 5; ++q5) {
-        float s[16];
-        tmem_ld16(ss_col(q5), s);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) s[u] = ex2(fmaf(s[u], sscale, -msc));
-        if (first || q5 == 0 || q5 == 4) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int j = 16 * q5 + u;
-            s[u] = (j >= jlo && j <= jhi) ? s[u] : 0.f;
-          }
-        }
-        la += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
-        lb += ((s[8] + s[9]) + (s[10] + s[11])) + ((s[12] + s[13]) + (s[14] + s[15]));
-        tmem_st16(ss_col(q5), s);
-      }
-      tmem_wait_st();
       // Z of the rows and the recurrent scores come with the feature tiles
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
       tc_fence_after();
@@ -1122,34 +1179,47 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float zrow = zq2[(c & 1) * 128 + r];
       const float bi = bsh[i];
       const float mrow = fast ? bsh[nv - 1] - bi : 0.f;
-      const float coef = beta * zrow * __expf(mrow) / (la + lb);
+      const float coef = beta * zrow * __expf(mrow) / (lsum.x + lsum.y);
       const float oscale = __expf(-mrow) / zrow;
+      const float2 coef2 = make_float2(coef, coef), gs2 = make_float2(gscale, gscale);
       // Probability tile over [previous | current] keys.  The recurrent tile covers the
       // same current keys (kk <= i) and multiplies the same values, so it is added to the
       // window tile's current half here: one P V product per half.  Group q5 holds the
       // current keys kk = 16 bb + u with bb = q5 + wq - 4 when bb >= 0.
-#pragma unroll 1
+#pragma unroll
       for (int q5 = 0; q5 < 5; ++q5) {
         const int bb = q5 + wq - 4;
-        float s[16], g[16];
-        tmem_ld16(ss_col(q5), s);
-        if (bb >= 0) tmem_ld16(lane_base + kColSg + 16 * bb, g);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) s[u] *= coef;
+        float* sv = s + 16 * q5;
         if (bb >= 0) {
+          float g[16];
+          tmem_ld16(lane_base + kColSg + 16 * bb, g);
+          tmem_wait_ld();
+          if (!fast) {   // exact mode: scores against phi(k); the decay per element
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int kk = 16 * bb + u;
-            // factored: the scores already carry e^{b_C - b_kk} / z_kk; exact: e_q e_k scores
-            float gv = fast ? g[u] * gscale : g[u] * (gscale * __expf(bi - bsh[kk]) * izk[kk]);
-            if (bb == wq) gv = kk <= i ? gv : 0.f;       // the diagonal block is causal
-            s[u] += gv;
+            for (int u = 0; u < 16; ++u) g[u] *= __expf(bi - bsh[16 * bb + u]);
+          }
+          if (bb == wq) {   // the diagonal block is causal
+#pragma unroll
+            for (int u = 0; u < 16; ++u) g[u] = 16 * bb + u <= i ? g[u] : 0.f;
+          }
+          // factored: the scores already carry e^{b_C - b_kk} / z_kk
+#pragma unroll
+          for (int u = 0; u < 16; u += 2) {
+            const float2 y = ffma2(make_float2(g[u], g[u + 1]), gs2, fmul2(make_float2(sv[u], sv[u + 1]), coef2));
+            sv[u] = y.x;
+            sv[u + 1] = y.y;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; u += 2) {
+            const float2 y = fmul2(make_float2(sv[u], sv[u + 1]), coef2);
+            sv[u] = y.x;
+            sv[u + 1] = y.y;
           }
         }
         uint32_t pw[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
+        for (int k = 0; k < 8; ++k) pw[k] = pack_bf16(sv[2 * k], sv[2 * k + 1]);
         tmem_st8u(lane_base + kColP + 8 * wq + 8 * q5, pw);
       }
       {   // zeros for the keys outside this quarter's band
@@ -1159,7 +1229,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(s_read);    // the scores are consumed: their TMEM may be reused
       mbar_arrive(p_ready);   // the probability tile is in TMEM
 
       // epilogue: O -> bf16 rows of out
@@ -1176,8 +1245,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
           tmem_wait_ld();
           if (store) {
             uint32_t pw[16];
+            const float2 os2 = make_float2(oscale, oscale);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) pw[u] = pack_bf16(v[2 * u] * oscale, v[2 * u + 1] * oscale);
+            for (int u = 0; u < 16; ++u) {
+              const float2 y = fmul2(make_float2(v[2 * u], v[2 * u + 1]), os2);
+              pw[u] = pack_bf16(y.x, y.y);
+            }
             if (p.out_v8) {   // two full 32-byte sectors per instruction
               st_global_v8(orow + col, pw);
               st_global_v8(orow + col + 16, pw + 8);
@@ -1277,6 +1350,9 @@ inline Plan make_plan(int B, int Hq, int Hkv, long T, int d, int n_seqs, bool va
   pl.off_segs = off;  off = al(off + sizeof(SegInfo) * (size_t)nseg);
   pl.off_lam = off;   off = al(off + sizeof(float) * (size_t)nseg * nsub * Hkv);
   pl.off_ds = off;    off = al(off + sizeof(float) * (size_t)nseg * nsub * Hkv * d * d);
+  pl.off_kimg = off;  off = al(off + (size_t)2 * C * d * (size_t)nseg * bestL * Hkv);
+  pl.off_bimg = off;  off = al(off + sizeof(float) * C * (size_t)nseg * bestL * Hkv);
+  pl.off_flags = off; off = al(off + sizeof(uint32_t) * (size_t)n_seqs * Hkv);
   pl.total = off;
   return pl;
 }
@@ -1332,12 +1408,10 @@ inline cudaError_t launch_chained(void (*kern)(KArgs...), dim3 grid, dim3 block,
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-template <int D>
-liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk) {
-  const bool varlen = pb.cu != nullptr;
-  const long NT = varlen ? pb.T : (long)pb.B * pb.T;
-  const Plan pl = make_plan(pb.B, pb.Hq, pb.Hkv, pb.T, D, pb.n_seqs, varlen);
-  char* w = static_cast<char*>(ws);
+// On return, *s0_flags (when not null) points at the per-(sequence, kv head) flags the scan
+// sets for groups whose initial-state copies differ (only meaningful with pb.s0).
+// Kernel parameters of a call whose workspace `w` follows plan `pl`.
+inline DevParams fill_params(const PrefillProblem& pb, char* w, const Plan& pl, long NT) {
   DevParams p{};
   p.seqs = reinterpret_cast<const SeqInfo*>(w + pl.off_seqs);
   p.segs = reinterpret_cast<const SegInfo*>(w + pl.off_segs);
@@ -1345,8 +1419,12 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   p.err = reinterpret_cast<uint32_t*>(w);
   p.lam = reinterpret_cast<float*>(w + pl.off_lam);
   p.ds = reinterpret_cast<float*>(w + pl.off_ds);
+  p.kimg = w + pl.off_kimg;
+  p.bimg = reinterpret_cast<float*>(w + pl.off_bimg);
   p.out = pb.out;
   p.final_state = pb.final_state;
+  p.s0 = pb.s0;
+  p.s0_flags = reinterpret_cast<uint32_t*>(w + pl.off_flags);
   p.cu = pb.cu;
   p.T = pb.T;
   p.NT = NT;
@@ -1360,6 +1438,17 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   p.alpha = pb.alpha;
   p.wait_ns = wait_limit_ns();
   p.out_v8 = (reinterpret_cast<uintptr_t>(pb.out) & 31u) == 0 ? 1 : 0;
+  return p;
+}
+
+template <int D>
+liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk,
+                           const uint32_t** s0_flags) {
+  const bool varlen = pb.cu != nullptr;
+  const long NT = varlen ? pb.T : (long)pb.B * pb.T;
+  const Plan pl = make_plan(pb.B, pb.Hq, pb.Hkv, pb.T, D, pb.n_seqs, varlen);
+  char* w = static_cast<char*>(ws);
+  DevParams p = fill_params(pb, w, pl, NT);
   p.inject_stall = take_injected_stall() ? 1 : 0;
 
   CUtensorMap mq, mk, mv;
@@ -1410,12 +1499,14 @@ liger_status run_prefill_d(const PrefillProblem& pb, void* ws, cudaStream_t s, c
   hk.after_main(s);
   hk.count(1);
   if (e != cudaSuccess) { g_msg = cudaGetErrorString(e); return LIGER_ERR_CUDA; }
+  if (s0_flags) *s0_flags = p.s0_flags;
   return LIGER_OK;
 }
 
-inline liger_status run_prefill(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk) {
+inline liger_status run_prefill(const PrefillProblem& pb, void* ws, cudaStream_t s, const LaunchHooks& hk,
+                                const uint32_t** s0_flags = nullptr) {
   g_msg = "";
-  return pb.d == 64 ? run_prefill_d<64>(pb, ws, s, hk) : run_prefill_d<128>(pb, ws, s, hk);
+  return pb.d == 64 ? run_prefill_d<64>(pb, ws, s, hk, s0_flags) : run_prefill_d<128>(pb, ws, s, hk, s0_flags);
 }
 
 }  // namespace tc

@@ -43,6 +43,11 @@ SIGNATURES = {
     "liger_attn_prefill_noalloc_status": (_i, []),
     "liger_attn_prefill_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                                      ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_size_t)]),
+    "liger_attn_prefill_backward_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
+    "liger_attn_prefill_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _i,
+                                         _vp, _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "liger_attn_full_causal": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp]),
+    "liger_attn_full_causal_status": (_i, []),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }
@@ -258,3 +263,81 @@ def prefill_status(workspace) -> int:
     if workspace is None:
         return LIGER_OK
     return int(load().liger_attn_prefill_status(_ptr(workspace), workspace.numel() * workspace.element_size()))
+
+
+def full_causal_attention(q, k, v, cu_seqlens=None, max_seqlen=None, out=None, stream=None):
+    """Causal softmax attention (the hybrid's standard attention layer), bf16.
+
+    q [B, T, Hq, d], k and v [B, T, Hkv, d]; cu_seqlens as for `prefill` (B must be 1), with
+    max_seqlen the longest sequence (computed from cu_seqlens when not given, which reads it
+    back to the host).  Returns out [B, T, Hq, d].
+    """
+    lib = load()
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, T, Hq, d] and k, v [B, T, Hkv, d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _expect(k, "k", (B, T, Hkv, d), q.dtype)
+    _expect(v, "v", (B, T, Hkv, d), q.dtype)
+    _expect(out, "out", (B, T, Hq, d), q.dtype)
+    if cu_seqlens is not None and (cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2
+                                   or cu_seqlens.dtype != torch.int32):
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of n + 1 offsets")
+    _need_cuda(q, k, v, out, cu_seqlens)
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item())
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib.liger_attn_full_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, Hq, Hkv, T, d, _dt(q),
+                                    _ptr(cu_seqlens), n, 0 if max_seqlen is None else int(max_seqlen),
+                                    _stream_ptr(stream))
+    _check(st)
+    return out
+
+
+def full_causal_status() -> int:
+    """LIGER_OK, or LIGER_ERR_TIMEOUT if a causal attention call gave up waiting since the last query."""
+    return int(load().liger_attn_full_causal_status())
+
+
+def prefill_backward_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:
+    return int(load().liger_attn_prefill_backward_workspace_size(
+        B, Hq, Hkv, T, d, n_seqs, LIGER_BF16 if dtype == torch.bfloat16 else LIGER_FP32))
+
+
+def prefill_backward(q, k, v, d_out, alpha: float = 0.5, w: int = 64, d_final_state=None,
+                     initial_state=None, cu_seqlens=None, want_d_initial_state: bool = False,
+                     workspace=None, stream=None):
+    """Gradient of `prefill` for L = sum(d_out * out) + sum(d_final_state * final_state).
+
+    initial_state and the returned d_initial_state are one per (sequence, kv head):
+    [n, Hkv, d, d] fp32.  Returns (dq, dk, dv, d_initial_state or None).
+    """
+    lib = load()
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, T, Hq, d] and k, v [B, T, Hkv, d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _expect(k, "k", (B, T, Hkv, d), q.dtype)
+    _expect(v, "v", (B, T, Hkv, d), q.dtype)
+    _expect(d_out, "d_out", (B, T, Hq, d), q.dtype)
+    if cu_seqlens is not None and (cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2
+                                   or cu_seqlens.dtype != torch.int32):
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of n + 1 offsets")
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    _expect(d_final_state, "d_final_state", (n, Hq, d, d), torch.float32)
+    _expect(initial_state, "initial_state", (n, Hkv, d, d), torch.float32)
+    _need_cuda(q, k, v, d_out, d_final_state, initial_state, cu_seqlens, workspace)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds0 = torch.empty(n, Hkv, d, d, device=q.device, dtype=torch.float32) if want_d_initial_state else None
+    need = prefill_backward_workspace_size(B, Hq, Hkv, T, d, n, q.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.liger_attn_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(d_out), _ptr(d_final_state), _ptr(initial_state), B, Hq, Hkv, T, d, w,
+        float(alpha), _dt(q), _ptr(cu_seqlens), n, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds0), _ptr(workspace),
+        ws_bytes, _stream_ptr(stream))
+    _check(st)
+    return dq, dk, dv, ds0

@@ -72,7 +72,7 @@ size_t liger_attn_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, i
 
 /*
  * The launch plan the tensor-core prefill (bf16, d in {64, 128}, even
- * Hq/Hkv, w = 64, no initial state) uses for these sizes.  Host only: no
+ * Hq/Hkv, w = 64) uses for these sizes.  Host only: no
  * device work; the planner reads the current device's SM count, or assumes
  * 148 when no device is present.  (The pages have no counterpart: the
  * sequence split is this implementation's way of filling the GPU.)
@@ -109,7 +109,12 @@ liger_status liger_attn_prefill_plan(int B, int Hq, int Hkv, int T, int d, int n
  *   final_state  [n, Hq, d, d]  fp32        (out, nullable) state after the last
  *                token of each sequence; every q head of a group gets its copy.
  *   initial_state[n, Hq, d, d]  fp32        (in, nullable = zero) seeds the
- *                recurrence; the window still starts at the first token.
+ *                recurrence; the window still starts at the first token.  The
+ *                tensor-core path runs the q heads of a group from one state; a
+ *                (sequence, group) whose heads' initial states differ is
+ *                recomputed by the general kernel within the same call (correct,
+ *                slower).  A final_state passed back as the next call's
+ *                initial_state always has equal copies.
  *   cu_seqlens   [n + 1]        int32       (in, nullable) packed variable-length
  *                sequences: offsets into the T axis, first 0, last T, non-
  *                decreasing; requires B == 1.  The state and the window restart
@@ -233,6 +238,59 @@ liger_status liger_attn_prefill_noalloc_status(void);
  *                                detection without a GPU fault); later calls
  *                                run normally
  */
+
+/*
+ * Gradient of liger_attn_prefill (bf16 tensor-core path).  The pages give no
+ * backward pass; the linearisation fine-tune of the news article on Liger
+ * (section "軽量ファインチューニング": LoRA on the Q/K/V projections, trained
+ * with next-token cross-entropy through this layer) needs one.  For the loss
+ * L = sum(d_out * out) + sum(d_final_state * final_state) of the prefill with
+ * the same q, k, v, w, alpha, cu_seqlens and initial state:
+ *   dq           [B, T, Hq, d]  bf16  (out)  dL/dq
+ *   dk, dv       [B, T, Hkv, d] bf16  (out)  dL/dk, dL/dv (summed over each group's q heads)
+ *   d_out        [B, T, Hq, d]  bf16  (in)
+ *   d_final_state[n, Hq, d, d]  fp32  (in, nullable = zero)
+ *   initial_state[n, Hkv, d, d] fp32  (in, nullable = zero) the initial state as the
+ *                recurrence carries it, one per (sequence, kv head); a per-q-head
+ *                state whose G copies are equal (as every final_state is) passes as
+ *                its first copy of each group.
+ *   d_initial_state [n, Hkv, d, d] fp32 (out, nullable) dL/d initial_state (the sum
+ *                over the group's heads of the per-head gradients).
+ *   workspace    liger_attn_prefill_backward_workspace_size() bytes of device scratch.
+ * Supported: bf16, d in {64, 128}, w = 64, even Hq/Hkv (else LIGER_ERR_UNSUPPORTED).
+ * Every internal wait is bounded; liger_attn_prefill_status(workspace, bytes)
+ * reports a timeout as for the forward.
+ */
+size_t liger_attn_prefill_backward_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                                  liger_dtype dt);
+liger_status liger_attn_prefill_backward(const void* q, const void* k, const void* v, const void* d_out,
+                                         const float* d_final_state, const float* initial_state, int B, int Hq,
+                                         int Hkv, int T, int d, int w, float alpha, liger_dtype dt,
+                                         const int32_t* cu_seqlens, int n_seqs, void* dq, void* dk, void* dv,
+                                         float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
+ * Causal softmax attention: the standard attention layer of the inter-layer
+ * hybrid (news article on Liger, section "ハイブリッドメカニズム": one full
+ * softmax attention layer after every seven Liger layers; Paper-Notes page,
+ * section "Liger 整体架构").  Per query head h with kv head h / (Hq/Hkv):
+ *   o_t = sum_{j <= t} softmax_j(q_t . k_j / sqrt(d)) v_j   within each sequence.
+ *
+ *   q, out  [B, T, Hq, d]  bf16;  k, v  [B, T, Hkv, d]  bf16
+ *   cu_seqlens [n + 1] int32 (device, nullable) packed sequences as for the
+ *           prefill (then B == 1 and n = n_seqs; otherwise n_seqs == B);
+ *   max_seqlen  the longest sequence (read only with cu_seqlens; it sizes the
+ *           grid, so it must be at least every sequence's length).
+ * Supported: bf16, d in {64, 128}.  fp32 returns LIGER_ERR_UNSUPPORTED.  Every
+ * internal wait is bounded (as for the prefill); liger_attn_full_causal_status()
+ * reports whether any call on the current device gave up since the last query
+ * (synchronous read; call it after the stream has completed; it clears the report).
+ */
+liger_status liger_attn_full_causal(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                    int Hkv, int T, int d, liger_dtype dt, const int32_t* cu_seqlens, int n_seqs,
+                                    int max_seqlen, void* stream);
+liger_status liger_attn_full_causal_status(void);
 
 /* Message of the last failure on the calling thread ("" if none). */
 const char* liger_last_error(void);

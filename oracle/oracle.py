@@ -233,3 +233,27 @@ def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthread
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
     return out, st, rg, ps
+
+
+def causal_attention_rows(q, k, v, rows, cu_seqlens=None):
+    """Causal softmax attention o_t = sum_{j <= t} softmax_j(q_t . k_j / sqrt(d)) v_j, written out
+    row by row for the requested rows only (numpy, float64); the sequence containing each row
+    bounds its keys.
+
+    q [B, T, Hq, d]; k, v [B, T, Hkv, d]; rows: iterable of (b, t, h).  Returns [len(rows), d].
+    This is the standard attention layer of the inter-layer hybrid (news article on Liger, section
+    ハイブリッドメカニズム: one full softmax attention layer after every seven Liger layers); it is
+    also the window branch with a window covering the whole sequence.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    G = Hq // k.shape[2]
+    starts = None if cu_seqlens is None else np.asarray(cu_seqlens, dtype=np.int64)
+    res = np.empty((len(rows), d))
+    for n, (b, t, h) in enumerate(rows):
+        t0 = 0 if starts is None else int(starts[np.searchsorted(starts, t, side="right") - 1])
+        kv = h // G
+        s = k[b, t0:t + 1, kv] @ q[b, t, h] / np.sqrt(d)
+        p = np.exp(s - s.max())
+        res[n] = (p / p.sum()) @ v[b, t0:t + 1, kv]
+    return res

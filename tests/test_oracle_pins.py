@@ -321,3 +321,30 @@ def test_decode_inplace_steps_equal_a_longer_prefill():
     np.testing.assert_array_equal(ps, pos_full)
     with pytest.raises(ValueError):
         oracle.decode_inplace(q[:, 0], k[:, 0], v[:, 0], st.astype(np.float32), rg, ps)
+
+
+def test_causal_attention_rows_equal_the_window_branch_and_sdpa():
+    """The row-wise causal attention reference equals the C oracle's window branch with a window
+    covering the sequence and alpha = 0, and torch's causal scaled_dot_product_attention (fp64);
+    with packed sequences each row sees only its own sequence."""
+    import torch
+    B, T, Hq, Hkv, d = 2, 13, 4, 2, 8
+    q, k, v = rand(B, T, Hq, d), rand(B, T, Hkv, d), rand(B, T, Hkv, d)
+    rows = [(b, t, h) for b in range(B) for t in range(T) for h in range(Hq)]
+    got = oracle.causal_attention_rows(q, k, v, rows)
+    ref = oracle.prefill(q, k, v, w=T, alpha=0.0)[0]
+    np.testing.assert_allclose(got, np.array([ref[b, t, h] for b, t, h in rows]), rtol=1e-12, atol=1e-13)
+    G = Hq // Hkv
+    qt = torch.tensor(q).permute(0, 2, 1, 3)
+    kt = torch.tensor(np.repeat(k, G, axis=2)).permute(0, 2, 1, 3)
+    vt = torch.tensor(np.repeat(v, G, axis=2)).permute(0, 2, 1, 3)
+    sd = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(got, np.array([sd[b, t, h] for b, t, h in rows]), rtol=1e-10, atol=1e-12)
+    cu = [0, 5, 5, 13]
+    q1, k1, v1 = q[:1], k[:1], v[:1]
+    rows1 = [(0, t, h) for t in range(T) for h in range(Hq)]
+    got1 = oracle.causal_attention_rows(q1, k1, v1, rows1, cu_seqlens=cu)
+    for a, b_ in ((0, 5), (5, 13)):
+        sep = oracle.causal_attention_rows(q1[:, a:b_], k1[:, a:b_], v1[:, a:b_],
+                                           [(0, t, h) for t in range(b_ - a) for h in range(Hq)])
+        np.testing.assert_allclose(got1[a * Hq:b_ * Hq], sep, rtol=1e-13, atol=1e-14)

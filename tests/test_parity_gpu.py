@@ -341,3 +341,67 @@ def test_decode_kvshared_matches_per_head_decode_full_shape(cuda_device):
         assert_close(np64(o2), np64(o1), wl.dtype, f"step {step}")
     assert_close(np64(st_kv), np64(st[:, ::G]), wl.dtype, "state")
     assert torch.equal(rg, rg2) and torch.equal(ps, ps2)
+
+
+# ----------------------------------------------------------------- initial states on the tensor-core path
+
+def _group_shared_state(n, Hq, Hkv, d, seed, differ_groups=()):
+    """Initial states whose G copies are equal within each group, except in the listed
+    (sequence, kv head) groups, whose heads get states of their own."""
+    G = Hq // Hkv
+    base = inputs.random_state(n, Hkv, d, seed=seed, scale=0.05)
+    s0 = base.repeat_interleave(G, dim=1).contiguous()
+    if differ_groups:
+        other = inputs.random_state(n, Hq, d, seed=seed + 1, scale=0.05)
+        for seq, kv in differ_groups:
+            s0[seq, kv * G:(kv + 1) * G] = other[seq, kv * G:(kv + 1) * G]
+    return s0
+
+
+@pytest.mark.parametrize("name,B,Hq,Hkv,T,d,seqlens,differ", [
+    ("shared_d128", 2, 8, 2, 300, 128, (), ()),
+    ("shared_d64_packed_empty", 1, 8, 4, 260, 64, (90, 0, 170), ()),
+    ("mixed_groups_d128", 2, 8, 2, 200, 128, (), ((0, 1), (1, 0))),
+    ("mixed_groups_d64_packed", 1, 8, 2, 210, 64, (70, 140), ((1, 1),)),
+])
+def test_prefill_initial_state_tensor_core(name, B, Hq, Hkv, T, d, seqlens, differ, cuda_device):
+    """bf16, w = 64, even G: the tensor-core path takes the initial state.  Groups whose heads
+    share a state run on it; groups whose heads differ are recomputed in the same call."""
+    wl = inputs.small(name, B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, seed=zlib.crc32(name.encode()) % 10000, seqlens=seqlens)
+    q, k, v = inputs.prefill_inputs(wl)
+    n = wl.n_seqs
+    s0 = _group_shared_state(n, Hq, Hkv, d, seed=13, differ_groups=differ)
+    cu = wl.cu_seqlens
+    dev = cuda_device
+    plan = ops.prefill_plan(B, Hq, Hkv, T, d, n, packed=cu is not None)
+    assert plan["chunks_per_segment"] >= 1   # the tensor-core path takes these sizes
+    out, fs = ops.prefill(q.to(dev), k.to(dev), v.to(dev), initial_state=s0.to(dev),
+                          cu_seqlens=None if cu is None else torch.tensor(cu, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    ro, rfs, _, _ = oracle.prefill(np64(q), np64(k), np64(v), cu_seqlens=cu, initial_state=np64(s0))
+    assert_close(np64(out), ro, torch.bfloat16, "out")
+    assert_close(np64(fs), rfs, torch.bfloat16, "final_state")
+
+
+def test_prefill_resume_llama8b_shape(cuda_device):
+    """Llama-3-8B shape: prefill of the first 4096 tokens, then of the next 4096 from its final
+    state, on the tensor-core path.  The second call matches the oracle run from the same
+    state; with alpha = 1 (the recurrent branch alone: the window restarts with each call)
+    the two calls reproduce one 8192-token prefill."""
+    wl = inputs.WORKLOADS["llama8b_prefill"]
+    q, k, v = inputs.prefill_inputs(wl)
+    dev = cuda_device
+    T1 = 4096
+    halves = [(t[:, :T1].contiguous(), t[:, T1:].contiguous()) for t in (q, k, v)]
+    (q1, q2), (k1, k2), (v1, v2) = halves
+    for alpha in (0.5, 1.0):
+        _, fs1 = ops.prefill(q1.to(dev), k1.to(dev), v1.to(dev), alpha=alpha)
+        out2, fs2 = ops.prefill(q2.to(dev), k2.to(dev), v2.to(dev), alpha=alpha, initial_state=fs1)
+        torch.cuda.synchronize()
+        ro2, rfs2, _, _ = oracle.prefill(np64(q2), np64(k2), np64(v2), alpha=alpha, initial_state=np64(fs1))
+        assert_close(np64(out2), ro2, wl.dtype, f"second call out (alpha {alpha})")
+        assert_close(np64(fs2), rfs2, wl.dtype, f"second call final state (alpha {alpha})")
+        if alpha == 1.0:
+            ro, rfs, _, _ = oracle.prefill(np64(q), np64(k), np64(v), alpha=1.0)
+            assert_close(np64(out2), ro[:, T1:], wl.dtype, "resumed recurrent branch vs one long prefill")
+            assert_close(np64(fs2), rfs, wl.dtype, "resumed final state vs one long prefill")

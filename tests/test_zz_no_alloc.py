@@ -42,7 +42,7 @@ def _noalloc(lib, q, k, v, out, fs, ring, pos, cu=None, n=None, alpha=0.5, w=64)
 def _fill_scratch_with_a_larger_call(lib, device):
     """A call of another, larger shape, so the compared calls find the shared scratch full of
     that call's tables and states."""
-    wl = inputs.small("filler", B=1, Hq=16, Hkv=4, T=6000, d=128, seed=5)
+    wl = inputs.small("filler", B=1, Hq=16, Hkv=4, T=2500, d=128, seed=5)
     q, k, v = (t.to(device) for t in inputs.prefill_inputs(wl))
     need = ops.prefill_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.B)
     assert need <= 16 * 1024 * 1024
