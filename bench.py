@@ -416,17 +416,23 @@ def run_ours(args, world, rank, local):
 
     # ---------------- the prefill's gradient (the fine-tune's backward pass)
     bwd = None
-    if args.only is None or args.only in ("prefill", "backward"):
+    if args.only is None or args.only == "backward":
         bwd = time_backward(PREFILL, args, world, dev, stream, pk, windows)
+
+    # ---------------- the per-dimension (vector) gate prefill
+    vgate = None
+    if args.only is None or args.only == "vgate":
+        vgate = time_vector_gate(PREFILL, args, world, dev, stream, pk, windows)
 
     # ---------------- the hybrid's standard attention layer (causal softmax attention)
     full = None
-    if args.only is None or args.only in ("prefill", "full"):
+    if args.only is None or args.only == "full":
         full = time_full_attention(PREFILL, args, world, dev, stream, pk, windows)
 
     # ---------------- decode
-    dec = None if args.only in ("prefill", "full", "backward") else run_decode(args, world, dev, stream, pk, windows)
-    dec_kv = (None if args.only in ("prefill", "full", "backward")
+    dec = (None if args.only in ("prefill", "full", "backward", "vgate")
+           else run_decode(args, world, dev, stream, pk, windows))
+    dec_kv = (None if args.only in ("prefill", "full", "backward", "vgate")
               else run_decode(args, world, dev, stream, pk, windows, kvshared=True))
 
     sampler.stop()
@@ -444,7 +450,7 @@ def run_ours(args, world, rank, local):
             "data": "synthetic (seeded N(0,1), Llama-3-8B attention shapes)",
             "config": workload_config(), "roofline": roofline, "prefill_call": res8["call"],
             "llama1b_prefill": others.get("llama1b_prefill"), "long_varlen": others.get("long_varlen"),
-            "full_attention": full, "backward": bwd,
+            "full_attention": full, "backward": bwd, "vector_gate": vgate,
             "decode": dec, "decode_kvshared": dec_kv, "e2e": e2e,
             "gpu_launches": prefill_launches, "clocks": clocks, "cpu_baseline": cpu,
         }
@@ -609,6 +615,38 @@ def time_backward(wl, args, world, dev, stream, pk, windows):
                          "algorithmic_flops": alg_flops,
                          "tensor_frac": alg_flops / (ms * 1e-3) / (pk["bf16_tflops"] * 1e12),
                          "peak_source": pk["source"]}}
+
+
+def time_vector_gate(wl, args, world, dev, stream, pk, windows):
+    """Times the prefill with one gate per key dimension (general CUDA-core kernel) on the
+    workload; the same algorithmic bytes as the scalar-gate prefill."""
+    from gated_linear_attention_liger_b200 import ops
+    q, k, v = (t.to(dev) for t in inputs.prefill_inputs(wl))
+    torch.cuda.synchronize()
+    for _ in range(min(args.warmup, 3)):
+        ops.prefill_vector_gate(q, k, v, alpha=wl.alpha, w=wl.w, stream=stream)
+    n = 3
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    a.record(stream)
+    for _ in range(n):
+        ops.prefill_vector_gate(q, k, v, alpha=wl.alpha, w=wl.w, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    windows.append((w0, time.perf_counter()))
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b) / n, world, dev)
+    alg_bytes, alg_flops = prefill_algorithmic(wl)
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    del q, k, v
+    return {"metric": "vector-gate prefill tokens/s (8B attn shape)", "value": world * wl.tokens / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": "general prefill (CUDA cores)",
+                         "algorithmic_bytes": alg_bytes, "peak_source": pk["source"]}}
 
 
 def full_attention_flops(wl):
@@ -795,7 +833,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-steps", type=int, default=1000, help="decode steps per captured graph")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the CPU baseline")
-    ap.add_argument("--only", choices=["prefill", "decode", "full", "backward"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "full", "backward", "vgate"], default=None,
                     help="run one part only (for profiling); the JSON line is then partial")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -33,6 +33,7 @@ struct DecodeArgs {
   const int32_t* pos;
   int Hq, Hkv, w;
   float alpha;
+  int vector_gate;   // one gate per key dimension, sigmoid(k[r]) on row r of the state
 };
 
 constexpr int kDecodeThreads = 256;
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   extern __shared__ __align__(16) unsigned char dsm[];
   Tin* rk_s = reinterpret_cast<Tin*>(dsm);          // [64][D]
   Tin* rv_s = rk_s + 64 * ring_row_elems<Tin, D>();  // [64][row]
-  __shared__ __align__(16) float qs[D], ks[D], vs[D], fq[D], fk[D];
+  __shared__ __align__(16) float qs[D], ks[D], vs[D], fq[D], fk[D], gv[D];
   __shared__ float sc[1][64];
   __shared__ __align__(16) float part[RGN][D];
   __shared__ __align__(16) float wsum[WV::NW][1][D];
@@ -289,6 +290,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
 #pragma unroll
     for (int j = 0; j < EPL; ++j) fk[lane + 32 * j] = x[j] / z;
     if (lane == 0) gsh = expf(log_sigmoid(sum / (float)D));
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      gv[lane + 32 * j] = a.vector_gate ? expf(log_sigmoid(ks[lane + 32 * j])) : 0.f;
   } else if (warp == 1) {
     float x[EPL], m = -INFINITY, z = 0.f;
 #pragma unroll
@@ -305,13 +309,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
   // 4. state update and readout on the streamed rows: the state goes back to memory
   //    before the window branch is computed
   {
-    const float g = gsh;
+    const float gs = gsh;
+    const bool vg = a.vector_gate != 0;
     const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int row = rg * RPT + r;
       const float kr = fk[row], qr = fq[row];
+      const float g = vg ? gv[row] : gs;
       float4 x = st[r];
       x.x = fmaf(g, x.x, kr * vv.x);
       x.y = fmaf(g, x.y, kr * vv.y);

@@ -112,10 +112,10 @@ liger_status check_common(int Hq, int Hkv, int d, int w, float alpha, liger_dtyp
   return LIGER_OK;
 }
 
-template <typename Tin, int D>
+template <typename Tin, int D, bool VG = false>
 liger_status launch_simt_prefill(const liger::SimtPrefillArgs& a, int n_seqs, cudaStream_t s) {
-  const size_t smem = liger::simt_prefill_smem_bytes<D>();
-  auto kern = liger::prefill_simt_kernel<Tin, D>;
+  const size_t smem = liger::simt_prefill_smem_bytes<D, VG>();
+  auto kern = liger::prefill_simt_kernel<Tin, D, VG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return cuda_check("cudaFuncSetAttribute(prefill_simt)");
   const long blocks = (long)n_seqs * a.Hq;
@@ -179,9 +179,9 @@ liger_status decode_kvshared_g(const liger::DecodeArgs& a, int G, unsigned block
   }
 }
 
-template <typename Tin>
+template <typename Tin, bool VG = false>
 liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, cudaStream_t s) {
-  return d == 64 ? launch_simt_prefill<Tin, 64>(a, n_seqs, s) : launch_simt_prefill<Tin, 128>(a, n_seqs, s);
+  return d == 64 ? launch_simt_prefill<Tin, 64, VG>(a, n_seqs, s) : launch_simt_prefill<Tin, 128, VG>(a, n_seqs, s);
 }
 
 // Error word of the causal-attention kernel (bit 0: a bounded wait gave up; word 1: the
@@ -353,10 +353,69 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
   return launch_ring<float>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
 }
 
+liger_status liger_attn_prefill_vector_gate(const void* q, const void* k, const void* v, void* out,
+                                            float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
+                                            float alpha, liger_dtype dt, const float* initial_state,
+                                            const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
+                                            int32_t* pos_out, void* stream) {
+  const NvtxRange range("liger_attn_prefill_vector_gate");
+  g_last_error.clear();
+  liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
+  if (st != LIGER_OK) return st;
+  if (B < 1 || T < 0) return fail(LIGER_ERR_INVALID_ARG, "need B >= 1 and T >= 0 (B=%d T=%d)", B, T);
+  if (cu_seqlens) {
+    if (B != 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (B=%d)", B);
+    if (n_seqs < 1) return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens requires n_seqs >= 1 (n_seqs=%d)", n_seqs);
+  } else if (n_seqs != B) {
+    return fail(LIGER_ERR_INVALID_ARG, "without cu_seqlens n_seqs must equal B (n_seqs=%d B=%d)", n_seqs, B);
+  }
+  if ((long)T * B * Hq > (1L << 40) / d || (long)T * B > 0x7fffffffL - 1024)
+    return fail(LIGER_ERR_UNSUPPORTED, "tensor too large");
+  if ((long)B * T > 0 && (!q || !k || !v || !out))
+    return fail(LIGER_ERR_INVALID_ARG, "q, k, v and out must be non-null");
+  const void* ptrs[] = {q, k, v, out, final_state, initial_state, swa_ring_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(LIGER_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+  if (pos_out && (reinterpret_cast<uintptr_t>(pos_out) & 3u))
+    return fail(LIGER_ERR_INVALID_ARG, "pos_out must be 4-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha, nullptr};
+  st = dt == LIGER_BF16 ? prefill_simt_dispatch<__nv_bfloat16, true>(a, d, n_seqs, s)
+                        : prefill_simt_dispatch<float, true>(a, d, n_seqs, s);
+  if (st != LIGER_OK) return st;
+  if (dt == LIGER_BF16)
+    return launch_ring<__nv_bfloat16>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
+  return launch_ring<float>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
+}
+
+namespace {
+liger_status decode_impl(const void* q, const void* k, const void* v, float* state, void* swa_ring, void* out,
+                         int32_t* pos, int B, int Hq, int Hkv, int d, int w, float alpha, liger_dtype dt,
+                         void* stream, int vector_gate);
+}
+
+liger_status liger_attn_decode_vector_gate(const void* q, const void* k, const void* v, float* state,
+                                           void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                                           int d, int w, float alpha, liger_dtype dt, void* stream) {
+  const NvtxRange range("liger_attn_decode_vector_gate");
+  return decode_impl(q, k, v, state, swa_ring, out, pos, B, Hq, Hkv, d, w, alpha, dt, stream, 1);
+}
+
 liger_status liger_attn_decode(const void* q, const void* k, const void* v, float* state,
                                void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                int d, int w, float alpha, liger_dtype dt, void* stream) {
   const NvtxRange range("liger_attn_decode");
+  return decode_impl(q, k, v, state, swa_ring, out, pos, B, Hq, Hkv, d, w, alpha, dt, stream, 0);
+}
+
+}  // extern "C"
+
+namespace {
+liger_status decode_impl(const void* q, const void* k, const void* v, float* state, void* swa_ring, void* out,
+                         int32_t* pos, int B, int Hq, int Hkv, int d, int w, float alpha, liger_dtype dt,
+                         void* stream, int vector_gate) {
   g_last_error.clear();
   liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
   if (st != LIGER_OK) return st;
@@ -370,7 +429,7 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
   if (reinterpret_cast<uintptr_t>(pos) & 3u) return fail(LIGER_ERR_INVALID_ARG, "pos must be 4-byte aligned");
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha};
+  liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha, vector_gate};
   const unsigned blocks = (unsigned)((long)B * Hq);
   if (dt == LIGER_BF16) st = d == 64 ? launch_decode<__nv_bfloat16, 64>(a, blocks, s)
                                      : launch_decode<__nv_bfloat16, 128>(a, blocks, s);
@@ -381,6 +440,9 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
   ++g_launches;
   return cuda_check("advance_pos launch");
 }
+}  // namespace
+
+extern "C" {
 
 liger_status liger_attn_prefill_status(const void* workspace, size_t workspace_bytes) {
   g_last_error.clear();
@@ -548,8 +610,9 @@ liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   liger::DecodeArgs a{q, k, v, state, swa_ring, out, pos, Hq, Hkv, w, alpha};
   const unsigned blocks = (unsigned)((long)B * Hkv);
-  if (dt == LIGER_BF16) st = d == 64 ? decode_kvshared_g<__nv_bfloat16, 64>(a, G, blocks, s)
-                                     : decode_kvshared_g<__nv_bfloat16, 128>(a, G, blocks, s);
+  if (dt == LIGER_BF16)
+    st = d == 64 ? decode_kvshared_g<__nv_bfloat16, 64>(a, G, blocks, s)
+                 : decode_kvshared_g<__nv_bfloat16, 128>(a, G, blocks, s);
   else st = d == 64 ? decode_kvshared_g<float, 64>(a, G, blocks, s) : decode_kvshared_g<float, 128>(a, G, blocks, s);
   if (st != LIGER_OK) return st;
   if (launch_pdl(liger::advance_pos_kernel, dim3((B + 255) / 256), dim3(256), 0, s, pos, B) != cudaSuccess)

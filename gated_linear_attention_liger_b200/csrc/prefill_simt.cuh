@@ -38,14 +38,16 @@ constexpr int kSimtChunk = 32;         // tokens per chunk
 constexpr int kSimtRing = 96;          // >= 64 + kSimtChunk - 1 window slots
 constexpr int kMaxWindow = 64;
 
-template <int D>
+// VG: one gate per key dimension, sigmoid(k_t[r]) on row r of the state (the
+// per-dimension form of the pooled key gate); otherwise the pooled scalar gate.
+template <int D, bool VG = false>
 constexpr size_t simt_prefill_smem_bytes() {
   constexpr int RG = kSimtThreads / D;
   return sizeof(float) * (size_t)(2 * kSimtRing * D + 3 * kSimtChunk * D + kSimtChunk * RG * D +
-                                  kSimtChunk * kMaxWindow + kSimtChunk);
+                                  kSimtChunk * kMaxWindow + kSimtChunk + (VG ? kSimtChunk * D : 0));
 }
 
-template <typename Tin, int D>
+template <typename Tin, int D, bool VG = false>
 __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillArgs a) {
   constexpr int NT = kSimtThreads, C = kSimtChunk, RING = kSimtRing, W64 = kMaxWindow;
   constexpr int RG = NT / D;      // row groups
@@ -60,6 +62,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
   float* part = fk + C * D;                 // [C][RG][D] partial readouts
   float* sc = part + C * RG * D;            // [C][W64] window scores / probabilities
   float* gate = sc + C * W64;               // [C]
+  float* gvec = gate + C;                   // [C][D] per-dimension gates (VG only)
 
   const Tin* __restrict__ q = static_cast<const Tin*>(a.q);
   const Tin* __restrict__ k = static_cast<const Tin*>(a.k);
@@ -110,7 +113,12 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       z = warp_sum(z);
 #pragma unroll
       for (int j = 0; j < EPL; ++j) fk[i * D + lane + 32 * j] = x[j] / z;
-      if (lane == 0) gate[i] = expf(log_sigmoid(sum / (float)D));
+      if (VG) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) gvec[i * D + lane + 32 * j] = expf(log_sigmoid(ring_k[slot * D + lane + 32 * j]));
+      } else if (lane == 0) {
+        gate[i] = expf(log_sigmoid(sum / (float)D));
+      }
       m = -INFINITY;
 #pragma unroll
       for (int j = 0; j < EPL; ++j) { x[j] = qbuf[i * D + lane + 32 * j]; m = fmaxf(m, x[j]); }
@@ -164,14 +172,15 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
     }
     // 4. token-serial recurrence on the register-resident state (no syncs)
     for (int i = 0; i < n; ++i) {
-      const float g = gate[i];
+      const float g = VG ? 1.f : gate[i];
       const float vc = ring_v[((int)((t0 + i - tb) % RING)) * D + c];
       const float* fki = fk + i * D + rg * RPT;
       const float* fqi = fq + i * D + rg * RPT;
       float acc = 0.f;
+      const float* gvi = gvec + i * D + rg * RPT;
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
-        s[r] = fmaf(g, s[r], fki[r] * vc);
+        s[r] = fmaf(VG ? gvi[r] : g, s[r], fki[r] * vc);
         acc = fmaf(fqi[r], s[r], acc);
       }
       part[(i * RG + rg) * D + c] = acc;

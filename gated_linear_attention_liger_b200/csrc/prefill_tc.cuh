@@ -866,10 +866,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         if (!fast) mma_commit(q_empty);   // exact decay: the readout read e^{b_i} e_q from the q buffer
       };
       // A chunk's P.V goes out before the next chunk's window scores: the window warps
-      // wait for it, while the next scores are needed only after their epilogue.  This
-      // order also guards the recurrent scores' TMEM: the window warps release the score
-      // columns (s_read) before they read the recurrent scores of the same chunk, and the
-      // next chunk's Sg is issued only after this chunk's P.V, which waits for p_ready.
+      // wait for it, while the next scores are needed only after their epilogue.
       issue_ss(0);
       issue_sg_state(0);
       issue_inter(0);
@@ -1134,41 +1131,49 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const int jlo = max(il + 1, t0 == sg.q0 ? 64 - 16 * wq : 0), jhi = il + 64;
       // score column of key x: (x + 64 (c & 1)) mod 128 (the two key slots form one operand)
       const int ss_rot = 16 * wq + ((c & 1) << 6);
+      auto ss_col = [&](int q5) { return lane_base + kColSs + ((ss_rot + 16 * q5) & 127); };
       mbar_wait(ss_done, c & 1, wc, wsite(4, 6, c));
       tc_fence_after();
-      // The row's 80 scores, loaded once and kept in registers.
-      float s[80];
-#pragma unroll
-      for (int q5 = 0; q5 < 5; ++q5) tmem_ld16(lane_base + kColSs + ((ss_rot + 16 * q5) & 127), s + 16 * q5);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_read);   // the score columns are in registers: their TMEM may be reused
-      // Columns 16..63 are inside every row's band except in the sequence's first chunk:
-      // only the outer groups (and that chunk) take the mask, as -inf, whose exponential is 0.
+      // The row's 80 scores, loaded once: mask (-inf, whose exponential is 0), maximum,
+      // exponentials and their sum in registers, then the exponentials written back over
+      // the scores for the rolled probability pass below (short code for the instruction
+      // caches the roles share).  Columns 16..63 are inside every row's band except in the
+      // sequence's first chunk: only the outer groups (and that chunk) take the mask.
       const bool first = t0 == sg.q0;
+      float lsum;
+      {
+        float s[80];
 #pragma unroll
-      for (int q5 = 0; q5 < 5; ++q5) {
-        if (first || q5 == 0 || q5 == 4) {
+        for (int q5 = 0; q5 < 5; ++q5) tmem_ld16(ss_col(q5), s + 16 * q5);
+        tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int j = 16 * q5 + u;
-            s[16 * q5 + u] = (j >= jlo && j <= jhi) ? s[16 * q5 + u] : -INFINITY;
+        for (int q5 = 0; q5 < 5; ++q5) {
+          if (first || q5 == 0 || q5 == 4) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const int j = 16 * q5 + u;
+              s[16 * q5 + u] = (j >= jlo && j <= jhi) ? s[16 * q5 + u] : -INFINITY;
+            }
           }
         }
-      }
-      float m = -INFINITY;
+        float m = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 80; u += 2) m = fmax3(m, s[u], s[u + 1]);
-      const float2 sc2 = make_float2(sscale, sscale), nmsc = make_float2(-m * sscale, -m * sscale);
-      float2 lsum = make_float2(0.f, 0.f);
+        for (int u = 0; u < 80; u += 2) m = fmax3(m, s[u], s[u + 1]);
+        const float2 sc2 = make_float2(sscale, sscale), nmsc = make_float2(-m * sscale, -m * sscale);
+        float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 80; u += 2) {
-        float2 y = ffma2(make_float2(s[u], s[u + 1]), sc2, nmsc);
-        y.x = ex2(y.x);
-        y.y = ex2(y.y);
-        s[u] = y.x;
-        s[u + 1] = y.y;
-        lsum = fadd2(lsum, y);
+        for (int u = 0; u < 80; u += 2) {
+          float2 y = ffma2(make_float2(s[u], s[u + 1]), sc2, nmsc);
+          y.x = ex2(y.x);
+          y.y = ex2(y.y);
+          s[u] = y.x;
+          s[u + 1] = y.y;
+          ls = fadd2(ls, y);
+        }
+        lsum = ls.x + ls.y;
+#pragma unroll
+        for (int q5 = 0; q5 < 5; ++q5) tmem_st16(ss_col(q5), s + 16 * q5);
+        tmem_wait_st();
       }
       // Z of the rows and the recurrent scores come with the feature tiles
       mbar_wait(sg_done, c & 1, wc, wsite(4, 1, c));
@@ -1179,21 +1184,21 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float zrow = zq2[(c & 1) * 128 + r];
       const float bi = bsh[i];
       const float mrow = fast ? bsh[nv - 1] - bi : 0.f;
-      const float coef = beta * zrow * __expf(mrow) / (lsum.x + lsum.y);
+      const float coef = beta * zrow * __expf(mrow) / lsum;
       const float oscale = __expf(-mrow) / zrow;
       const float2 coef2 = make_float2(coef, coef), gs2 = make_float2(gscale, gscale);
       // Probability tile over [previous | current] keys.  The recurrent tile covers the
       // same current keys (kk <= i) and multiplies the same values, so it is added to the
       // window tile's current half here: one P V product per half.  Group q5 holds the
       // current keys kk = 16 bb + u with bb = q5 + wq - 4 when bb >= 0.
-#pragma unroll
+#pragma unroll 1
       for (int q5 = 0; q5 < 5; ++q5) {
         const int bb = q5 + wq - 4;
-        float* sv = s + 16 * q5;
+        float sv[16], g[16];
+        tmem_ld16(ss_col(q5), sv);
+        if (bb >= 0) tmem_ld16(lane_base + kColSg + 16 * bb, g);
+        tmem_wait_ld();
         if (bb >= 0) {
-          float g[16];
-          tmem_ld16(lane_base + kColSg + 16 * bb, g);
-          tmem_wait_ld();
           if (!fast) {   // exact mode: scores against phi(k); the decay per element
 #pragma unroll
             for (int u = 0; u < 16; ++u) g[u] *= __expf(bi - bsh[16 * bb + u]);
@@ -1229,6 +1234,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
+      mbar_arrive(s_read);    // the scores are consumed: their TMEM may be reused
       mbar_arrive(p_ready);   // the probability tile is in TMEM
 
       // epilogue: O -> bf16 rows of out

@@ -46,6 +46,10 @@ SIGNATURES = {
     "liger_attn_prefill_backward_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
     "liger_attn_prefill_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _i,
                                          _vp, _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "liger_attn_prefill_vector_gate": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
+                                            _i, _vp, _vp, _i, _vp, _vp, _vp]),
+    "liger_attn_decode_vector_gate": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
+                                           _i, _vp]),
     "liger_attn_full_causal": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp]),
     "liger_attn_full_causal_status": (_i, []),
     "liger_set_timing_events": (None, [_vp, _vp]),
@@ -341,3 +345,44 @@ def prefill_backward(q, k, v, d_out, alpha: float = 0.5, w: int = 64, d_final_st
         ws_bytes, _stream_ptr(stream))
     _check(st)
     return dq, dk, dv, ds0
+
+
+def prefill_vector_gate(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seqlens=None,
+                        return_ring: bool = False, stream=None):
+    """The prefill with one gate per key dimension (sigmoid(k_t[r]) on row r of the state).
+    Returns (out, final_state) or, with return_ring, (out, final_state, ring, pos)."""
+    lib = load()
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, T, Hq, d] and k, v [B, T, Hkv, d]")
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _expect(k, "k", (B, T, Hkv, d), q.dtype)
+    _expect(v, "v", (B, T, Hkv, d), q.dtype)
+    if cu_seqlens is not None and (cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2
+                                   or cu_seqlens.dtype != torch.int32):
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor of n + 1 offsets")
+    n = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    _expect(initial_state, "initial_state", (n, Hq, d, d), torch.float32)
+    _need_cuda(q, k, v, initial_state, cu_seqlens)
+    out = torch.empty_like(q)
+    fs = torch.empty(n, Hq, d, d, device=q.device, dtype=torch.float32)
+    ring = torch.empty(n, Hkv, 2, w, d, device=q.device, dtype=q.dtype) if return_ring else None
+    pos = torch.empty(n, device=q.device, dtype=torch.int32) if return_ring else None
+    st = lib.liger_attn_prefill_vector_gate(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(fs), B, Hq, Hkv, T, d, w, float(alpha), _dt(q),
+        _ptr(initial_state), _ptr(cu_seqlens), n, _ptr(ring), _ptr(pos), _stream_ptr(stream))
+    _check(st)
+    return (out, fs, ring, pos) if return_ring else (out, fs)
+
+
+def decode_vector_gate(q, k, v, state, ring, pos, alpha: float = 0.5, out=None, stream=None):
+    """One decode step with one gate per key dimension; updates state, ring and pos in place."""
+    lib = load()
+    B, Hq, Hkv, d, w = _check_decode(q, k, v, state, ring, pos, out, per_head=True)
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib.liger_attn_decode_vector_gate(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos), B, Hq, Hkv, d, w,
+        float(alpha), _dt(q), _stream_ptr(stream))
+    _check(st)
+    return out

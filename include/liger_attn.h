@@ -240,6 +240,25 @@ liger_status liger_attn_prefill_noalloc_status(void);
  */
 
 /*
+ * The gated recurrent branch with one gate per key dimension (the survey's
+ * vector gate; Paper-Notes page, section 统一的门控线性循环框架: Liger adapts to
+ * GLA, Mamba2, mLSTM, HGRN2 and RWKV6 through the form of the gate G_t in
+ * S_t = G_t (.) S_{t-1} + phi(k_t)^T v_t).  The pooling of the key is taken per
+ * element: G_t[r] = sigmoid(k_t[r]) scales row r (key dimension) of the state,
+ * as GLA's diagonal gate does; the window branch and the mix are unchanged.
+ * Arguments, layouts and errors as liger_attn_prefill / liger_attn_decode (the
+ * prefill takes no workspace: it runs the general CUDA-core kernel).
+ */
+liger_status liger_attn_prefill_vector_gate(const void* q, const void* k, const void* v, void* out,
+                                            float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
+                                            float alpha, liger_dtype dt, const float* initial_state,
+                                            const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
+                                            int32_t* pos_out, void* stream);
+liger_status liger_attn_decode_vector_gate(const void* q, const void* k, const void* v, float* state,
+                                           void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
+                                           int d, int w, float alpha, liger_dtype dt, void* stream);
+
+/*
  * Gradient of liger_attn_prefill (bf16 tensor-core path).  The pages give no
  * backward pass; the linearisation fine-tune of the news article on Liger
  * (section "軽量ファインチューニング": LoRA on the Q/K/V projections, trained

@@ -15,6 +15,12 @@
  *   [N-rec]   same page, section "统一的门控线性循环框架", recurrence
  *             S_t = G_t (.) S_{t-1} + phi(k_t)^T v_t,  o_t = phi(q_t) S_t,
  *             with phi = Softmax (no learned feature map).
+ *   [N-vgate] same page, same section: Liger adapts to other gated recurrent
+ *             structures (GLA, Mamba2, mLSTM, HGRN2, RWKV6) by the form of G_t;
+ *             read here as GLA's per-dimension gate with the parameter-free
+ *             pooling of the key taken per element: G_t[r] = sigmoid(k_t[r])
+ *             acting on row r (key dimension) of S, so G_t (.) S_{t-1} is
+ *             diag(G_t) S_{t-1}.
  *   [N-mix]   same page, section "Liger Attention：层内混合注意力",
  *             o_t = alpha*GRM + beta*SWA, alpha + beta = 1 (0.5 each), w = 64.
  *   [J-method] news article on Liger (Japanese), section "手法の説明":
@@ -102,11 +108,14 @@ static void prefill_unit(const prefill_job* J, int seq, int h) {
     const double* kt = J->k + (t * Hkv + kv) * d;
     const double* vt = J->v + (t * Hkv + kv) * d;
     /* gated recurrent branch [N-gate], [N-rec] */
-    const double g = J->gate_off ? 1.0 : exp(oracle_log_gate(kt, d));
+    const double g = J->gate_off == 1 ? 1.0 : exp(oracle_log_gate(kt, d));
     oracle_feature_map(kt, d, pk);
     oracle_feature_map(qt, d, pq);
-    for (int r = 0; r < d; ++r)
-      for (int c = 0; c < d; ++c) S[r * d + c] = g * S[r * d + c] + pk[r] * vt[c];
+    for (int r = 0; r < d; ++r) {
+      /* gate_off == 2: one gate per key dimension, sigmoid(k[r]) on row r [N-vgate] */
+      const double gr = J->gate_off == 2 ? exp(oracle_log_gate(kt + r, 1)) : g;
+      for (int c = 0; c < d; ++c) S[r * d + c] = gr * S[r * d + c] + pk[r] * vt[c];
+    }
     double* o = J->out + (t * Hq + h) * d;
     for (int c = 0; c < d; ++c) {
       double a = 0.0;
@@ -168,7 +177,10 @@ static void* prefill_worker(void* arg) {
  *   ring_out      [n_seqs, Hkv, 2, w, d] or NULL: the last min(len, w) keys and
  *                 values, position p at slot p mod w, other slots zero.
  *   pos_out       [n_seqs] or NULL: the sequence lengths.
- *   gate_off      test switch: 1 forces g = 1 (ungated linear attention).
+ *   gate_off      gate form: 0 the pooled scalar gate sigmoid(mean_d k_t) [N-gate];
+ *                 1 forces g = 1 (ungated linear attention, a test switch);
+ *                 2 one gate per key dimension, sigmoid(k_t[r]) scaling row r of
+ *                 the state [N-vgate].
  * Returns 0, or -1 on a bad argument.
  */
 int oracle_prefill(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
@@ -379,7 +391,7 @@ int oracle_prefill_backward(const double* q, const double* k, const double* v, i
                             const double* d_out, const double* d_final_state, double* dq,
                             double* dk, double* dv, double* d_initial_state, int gate_off,
                             int nthreads) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || d < 1 || w < 1 || !d_out) return -1;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || d < 1 || w < 1 || !d_out || gate_off == 2) return -1;
   if (cu_seqlens) {
     if (B != 1 || n_seqs < 1 || cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T) return -1;
     for (int i = 0; i < n_seqs; ++i)
@@ -440,11 +452,13 @@ static void decode_row(const decode_job* J, int b) {
     const double* kt = J->k + ((long)b * Hkv + kv) * d;
     const double* vt = J->v + ((long)b * Hkv + kv) * d;
     double* S = J->state + ((long)b * Hq + h) * d * d;
-    const double g = J->gate_off ? 1.0 : exp(oracle_log_gate(kt, d));
+    const double g = J->gate_off == 1 ? 1.0 : exp(oracle_log_gate(kt, d));
     oracle_feature_map(kt, d, pk);
     oracle_feature_map(qt, d, pq);
-    for (int r = 0; r < d; ++r)
-      for (int c = 0; c < d; ++c) S[r * d + c] = g * S[r * d + c] + pk[r] * vt[c];
+    for (int r = 0; r < d; ++r) {
+      const double gr = J->gate_off == 2 ? exp(oracle_log_gate(kt + r, 1)) : g;   /* [N-vgate] */
+      for (int c = 0; c < d; ++c) S[r * d + c] = gr * S[r * d + c] + pk[r] * vt[c];
+    }
     double* o = J->out + ((long)b * Hq + h) * d;
     for (int c = 0; c < d; ++c) {
       double a = 0.0;

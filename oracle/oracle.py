@@ -106,9 +106,18 @@ def log_gate(k):
     return res.reshape(k.shape[:-1])
 
 
+def _gate_mode(gate_off, vector_gate):
+    if gate_off and vector_gate:
+        raise ValueError("gate_off and vector_gate exclude each other")
+    return 1 if gate_off else (2 if vector_gate else 0)
+
+
 def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_off=False,
-            nthreads=None):
+            nthreads=None, vector_gate=False):
     """Token-by-token prefill.  Returns (out, final_state, ring, pos).
+
+    vector_gate: one gate per key dimension, sigmoid(k_t[r]) scaling row r of the state
+    (the per-dimension form of the pooled key gate), instead of sigmoid(mean_d k_t).
 
     q [B, T, Hq, d]; k, v [B, T, Hkv, d]; cu_seqlens (optional, B == 1) lists
     n_seqs + 1 offsets into T.  out [B, T, Hq, d], final_state [n, Hq, d, d],
@@ -135,7 +144,7 @@ def prefill(q, k, v, w=64, alpha=0.5, initial_state=None, cu_seqlens=None, gate_
     pos = np.zeros(n, dtype=np.int32)
     rc = lib.oracle_prefill(
         _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, T, d, w, float(alpha), _ptr(s0),
-        _ptr(cu, _ip), n, _ptr(out), _ptr(fs), _ptr(ring), _ptr(pos, _ip), int(bool(gate_off)),
+        _ptr(cu, _ip), n, _ptr(out), _ptr(fs), _ptr(ring), _ptr(pos, _ip), _gate_mode(gate_off, vector_gate),
         nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle_prefill rejected its arguments")
@@ -180,7 +189,7 @@ def prefill_backward(q, k, v, d_out, w=64, alpha=0.5, initial_state=None, cu_seq
     return dq, dk, dv, ds0
 
 
-def decode_inplace(q, k, v, state, ring, pos, alpha=0.5, gate_off=False, nthreads=None):
+def decode_inplace(q, k, v, state, ring, pos, alpha=0.5, gate_off=False, nthreads=None, vector_gate=False):
     """One decode step that updates state, ring and pos in place and returns out.
 
     state [B, Hq, d, d] and ring [B, Hkv, 2, w, d] must be C-contiguous float64 arrays and pos a
@@ -201,13 +210,13 @@ def decode_inplace(q, k, v, state, ring, pos, alpha=0.5, gate_off=False, nthread
     out = np.zeros_like(q)
     rc = lib.oracle_decode(
         _ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(ring), _ptr(out), _ptr(pos, _ip), B, Hq, Hkv, d, w,
-        float(alpha), int(bool(gate_off)), nthreads or default_threads())
+        float(alpha), _gate_mode(gate_off, vector_gate), nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
     return out
 
 
-def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthreads=None):
+def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthreads=None, vector_gate=False):
     """One decode step.  Returns (out, new_state, new_ring, new_pos); inputs are not modified.
 
     q [B, Hq, d]; k, v [B, Hkv, d]; state [B, Hq, d, d]; ring [B, Hkv, 2, w, d]; pos [B].
@@ -229,7 +238,7 @@ def decode(q, k, v, state, ring, pos, w=None, alpha=0.5, gate_off=False, nthread
     out = np.zeros_like(q)
     rc = lib.oracle_decode(
         _ptr(q), _ptr(k), _ptr(v), _ptr(st), _ptr(rg), _ptr(out), _ptr(ps, _ip), B, Hq, Hkv, d, w,
-        float(alpha), int(bool(gate_off)), nthreads or default_threads())
+        float(alpha), _gate_mode(gate_off, vector_gate), nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle_decode rejected its arguments")
     return out, st, rg, ps

@@ -348,3 +348,59 @@ def test_causal_attention_rows_equal_the_window_branch_and_sdpa():
         sep = oracle.causal_attention_rows(q1[:, a:b_], k1[:, a:b_], v1[:, a:b_],
                                            [(0, t, h) for t in range(b_ - a) for h in range(Hq)])
         np.testing.assert_allclose(got1[a * Hq:b_ * Hq], sep, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- per-dimension gate
+
+def _sig(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _phi(x):
+    e = np.exp(x - x.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def test_vector_gate_equals_scalar_gate_for_uniform_keys():
+    """When every element of a key is the same value, its mean is that value: the per-dimension
+    gate and the pooled scalar gate coincide."""
+    B, T, Hq, Hkv, d = 1, 9, 2, 1, 6
+    q, v = rand(B, T, Hq, d), rand(B, T, Hkv, d)
+    k = np.repeat(rand(B, T, Hkv, 1), d, axis=-1)
+    a = oracle.prefill(q, k, v, w=4, vector_gate=True)
+    b = oracle.prefill(q, k, v, w=4)
+    np.testing.assert_allclose(a[0], b[0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(a[1], b[1], rtol=1e-12, atol=1e-14)
+
+
+def test_vector_gate_equals_masked_parallel_form():
+    """alpha = 1: o_t = sum_{s<=t} sum_r phi q_t[r] (prod_{u=s+1..t} g_u[r]) phi k_s[r] v_s, the gate
+    acting on the key dimension r; the final state is sum_s (prod_{u>s} g_u[r]) phi k_s[r] v_s[c]
+    plus the decayed initial state.  (A gate applied to the value dimension fails both.)"""
+    T, d = 7, 5
+    q, k, v = rand(1, T, 1, d), rand(1, T, 1, d), rand(1, T, 1, d)
+    s0 = rand(1, 1, d, d, scale=0.3)
+    out, fs, _, _ = oracle.prefill(q, k, v, w=3, alpha=1.0, vector_gate=True, initial_state=s0)
+    pq, pk, g = _phi(q[0, :, 0]), _phi(k[0, :, 0]), _sig(k[0, :, 0])
+    for t in range(T):
+        ref = np.zeros(d)
+        for s in range(t + 1):
+            dec = np.prod(g[s + 1:t + 1], axis=0)                       # [d] over the key dim
+            ref += (pq[t] * dec * pk[s]).sum() * v[0, s, 0]
+        ref += (pq[t] * np.prod(g[:t + 1], axis=0)) @ s0[0, 0]
+        np.testing.assert_allclose(out[0, t, 0], ref, rtol=1e-11, atol=1e-13)
+    ref_s = np.prod(g, axis=0)[:, None] * s0[0, 0]
+    for s in range(T):
+        ref_s += np.outer(np.prod(g[s + 1:], axis=0) * pk[s], v[0, s, 0])
+    np.testing.assert_allclose(fs[0, 0], ref_s, rtol=1e-11, atol=1e-13)
+
+
+def test_vector_gate_decode_continues_prefill():
+    B, Hq, Hkv, T1, T2, d, w = 2, 4, 2, 8, 4, 8, 4
+    q, k, v = rand(B, T1 + T2, Hq, d), rand(B, T1 + T2, Hkv, d), rand(B, T1 + T2, Hkv, d)
+    full = oracle.prefill(q, k, v, w=w, vector_gate=True)
+    _, st, rg, ps = oracle.prefill(q[:, :T1], k[:, :T1], v[:, :T1], w=w, vector_gate=True)
+    for t in range(T1, T1 + T2):
+        o, st, rg, ps = oracle.decode(q[:, t], k[:, t], v[:, t], st, rg, ps, vector_gate=True)
+        np.testing.assert_allclose(o, full[0][:, t], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(st, full[1], rtol=1e-12, atol=1e-14)
