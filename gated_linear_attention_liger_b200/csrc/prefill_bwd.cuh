@@ -297,6 +297,10 @@ struct WinSmem {
 __device__ __forceinline__ void red_add(float* p, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
+// Adds four consecutive fp32 (16-byte aligned) in one instruction.
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
 
 // Per (chunk, q-head pair): rows 2 * token + head against keys [previous chunk | current
 // chunk].  Grid (slots * Hq / 2), 160 threads: warps 0-3 one row each, warp 4 lane 0
@@ -396,7 +400,7 @@ __global__ void __launch_bounds__(160, 1)
     for (int x = 0; x < 2 * C; ++x) P[x] *= il;
     // D_i = sum_x P dP with dP = beta dO . v_x
     float Dsum = 0.f;
-#pragma unroll 1
+#pragma unroll
     for (int x0 = 0; x0 < 2 * C; x0 += 32) {
       float g[32];
       tmem_ld32(lb + 128 + x0, g);
@@ -407,7 +411,7 @@ __global__ void __launch_bounds__(160, 1)
     Dsum *= beta;
     // dS = P (dP - D) / sqrt(d) and beta P, bf16 rows of the two key tiles
     const float isd = 1.f / sqrtf((float)D);
-#pragma unroll 1
+#pragma unroll
     for (int x0 = 0; x0 < 2 * C; x0 += 32) {
       float g[32];
       tmem_ld32(lb + 128 + x0, g);
@@ -438,15 +442,15 @@ __global__ void __launch_bounds__(160, 1)
     for (int kk = 0; kk < 2 * C / 16; ++kk)
       mma_bf16_ss(tmem + 256, sdesc_sw128(smem_u32(smem + L::DSW) + (kk >> 2) * (ROWS * 128) + (kk & 3) * 32, 16, 1024),
                   sdesc_sw128(smem_u32(smem + L::K0) + kk * 2048, 2 * C * 128, 1024), id_q, kk > 0);
-    // dk_win^T = Q^T dS and dv_win^T = dO^T (beta P): M = D (D = 64 duplicates rows), N = 128 keys, K = 128 rows
-    const uint32_t id_t = idesc_bf16(128, 2 * C, 1, 1);
-    const uint32_t lbo_a = D == 128 ? ROWS * 128 : 0;
+    // dk_win = dS^T Q and dv_win = (beta P)^T dO with the keys on the lanes: M = 128 keys
+    // (A = the key tiles, MN-major), N = D, K = 128 rows
+    const uint32_t id_t = idesc_bf16(128, D, 1, 1);
 #pragma unroll
     for (int kk = 0; kk < ROWS / 16; ++kk) {
-      mma_bf16_ss(tmem, sdesc_sw128(smem_u32(smem + L::Q0) + kk * 2048, lbo_a, 1024),
-                  sdesc_sw128(smem_u32(smem + L::DSW) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
-      mma_bf16_ss(tmem + 128, sdesc_sw128(smem_u32(smem + L::DO0) + kk * 2048, lbo_a, 1024),
-                  sdesc_sw128(smem_u32(smem + L::PW) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
+      mma_bf16_ss(tmem, sdesc_sw128(smem_u32(smem + L::DSW) + kk * 2048, ROWS * 128, 1024),
+                  sdesc_sw128(smem_u32(smem + L::Q0) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
+      mma_bf16_ss(tmem + 128, sdesc_sw128(smem_u32(smem + L::PW) + kk * 2048, ROWS * 128, 1024),
+                  sdesc_sw128(smem_u32(smem + L::DO0) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
     }
     mma_commit(mma2);
   }
@@ -467,25 +471,21 @@ __global__ void __launch_bounds__(160, 1)
         for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
       }
     }
-    // key side: lane = key-dim (dk) or value-dim (dv) row, column = key of [previous | current]
-    const int r = row;
+    // key side: lane = key x of [previous | current], columns = its d-vector
+    const int x = row;
+    const bool key_ok = x < C ? !cr.first : (x - C) < cr.nv;
+    if (key_ok) {
+      const size_t base = ((size_t)(cr.t0 + x - C) * p.Hkv + cr.kv) * D;
 #pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
+      for (int which = 0; which < 2; ++which) {
+        float* dst = (which == 0 ? bp.dkw : bp.dv_acc) + base;
 #pragma unroll 1
-      for (int x0 = 0; x0 < 2 * C; x0 += 32) {
-        float v[32];
-        tmem_ld32(lb + which * 128 + x0, v);
-        tmem_wait_ld();
-        if (r < D) {
-#pragma unroll 4
-          for (int u = 0; u < 32; ++u) {
-            const int x = x0 + u;
-            const bool key_ok = x < C ? !cr.first : (x - C) < cr.nv;
-            if (key_ok) {
-              const size_t tok = (size_t)(cr.t0 + x - C);
-              red_add((which == 0 ? bp.dkw : bp.dv_acc) + (tok * p.Hkv + cr.kv) * D + r, v[u]);
-            }
-          }
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(lb + which * 128 + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) red_add4(dst + c0 + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
         }
       }
     }
@@ -696,7 +696,7 @@ __global__ void __launch_bounds__(160, 1)
       rowsum = fmaf(a, g[j], rowsum);
     }
     // column sums over the pair's rows: warp sums, then shared atomics
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < C; ++j) {
       const float cs = warp_sum(av[j] * g[j]);
       if (lane == 0) atomicAdd(&colsum[j], cs);
@@ -720,32 +720,17 @@ __global__ void __launch_bounds__(160, 1)
     for (int kk = 0; kk < C / 16; ++kk)
       mma_bf16_ss(tmem + 128, sdesc_sw128(smem_u32(smem + L::GM) + kk * 32, 16, 1024),
                   sdesc_sw128(smem_u32(smem + L::IMG) + kk * 2048, C * 128, 1024), id_q, kk > 0);
-    // transposed products, M = D (D = 64 duplicates rows), N = 64 keys
-    const uint32_t id_t = idesc_bf16(128, C, 1, 1);
-    const uint32_t lbo_q = D == 128 ? ROWS * 128 : 0;
+    // key side with the keys on the lanes: M = 128 over the 64 keys (LBO 0 repeats them;
+    // lanes 64-127 are not read), N = D, K = 128 rows
+    const uint32_t id_t = idesc_bf16(128, D, 1, 1);
 #pragma unroll
     for (int kk = 0; kk < ROWS / 16; ++kk) {
-      // d phi k^T = Qr^T GM
-      mma_bf16_ss(tmem + 256, sdesc_sw128(smem_u32(smem + L::H0) + kk * 2048, lbo_q, 1024),
-                  sdesc_sw128(smem_u32(smem + L::GM) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
-      // dv^T = dO^T (alpha A)
-      mma_bf16_ss(tmem + 384, sdesc_sw128(smem_u32(smem + L::DO0) + kk * 2048, lbo_q, 1024),
-                  sdesc_sw128(smem_u32(smem + L::AT) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
-    }
-    if (pair_first) {
-      // (v_j dS'^T)^T = dS' Vc^T: A = dS' K-major (rows r), B = Vc K-major; K = D
-      const uint32_t id_kk = idesc_bf16(128, C, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_bf16_ss(tmem + 320, sdesc_sw128(smem_u32(smem + L::DH0) + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024),
-                    sdesc_sw128(smem_u32(smem + L::V0) + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024), id_kk, kk > 0);
-      // (Img_j dS')^T: A[c][r] = dS'[r][c] (MN-major), B[r][j] = Img[j][r] (K-major); K = D
-      const uint32_t id_mk = idesc_bf16(128, C, 1, 0);
-      const uint32_t lbo_s = D == 128 ? D * 128 : 0;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        mma_bf16_ss(tmem + 448, sdesc_sw128(smem_u32(smem + L::DH0) + kk * 2048, lbo_s, 1024),
-                    sdesc_sw128(smem_u32(smem + L::IMG) + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024), id_mk, kk > 0);
+      // d phi k (the group's rows) = GM^T Qr
+      mma_bf16_ss(tmem + 256, sdesc_sw128(smem_u32(smem + L::GM) + kk * 2048, 0, 1024),
+                  sdesc_sw128(smem_u32(smem + L::H0) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
+      // dv (the group's rows) = (alpha A)^T dO
+      mma_bf16_ss(tmem + 384, sdesc_sw128(smem_u32(smem + L::AT) + kk * 2048, 0, 1024),
+                  sdesc_sw128(smem_u32(smem + L::DO0) + kk * 2048, ROWS * 128, 1024), id_t, kk > 0);
     }
     mma_commit(mma3);
   }
@@ -754,106 +739,119 @@ __global__ void __launch_bounds__(160, 1)
   if (threadIdx.x < 128 && ok && !*abort_flag) {
     const float bi = bsh[i];
     // dq = phi q (d phi q - <d phi q, phi q>) + the window part
-    {
-      const float rq = fast ? __expf(bi - bC) : 1.f;
-      const float eb = alpha * __expf(bi);
-      const char* qb = smem + L::Q0;
-      const float izq = 1.f / zq;
-      float dot = 0.f;
+    const float rq = fast ? __expf(bi - bC) : 1.f;
+    const float eb = alpha * __expf(bi);
+    const char* qb = smem + L::Q0;
+    const float izq = 1.f / zq;
+    float dot = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float xv[32], mv[32];
-        tmem_ld32(lb + c0, xv);
-        tmem_ld32(lb + 128 + c0, mv);
-        tmem_wait_ld();
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float xv[32], mv[32];
+      tmem_ld32(lb + c0, xv);
+      tmem_ld32(lb + 128 + c0, mv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u8 = 0; u8 < 32; u8 += 8) {
+        float x[8];
+        tc::ld_chunk8(qb, kmajor_off(row, c0 + u8, ROWS * 128), x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float ph = ex2(fmaf(x[q], kL2e, -mq)) * izq;
+          dot = fmaf(ph, fmaf(eb, xv[u8 + q], rq * mv[u8 + q]), dot);
+        }
+      }
+    }
+    const size_t o = ((size_t)(cr.t0 + i) * p.Hq + h0 + hh) * D;
+    __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(bp.dq);
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float xv[32], mv[32];
+      tmem_ld32(lb + c0, xv);
+      tmem_ld32(lb + 128 + c0, mv);
+      tmem_wait_ld();
+      if (live) {
 #pragma unroll
         for (int u8 = 0; u8 < 32; u8 += 8) {
           float x[8];
           tc::ld_chunk8(qb, kmajor_off(row, c0 + u8, ROWS * 128), x);
+          uint32_t w[4];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float ph = ex2(fmaf(x[q], kL2e, -mq)) * izq;
-            dot = fmaf(ph, fmaf(eb, xv[u8 + q], rq * mv[u8 + q]), dot);
-          }
-        }
-      }
-      const size_t o = ((size_t)(cr.t0 + i) * p.Hq + h0 + hh) * D;
-      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(bp.dq);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        float xv[32], mv[32];
-        tmem_ld32(lb + c0, xv);
-        tmem_ld32(lb + 128 + c0, mv);
-        tmem_wait_ld();
-        if (live) {
+          for (int q = 0; q < 8; q += 2) {
+            float y[2];
 #pragma unroll
-          for (int u8 = 0; u8 < 32; u8 += 8) {
-            float x[8];
-            tc::ld_chunk8(qb, kmajor_off(row, c0 + u8, ROWS * 128), x);
-            uint32_t w[4];
-#pragma unroll
-            for (int q = 0; q < 8; q += 2) {
-              float y[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const float ph = ex2(fmaf(x[q + e], kL2e, -mq)) * izq;
-                const float dphi = fmaf(eb, xv[u8 + q + e], rq * mv[u8 + q + e]);
-                y[e] = fmaf(ph, dphi - dot, bp.dq_acc[o + c0 + u8 + q + e]);
-              }
-              w[q / 2] = pack_bf16(y[0], y[1]);
+            for (int e = 0; e < 2; ++e) {
+              const float ph = ex2(fmaf(x[q + e], kL2e, -mq)) * izq;
+              const float dphi = fmaf(eb, xv[u8 + q + e], rq * mv[u8 + q + e]);
+              y[e] = fmaf(ph, dphi - dot, bp.dq_acc[o + c0 + u8 + q + e]);
             }
-            *reinterpret_cast<uint4*>(dq + o + c0 + u8) = make_uint4(w[0], w[1], w[2], w[3]);
+            w[q / 2] = pack_bf16(y[0], y[1]);
           }
+          *reinterpret_cast<uint4*>(dq + o + c0 + u8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
-    // key side: lane = key-dim (d phi k) or value-dim (dv) row, column = key of the chunk
-    const int r = row;
+  }
+  tc_fence_before();
+  __syncthreads();   // X and d phi q are read: their columns take the state-gradient terms
+  if (pair_first && issuer && ok) {
+    tc_fence_after();
+    // v_j dS'^T (A = Vc K-major, B = dS' K-major) and Img_j dS' (A = Img K-major, B = dS'
+    // MN-major); keys on the lanes, K = D
+    const uint32_t id_kk = idesc_bf16(128, D, 0, 0), id_km = idesc_bf16(128, D, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      mma_bf16_ss(tmem, sdesc_sw128(smem_u32(smem + L::V0) + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(smem_u32(smem + L::DH0) + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024), id_kk,
+                  kk > 0);
+      mma_bf16_ss(tmem + 128, sdesc_sw128(smem_u32(smem + L::IMG) + (kk >> 2) * (C * 128) + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(smem_u32(smem + L::DH0) + kk * 2048, D * 128, 1024), id_km, kk > 0);
+    }
+    mma_commit(mma1);   // (second phase of this barrier)
+  }
+  if (pair_first) {
+    ok = bwait(mma1, 1, wc, wsite(2, 4, 0)) && ok;
+    tc_fence_after();
+  }
+  if (threadIdx.x < 128 && ok && !*abort_flag && threadIdx.x < cr.nv) {
+    // key j = this lane: d phi k and dv rows, and (once per kv head) the state terms
+    const int j = threadIdx.x;
+    const float cj = __expf(bC - bsh[j]);
+    const size_t base = ((size_t)(cr.t0 + j) * p.Hkv + cr.kv) * D;
+    float es = 0.f;   // e^{b_C - b_j} phi k_j dS' . v_j
 #pragma unroll 1
-    for (int j0 = 0; j0 < C; j0 += 32) {
+    for (int c0 = 0; c0 < D; c0 += 32) {
       float t1[32], t2[32], d2[32], d4[32];
-      tmem_ld32(lb + 256 + j0, t1);
-      tmem_ld32(lb + 384 + j0, t2);
+      tmem_ld32(lb + 256 + c0, t1);
+      tmem_ld32(lb + 384 + c0, t2);
       if (pair_first) {
-        tmem_ld32(lb + 320 + j0, d2);
-        tmem_ld32(lb + 448 + j0, d4);
+        tmem_ld32(lb + c0, d2);
+        tmem_ld32(lb + 128 + c0, d4);
       }
       tmem_wait_ld();
-      float es[32];   // this lane's share of e^{b_C - b_j} phi k_j dS' . v_j
-#pragma unroll 4
+#pragma unroll
       for (int u = 0; u < 32; ++u) {
-        const int j = j0 + u;
-        const float cj = __expf(bC - bsh[j]);
         float dk = t1[u], dvv = t2[u];
-        es[u] = 0.f;
         if (pair_first) {
           dk = fast ? cj * (dk + d2[u]) : dk + cj * d2[u];
           const float e4 = fast ? d4[u] : cj * d4[u];
           dvv += e4;
-          if (r < D) {
-            // v_j[c] for c = r: element (j, r) of the values tile
-            const uint32_t off = kmajor_off(j, r, C * 128);
-            es[u] = e4 * bf16_lo(*reinterpret_cast<const uint16_t*>(smem + L::V0 + off));
-          }
+          // v_j[c] for c = c0 + u: element (j, c) of the values tile
+          es = fmaf(e4, bf16_lo(*reinterpret_cast<const uint16_t*>(smem + L::V0 + kmajor_off(j, c0 + u, C * 128))), es);
         } else if (fast) {
           dk *= cj;
         }
-        if (r < D && j < cr.nv) {
-          const size_t base = ((size_t)(cr.t0 + j) * p.Hkv + cr.kv) * D + r;
-          red_add(bp.dphik + base, dk);
-          red_add(bp.dv_acc + base, dvv);
-        }
+        t1[u] = dk;
+        t2[u] = dvv;
       }
-      if (pair_first) {
-        float etot = 0.f;
-#pragma unroll 4
-        for (int u = 0; u < 32; ++u) {
-          const float e = warp_sum(es[u]);   // this warp's part of E_j = e^{b_C - b_j} phi k_j dS' . v_j
-          etot += e;
-          if (lane == 0) atomicAdd(&dbt[j0 + u], -e);
-        }
-        if (lane == 0) atomicAdd(&red[4 + warp], etot);
+#pragma unroll
+      for (int u = 0; u < 32; u += 4) {
+        red_add4(bp.dphik + base + c0 + u, t1[u], t1[u + 1], t1[u + 2], t1[u + 3]);
+        red_add4(bp.dv_acc + base + c0 + u, t2[u], t2[u + 1], t2[u + 2], t2[u + 3]);
       }
+    }
+    if (pair_first) {
+      atomicAdd(&dbt[j], -es);
+      atomicAdd(&red[4], es);
     }
   }
   tc_fence_before();
@@ -869,7 +867,7 @@ __global__ void __launch_bounds__(160, 1)
     // the last token's gate also scales the state it hands on:
     // <dS', S'> = e^{b_C} <dS', S> + sum_j E_j
     const float sds = red[0] + red[1] + red[2] + red[3];
-    const float esum = red[4] + red[5] + red[6] + red[7];
+    const float esum = red[4];
     atomicAdd(&dbt[cr.nv - 1], __expf(bC) * sds + esum);
   }
   __syncthreads();

@@ -22,23 +22,23 @@
 //   chunk     : per (segment, pair of q heads of one kv head) the fused pass.
 //               Its prologue loads the entering state into TMEM; after the last
 //               chunk of a sequence it writes the final state.  TMA stages q/k/v
-//               chunks; an 8-warp feature group computes the key features,
-//               gates and decay-scaled keys, then e_q, then the bf16 state copy
-//               for the readout; four window warps run the window softmax, the
-//               recurrent probability tile and the epilogue on TMEM rows; one
-//               thread issues the tcgen05 MMAs:
+//               chunks and the state pass's key-tile images; an 8-warp feature
+//               group computes e_q, the bf16 state copy for the readout and, one
+//               chunk behind, scales and stores the output; four window warps run
+//               the window softmax and the recurrent probability tile on TMEM rows;
+//               one thread issues the tcgen05 MMAs:
 //                 Ss = Q [K_slot0 | K_slot1]^T   raw scores of the window band
-//                 Sg = e_Q (e^{b_C-b_j} phi(K))^T recurrent scores (e_Q e_K^T when the
-//                                                decay does not factor)
+//                 Sg = e_Q (e^{b_C-b_j} phi(K))^T recurrent scores (e_Q phi(K)^T when
+//                                                the decay does not factor)
 //                 O  = e_Q (e^{b_C} S)           inter-chunk readout (e^{b_i} e_Q and S
 //                                                when the decay does not factor)
 //                 S += (e^{b_C-b_j} phi(K))^T V  state carry (fp32, in TMEM)
 //                 O += P_prev V_prev + P_cur V_cur + A_grm V_cur
 //               (P and A_grm are written to TMEM and read from there as the A
-//               operand); e_Q (which also carries alpha) and e_K are unnormalised
+//               operand); e_Q (which also carries alpha) holds unnormalised
 //               exponentials, their sums and the row factor e^{b_i - b_C} of the
-//               decay are folded into per-row scalars, and the epilogue stores bf16
-//               rows.
+//               decay are folded into per-row scalars, and the output is stored as
+//               bf16 rows.
 // Rows of the MMA tile interleave the two heads: row = 2 * token + head, which
 // is exactly the order a TMA box over (d, head, token) produces.
 #pragma once
@@ -633,7 +633,7 @@ constexpr uint32_t kColSg = 128;   // recurrent scores (64)
 constexpr uint32_t kColP = 192;    // probability tile, bf16 pairs: previous keys, current keys (64)
 constexpr uint32_t kColO = 256;    // output accumulator (D); the state follows it (D)
 
-// warps 0-3 window/epilogue, 4-11 features, 12 TMA, 13 MMA
+// warps 0-3 window, 4-11 features (and the output), 12 TMA, 13 MMA
 constexpr int kFeatWarp0 = 4;
 constexpr int kTmaWarp = kFeatWarp0 + 8, kMmaWarp = kTmaWarp + 1;
 constexpr int kChunkThreads = 32 * (kMmaWarp + 1);
@@ -674,6 +674,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
   float* bsh2 = reinterpret_cast<float*>(smem + L::SMALL + 256 + 64);  // [2][64] running log-gate sums
   float* zq2 = bsh2 + 128;                                     // [2][128] Z = sum_d e_q per row
   float* fast2 = zq2 + 256;                                     // [2] factored decay usable
+  float* osc2 = reinterpret_cast<float*>(smem + L::SMALL + 1920);  // [2][128] output row scales
 
   const int npairs = p.Hq / 2;
   const int seg = blockIdx.x / npairs, pair = blockIdx.x % npairs;
@@ -690,7 +691,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     mbar_init(q_full, 1); mbar_init(q_empty, 2);
     mbar_init(ss_done, 1); mbar_init(feat, 256); mbar_init(sg_done, 1); mbar_init(mma2_done, 1);
     mbar_init(state_ready, 256); mbar_init(state_done, 1);
-    mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 128);
+    mbar_init(s_read, 128); mbar_init(p_ready, 128); mbar_init(o_done, 1); mbar_init(o_free, 256);
     mbar_init(drain, 1);
     for (int i = 0; i < 2; ++i) { mbar_init(&kimg_full[i], 1); mbar_init(&kimg_empty[i], 1); }
     *abort_flag = 0u;
@@ -865,8 +866,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mma_commit(mma2_done);
         if (!fast) mma_commit(q_empty);   // exact decay: the readout read e^{b_i} e_q from the q buffer
       };
-      // A chunk's P.V goes out before the next chunk's window scores: the window warps
-      // wait for it, while the next scores are needed only after their epilogue.
+      // A chunk's P.V goes out before the next chunk's window scores (the scores' TMEM
+      // holds the probability tile until then); the readout of a chunk waits for the
+      // feature warps to have stored the previous chunk's output.
       issue_ss(0);
       issue_sg_state(0);
       issue_inter(0);
@@ -900,6 +902,44 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     const float qa = p.alpha >= 0x1p-20f ? p.alpha : 1.f;
     const float lqa = log2f(qa), iqa = 1.f / qa;
     const float copy_scale = p.alpha / qa;   // 1, or alpha when it stays on the copy
+
+    // Output of chunk cc: this warp's lane quarter (rows 2 * token + head), its column half;
+    // O / Z times the row factor from the window warps, bf16.  Frees the accumulator.
+    __nv_bfloat16* const out = static_cast<__nv_bfloat16*>(p.out);
+    auto epilogue = [&](int cc) {
+      const bool live = mbar_wait(o_done, cc & 1, wc, wsite(3, 8, cc)) && !*abort_flag;
+      tc_fence_after();
+      const int t0c = sg.t_begin + cc * C, nvc = min(C, sg.t_end - t0c);
+      const int i = lrow >> 1;
+      const float os = osc2[(cc & 1) * 128 + lrow];
+      __nv_bfloat16* orow = out + ((size_t)((long)t0c + i) * p.Hq + h0 + (lrow & 1)) * D;
+      const bool store = i < nvc && live;
+      const float2 os2 = make_float2(os, os);
+#pragma unroll 1
+      for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {
+        float v[32];
+        tmem_ld32(lane_base + kColO + col, v);
+        tmem_wait_ld();
+        if (store) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float2 y = fmul2(make_float2(v[2 * u], v[2 * u + 1]), os2);
+            pw[u] = pack_bf16(y.x, y.y);
+          }
+          if (p.out_v8) {   // two full 32-byte sectors per instruction
+            st_global_v8(orow + col, pw);
+            st_global_v8(orow + col + 16, pw + 8);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 16; u += 4)
+              *reinterpret_cast<uint4*>(orow + col + 2 * u) = make_uint4(pw[u], pw[u + 1], pw[u + 2], pw[u + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(o_free);
+    };
 
     // state entering the segment: this warp's quarter of the first half of the columns
     // (the window warps load the second half)
@@ -1081,7 +1121,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(state_ready);
+      // the previous chunk's output (its P.V finished long ago); the readout of this chunk
+      // waits for the accumulator to be free
+      if (c > 0) epilogue(c - 1);
     }
+    if (nch > 0) epilogue(nch - 1);
     // final state of the sequence: the carry after the last chunk of its last segment
     const SeqInfo si = p.seqs[sg.seq];
     const bool last = seg == si.first_seg + si.n_seg - 1;
@@ -1103,16 +1147,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         }
       }
     }
-  } else {   // ---------------- window softmax and epilogue (128 threads, warps 0-3)
+  } else {   // ---------------- window softmax and the probability tile (128 threads, warps 0-3)
     const int r = threadIdx.x;
-    const int i = r >> 1, hl = r & 1;
+    const int i = r >> 1;
     const int wq = warp, il = i - 16 * wq;
     const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
     const float alpha = p.alpha, beta = 1.0f - p.alpha;
     // the part of alpha that the e_q tile (and so the recurrent scores) does not carry
     const float gscale = alpha / (alpha >= 0x1p-20f ? alpha : 1.f);
     const float sscale = 1.4426950408889634f / sqrtf((float)D);
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
     // state entering the segment, second half of the columns (the feature warps load the
     // first half; TMEM: the state follows O)
     entering_state<D, D / 2>(p, seg, kv, r % D, lane_base + kColO + D, D / 2);
@@ -1185,7 +1228,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       const float bi = bsh[i];
       const float mrow = fast ? bsh[nv - 1] - bi : 0.f;
       const float coef = beta * zrow * __expf(mrow) / lsum;
-      const float oscale = __expf(-mrow) / zrow;
+      osc2[(c & 1) * 128 + r] = __expf(-mrow) / zrow;   // the feature warps scale and store the output
       const float2 coef2 = make_float2(coef, coef), gs2 = make_float2(gscale, gscale);
       // Probability tile over [previous | current] keys.  The recurrent tile covers the
       // same current keys (kk <= i) and multiplies the same values, so it is added to the
@@ -1237,39 +1280,6 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
       mbar_arrive(s_read);    // the scores are consumed: their TMEM may be reused
       mbar_arrive(p_ready);   // the probability tile is in TMEM
 
-      // epilogue: O -> bf16 rows of out
-      const bool live = mbar_wait(o_done, c & 1, wc, wsite(4, 2, c)) && !*abort_flag;
-      tc_fence_after();
-      {
-        const long t = (long)t0 + i;
-        __nv_bfloat16* orow = out + ((size_t)t * p.Hq + h0 + hl) * D;
-        const bool store = i < nv && live;
-#pragma unroll 1
-        for (int col = 0; col < D; col += 32) {
-          float v[32];
-          tmem_ld32(lane_base + kColO + col, v);
-          tmem_wait_ld();
-          if (store) {
-            uint32_t pw[16];
-            const float2 os2 = make_float2(oscale, oscale);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const float2 y = fmul2(make_float2(v[2 * u], v[2 * u + 1]), os2);
-              pw[u] = pack_bf16(y.x, y.y);
-            }
-            if (p.out_v8) {   // two full 32-byte sectors per instruction
-              st_global_v8(orow + col, pw);
-              st_global_v8(orow + col + 16, pw + 8);
-            } else {
-#pragma unroll
-              for (int u = 0; u < 16; u += 4)
-                *reinterpret_cast<uint4*>(orow + col + 2 * u) = make_uint4(pw[u], pw[u + 1], pw[u + 2], pw[u + 3]);
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(o_free);
     }
   }
   __syncthreads();
