@@ -20,6 +20,7 @@
 #include "decode.cuh"
 #include "full_attn.cuh"
 #include "prefill_bwd.cuh"
+#include "prefill_seg.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
 
@@ -113,18 +114,56 @@ liger_status check_common(int Hq, int Hkv, int d, int w, float alpha, liger_dtyp
 }
 
 template <typename Tin, int D, bool VG = false>
-liger_status launch_simt_prefill(const liger::SimtPrefillArgs& a, int n_seqs, cudaStream_t s) {
+liger_status launch_simt_prefill(const liger::SimtPrefillArgs& a, long units, cudaStream_t s, bool timed = true) {
   const size_t smem = liger::simt_prefill_smem_bytes<D, VG>();
   auto kern = liger::prefill_simt_kernel<Tin, D, VG>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return cuda_check("cudaFuncSetAttribute(prefill_simt)");
-  const long blocks = (long)n_seqs * a.Hq;
+  const long blocks = units * a.Hq;
   if (blocks > 0x7fffffffL) return fail(LIGER_ERR_UNSUPPORTED, "too many (sequence, head) units");
-  mark_start(s);
+  if (timed) mark_start(s);
   kern<<<(unsigned)blocks, liger::kSimtThreads, smem, s>>>(a);
-  mark_stop(s);
+  if (timed) mark_stop(s);
   ++g_launches;
   return cuda_check("prefill_simt launch");
+}
+
+// Segment-parallel general prefill: plan, per-segment states, scan, the general kernel per
+// (segment, q head); groups whose initial-state copies differ are rerun unsegmented.
+template <typename Tin, int D, bool VG>
+liger_status run_segmented(const liger::SimtPrefillArgs& a, int n_seqs, long T_total, void* ws,
+                           cudaStream_t s) {
+  namespace sg = liger::seg;
+  const sg::Layout L = sg::layout(T_total, n_seqs, a.Hkv, D);
+  char* w = static_cast<char*>(ws);
+  auto* segs = reinterpret_cast<liger::SimtSeg*>(w + L.off_segs);
+  int* count = reinterpret_cast<int*>(w);
+  float* lam = reinterpret_cast<float*>(w + L.off_lam);
+  float* ds = reinterpret_cast<float*>(w + L.off_ds);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(w + L.off_flags);
+  if (L.cap * a.Hkv > 0x7fffffffL || L.cap * a.Hq > 0x7fffffffL || (long)n_seqs * a.Hkv > 0x7fffffffL)
+    return fail(LIGER_ERR_UNSUPPORTED, "too many segments");
+  sg::plan_kernel<<<1, 32, 0, s>>>(a.cu, a.T, n_seqs, T_total, segs, count, L.cap, flags, a.Hkv);
+  ++g_launches;
+  sg::seg_state_kernel<Tin, D, VG><<<(unsigned)(L.cap * a.Hkv), sg::kSegThreads, 0, s>>>(
+      static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.Hkv, segs, count, ds, lam);
+  ++g_launches;
+  sg::scan_kernel<D><<<(unsigned)((long)n_seqs * a.Hkv), sg::kSegThreads, 0, s>>>(segs, count, a.Hq, a.Hkv,
+                                                                                   a.init_state, ds, lam, flags);
+  ++g_launches;
+  liger_status st = cuda_check("segmented prefill launch");
+  if (st != LIGER_OK) return st;
+  liger::SimtPrefillArgs b = a;
+  b.segs = segs;
+  b.n_segs = count;
+  b.seg_state = ds;
+  b.only_flagged = nullptr;
+  st = launch_simt_prefill<Tin, D, VG>(b, L.cap, s);
+  if (st != LIGER_OK || !a.init_state) return st;
+  liger::SimtPrefillArgs f = a;
+  f.segs = nullptr;
+  f.only_flagged = flags;
+  return launch_simt_prefill<Tin, D, VG>(f, n_seqs, s, false);
 }
 
 template <typename Tin>
@@ -182,6 +221,13 @@ liger_status decode_kvshared_g(const liger::DecodeArgs& a, int G, unsigned block
 template <typename Tin, bool VG = false>
 liger_status prefill_simt_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, cudaStream_t s) {
   return d == 64 ? launch_simt_prefill<Tin, 64, VG>(a, n_seqs, s) : launch_simt_prefill<Tin, 128, VG>(a, n_seqs, s);
+}
+
+template <typename Tin, bool VG>
+liger_status segmented_dispatch(const liger::SimtPrefillArgs& a, int d, int n_seqs, long T_total, void* ws,
+                                cudaStream_t s) {
+  return d == 64 ? run_segmented<Tin, 64, VG>(a, n_seqs, T_total, ws, s)
+                 : run_segmented<Tin, 128, VG>(a, n_seqs, T_total, ws, s);
 }
 
 // Error word of the causal-attention kernel (bit 0: a bounded wait gave up; word 1: the
@@ -353,11 +399,23 @@ liger_status liger_attn_prefill(const void* q, const void* k, const void* v, voi
   return launch_ring<float>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);
 }
 
+size_t liger_attn_prefill_vector_gate_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                                     liger_dtype dt) {
+  if (B < 1 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || (d != 64 && d != 128)) return 0;
+  if (dt != LIGER_BF16 && dt != LIGER_FP32) return 0;
+  const int n = n_seqs > 0 ? n_seqs : B;
+  // packed input (B == 1, n sequences) and B separate sequences: the larger layout
+  const size_t a = liger::seg::layout((long)B * T, B, Hkv, d).total;
+  const size_t b = liger::seg::layout((long)B * T, n, Hkv, d).total;
+  return a > b ? a : b;
+}
+
 liger_status liger_attn_prefill_vector_gate(const void* q, const void* k, const void* v, void* out,
                                             float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
                                             float alpha, liger_dtype dt, const float* initial_state,
                                             const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
-                                            int32_t* pos_out, void* stream) {
+                                            int32_t* pos_out, void* workspace, size_t workspace_bytes,
+                                            void* stream) {
   const NvtxRange range("liger_attn_prefill_vector_gate");
   g_last_error.clear();
   liger_status st = check_common(Hq, Hkv, d, w, alpha, dt);
@@ -380,10 +438,21 @@ liger_status liger_attn_prefill_vector_gate(const void* q, const void* k, const 
     return fail(LIGER_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
   if (pos_out && (reinterpret_cast<uintptr_t>(pos_out) & 3u))
     return fail(LIGER_ERR_INVALID_ARG, "pos_out must be 4-byte aligned");
+  if (workspace && !aligned16(workspace))
+    return fail(LIGER_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  const long T_total = (long)B * T;
+  const size_t need = T_total > 0 ? liger::seg::layout(T_total, n_seqs, Hkv, d).total : 0;
+  if (need > workspace_bytes || (need && !workspace))
+    return fail(LIGER_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, workspace_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   liger::SimtPrefillArgs a{q, k, v, out, final_state, initial_state, cu_seqlens, Hq, Hkv, w, (long)T, alpha, nullptr};
-  st = dt == LIGER_BF16 ? prefill_simt_dispatch<__nv_bfloat16, true>(a, d, n_seqs, s)
-                        : prefill_simt_dispatch<float, true>(a, d, n_seqs, s);
+  if (T_total > 0) {
+    st = dt == LIGER_BF16 ? segmented_dispatch<__nv_bfloat16, true>(a, d, n_seqs, T_total, workspace, s)
+                          : segmented_dispatch<float, true>(a, d, n_seqs, T_total, workspace, s);
+  } else {
+    st = dt == LIGER_BF16 ? prefill_simt_dispatch<__nv_bfloat16, true>(a, d, n_seqs, s)
+                          : prefill_simt_dispatch<float, true>(a, d, n_seqs, s);
+  }
   if (st != LIGER_OK) return st;
   if (dt == LIGER_BF16)
     return launch_ring<__nv_bfloat16>(k, v, swa_ring_out, pos_out, cu_seqlens, T, n_seqs, Hkv, d, w, s);

@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(160, 1)
     mbar_wait(ld_q, (pairs_issued - 1) & 1, dw);
   }
   // both accumulators to global, one key-dim row per thread
-  if (threadIdx.x < 128 && ok && !*abort_flag) {
+  if (threadIdx.x < 128 && warp_all(ok && !*abort_flag)) {
     const int r = threadIdx.x;
     const uint32_t lb = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll 1
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(160, 1)
   }
   ok = bwait(mma2, 0, wc, wsite(2, 2, 0)) && ok;
   tc_fence_after();
-  if (threadIdx.x < 128 && ok && !*abort_flag) {
+  if (threadIdx.x < 128 && warp_all(ok && !*abort_flag)) {
     const int row = threadIdx.x, i = row >> 1, hh = row & 1;
     const uint32_t lb = tmem + ((uint32_t)(warp * 32) << 16);
     // the window part of dq, kept in fp32 for the recurrent kernel
@@ -471,19 +471,20 @@ __global__ void __launch_bounds__(160, 1)
         for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
       }
     }
-    // key side: lane = key x of [previous | current], columns = its d-vector
+    // key side: lane = key x of [previous | current], columns = its d-vector.  The TMEM
+    // loads are warp-collective: every lane takes them, only live keys add.
     const int x = row;
     const bool key_ok = x < C ? !cr.first : (x - C) < cr.nv;
-    if (key_ok) {
-      const size_t base = ((size_t)(cr.t0 + x - C) * p.Hkv + cr.kv) * D;
+    const size_t base = key_ok ? ((size_t)(cr.t0 + x - C) * p.Hkv + cr.kv) * D : 0;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        float* dst = (which == 0 ? bp.dkw : bp.dv_acc) + base;
+    for (int which = 0; which < 2; ++which) {
+      float* dst = (which == 0 ? bp.dkw : bp.dv_acc) + base;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(lb + which * 128 + c0, v);
-          tmem_wait_ld();
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float v[32];
+        tmem_ld32(lb + which * 128 + c0, v);
+        tmem_wait_ld();
+        if (key_ok) {
 #pragma unroll
           for (int u = 0; u < 32; u += 4) red_add4(dst + c0 + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
         }
@@ -736,7 +737,7 @@ __global__ void __launch_bounds__(160, 1)
   }
   ok = bwait(mma3, 0, wc, wsite(2, 3, 0)) && ok;
   tc_fence_after();
-  if (threadIdx.x < 128 && ok && !*abort_flag) {
+  if (threadIdx.x < 128 && warp_all(ok && !*abort_flag)) {
     const float bi = bsh[i];
     // dq = phi q (d phi q - <d phi q, phi q>) + the window part
     const float rq = fast ? __expf(bi - bC) : 1.f;
@@ -812,11 +813,13 @@ __global__ void __launch_bounds__(160, 1)
     ok = bwait(mma1, 1, wc, wsite(2, 4, 0)) && ok;
     tc_fence_after();
   }
-  if (threadIdx.x < 128 && ok && !*abort_flag && threadIdx.x < cr.nv) {
-    // key j = this lane: d phi k and dv rows, and (once per kv head) the state terms
+  if (threadIdx.x < 128 && warp_all(ok && !*abort_flag)) {
+    // key j = this lane: d phi k and dv rows, and (once per kv head) the state terms.  The
+    // TMEM loads are warp-collective: every lane takes them, only keys j < nv add.
     const int j = threadIdx.x;
-    const float cj = __expf(bC - bsh[j]);
-    const size_t base = ((size_t)(cr.t0 + j) * p.Hkv + cr.kv) * D;
+    const bool jl = j < cr.nv;
+    const float cj = __expf(bC - bsh[j & (C - 1)]);
+    const size_t base = jl ? ((size_t)(cr.t0 + j) * p.Hkv + cr.kv) * D : 0;
     float es = 0.f;   // e^{b_C - b_j} phi k_j dS' . v_j
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -836,20 +839,22 @@ __global__ void __launch_bounds__(160, 1)
           const float e4 = fast ? d4[u] : cj * d4[u];
           dvv += e4;
           // v_j[c] for c = c0 + u: element (j, c) of the values tile
-          es = fmaf(e4, bf16_lo(*reinterpret_cast<const uint16_t*>(smem + L::V0 + kmajor_off(j, c0 + u, C * 128))), es);
+          es = fmaf(e4, bf16_lo(*reinterpret_cast<const uint16_t*>(smem + L::V0 + kmajor_off(j & (C - 1), c0 + u, C * 128))), es);
         } else if (fast) {
           dk *= cj;
         }
         t1[u] = dk;
         t2[u] = dvv;
       }
+      if (jl) {
 #pragma unroll
-      for (int u = 0; u < 32; u += 4) {
-        red_add4(bp.dphik + base + c0 + u, t1[u], t1[u + 1], t1[u + 2], t1[u + 3]);
-        red_add4(bp.dv_acc + base + c0 + u, t2[u], t2[u + 1], t2[u + 2], t2[u + 3]);
+        for (int u = 0; u < 32; u += 4) {
+          red_add4(bp.dphik + base + c0 + u, t1[u], t1[u + 1], t1[u + 2], t1[u + 3]);
+          red_add4(bp.dv_acc + base + c0 + u, t2[u], t2[u + 1], t2[u + 2], t2[u + 3]);
+        }
       }
     }
-    if (pair_first) {
+    if (pair_first && jl) {
       atomicAdd(&dbt[j], -es);
       atomicAdd(&red[4], es);
     }

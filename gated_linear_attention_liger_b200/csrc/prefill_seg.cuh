@@ -1,0 +1,209 @@
+// prefill_seg.cuh -- segment-parallel general prefill (CUDA cores, fp32 arithmetic).
+//
+// The general kernel steps the recurrence token by token, one CTA per (sequence,
+// q head).  This file splits each sequence into segments of kSegTokens tokens so
+// that the token-serial work runs on many CTAs at once:
+//   1. plan          the segment table from the sequence lengths (device side);
+//   2. seg_state     per (segment, kv head): the segment's own contribution to the
+//                    state, dS = sum_j diag(e^{B - B_j}) phi(k_j)^T v_j, and its total
+//                    log gate B (a vector over the key dimensions, or one value
+//                    repeated, for the pooled gate), B_j the running sum up to j;
+//   3. scan          per (sequence, kv head): the state entering each segment,
+//                    S_in(s+1) = diag(e^{B_s}) S_in(s) + dS_s, written over dS_s;
+//   4. the general kernel in segmented mode, per (segment, q head), from S_in.
+// The state is carried per kv head (the recurrence never reads q); an initial
+// state whose G copies in a group differ is handled by the caller, which reruns
+// those groups with the unsegmented kernel.
+//
+// Recurrence: "Liger: Linearizing Large Language Models to Gated Recurrent
+// Structures" (Paper-Notes page), section 统一的门控线性循环框架; the state of a
+// run of tokens is the sum of its tokens' outer products, each decayed by the
+// gates after it, which is what makes the scan associative.
+#pragma once
+
+#include "prefill_simt.cuh"
+
+namespace liger {
+namespace seg {
+
+constexpr int kSegTokens = 256;   // tokens per segment
+constexpr int kSegThreads = 256;
+constexpr int kStage = 16;        // tokens staged in shared memory at a time
+
+// Upper bound of the segment count: every sequence adds at most one partial (or empty)
+// segment.
+inline long max_segments(long T_total, int n_seqs) { return T_total / kSegTokens + n_seqs; }
+
+// One thread: walks the sequences and writes the segment table and its length.
+// Also clears the per-(sequence, kv head) flags the scan sets.
+__global__ void plan_kernel(const int32_t* cu, long T, int n_seqs, long T_total, SimtSeg* segs, int* n_segs,
+                            long cap, uint32_t* flags, int Hkv) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  for (long i = 0; i < (long)n_seqs * Hkv; ++i) flags[i] = 0u;
+  long n = 0;
+  for (int s = 0; s < n_seqs; ++s) {
+    long b, e;
+    seq_range(cu, s, T, T_total, &b, &e);
+    // an empty sequence still gets one (empty) segment: it writes the final state
+    for (long t = b; (t < e || t == b) && n < cap; t += kSegTokens, ++n) {
+      SimtSeg g;
+      g.t_begin = t;
+      g.t_end = min(e, t + kSegTokens);
+      g.seq_begin = b;
+      g.seq = s;
+      g.flags = (t == b ? 1 : 0) | (g.t_end == e ? 2 : 0);
+      segs[n] = g;
+    }
+  }
+  *n_segs = (int)n;
+}
+
+// Per (segment slot, kv head), 256 threads: thread (column c, row group rg) owns
+// rows rg*RPT .. rg*RPT+RPT-1 of column c of dS.  Tokens are staged 16 at a time,
+// last to first: lam[r] = B - B_j (the gates after token j) is then known when j is
+// reached, and w_j[r] = e^{lam[r]} phi(k_j)[r] <= phi(k_j)[r].
+template <typename Tin, int D, bool VG>
+__global__ void __launch_bounds__(kSegThreads) seg_state_kernel(const Tin* __restrict__ k,
+                                                                const Tin* __restrict__ v, int Hkv,
+                                                                const SimtSeg* segs, const int* n_segs,
+                                                                float* __restrict__ ds, float* __restrict__ lam_out) {
+  constexpr int NT = kSegThreads, S = kStage;
+  constexpr int RG = NT / D, RPT = D / RG, EPL = D / 32;
+  __shared__ __align__(16) float kw[S][D];   // raw keys, then the weights w_j
+  __shared__ __align__(16) float vs[S][D];
+  __shared__ float lg[S][VG ? D : 1];        // log gates
+  __shared__ float lam[D];                   // gates after the staged block
+  const int slot = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
+  if (slot >= *n_segs) return;
+  const SimtSeg sg = segs[slot];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid % D, rg = tid / D;
+  float acc[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) acc[r] = 0.f;
+  if (tid < D) lam[tid] = 0.f;
+  for (long t1 = sg.t_end; t1 > sg.t_begin; t1 -= S) {
+    const long t0 = max(sg.t_begin, t1 - S);
+    const int n = (int)(t1 - t0);
+    __syncthreads();   // the previous block's weights are consumed
+    for (int idx = tid; idx < n * D; idx += NT) {
+      const int i = idx / D, e = idx % D;
+      kw[i][e] = io<Tin>::ld(k + ((size_t)(t0 + i) * Hkv + kv) * D + e);
+      vs[i][e] = io<Tin>::ld(v + ((size_t)(t0 + i) * Hkv + kv) * D + e);
+    }
+    __syncthreads();
+    // phi(k) and the log gates, one warp per token
+    for (int i = warp; i < n; i += NT / 32) {
+      float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = kw[i][lane + 32 * j]; m = fmaxf(m, x[j]); sum += x[j]; }
+      m = warp_max(m);
+      sum = warp_sum(sum);
+      if (VG) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) lg[i][VG ? lane + 32 * j : 0] = log_sigmoid(x[j]);
+      } else if (lane == 0) {
+        lg[i][0] = log_sigmoid(sum / (float)D);
+      }
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
+      z = warp_sum(z);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) kw[i][lane + 32 * j] = x[j] / z;
+    }
+    __syncthreads();
+    // weights, last token first: one thread per key dimension
+    if (tid < D) {
+      float l = lam[tid];
+      for (int i = n - 1; i >= 0; --i) {
+        kw[i][tid] *= expf(l);
+        l += lg[i][VG ? tid : 0];
+      }
+      lam[tid] = l;
+    }
+    __syncthreads();
+    for (int i = 0; i < n; ++i) {
+      const float vc = vs[i][c];
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) acc[r] = fmaf(kw[i][rg * RPT + r], vc, acc[r]);
+    }
+  }
+  float* dst = ds + ((size_t)slot * Hkv + kv) * D * D;
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) dst[(size_t)(rg * RPT + r) * D + c] = acc[r];
+  __syncthreads();
+  if (tid < D) lam_out[((size_t)slot * Hkv + kv) * D + tid] = lam[tid];
+}
+
+// Per (sequence, kv head): folds the segments' contributions in order, overwriting
+// each segment's dS with the state entering it.  The scan starts from the group's
+// first copy of the initial state; when another copy of the group differs, the
+// (sequence, kv head) flag is set and the caller recomputes that group unsegmented.
+template <int D>
+__global__ void __launch_bounds__(kSegThreads) scan_kernel(const SimtSeg* segs, const int* n_segs, int Hq,
+                                                           int Hkv, const float* __restrict__ init_state,
+                                                           float* __restrict__ ds, const float* __restrict__ lam,
+                                                           uint32_t* flags) {
+  constexpr int NT = kSegThreads, RG = NT / D, RPT = D / RG;
+  const int seq = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
+  const int tid = threadIdx.x, c = tid % D, rg = tid / D;
+  const int G = Hq / Hkv;
+  float s[RPT];
+  bool differ = false;
+  if (init_state) {
+    const float* s0 = init_state + ((size_t)seq * Hq + (size_t)kv * G) * D * D;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = s0[(size_t)(rg * RPT + r) * D + c];
+    for (int hh = 1; hh < G; ++hh) {
+      const float* sh = s0 + (size_t)hh * D * D;
+#pragma unroll
+      for (int r = 0; r < RPT; ++r) differ |= sh[(size_t)(rg * RPT + r) * D + c] != s[r];
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = 0.f;
+  }
+  if (__syncthreads_or(differ) && tid == 0) flags[(size_t)seq * Hkv + kv] = 1u;
+  // the segments of one sequence are consecutive in the table, which is sorted by
+  // sequence: the first is found by bisection
+  const int n = *n_segs;
+  int first = 0, hi = n;
+  while (first < hi) {
+    const int mid = (first + hi) >> 1;
+    if (segs[mid].seq < seq) first = mid + 1;
+    else hi = mid;
+  }
+  for (int slot = first; slot < n && segs[slot].seq == seq; ++slot) {
+    float* p = ds + ((size_t)slot * Hkv + kv) * D * D;
+    const float* l = lam + ((size_t)slot * Hkv + kv) * D;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const size_t o = (size_t)(rg * RPT + r) * D + c;
+      const float d = p[o];
+      p[o] = s[r];
+      s[r] = fmaf(expf(l[rg * RPT + r]), s[r], d);
+    }
+  }
+}
+
+// Workspace of the segmented prefill: segment count, segment table, per (slot, kv
+// head) the total log gate [D] and dS / the entering state [D][D], the flags.
+struct Layout {
+  long cap;
+  size_t off_segs, off_lam, off_ds, off_flags, total;
+};
+inline Layout layout(long T_total, int n_seqs, int Hkv, int d) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  Layout L{};
+  L.cap = max_segments(T_total, n_seqs);
+  size_t off = 256;   // header: the segment count
+  L.off_segs = off;   off = al(off + sizeof(SimtSeg) * (size_t)L.cap);
+  L.off_lam = off;    off = al(off + sizeof(float) * (size_t)L.cap * Hkv * d);
+  L.off_ds = off;     off = al(off + sizeof(float) * (size_t)L.cap * Hkv * d * d);
+  L.off_flags = off;  off = al(off + sizeof(uint32_t) * (size_t)n_seqs * Hkv);
+  L.total = off;
+  return L;
+}
+
+}  // namespace seg
+}  // namespace liger

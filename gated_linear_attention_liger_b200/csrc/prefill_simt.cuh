@@ -7,7 +7,9 @@
 // rows), so the token-serial update S <- g S + phi(k)^T v and the readout
 // phi(q) S need no synchronisation inside a chunk.  Everything that is
 // parallel across the tokens of a chunk (feature maps, gates, window scores,
-// window softmax and its value sum) is done first, chunk by chunk.
+// window softmax and its value sum) is done first, chunk by chunk.  In segmented
+// mode (prefill_seg.cuh) one CTA takes one segment of a sequence per q head, from the
+// state a segment scan computed, with the window reaching back before the segment.
 //
 // Recurrence and hybrid: "Liger: Linearizing Large Language Models to Gated
 // Recurrent Structures" (Paper-Notes page), sections 统一的门控线性循环框架 and
@@ -17,6 +19,16 @@
 #include "common.cuh"
 
 namespace liger {
+
+// A run of tokens of one sequence that one CTA per q head processes (segmented mode):
+// the state entering it comes from a segment scan, the window reaches back into the
+// tokens before it.
+struct SimtSeg {
+  long t_begin, t_end;   // the segment's tokens
+  long seq_begin;        // first token of its sequence (the window starts no earlier)
+  int seq;               // sequence index
+  int flags;             // bit 0: first segment of its sequence; bit 1: last
+};
 
 struct SimtPrefillArgs {
   const void* q;
@@ -31,6 +43,12 @@ struct SimtPrefillArgs {
   float alpha;
   const uint32_t* only_flagged;   // [n][Hkv] or null: when set, a CTA works only if its
                                   // (sequence, kv head) flag is set, and returns at once otherwise
+  // Segmented mode (segs non-null): the grid is (segment slot, q head); a segment that is
+  // not its sequence's first starts from seg_state[slot][kv] (the state entering it, one
+  // per kv head) instead of init_state; only a last segment writes the final state.
+  const SimtSeg* segs;
+  const int* n_segs;
+  const float* seg_state;   // [slots][Hkv][D][D]
 };
 
 constexpr int kSimtThreads = 256;
@@ -69,11 +87,25 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
   const Tin* __restrict__ v = static_cast<const Tin*>(a.v);
   Tin* __restrict__ out = static_cast<Tin*>(a.out);
   const int Hq = a.Hq, Hkv = a.Hkv, w = a.w;
-  const int seq = blockIdx.x / Hq, h = blockIdx.x % Hq, kv = h / (Hq / Hkv);
+  const int unit = blockIdx.x / Hq, h = blockIdx.x % Hq, kv = h / (Hq / Hkv);
+  int seq = unit;
+  long tb, te, sb;          // sequence start, end of this CTA's tokens, first token of them
+  bool first = true, last = true;
+  if (a.segs) {
+    if (unit >= *a.n_segs) return;
+    const SimtSeg sg = a.segs[unit];
+    seq = sg.seq;
+    tb = sg.seq_begin;
+    sb = sg.t_begin;
+    te = sg.t_end;
+    first = (sg.flags & 1) != 0;
+    last = (sg.flags & 2) != 0;
+  } else {
+    const long T_total = a.cu ? a.T : (long)gridDim.x / Hq * a.T;
+    seq_range(a.cu, seq, a.T, T_total, &tb, &te);
+    sb = tb;
+  }
   if (a.only_flagged && a.only_flagged[(size_t)seq * Hkv + kv] == 0u) return;
-  const long T_total = a.cu ? a.T : (long)gridDim.x / Hq * a.T;
-  long tb, te;
-  seq_range(a.cu, seq, a.T, T_total, &tb, &te);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = tid % D, rg = tid / D;
@@ -82,11 +114,21 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
 
   float s[RPT];
   const size_t st_off = ((size_t)seq * Hq + h) * D * D;
+  const float* s_in = first ? (a.init_state ? a.init_state + st_off : nullptr)
+                            : a.seg_state + ((size_t)unit * Hkv + kv) * D * D;
 #pragma unroll
-  for (int r = 0; r < RPT; ++r)
-    s[r] = a.init_state ? a.init_state[st_off + (size_t)(rg * RPT + r) * D + c] : 0.f;
+  for (int r = 0; r < RPT; ++r) s[r] = s_in ? s_in[(size_t)(rg * RPT + r) * D + c] : 0.f;
 
-  for (long t0 = tb; t0 < te; t0 += C) {
+  // the window's keys and values before the first token (segmented mode)
+  for (long idx = tid; idx < (sb - max(tb, sb - (w - 1))) * D; idx += NT) {
+    const long t = max(tb, sb - (w - 1)) + idx / D;
+    const int e = (int)(idx % D);
+    const int slot = (int)((t - tb) % RING);
+    ring_k[slot * D + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
+    ring_v[slot * D + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
+  }
+
+  for (long t0 = sb; t0 < te; t0 += C) {
     const int n = (int)min((long)C, te - t0);
     // 1. stage the chunk: q rows, and k/v rows into the window ring
     for (int idx = tid; idx < n * D; idx += NT) {
@@ -196,7 +238,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
     }
     __syncthreads();
   }
-  if (a.final_state) {
+  if (a.final_state && last) {
 #pragma unroll
     for (int r = 0; r < RPT; ++r) a.final_state[st_off + (size_t)(rg * RPT + r) * D + c] = s[r];
   }

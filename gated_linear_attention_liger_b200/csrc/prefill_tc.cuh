@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       mbar_arrive(feat);
       named_bar(1, 256);   // lg is rewritten by the next chunk
     }
-    if (nch > 0 && mbar_wait(&mma_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, wc) && !*abort_flag) {
+    if (nch > 0 && warp_all(mbar_wait(&mma_done[(nch - 1) & 1], ((nch - 1) >> 1) & 1, wc) && !*abort_flag)) {
       tc_fence_after();
       float* dst = ds_out + (size_t)row * D;
 #pragma unroll 1
@@ -866,15 +866,18 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
         mma_commit(mma2_done);
         if (!fast) mma_commit(q_empty);   // exact decay: the readout read e^{b_i} e_q from the q buffer
       };
-      // A chunk's P.V goes out before the next chunk's window scores (the scores' TMEM
-      // holds the probability tile until then); the readout of a chunk waits for the
-      // feature warps to have stored the previous chunk's output.
+      // The next chunk's window scores go out as soon as the window warps have read the
+      // previous scores, ahead of the previous chunk's P.V, so the window warps' next
+      // softmax does not wait for that product.  The probability tile is rewritten only
+      // after the recurrent scores' completion, which the tensor pipe signals after every
+      // earlier product, P.V included.  The readout of a chunk waits for the feature
+      // warps to have stored the previous chunk's output.
       issue_ss(0);
       issue_sg_state(0);
       issue_inter(0);
       for (int c = 1; c < nch && ok; ++c) {
-        issue_pv(c - 1);
         issue_ss(c);
+        issue_pv(c - 1);
         issue_sg_state(c);
         issue_inter(c);
       }
@@ -1129,7 +1132,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1)
     // final state of the sequence: the carry after the last chunk of its last segment
     const SeqInfo si = p.seqs[sg.seq];
     const bool last = seg == si.first_seg + si.n_seg - 1;
-    if (p.final_state && last && mbar_wait(mma2_done, (nch - 1) & 1, wc, wsite(3, 5, nch)) && !*abort_flag) {
+    if (p.final_state && last && warp_all(mbar_wait(mma2_done, (nch - 1) & 1, wc, wsite(3, 5, nch)) && !*abort_flag)) {
       tc_fence_after();
 #pragma unroll 1
       for (int col = half * (D / 2); col < (half + 1) * (D / 2); col += 32) {

@@ -282,6 +282,13 @@ __device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* v) {
 }
 
 // 2^x on the special-function unit (approximate; flushes subnormal results to zero).
+// A predicate made the same on every lane of the warp (true only if true on all).
+// Warp-collective TMEM instructions (tcgen05.ld / st .sync.aligned) must be reached by
+// every lane together: a guard in front of them that could differ between lanes -- a
+// bounded wait that gave up on some lanes only, an abort flag read at different times --
+// goes through this first.  Every lane of the warp must call it.
+__device__ __forceinline__ bool warp_all(bool p) { return __all_sync(0xffffffffu, p); }
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

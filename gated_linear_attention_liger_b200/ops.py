@@ -46,8 +46,9 @@ SIGNATURES = {
     "liger_attn_prefill_backward_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
     "liger_attn_prefill_backward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float, _i,
                                          _vp, _i, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "liger_attn_prefill_vector_gate_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
     "liger_attn_prefill_vector_gate": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_float,
-                                            _i, _vp, _vp, _i, _vp, _vp, _vp]),
+                                            _i, _vp, _vp, _i, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "liger_attn_decode_vector_gate": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float,
                                            _i, _vp]),
     "liger_attn_full_causal": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp]),
@@ -347,10 +348,17 @@ def prefill_backward(q, k, v, d_out, alpha: float = 0.5, w: int = 64, d_final_st
     return dq, dk, dv, ds0
 
 
+def prefill_vector_gate_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:
+    return int(load().liger_attn_prefill_vector_gate_workspace_size(
+        B, Hq, Hkv, T, d, n_seqs, LIGER_BF16 if dtype == torch.bfloat16 else LIGER_FP32))
+
+
 def prefill_vector_gate(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=None, cu_seqlens=None,
-                        return_ring: bool = False, stream=None):
+                        return_ring: bool = False, workspace=None, stream=None):
     """The prefill with one gate per key dimension (sigmoid(k_t[r]) on row r of the state).
-    Returns (out, final_state) or, with return_ring, (out, final_state, ring, pos)."""
+    Returns (out, final_state) or, with return_ring, (out, final_state, ring, pos).
+    workspace: uint8 CUDA tensor of prefill_vector_gate_workspace_size() bytes (allocated
+    here when None)."""
     lib = load()
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q must be [B, T, Hq, d] and k, v [B, T, Hkv, d]")
@@ -368,9 +376,16 @@ def prefill_vector_gate(q, k, v, alpha: float = 0.5, w: int = 64, initial_state=
     fs = torch.empty(n, Hq, d, d, device=q.device, dtype=torch.float32)
     ring = torch.empty(n, Hkv, 2, w, d, device=q.device, dtype=q.dtype) if return_ring else None
     pos = torch.empty(n, device=q.device, dtype=torch.int32) if return_ring else None
+    need = lib.liger_attn_prefill_vector_gate_workspace_size(B, Hq, Hkv, T, d, n, _dt(q))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    _need_cuda(workspace)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor")
     st = lib.liger_attn_prefill_vector_gate(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(fs), B, Hq, Hkv, T, d, w, float(alpha), _dt(q),
-        _ptr(initial_state), _ptr(cu_seqlens), n, _ptr(ring), _ptr(pos), _stream_ptr(stream))
+        _ptr(initial_state), _ptr(cu_seqlens), n, _ptr(ring), _ptr(pos), _ptr(workspace), workspace.numel(),
+        _stream_ptr(stream))
     _check(st)
     return (out, fs, ring, pos) if return_ring else (out, fs)
 

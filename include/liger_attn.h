@@ -246,14 +246,22 @@ liger_status liger_attn_prefill_noalloc_status(void);
  * S_t = G_t (.) S_{t-1} + phi(k_t)^T v_t).  The pooling of the key is taken per
  * element: G_t[r] = sigmoid(k_t[r]) scales row r (key dimension) of the state,
  * as GLA's diagonal gate does; the window branch and the mix are unchanged.
- * Arguments, layouts and errors as liger_attn_prefill / liger_attn_decode (the
- * prefill takes no workspace: it runs the general CUDA-core kernel).
+ * Arguments, layouts and errors as liger_attn_prefill / liger_attn_decode.  The
+ * prefill runs on the CUDA cores in fp32, split into segments of 256 tokens that
+ * are processed in parallel after a scan over the segments' states; workspace
+ * is device scratch of at least liger_attn_prefill_vector_gate_workspace_size()
+ * bytes (16-byte aligned; a smaller one is LIGER_ERR_INVALID_ARG), owned by the
+ * caller and not read after the call's kernels end.  Supported: d in {64, 128},
+ * bf16 or fp32, w <= 64, any group size.
  */
+size_t liger_attn_prefill_vector_gate_workspace_size(int B, int Hq, int Hkv, int T, int d, int n_seqs,
+                                                     liger_dtype dt);
 liger_status liger_attn_prefill_vector_gate(const void* q, const void* k, const void* v, void* out,
                                             float* final_state, int B, int Hq, int Hkv, int T, int d, int w,
                                             float alpha, liger_dtype dt, const float* initial_state,
                                             const int32_t* cu_seqlens, int n_seqs, void* swa_ring_out,
-                                            int32_t* pos_out, void* stream);
+                                            int32_t* pos_out, void* workspace, size_t workspace_bytes,
+                                            void* stream);
 liger_status liger_attn_decode_vector_gate(const void* q, const void* k, const void* v, float* state,
                                            void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                            int d, int w, float alpha, liger_dtype dt, void* stream);

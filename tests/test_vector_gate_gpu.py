@@ -1,5 +1,5 @@
-"""The per-dimension (vector) gate on the GPU against the oracle: the prefill (general kernel)
-and decode steps, bf16 and fp32, with ragged and packed sequences and an initial state; the
+"""The per-dimension (vector) gate on the GPU against the oracle: the prefill (segment-parallel
+general kernels) and decode steps, bf16 and fp32, with ragged and packed sequences and an initial state; the
 Llama-3-8B-shape prefill in full.  Tolerances: bf16 max-abs 2e-2 and rel-L2 5e-3, fp32 1e-4."""
 import zlib
 
@@ -18,6 +18,11 @@ CASES = [
     ("bf16_d64_packed", 1, 4, 2, 230, 64, torch.bfloat16, (100, 0, 130), False),
     ("fp32_d64_s0", 1, 4, 4, 130, 64, torch.float32, (), True),
     ("fp32_d128", 1, 2, 1, 90, 128, torch.float32, (), False),
+    # several 256-token segments (a ragged last one), packed sequences across segment
+    # boundaries, an initial state shared by each group (the segment scan starts from it)
+    ("bf16_d128_segments", 1, 8, 2, 700, 128, torch.bfloat16, (), False),
+    ("bf16_d64_packed_segments", 1, 4, 2, 1100, 64, torch.bfloat16, (300, 0, 530, 270), False),
+    ("fp32_d64_shared_s0_segments", 2, 4, 2, 600, 64, torch.float32, (), "shared"),
 ]
 
 
@@ -29,6 +34,9 @@ def test_vector_gate_prefill_then_decode(case, cuda_device):
     q, k, v = inputs.prefill_inputs(wl)
     n = wl.n_seqs
     s0 = inputs.random_state(n, Hq, d, seed=4, scale=0.05) if with_s0 else None
+    if with_s0 == "shared":   # the copies of a group equal: one state per kv head
+        s0 = s0.view(n, Hkv, Hq // Hkv, d, d)[:, :, :1].expand(n, Hkv, Hq // Hkv, d, d).reshape(n, Hq, d, d)
+        s0 = s0.contiguous()
     cu = wl.cu_seqlens
     dev = cuda_device
     out, fs, ring, pos = ops.prefill_vector_gate(
