@@ -20,8 +20,12 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace liger {
+
+using sm100::ffma2;
+using sm100::fmul2;
 
 struct DecodeArgs {
   const void* q;
@@ -123,9 +127,9 @@ __device__ __forceinline__ void window_scores(const float (*qv)[D], const float*
   if (jj < 64) {   // all four lanes of a slot take part in the shuffles
     const int j = p - (w - 1) + jj;
     const bool live = jj < w && j >= 0;
-    float acc[NH];
+    float2 acc[NH];   // two partial sums (packed multiply-adds)
 #pragma unroll
-    for (int h = 0; h < NH; ++h) acc[h] = 0.f;
+    for (int h = 0; h < NH; ++h) acc[h] = make_float2(0.f, 0.f);
     if (live) {
 #pragma unroll
       for (int pc = qq; pc < NP; pc += 4) {
@@ -144,17 +148,15 @@ __device__ __forceinline__ void window_scores(const float (*qv)[D], const float*
 #pragma unroll
           for (int e = 0; e < EPP; e += 4) {
             const float4 qf = *reinterpret_cast<const float4*>(&qv[h][pc * EPP + e]);
-            acc[h] = fmaf(qf.x, x[e], acc[h]);
-            acc[h] = fmaf(qf.y, x[e + 1], acc[h]);
-            acc[h] = fmaf(qf.z, x[e + 2], acc[h]);
-            acc[h] = fmaf(qf.w, x[e + 3], acc[h]);
+            acc[h] = ffma2(make_float2(qf.x, qf.y), make_float2(x[e], x[e + 1]), acc[h]);
+            acc[h] = ffma2(make_float2(qf.z, qf.w), make_float2(x[e + 2], x[e + 3]), acc[h]);
           }
         }
       }
     }
 #pragma unroll
     for (int h = 0; h < NH; ++h) {
-      float t = acc[h];
+      float t = acc[h].x + acc[h].y;
       t += __shfl_xor_sync(0xffffffffu, t, 1);
       t += __shfl_xor_sync(0xffffffffu, t, 2);
       if (qq == 0 && jj < w) sc[h][jj] = live ? t * (1.0f / sqrtf((float)D)) : -INFINITY;
@@ -190,11 +192,11 @@ struct WindowValues {
     }
     constexpr int RS = ring_row_elems<Tin, D>();
     const int cp = tid % NPC, sg = tid / NPC;
-    float acc[NH][EPP];
+    float2 acc[NH][EPP / 2];   // element pairs (packed multiply-adds)
 #pragma unroll
     for (int h = 0; h < NH; ++h)
 #pragma unroll
-      for (int e = 0; e < EPP; ++e) acc[h][e] = 0.f;
+      for (int e = 0; e < EPP / 2; ++e) acc[h][e] = make_float2(0.f, 0.f);
     for (int jj = sg; jj < w; jj += NSG) {
       const int j = p - (w - 1) + jj;
       if (j < 0) continue;
@@ -208,8 +210,9 @@ struct WindowValues {
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         const float ph = expf(sc[h][jj] - mh[h]) * izh[h];
+        const float2 ph2 = make_float2(ph, ph);
 #pragma unroll
-        for (int e = 0; e < EPP; ++e) acc[h][e] = fmaf(ph, x[e], acc[h][e]);
+        for (int e = 0; e < EPP / 2; ++e) acc[h][e] = ffma2(ph2, make_float2(x[2 * e], x[2 * e + 1]), acc[h][e]);
       }
     }
 #pragma unroll
@@ -217,14 +220,17 @@ struct WindowValues {
 #pragma unroll
       for (int h = 0; h < NH; ++h)
 #pragma unroll
-        for (int e = 0; e < EPP; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
+        for (int e = 0; e < EPP / 2; ++e) {
+          acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+          acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
+        }
     if (lane < NPC) {
 #pragma unroll
       for (int h = 0; h < NH; ++h)
 #pragma unroll
-        for (int e = 0; e < EPP; e += 4)
-          *reinterpret_cast<float4*>(&wsum[tid >> 5][h][cp * EPP + e]) =
-              make_float4(acc[h][e], acc[h][e + 1], acc[h][e + 2], acc[h][e + 3]);
+        for (int e = 0; e < EPP / 2; e += 2)
+          *reinterpret_cast<float4*>(&wsum[tid >> 5][h][cp * EPP + 2 * e]) =
+              make_float4(acc[h][e].x, acc[h][e].y, acc[h][e + 1].x, acc[h][e + 1].y);
     }
   }
 };
@@ -312,24 +318,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kernel(DecodeArgs a)
     const float gs = gsh;
     const bool vg = a.vector_gate != 0;
     const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float2 v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
+    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int row = rg * RPT + r;
       const float kr = fk[row], qr = fq[row];
       const float g = vg ? gv[row] : gs;
-      float4 x = st[r];
-      x.x = fmaf(g, x.x, kr * vv.x);
-      x.y = fmaf(g, x.y, kr * vv.y);
-      x.z = fmaf(g, x.z, kr * vv.z);
-      x.w = fmaf(g, x.w, kr * vv.w);
-      acc.x = fmaf(qr, x.x, acc.x);
-      acc.y = fmaf(qr, x.y, acc.y);
-      acc.z = fmaf(qr, x.z, acc.z);
-      acc.w = fmaf(qr, x.w, acc.w);
-      st_stream(S + (size_t)row * D + 4 * cq, x);
+      const float2 g2 = make_float2(g, g), k2 = make_float2(kr, kr), q2 = make_float2(qr, qr);
+      const float2 x01 = ffma2(g2, make_float2(st[r].x, st[r].y), fmul2(k2, v01));
+      const float2 x23 = ffma2(g2, make_float2(st[r].z, st[r].w), fmul2(k2, v23));
+      a01 = ffma2(q2, x01, a01);
+      a23 = ffma2(q2, x23, a23);
+      st_stream(S + (size_t)row * D + 4 * cq, make_float4(x01.x, x01.y, x23.x, x23.y));
     }
-    *reinterpret_cast<float4*>(&part[rg][4 * cq]) = acc;
+    *reinterpret_cast<float4*>(&part[rg][4 * cq]) = make_float4(a01.x, a01.y, a23.x, a23.y);
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
@@ -454,30 +457,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
   {
     const float g = gsh;
     const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
-    float4 acc[G];
+    const float2 g2 = make_float2(g, g), v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
+    float2 a01[G], a23[G];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int hh = 0; hh < G; ++hh) a01[hh] = a23[hh] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
       const int row = rg * RPT + r;
       const float kr = fk[row];
-      float4 x = st[r];
-      x.x = fmaf(g, x.x, kr * vv.x);
-      x.y = fmaf(g, x.y, kr * vv.y);
-      x.z = fmaf(g, x.z, kr * vv.z);
-      x.w = fmaf(g, x.w, kr * vv.w);
+      const float2 k2 = make_float2(kr, kr);
+      const float2 x01 = ffma2(g2, make_float2(st[r].x, st[r].y), fmul2(k2, v01));
+      const float2 x23 = ffma2(g2, make_float2(st[r].z, st[r].w), fmul2(k2, v23));
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         const float qr = fq[hh][row];
-        acc[hh].x = fmaf(qr, x.x, acc[hh].x);
-        acc[hh].y = fmaf(qr, x.y, acc[hh].y);
-        acc[hh].z = fmaf(qr, x.z, acc[hh].z);
-        acc[hh].w = fmaf(qr, x.w, acc[hh].w);
+        const float2 q2 = make_float2(qr, qr);
+        a01[hh] = ffma2(q2, x01, a01[hh]);
+        a23[hh] = ffma2(q2, x23, a23[hh]);
       }
-      st_stream(S + (size_t)row * D + 4 * cq, x);
+      st_stream(S + (size_t)row * D + 4 * cq, make_float4(x01.x, x01.y, x23.x, x23.y));
     }
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = acc[hh];
+    for (int hh = 0; hh < G; ++hh)
+      *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = make_float4(a01[hh].x, a01[hh].y, a23[hh].x, a23[hh].y);
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
