@@ -17,6 +17,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace liger {
 
@@ -55,31 +56,40 @@ constexpr int kSimtThreads = 256;
 constexpr int kSimtChunk = 32;         // tokens per chunk
 constexpr int kSimtRing = 96;          // >= 64 + kSimtChunk - 1 window slots
 constexpr int kMaxWindow = 64;
+// Shared-memory ring rows are padded by 4 floats: consecutive slots then sit in different
+// 16-byte bank groups, so eight lanes reading eight slots at the same column do not conflict.
+template <int D>
+constexpr int simt_ring_stride() { return D + 4; }
 
 // VG: one gate per key dimension, sigmoid(k_t[r]) on row r of the state (the
 // per-dimension form of the pooled key gate); otherwise the pooled scalar gate.
 template <int D, bool VG = false>
 constexpr size_t simt_prefill_smem_bytes() {
   constexpr int RG = kSimtThreads / D;
-  return sizeof(float) * (size_t)(2 * kSimtRing * D + 3 * kSimtChunk * D + kSimtChunk * RG * D +
-                                  kSimtChunk * kMaxWindow + kSimtChunk + (VG ? kSimtChunk * D : 0));
+  return sizeof(float) * (size_t)(2 * kSimtRing * simt_ring_stride<D>() + 3 * kSimtChunk * D + kSimtChunk * RG * D +
+                                  kSimtChunk * kSimtRing + kSimtChunk + (VG ? kSimtChunk * D : 0));
 }
 
 template <typename Tin, int D, bool VG = false>
 __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillArgs a) {
-  constexpr int NT = kSimtThreads, C = kSimtChunk, RING = kSimtRing, W64 = kMaxWindow;
+  constexpr int NT = kSimtThreads, C = kSimtChunk, RING = kSimtRing;
+  constexpr int RS = simt_ring_stride<D>();
   constexpr int RG = NT / D;      // row groups
   constexpr int RPT = D / RG;     // key rows per thread
   constexpr int EPL = D / 32;     // elements per lane for row-wise work
+  constexpr int TPW = C / (NT / 32);   // window: tokens per warp
+  constexpr int XPL = RING / 32;       // window: ring positions per lane
+  static_assert(RING == C + kMaxWindow && RING % 32 == 0 && C % (NT / 32) == 0 && RPT % 4 == 0 &&
+                (EPL == 2 || EPL == 4), "window and row tiling");
   extern __shared__ float smem[];
-  float* ring_k = smem;                     // [RING][D]
-  float* ring_v = ring_k + RING * D;        // [RING][D]
-  float* qbuf = ring_v + RING * D;          // [C][D]  raw q, later the window output
+  float* ring_k = smem;                     // [RING][RS]
+  float* ring_v = ring_k + RING * RS;       // [RING][RS]
+  float* qbuf = ring_v + RING * RS;         // [C][D]  raw q, later the window output
   float* fq = qbuf + C * D;                 // [C][D]  phi(q)
   float* fk = fq + C * D;                   // [C][D]  phi(k)
   float* part = fk + C * D;                 // [C][RG][D] partial readouts
-  float* sc = part + C * RG * D;            // [C][W64] window scores / probabilities
-  float* gate = sc + C * W64;               // [C]
+  float* sc = part + C * RG * D;            // [C][RING] window probabilities over the ring positions
+  float* gate = sc + C * RING;              // [C]
   float* gvec = gate + C;                   // [C][D] per-dimension gates (VG only)
 
   const Tin* __restrict__ q = static_cast<const Tin*>(a.q);
@@ -124,8 +134,8 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
     const long t = max(tb, sb - (w - 1)) + idx / D;
     const int e = (int)(idx % D);
     const int slot = (int)((t - tb) % RING);
-    ring_k[slot * D + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
-    ring_v[slot * D + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
+    ring_k[slot * RS + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
+    ring_v[slot * RS + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
   }
 
   for (long t0 = sb; t0 < te; t0 += C) {
@@ -136,8 +146,8 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       const long t = t0 + i;
       const int slot = (int)((t - tb) % RING);
       qbuf[idx] = io<Tin>::ld(q + ((size_t)t * Hq + h) * D + e);
-      ring_k[slot * D + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
-      ring_v[slot * D + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
+      ring_k[slot * RS + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
+      ring_v[slot * RS + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
     }
     __syncthreads();
     // 2. feature maps and gate, one warp per token
@@ -146,7 +156,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       float x[EPL];
       float m = -INFINITY, sum = 0.f;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = ring_k[slot * D + lane + 32 * j]; m = fmaxf(m, x[j]); sum += x[j]; }
+      for (int j = 0; j < EPL; ++j) { x[j] = ring_k[slot * RS + lane + 32 * j]; m = fmaxf(m, x[j]); sum += x[j]; }
       m = warp_max(m);
       sum = warp_sum(sum);
       float z = 0.f;
@@ -157,7 +167,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       for (int j = 0; j < EPL; ++j) fk[i * D + lane + 32 * j] = x[j] / z;
       if (VG) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) gvec[i * D + lane + 32 * j] = expf(log_sigmoid(ring_k[slot * D + lane + 32 * j]));
+        for (int j = 0; j < EPL; ++j) gvec[i * D + lane + 32 * j] = expf(log_sigmoid(ring_k[slot * RS + lane + 32 * j]));
       } else if (lane == 0) {
         gate[i] = expf(log_sigmoid(sum / (float)D));
       }
@@ -172,60 +182,128 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
 #pragma unroll
       for (int j = 0; j < EPL; ++j) fq[i * D + lane + 32 * j] = x[j] / z;
     }
-    // 3a. window scores q_t . k_j / sqrt(d) for j = t-w+1 .. t, one warp per pair
-    for (int pr = warp; pr < n * w; pr += NT / 32) {
-      const int i = pr / w, jj = pr % w;
-      const long j = t0 + i - (w - 1) + jj;
-      float dot = -INFINITY;
-      if (j >= tb) {
-        const int slot = (int)((j - tb) % RING);
-        float acc = 0.f;
+    __syncthreads();   // features and gates of every token (phase 2 rows are spread over the warps)
+    // 3. window branch over the ring, which holds positions t0 - 64 .. t0 + C - 1 (ring
+    //    position x holds t0 - 64 + x; slot = (position - tb) mod RING).  Warp w takes the
+    //    tokens w TPW .. w TPW + TPW - 1, lane l the ring positions l, l + 32, l + 64: each
+    //    thread forms its TPW x XPL scores in registers (row i sees x in [i + 64 - w + 1,
+    //    i + 64] at positions >= tb), the warp reduces each row's softmax statistics.
+    const int i0 = warp * TPW;
+    const long pbase = t0 - kMaxWindow;   // position of ring position 0
+    const int slot0 = (int)((((pbase - tb) % RING) + RING) % RING);
+    {
+      int xslot[XPL];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          acc = fmaf(qbuf[i * D + lane + 32 * e], ring_k[slot * D + lane + 32 * e], acc);
-        dot = warp_sum(acc) * inv_sqrt_d;
+      for (int u = 0; u < XPL; ++u) {
+        const int sl = slot0 + lane + 32 * u;
+        xslot[u] = sl >= RING ? sl - RING : sl;
       }
-      if (lane == 0) sc[i * W64 + jj] = dot;
-    }
-    __syncthreads();
-    // 3b. window softmax, one warp per token row
-    for (int i = warp; i < n; i += NT / 32) {
-      const float x0 = lane < w ? sc[i * W64 + lane] : -INFINITY;
-      const float x1 = lane + 32 < w ? sc[i * W64 + lane + 32] : -INFINITY;
-      const float m = warp_max(fmaxf(x0, x1));   // the token itself is always valid
-      const float e0 = lane < w ? expf(x0 - m) : 0.f;
-      const float e1 = lane + 32 < w ? expf(x1 - m) : 0.f;
-      const float z = warp_sum(e0 + e1);
-      if (lane < w) sc[i * W64 + lane] = e0 / z;
-      if (lane + 32 < w) sc[i * W64 + lane + 32] = e1 / z;
-    }
-    __syncthreads();
-    // 3c. window output into qbuf (raw q no longer needed)
-    for (int idx = tid; idx < n * D; idx += NT) {
-      const int i = idx / D, e = idx % D;
-      const long t = t0 + i;
-      float acc = 0.f;
-      for (int jj = 0; jj < w; ++jj) {
-        const long j = t - (w - 1) + jj;
-        if (j < tb) continue;
-        acc = fmaf(sc[i * W64 + jj], ring_v[((int)((j - tb) % RING)) * D + e], acc);
+      float acc[TPW][XPL];
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+        for (int u = 0; u < XPL; ++u) acc[tt][u] = 0.f;
+#pragma unroll 4
+      for (int e = 0; e < D; e += 4) {
+        float4 kq[XPL];
+#pragma unroll
+        for (int u = 0; u < XPL; ++u) kq[u] = *reinterpret_cast<const float4*>(ring_k + xslot[u] * RS + e);
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+          const float4 qq = *reinterpret_cast<const float4*>(qbuf + (i0 + tt) * D + e);
+#pragma unroll
+          for (int u = 0; u < XPL; ++u)
+            acc[tt][u] = fmaf(qq.x, kq[u].x, fmaf(qq.y, kq[u].y, fmaf(qq.z, kq[u].z, fmaf(qq.w, kq[u].w, acc[tt][u]))));
+        }
       }
-      qbuf[idx] = acc;
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt) {
+        const int i = i0 + tt;
+        float sv[XPL], m = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < XPL; ++u) {
+          const int x = lane + 32 * u;
+          const bool ok = i < n && x >= i + kMaxWindow - w + 1 && x <= i + kMaxWindow && pbase + x >= tb;
+          sv[u] = ok ? acc[tt][u] * inv_sqrt_d : -INFINITY;
+          m = fmaxf(m, sv[u]);
+        }
+        m = warp_max(m);   // finite for i < n: the token itself is always in its window
+        float z = 0.f;
+#pragma unroll
+        for (int u = 0; u < XPL; ++u) {
+          sv[u] = sv[u] == -INFINITY ? 0.f : expf(sv[u] - m);
+          z += sv[u];
+        }
+        z = warp_sum(z);
+        const float iz = z > 0.f ? 1.f / z : 0.f;
+#pragma unroll
+        for (int u = 0; u < XPL; ++u) sc[i * RING + lane + 32 * u] = sv[u] * iz;
+      }
     }
-    // 4. token-serial recurrence on the register-resident state (no syncs)
+    __syncwarp();
+    // window output into qbuf (this warp's tokens; lane l holds elements EPL l .. EPL l + EPL - 1)
+    {
+      float o[TPW][EPL];
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) o[tt][q] = 0.f;
+      // positions of this warp's windows that hold this chunk's or earlier tokens of the
+      // sequence (the others hold no value of it and have zero weight)
+      const int xlo = max(max(0, i0 + kMaxWindow - w + 1), (int)max(0L, tb - pbase));
+      const int xhi = min(min(RING - 1, i0 + TPW - 1 + kMaxWindow), n - 1 + kMaxWindow);
+      int sl = slot0 + xlo;
+      sl = sl >= RING ? sl - RING : sl;
+#pragma unroll 2
+      for (int x = xlo; x <= xhi; ++x) {
+        float vv[EPL];
+        if (EPL == 4) {
+          const float4 t4 = *reinterpret_cast<const float4*>(ring_v + sl * RS + EPL * lane);
+          vv[0] = t4.x; vv[1] = t4.y; vv[EPL > 2 ? 2 : 0] = t4.z; vv[EPL > 3 ? 3 : 0] = t4.w;
+        } else {
+          const float2 t2 = *reinterpret_cast<const float2*>(ring_v + sl * RS + EPL * lane);
+          vv[0] = t2.x; vv[1] = t2.y;
+        }
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+          const float pr = sc[(i0 + tt) * RING + x];
+#pragma unroll
+          for (int q = 0; q < EPL; ++q) o[tt][q] = fmaf(pr, vv[q], o[tt][q]);
+        }
+        sl = sl + 1 == RING ? 0 : sl + 1;
+      }
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) qbuf[(i0 + tt) * D + EPL * lane + q] = o[tt][q];
+    }
+    // 4. token-serial recurrence on the register-resident state (no syncs); rows in fours
+    //    from shared memory, pairs of rows in packed multiply-adds
     for (int i = 0; i < n; ++i) {
       const float g = VG ? 1.f : gate[i];
-      const float vc = ring_v[((int)((t0 + i - tb) % RING)) * D + c];
+      const float vc = ring_v[((int)((t0 + i - tb) % RING)) * RS + c];
       const float* fki = fk + i * D + rg * RPT;
       const float* fqi = fq + i * D + rg * RPT;
-      float acc = 0.f;
       const float* gvi = gvec + i * D + rg * RPT;
+      const float2 vc2 = make_float2(vc, vc), g2 = make_float2(g, g);
+      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        s[r] = fmaf(VG ? gvi[r] : g, s[r], fki[r] * vc);
-        acc = fmaf(fqi[r], s[r], acc);
+      for (int r = 0; r < RPT; r += 4) {
+        const float4 kf = *reinterpret_cast<const float4*>(fki + r);
+        const float4 qf = *reinterpret_cast<const float4*>(fqi + r);
+        float2 ga = g2, gb = g2;
+        if (VG) {
+          const float4 gf = *reinterpret_cast<const float4*>(gvi + r);
+          ga = make_float2(gf.x, gf.y);
+          gb = make_float2(gf.z, gf.w);
+        }
+        const float2 s01 = sm100::ffma2(ga, make_float2(s[r], s[r + 1]), sm100::fmul2(make_float2(kf.x, kf.y), vc2));
+        const float2 s23 = sm100::ffma2(gb, make_float2(s[r + 2], s[r + 3]), sm100::fmul2(make_float2(kf.z, kf.w), vc2));
+        s[r] = s01.x; s[r + 1] = s01.y; s[r + 2] = s23.x; s[r + 3] = s23.y;
+        a01 = sm100::ffma2(make_float2(qf.x, qf.y), s01, a01);
+        a23 = sm100::ffma2(make_float2(qf.z, qf.w), s23, a23);
       }
-      part[(i * RG + rg) * D + c] = acc;
+      part[(i * RG + rg) * D + c] = (a01.x + a01.y) + (a23.x + a23.y);
     }
     __syncthreads();
     // 5. mix and store
