@@ -693,7 +693,7 @@ def time_full_attention(wl, args, world, dev, stream, pk, windows):
     return {"metric": "causal attention tokens/s (8B attn shape)", "value": world * wl.tokens / (k_ms * 1e-3),
             "unit": "tokens/s", "ms_per_step": k_ms, "steps": n, "status": ops.STATUS_NAMES.get(status, status),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / pk["bf16_tflops"], "traffic": None, "kernel": "causal attention",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": measured_traffic("full_attn_kernel<128>"), "kernel": "causal attention",
                          "kernel_ms": k_ms, "algorithmic_flops": flops, "peak_source": pk["source"],
                          "frac_of": f"{pk['source']} cuBLAS bf16 burst"}}
 
