@@ -141,15 +141,20 @@ liger_status run_segmented(const liger::SimtPrefillArgs& a, int n_seqs, long T_t
   float* lam = reinterpret_cast<float*>(w + L.off_lam);
   float* ds = reinterpret_cast<float*>(w + L.off_ds);
   uint32_t* flags = reinterpret_cast<uint32_t*>(w + L.off_flags);
-  if (L.cap * a.Hkv > 0x7fffffffL || L.cap * a.Hq > 0x7fffffffL || (long)n_seqs * a.Hkv > 0x7fffffffL)
+  if (L.cap * a.Hkv > 0x7fffffffL || L.cap * a.Hq > 0x7fffffffL ||
+      (long)n_seqs * a.Hkv * (D * D / liger::seg::kScanThreads) > 0x7fffffffL)
     return fail(LIGER_ERR_UNSUPPORTED, "too many segments");
   sg::plan_kernel<<<1, 32, 0, s>>>(a.cu, a.T, n_seqs, T_total, segs, count, L.cap, flags, a.Hkv);
   ++g_launches;
-  sg::seg_state_kernel<Tin, D, VG><<<(unsigned)(L.cap * a.Hkv), sg::kSegThreads, 0, s>>>(
+  constexpr size_t seg_smem = sg::seg_state_smem_bytes<D, VG>();
+  if (cudaFuncSetAttribute(sg::seg_state_kernel<Tin, D, VG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)seg_smem) != cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(segment states)");
+  sg::seg_state_kernel<Tin, D, VG><<<(unsigned)(L.cap * a.Hkv), sg::kSegThreads, seg_smem, s>>>(
       static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.Hkv, segs, count, ds, lam);
   ++g_launches;
-  sg::scan_kernel<D><<<(unsigned)((long)n_seqs * a.Hkv), sg::kSegThreads, 0, s>>>(segs, count, a.Hq, a.Hkv,
-                                                                                   a.init_state, ds, lam, flags);
+  sg::scan_kernel<D><<<(unsigned)((long)n_seqs * a.Hkv * (D * D / sg::kScanThreads)), sg::kScanThreads, 0, s>>>(
+      segs, count, a.Hq, a.Hkv, a.init_state, ds, lam, flags);
   ++g_launches;
   liger_status st = cuda_check("segmented prefill launch");
   if (st != LIGER_OK) return st;

@@ -28,7 +28,7 @@ namespace seg {
 
 constexpr int kSegTokens = 256;   // tokens per segment
 constexpr int kSegThreads = 256;
-constexpr int kStage = 16;        // tokens staged in shared memory at a time
+constexpr int kStage = 64;        // tokens staged in shared memory at a time
 
 // Upper bound of the segment count: every sequence adds at most one partial (or empty)
 // segment.
@@ -59,7 +59,7 @@ __global__ void plan_kernel(const int32_t* cu, long T, int n_seqs, long T_total,
 }
 
 // Per (segment slot, kv head), 256 threads: thread (column c, row group rg) owns
-// rows rg*RPT .. rg*RPT+RPT-1 of column c of dS.  Tokens are staged 16 at a time,
+// rows rg*RPT .. rg*RPT+RPT-1 of column c of dS.  Tokens are staged 64 at a time,
 // last to first: lam[r] = B - B_j (the gates after token j) is then known when j is
 // reached, and w_j[r] = e^{lam[r]} phi(k_j)[r] <= phi(k_j)[r].
 template <typename Tin, int D, bool VG>
@@ -69,9 +69,10 @@ __global__ void __launch_bounds__(kSegThreads) seg_state_kernel(const Tin* __res
                                                                 float* __restrict__ ds, float* __restrict__ lam_out) {
   constexpr int NT = kSegThreads, S = kStage;
   constexpr int RG = NT / D, RPT = D / RG, EPL = D / 32;
-  __shared__ __align__(16) float kw[S][D];   // raw keys, then the weights w_j
-  __shared__ __align__(16) float vs[S][D];
-  __shared__ float lg[S][VG ? D : 1];        // log gates
+  extern __shared__ __align__(16) float seg_smem[];
+  float (*kw)[D] = reinterpret_cast<float (*)[D]>(seg_smem);            // [S][D] raw keys, then the weights w_j
+  float (*vs)[D] = reinterpret_cast<float (*)[D]>(seg_smem + S * D);    // [S][D]
+  float (*lg)[VG ? D : 1] = reinterpret_cast<float (*)[VG ? D : 1]>(seg_smem + 2 * S * D);   // [S] log gates
   __shared__ float lam[D];                   // gates after the staged block
   const int slot = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
   if (slot >= *n_segs) return;
@@ -135,35 +136,34 @@ __global__ void __launch_bounds__(kSegThreads) seg_state_kernel(const Tin* __res
   if (tid < D) lam_out[((size_t)slot * Hkv + kv) * D + tid] = lam[tid];
 }
 
-// Per (sequence, kv head): folds the segments' contributions in order, overwriting
-// each segment's dS with the state entering it.  The scan starts from the group's
-// first copy of the initial state; when another copy of the group differs, the
-// (sequence, kv head) flag is set and the caller recomputes that group unsegmented.
+template <int D, bool VG>
+constexpr size_t seg_state_smem_bytes() { return sizeof(float) * (size_t)kStage * (2 * D + (VG ? D : 1)); }
+
+// Per (sequence, kv head, block of 256 state elements): folds the segments'
+// contributions in order, overwriting each segment's dS with the state entering it
+// (every element of the state evolves on its own: S_in(s+1)[r][c] = e^{B_s[r]} S_in(s)[r][c]
+// + dS_s[r][c]).  The scan starts from the group's first copy of the initial state; when
+// another copy of the group differs, the (sequence, kv head) flag is set and the caller
+// recomputes that group unsegmented.
+constexpr int kScanThreads = 256;
 template <int D>
-__global__ void __launch_bounds__(kSegThreads) scan_kernel(const SimtSeg* segs, const int* n_segs, int Hq,
-                                                           int Hkv, const float* __restrict__ init_state,
-                                                           float* __restrict__ ds, const float* __restrict__ lam,
-                                                           uint32_t* flags) {
-  constexpr int NT = kSegThreads, RG = NT / D, RPT = D / RG;
-  const int seq = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
-  const int tid = threadIdx.x, c = tid % D, rg = tid / D;
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const SimtSeg* segs, const int* n_segs, int Hq,
+                                                            int Hkv, const float* __restrict__ init_state,
+                                                            float* __restrict__ ds, const float* __restrict__ lam,
+                                                            uint32_t* flags) {
+  constexpr int BPU = D * D / kScanThreads;   // blocks per (sequence, kv head)
+  const int unit = blockIdx.x / BPU, blk = blockIdx.x % BPU;
+  const int seq = unit / Hkv, kv = unit % Hkv;
+  const int e = blk * kScanThreads + threadIdx.x, r = e / D;
   const int G = Hq / Hkv;
-  float s[RPT];
-  bool differ = false;
+  float s = 0.f;
   if (init_state) {
-    const float* s0 = init_state + ((size_t)seq * Hq + (size_t)kv * G) * D * D;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) s[r] = s0[(size_t)(rg * RPT + r) * D + c];
-    for (int hh = 1; hh < G; ++hh) {
-      const float* sh = s0 + (size_t)hh * D * D;
-#pragma unroll
-      for (int r = 0; r < RPT; ++r) differ |= sh[(size_t)(rg * RPT + r) * D + c] != s[r];
-    }
-  } else {
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) s[r] = 0.f;
+    const float* s0 = init_state + ((size_t)seq * Hq + (size_t)kv * G) * D * D + e;
+    s = s0[0];
+    bool differ = false;
+    for (int hh = 1; hh < G; ++hh) differ |= s0[(size_t)hh * D * D] != s;
+    if (__syncthreads_or(differ) && threadIdx.x == 0) atomicOr(&flags[(size_t)seq * Hkv + kv], 1u);
   }
-  if (__syncthreads_or(differ) && tid == 0) flags[(size_t)seq * Hkv + kv] = 1u;
   // the segments of one sequence are consecutive in the table, which is sorted by
   // sequence: the first is found by bisection
   const int n = *n_segs;
@@ -174,15 +174,10 @@ __global__ void __launch_bounds__(kSegThreads) scan_kernel(const SimtSeg* segs, 
     else hi = mid;
   }
   for (int slot = first; slot < n && segs[slot].seq == seq; ++slot) {
-    float* p = ds + ((size_t)slot * Hkv + kv) * D * D;
-    const float* l = lam + ((size_t)slot * Hkv + kv) * D;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const size_t o = (size_t)(rg * RPT + r) * D + c;
-      const float d = p[o];
-      p[o] = s[r];
-      s[r] = fmaf(expf(l[rg * RPT + r]), s[r], d);
-    }
+    float* pp = ds + ((size_t)slot * Hkv + kv) * D * D + e;
+    const float d = *pp;
+    *pp = s;
+    s = fmaf(expf(lam[((size_t)slot * Hkv + kv) * D + r]), s, d);
   }
 }
 

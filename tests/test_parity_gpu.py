@@ -288,16 +288,18 @@ def test_full_llama8b_decode(cuda_device):
 
 # ----------------------------------------------------------------- shared-state decode
 
-@pytest.mark.parametrize("dtype,d,w,T0,G", [
-    (torch.bfloat16, 128, 64, 70, 4),
-    (torch.bfloat16, 64, 64, 0, 2),
-    (torch.bfloat16, 64, 16, 5, 1),
-    (torch.float32, 128, 64, 100, 4),
+@pytest.mark.parametrize("dtype,d,w,T0,G,B", [
+    (torch.bfloat16, 128, 64, 70, 4, 3),
+    (torch.bfloat16, 64, 64, 0, 2, 3),
+    (torch.bfloat16, 64, 16, 5, 1, 3),
+    (torch.float32, 128, 64, 100, 4, 3),
+    # more (sequence, kv head) units than SMs
+    (torch.bfloat16, 64, 64, 30, 4, 170),
 ])
-def test_decode_kvshared_parity(dtype, d, w, T0, G, cuda_device):
+def test_decode_kvshared_parity(dtype, d, w, T0, G, B, cuda_device):
     """One state per kv head: the oracle runs with that state copied to every q head of
     the group; outputs, the (shared) state, ring and positions must match."""
-    B, Hkv, steps = 3, 2, 10
+    Hkv, steps = 2, 10
     Hq = Hkv * G
     wl = inputs.small("deckv", B=B, Hq=Hq, Hkv=Hkv, T=T0 + steps, d=d, dtype=dtype, seed=29)
     q, k, v = inputs.prefill_inputs(wl)
