@@ -246,7 +246,7 @@ liger_status launch_full_attn(const CUtensorMap& mq, const CUtensorMap& mk, cons
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)liger::fa::Smem<D>::BYTES) !=
       cudaSuccess)
     return cuda_check("cudaFuncSetAttribute(full_attn)");
-  const dim3 grid((unsigned)prm.n_qblk, (unsigned)Hq, (unsigned)n_seqs);
+  const dim3 grid((unsigned)((prm.n_qblk + 1) / 2), (unsigned)Hq, (unsigned)n_seqs);   // pairs of query blocks
   mark_start(s);
   kern<<<grid, liger::fa::kThreads, liger::fa::Smem<D>::BYTES, s>>>(mq, mk, mv, prm);
   mark_stop(s);
