@@ -775,6 +775,10 @@ __global__ void __launch_bounds__(160, 1)
         for (int u8 = 0; u8 < 32; u8 += 8) {
           float x[8];
           tc::ld_chunk8(qb, kmajor_off(row, c0 + u8, ROWS * 128), x);
+          // the window part of dq: eight consecutive fp32 in two 16-byte loads
+          const float4 wa = *reinterpret_cast<const float4*>(bp.dq_acc + o + c0 + u8);
+          const float4 wb = *reinterpret_cast<const float4*>(bp.dq_acc + o + c0 + u8 + 4);
+          const float wq[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
           uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 8; q += 2) {
@@ -783,7 +787,7 @@ __global__ void __launch_bounds__(160, 1)
             for (int e = 0; e < 2; ++e) {
               const float ph = ex2(fmaf(x[q + e], kL2e, -mq)) * izq;
               const float dphi = fmaf(eb, xv[u8 + q + e], rq * mv[u8 + q + e]);
-              y[e] = fmaf(ph, dphi - dot, bp.dq_acc[o + c0 + u8 + q + e]);
+              y[e] = fmaf(ph, dphi - dot, wq[q + e]);
             }
             w[q / 2] = pack_bf16(y[0], y[1]);
           }
