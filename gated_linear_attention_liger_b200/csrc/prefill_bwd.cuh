@@ -696,12 +696,6 @@ __global__ void __launch_bounds__(160, 1)
       av[j] = a;
       rowsum = fmaf(a, g[j], rowsum);
     }
-    // column sums over the pair's rows: warp sums, then shared atomics
-#pragma unroll
-    for (int j = 0; j < C; ++j) {
-      const float cs = warp_sum(av[j] * g[j]);
-      if (lane == 0) atomicAdd(&colsum[j], cs);
-    }
 #pragma unroll
     for (int j8 = 0; j8 < C; j8 += 8) {
       float x[8];
@@ -710,6 +704,24 @@ __global__ void __launch_bounds__(160, 1)
       tc::st_chunk8(smem + L::AT, kmajor_off(row, j8, ROWS * 128), x);
     }
     fence_proxy_async_smem();
+    // column sums over the pair's rows: a reduce-scatter across the warp (each exchange
+    // halves the columns a lane holds; lane l ends with columns 2 l and 2 l + 1), then
+    // shared atomics across the warps
+#pragma unroll
+    for (int j = 0; j < C; ++j) av[j] *= g[j];
+    static_assert(C == 64, "two columns per lane at the end");
+#pragma unroll
+    for (int half = C / 2, mask = 16; half >= 2; half >>= 1, mask >>= 1) {
+      const bool up = (lane & mask) != 0;   // this lane keeps the upper half of its columns
+#pragma unroll
+      for (int k = 0; k < half; ++k) {
+        const float keep = up ? av[k + half] : av[k];
+        const float send = up ? av[k] : av[k + half];
+        av[k] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+      }
+    }
+    atomicAdd(&colsum[2 * lane], av[0]);
+    atomicAdd(&colsum[2 * lane + 1], av[1]);
   }
   tc_fence_before();
   __syncthreads();
