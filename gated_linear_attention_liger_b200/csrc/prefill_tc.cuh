@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::SMALL);
   uint64_t* k_full = bars;         // [2]
-  uint64_t* k_empty = bars + 2;    // [2] (256 arrivals)
+  uint64_t* img_ready = bars + 2;  // [2] the chunk's key image written over its raw keys (256 arrivals)
   uint64_t* v_full = bars + 4;     // [2]
   uint64_t* v_empty = bars + 7;    // [2]
   uint64_t* feat = bars + 10;
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kSegThreads, 2)
   constexpr uint32_t TCOLS = D < 32 ? 32 : D;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 256); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&k_full[i], 1); mbar_init(&img_ready[i], 256); }
     for (int i = 0; i < 2; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(feat, 256); mbar_init(&mma_done[0], 1); mbar_init(&mma_done[1], 1); mbar_init(drain, 1);
     *abort_flag = 0u;
@@ -475,11 +475,23 @@ __global__ void __launch_bounds__(kSegThreads, 2)
     if (lane == 0) {
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
-      int k_issued = 0, v_issued = 0;
+      // The key image of step c is written by the row warps over step c's raw keys; this
+      // thread stores it to the workspace in one bulk copy and then refills the slot.
+      auto store_img = [&](int c) {
+        const size_t ci = (size_t)(seg * p.L + sub * p.Ls + (nch - 1 - c)) * p.Hkv + kv;
+        bulk_store(p.kimg + ci * L::KV, smem + L::K0 + (c & 1) * L::KV, L::KV);
+        bulk_commit();
+      };
+      int k_issued = 0, v_issued = 0, stored = 0;
       for (int c = 0; c < nch; ++c) {   // step c handles chunk nch - 1 - c (last to first)
         const int t = sg.t_begin + (nch - 1 - c) * C;
         const int ks = c & 1, vs = c & 1;
-        if (c >= 2 && !mbar_wait(&k_empty[ks], ((c >> 1) - 1) & 1, wc)) break;
+        if (c >= 2) {
+          if (!mbar_wait(&img_ready[ks], ((c >> 1) - 1) & 1, wc)) break;
+          store_img(c - 2);
+          stored = c - 1;
+          bulk_wait_read_all();   // the slot's image is read out: it may take the next keys
+        }
         mbar_arrive_expect_tx(&k_full[ks], L::KV);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
@@ -492,6 +504,12 @@ __global__ void __launch_bounds__(kSegThreads, 2)
           tma_load_3d(smem + L::V0 + vs * L::KV + kb * C * 128, &tmv, &v_full[vs], kb * 64, kv, t);
         v_issued = c + 1;
       }
+      // the images of the last steps
+      for (int c = stored; c < k_issued; ++c) {
+        if (!mbar_wait(&img_ready[c & 1], (c >> 1) & 1, wc)) break;
+        store_img(c);
+      }
+      bulk_wait_all();   // the images are in the workspace before the CTA ends
       // never leave the CTA with copies in flight
       const WaitCtx dw{never, nullptr, p.wait_ns};
       for (int c = (k_issued > 2 ? k_issued - 2 : 0); c < k_issued; ++c) mbar_wait(&k_full[c & 1], (c >> 1) & 1, dw);
@@ -537,17 +555,20 @@ __global__ void __launch_bounds__(kSegThreads, 2)
       mbar_wait(&k_full[slot], (c >> 1) & 1, wc);
       GateSums gs;
       uint32_t ek[D / 8];
+      // (key_features ends with a barrier of the group after its last read of the raw keys)
       const float iz = key_features<D, 4>(smem + L::K0 + slot * L::KV, nullptr, lg, nullptr, r, nv, gs, ek);
-      mbar_arrive(&k_empty[slot]);   // this thread is done with the raw keys
       const float bC = gs.at(nv - 1);
       const float bj = gs.at(r >> 2);
       const bool live = (r >> 2) < nv;
       // The chunk pass's key tile for this chunk (written once, read by its q-head
-      // pairs): factored at the chunk end when the chunk's decay allows, else phi(k).
+      // pairs): factored at the chunk end when the chunk's decay allows, else phi(k).  It
+      // goes over the raw keys in shared memory, and the TMA warp stores it in one bulk copy.
       {
         const size_t ci = (size_t)(seg * p.L + sub * p.Ls + cc) * p.Hkv + kv;
         const float sc = live ? (bC >= kFactorFloor ? __expf(bC - bj) * iz : iz) : 0.f;
-        write_ktilde<D, 4>(ek, p.kimg + ci * L::KV, r, sc);
+        write_ktilde<D, 4>(ek, smem + L::K0 + slot * L::KV, r, sc);
+        fence_proxy_async_smem();
+        mbar_arrive(&img_ready[slot]);
         if (r < 32) {
           p.bimg[ci * C + 2 * r] = gs.b0;
           p.bimg[ci * C + 2 * r + 1] = gs.b1;
