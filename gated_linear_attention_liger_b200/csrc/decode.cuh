@@ -113,20 +113,24 @@ template <> __device__ __forceinline__ void ld16_vals<float>(const float* p, flo
 }
 
 // Window scores q_h . k_j / sqrt(d) of NH heads for the w slots, four threads per
-// slot; thread quarter qq takes the 16-byte pieces qq, qq+4, ... of the row
-// (conflict-free on the padded rows), loads each key piece once for all heads and
-// reduces with two shuffles.  qv[h] is head h's query row (fp32, 16-byte aligned).
-// Needs blockDim >= 4 * w.
-template <typename Tin, int D, int NH>
+// slot; thread quarter qq takes the 16-byte pieces qq, qq+4, ... of the row, loads
+// each key piece once for all heads and reduces with two shuffles.  qv[h] is head
+// h's query row (fp32, 16-byte aligned).  Window position jj sits in shared-memory
+// row (row0 + jj) mod wrap of stride RS elements (on unpadded rows the two rows of
+// a quarter-warp share banks, a two-way conflict on the key loads only; the query
+// loads, eight times as many, stay one wavefront each).  Needs blockDim >= 4 * w.
+template <typename Tin, int D, int NH, int RS = ring_row_elems<Tin, D>()>
 __device__ __forceinline__ void window_scores(const float (*qv)[D], const float* ks, const Tin* rk_s,
-                                              float (*sc)[64], int p, int w, int tid) {
+                                              float (*sc)[64], int p, int w, int tid, int row0 = 0,
+                                              int wrap = 64) {
   constexpr int EPP = 16 / (int)sizeof(Tin);      // elements per 16-byte piece
   constexpr int NP = D / EPP;                     // pieces per row
-  constexpr int RS = ring_row_elems<Tin, D>();
   const int jj = tid >> 2, qq = tid & 3;
   if (jj < 64) {   // all four lanes of a slot take part in the shuffles
     const int j = p - (w - 1) + jj;
     const bool live = jj < w && j >= 0;
+    int row = row0 + jj;
+    row = row >= wrap ? row - wrap : row;
     float2 acc[NH];   // two partial sums (packed multiply-adds)
 #pragma unroll
     for (int h = 0; h < NH; ++h) acc[h] = make_float2(0.f, 0.f);
@@ -141,7 +145,7 @@ __device__ __forceinline__ void window_scores(const float (*qv)[D], const float*
             x[e] = t.x; x[e + 1] = t.y; x[e + 2] = t.z; x[e + 3] = t.w;
           }
         } else {
-          ld16_vals<Tin>(rk_s + jj * RS + pc * EPP, x);
+          ld16_vals<Tin>(rk_s + row * RS + pc * EPP, x);
         }
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
@@ -164,14 +168,31 @@ __device__ __forceinline__ void window_scores(const float (*qv)[D], const float*
   }
 }
 
+// Window softmax of head h = warp (warps 0 .. NH-1): the scores sc[h][0..w) (-inf for
+// positions before the sequence start) become probabilities in place.
+template <int NH>
+__device__ __forceinline__ void window_probs(float (*sc)[64], int w, int warp, int lane) {
+  if (warp < NH) {
+    const float x0 = lane < w ? sc[warp][lane] : -INFINITY;
+    const float x1 = lane + 32 < w ? sc[warp][lane + 32] : -INFINITY;
+    const float m = warp_max(fmaxf(x0, x1));   // finite: the current position is always live
+    const float e0 = lane < w ? expf(x0 - m) : 0.f;
+    const float e1 = lane + 32 < w ? expf(x1 - m) : 0.f;
+    const float iz = 1.0f / warp_sum(e0 + e1);
+    if (lane < w) sc[warp][lane] = e0 * iz;
+    if (lane + 32 < w) sc[warp][lane + 32] = e1 * iz;
+  }
+}
+
 // Window softmax and value sums for NH heads.  sc[h][0..w) holds the scores (-inf
 // for positions before the sequence start).  Every warp reduces the maxima and sums
 // itself (no single-warp phase, no extra barrier).  Thread layout: 16-byte column
 // piece cp = tid % NPC, slot group sg = tid / NPC, slots sg, sg + NSG, ...; each thread
 // accumulates p_h(slot) v(slot) over its pieces, the slot groups of a warp are added
 // with shuffles, and each warp writes wsum[warp][h][...]; the caller adds the NW
-// partial sums.
-template <typename Tin, int D, int NT, int NH>
+// partial sums.  Window position jj sits in row (row0 + jj) mod wrap of stride RS.
+// With PROBS, sc already holds the probabilities (window_probs).
+template <typename Tin, int D, int NT, int NH, int RS = ring_row_elems<Tin, D>(), bool PROBS = false>
 struct WindowValues {
   static constexpr int EPP = 16 / (int)sizeof(Tin);   // elements per 16-byte piece
   static constexpr int NPC = D / EPP;                 // pieces per row
@@ -179,10 +200,11 @@ struct WindowValues {
   static constexpr int NSG = NT / NPC;                // slot groups
   static constexpr int NW = NT / 32;                  // warps (partial sums)
   __device__ __forceinline__ static void run(const float (*sc)[64], const Tin* rv_s, const float* vs,
-                                             float (*wsum)[NH][D], int p, int w, int tid, int lane) {
-    float mh[NH], izh[NH];
+                                             float (*wsum)[NH][D], int p, int w, int tid, int lane,
+                                             int row0 = 0, int wrap = 64) {
+    float mh[NH], izh[NH];   // unused when sc already holds probabilities (PROBS)
 #pragma unroll
-    for (int h = 0; h < NH; ++h) {
+    for (int h = 0; h < NH && !PROBS; ++h) {
       const float x0 = lane < w ? sc[h][lane] : -INFINITY;
       const float x1 = lane + 32 < w ? sc[h][lane + 32] : -INFINITY;
       const float m = warp_max(fmaxf(x0, x1));
@@ -190,26 +212,29 @@ struct WindowValues {
       mh[h] = m;
       izh[h] = 1.0f / z;
     }
-    constexpr int RS = ring_row_elems<Tin, D>();
     const int cp = tid % NPC, sg = tid / NPC;
     float2 acc[NH][EPP / 2];   // element pairs (packed multiply-adds)
 #pragma unroll
     for (int h = 0; h < NH; ++h)
 #pragma unroll
       for (int e = 0; e < EPP / 2; ++e) acc[h][e] = make_float2(0.f, 0.f);
-    for (int jj = sg; jj < w; jj += NSG) {
+#pragma unroll
+    for (int it = 0; it < (64 + NSG - 1) / NSG; ++it) {
+      const int jj = sg + it * NSG;
       const int j = p - (w - 1) + jj;
-      if (j < 0) continue;
+      if (jj >= w || j < 0) continue;
       float x[EPP];
       if (j == p) {
 #pragma unroll
         for (int e = 0; e < EPP; ++e) x[e] = vs[cp * EPP + e];
       } else {
-        ld16_vals<Tin>(rv_s + jj * RS + cp * EPP, x);
+        int row = row0 + jj;
+        row = row >= wrap ? row - wrap : row;
+        ld16_vals<Tin>(rv_s + row * RS + cp * EPP, x);
       }
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        const float ph = expf(sc[h][jj] - mh[h]) * izh[h];
+        const float ph = PROBS ? sc[h][jj] : expf(sc[h][jj] - mh[h]) * izh[h];
         const float2 ph2 = make_float2(ph, ph);
 #pragma unroll
         for (int e = 0; e < EPP / 2; ++e) acc[h][e] = ffma2(ph2, make_float2(x[2 * e], x[2 * e + 1]), acc[h][e]);
@@ -507,4 +532,293 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
   }
 }
 
+}  // namespace liger
+
+namespace liger {
+namespace kvs {
+
+// Shared-state decode as a persistent stream.  One CTA per SM walks the
+// (sequence, kv head) units blockIdx.x, blockIdx.x + gridDim.x, ...  A producer
+// warp moves each unit's fp32 state, its window ring (keys, then values, w slots
+// each, in slot order) and the step's rows q_h (G of them), k and v into one of
+// two shared-memory stages by bulk copies, so that the next unit's bytes are in
+// flight while eight consumer warps compute this one.  The updated state goes
+// back to HBM by bulk copies as soon as the consumers have written it, before
+// they run the window branch.  Every wait is bounded; a wait that gives up
+// records the timeout in the device error word and the CTA winds down with no
+// copy in flight.
+
+constexpr int kConsumers = 256;               // eight consumer warps
+constexpr int kThreads = kConsumers + 32;     // and the producer warp
+constexpr int kStages = 2;
+
+template <typename Tin, int D, int G>
+struct Layout {
+  static constexpr uint32_t STATE = D * D * 4;
+  static constexpr uint32_t RING = 2 * 64 * D * sizeof(Tin);    // room for w = 64
+  static constexpr uint32_t QKV = (G + 2) * D * sizeof(Tin);     // q_0 .. q_{G-1}, k, v
+  static constexpr uint32_t STAGE = STATE + RING + QKV;
+  static constexpr int CQ = D / 4;                  // column quads
+  static constexpr int RGN = kConsumers / CQ;       // row groups
+  static constexpr int RPT = D / RGN;               // rows per thread
+  using WV = WindowValues<Tin, D, kConsumers, G, D, true>;
+  static constexpr uint32_t PART = RGN * G * D * 4;              // readout partial sums
+  static constexpr uint32_t WSUM = WV::NW * G * D * 4;           // window partial sums (same room)
+  static constexpr uint32_t SCRATCH = PART > WSUM ? PART : WSUM;
+  static constexpr uint32_t OFF_SCRATCH = kStages * STAGE;
+  static constexpr uint32_t OFF_FQ = OFF_SCRATCH + SCRATCH;      // [G][D] phi(q_h)
+  static constexpr uint32_t OFF_QF = OFF_FQ + G * D * 4;         // [G][D] q_h in fp32
+  static constexpr uint32_t OFF_GRM = OFF_QF + G * D * 4;        // [G][D] recurrent readout
+  static constexpr uint32_t OFF_FK = OFF_GRM + G * D * 4;        // [D] phi(k)
+  static constexpr uint32_t OFF_KS = OFF_FK + D * 4;             // [D] k in fp32
+  static constexpr uint32_t OFF_VS = OFF_KS + D * 4;             // [D] v in fp32
+  static constexpr uint32_t OFF_SC = OFF_VS + D * 4;             // [G][64] window scores
+  static constexpr uint32_t OFF_MISC = OFF_SC + G * 64 * 4;      // barriers, gate, positions, abort
+  static constexpr uint32_t BYTES = OFF_MISC + 128;
+  static_assert(STAGE % 16 == 0 && STATE % 4096 == 0, "bulk copies need 16-byte sizes");
+  static_assert(RGN * RPT == D && RPT >= 1, "row split");
+};
+
+// Whether the two stages fit one CTA's shared memory (fp32 rows at d = 128 do not).
+template <typename Tin, int D, int G>
+constexpr bool fits() {
+  return Layout<Tin, D, G>::BYTES <= 227u * 1024u;
+}
+
+struct Args {
+  DecodeArgs d;
+  int units;           // B * Hkv
+  uint32_t* err;       // device error word (timeouts)
+  uint64_t wait_ns;    // give-up time of each wait
+};
+
+template <typename Tin, int D, int G>
+__global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Args c) {
+  using L = Layout<Tin, D, G>;
+  using sm100::mbar_wait;
+  extern __shared__ __align__(128) unsigned char sm[];
+  float* fq = reinterpret_cast<float*>(sm + L::OFF_FQ);
+  float* qf = reinterpret_cast<float*>(sm + L::OFF_QF);
+  float* grm = reinterpret_cast<float*>(sm + L::OFF_GRM);
+  float* fk = reinterpret_cast<float*>(sm + L::OFF_FK);
+  float* ks = reinterpret_cast<float*>(sm + L::OFF_KS);
+  float* vs = reinterpret_cast<float*>(sm + L::OFF_VS);
+  float(*sc)[64] = reinterpret_cast<float(*)[64]>(sm + L::OFF_SC);
+  float(*part)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
+  float(*wsum)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::OFF_MISC);   // [2] stage loaded
+  uint64_t* sdone = full + 2;                                        // [2] state updated in place
+  uint64_t* cons = full + 4;                                         // [2] stage no longer read
+  float* gsh = reinterpret_cast<float*>(full + 6);
+  int* pos_s = reinterpret_cast<int*>(gsh + 1);                      // [2]
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(pos_s + 2);
+
+  const DecodeArgs& a = c.d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hkv = a.Hkv, Hq = a.Hq, w = a.w;
+  const uint32_t ring_bytes = 2u * (uint32_t)w * D * sizeof(Tin);
+  auto stage = [&](int s) { return sm + (size_t)s * L::STAGE; };
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&sdone[s], kConsumers);
+      sm100::mbar_init(&cons[s], kConsumers);
+    }
+    *abort_flag = 0u;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_launch_dependents();
+  const sm100::WaitCtx wc{abort_flag, c.err, c.wait_ns};
+  const int n_local = c.units > (int)blockIdx.x ? (c.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == kConsumers / 32) {
+    // ---------------------------------------------------------------- producer
+    if (lane != 0) return;
+    auto issue = [&](int i) {
+      const int s = i % kStages;
+      const long u = (long)blockIdx.x + (long)i * gridDim.x;
+      const long b = u / Hkv, kv = u % Hkv;
+      unsigned char* st = stage(s);
+      pos_s[s] = max(a.pos[b], 0);   // a negative position is read as 0
+      sm100::mbar_arrive_expect_tx(&full[s], L::STATE + ring_bytes + L::QKV);
+      const float* S = a.state + (size_t)u * D * D;
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece)
+        sm100::bulk_load(st + piece * (L::STATE / 4), S + piece * (D * D / 4), L::STATE / 4, &full[s]);
+      sm100::bulk_load(st + L::STATE, static_cast<const Tin*>(a.ring) + (size_t)u * 2 * w * D, ring_bytes,
+                       &full[s]);
+      unsigned char* qkv = st + L::STATE + L::RING;
+      sm100::bulk_load(qkv, static_cast<const Tin*>(a.q) + ((size_t)b * Hq + kv * G) * D, G * D * sizeof(Tin),
+                       &full[s]);
+      sm100::bulk_load(qkv + G * D * sizeof(Tin), static_cast<const Tin*>(a.k) + (size_t)u * D, D * sizeof(Tin),
+                       &full[s]);
+      sm100::bulk_load(qkv + (G + 1) * D * sizeof(Tin), static_cast<const Tin*>(a.v) + (size_t)u * D,
+                       D * sizeof(Tin), &full[s]);
+    };
+    int issued = 0;
+    for (; issued < kStages && issued < n_local; ++issued) issue(issued);
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i % kStages;
+      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+      if (!mbar_wait(&sdone[s], ph, wc, sm100::wsite(7, 1, i))) break;
+      const long u = (long)blockIdx.x + (long)i * gridDim.x;
+      float* S = a.state + (size_t)u * D * D;
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece)
+        sm100::bulk_store(S + piece * (D * D / 4), stage(s) + piece * (L::STATE / 4), L::STATE / 4);
+      sm100::bulk_commit();
+      if (i + kStages < n_local) {
+        if (!mbar_wait(&cons[s], ph, wc, sm100::wsite(7, 2, i))) break;
+        sm100::bulk_wait_read_all();   // this unit's state has left the stage
+        issue(issued++);
+      }
+    }
+    // never leave with copies in flight: the last load of each stage, then the stores
+    volatile uint32_t never = 0u;
+    const sm100::WaitCtx drain{&never, nullptr, c.wait_ns};
+    for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+      mbar_wait(&full[i % kStages], (uint32_t)(i / kStages) & 1u, drain);
+    sm100::bulk_wait_all();
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int cq = tid % L::CQ, rg = tid / L::CQ;
+  for (int i = 0; i < n_local; ++i) {
+    const int s = i % kStages;
+    const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+    const bool ok = mbar_wait(&full[s], ph, wc, sm100::wsite(6, 1, i));
+    if (sm100::named_bar_or(1, kConsumers, !ok)) break;
+    const long u = (long)blockIdx.x + (long)i * gridDim.x;
+    const long b = u / Hkv, kv = u % Hkv;
+    unsigned char* st = stage(s);
+    float* Ss = reinterpret_cast<float*>(st);
+    const Tin* rk = reinterpret_cast<const Tin*>(st + L::STATE);
+    const Tin* rv = rk + (size_t)w * D;
+    const Tin* qin = reinterpret_cast<const Tin*>(st + L::STATE + L::RING);
+    const Tin* kin = qin + G * D;
+    const Tin* vin = kin + D;
+    const int p = pos_s[s];
+
+    // phi(k) and the gate (warp 0), phi(q_h) (warps 1..G), fp32 copies of q, k, v (the rest)
+    constexpr int EPL = D / 32;
+    if (warp == 0) {
+      float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = io<Tin>::ld(kin + lane + 32 * j); m = fmaxf(m, x[j]); sum += x[j]; }
+      m = warp_max(m);
+      sum = warp_sum(sum);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
+      z = warp_sum(z);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) fk[lane + 32 * j] = x[j] / z;
+      if (lane == 0) *gsh = expf(log_sigmoid(sum / (float)D));
+    } else if (warp <= G) {
+      const int hh = warp - 1;
+      float x[EPL], m = -INFINITY, z = 0.f;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = io<Tin>::ld(qin + hh * D + lane + 32 * j); m = fmaxf(m, x[j]); }
+      m = warp_max(m);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
+      z = warp_sum(z);
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) fq[hh * D + lane + 32 * j] = x[j] / z;
+    } else {
+      constexpr int first = 32 * (G + 1), nconv = kConsumers - first;
+      for (int idx = tid - first; idx < (G + 2) * D; idx += nconv) {
+        const float x = io<Tin>::ld(qin + idx);   // q rows, then k, then v
+        if (idx < G * D) qf[idx] = x;
+        else if (idx < (G + 1) * D) ks[idx - G * D] = x;
+        else vs[idx - (G + 1) * D] = x;
+      }
+    }
+    sm100::named_bar(1, kConsumers);
+
+    // state update in place, readout for every head of the group; the producer sends
+    // the state back as soon as every consumer has written its rows
+    {
+      const float g = *gsh;
+      const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
+      const float2 g2 = make_float2(g, g), v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
+      float2 a01[G], a23[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) a01[hh] = a23[hh] = make_float2(0.f, 0.f);
+      static_assert(L::RPT % 4 == 0, "rows in quads");
+#pragma unroll
+      for (int r4 = 0; r4 < L::RPT; r4 += 4) {
+        const int row4 = rg * L::RPT + r4;
+        const float4 k4 = *reinterpret_cast<const float4*>(fk + row4);   // phi(k) of four rows
+        float4 q4[G];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) q4[hh] = *reinterpret_cast<const float4*>(fq + hh * D + row4);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float4* sp = reinterpret_cast<float4*>(Ss + (size_t)(row4 + r) * D + 4 * cq);
+          const float4 sv = *sp;
+          const float kr = r == 0 ? k4.x : r == 1 ? k4.y : r == 2 ? k4.z : k4.w;
+          const float2 k2 = make_float2(kr, kr);
+          const float2 x01 = ffma2(g2, make_float2(sv.x, sv.y), fmul2(k2, v01));
+          const float2 x23 = ffma2(g2, make_float2(sv.z, sv.w), fmul2(k2, v23));
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float qr = r == 0 ? q4[hh].x : r == 1 ? q4[hh].y : r == 2 ? q4[hh].z : q4[hh].w;
+            const float2 q2 = make_float2(qr, qr);
+            a01[hh] = ffma2(q2, x01, a01[hh]);
+            a23[hh] = ffma2(q2, x23, a23[hh]);
+          }
+          *sp = make_float4(x01.x, x01.y, x23.x, x23.y);
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+        *reinterpret_cast<float4*>(&part[rg][hh][4 * cq]) = make_float4(a01[hh].x, a01[hh].y, a23[hh].x, a23[hh].y);
+    }
+    sm100::fence_proxy_async_smem();   // the rows written above are read by the bulk copy out
+    sm100::mbar_arrive(&sdone[s]);
+    sm100::named_bar(1, kConsumers);
+
+    // window scores on the ring in slot order (window position jj is slot (p+1+jj) mod w)
+    const int row0 = (p + 1) % w;
+    window_scores<Tin, D, G, D>(reinterpret_cast<const float(*)[D]>(qf), ks, rk, sc, p, w, tid, row0, w);
+    sm100::named_bar(1, kConsumers);
+    // window softmax, one warp per head; the other warps add up the readout partial sums
+    if (warp < G) {
+      window_probs<G>(sc, w, warp, lane);
+    } else {
+      for (int idx = tid - 32 * G; idx < G * D; idx += kConsumers - 32 * G) {
+        float t = 0.f;
+#pragma unroll
+        for (int r = 0; r < L::RGN; ++r) t += part[r][idx / D][idx % D];
+        grm[idx] = t;
+      }
+    }
+    sm100::named_bar(1, kConsumers);
+    L::WV::run(sc, rv, vs, wsum, p, w, tid, lane, row0, w);   // window value sums
+    sm100::named_bar(1, kConsumers);
+    for (int idx = tid; idx < G * D; idx += kConsumers) {
+      const int hh = idx / D, e = idx % D;
+      float swa = 0.f;
+#pragma unroll
+      for (int r = 0; r < L::WV::NW; ++r) swa += wsum[r][hh][e];
+      Tin* orow = static_cast<Tin*>(a.out) + ((size_t)b * Hq + kv * G + hh) * D;
+      io<Tin>::st(orow + e, a.alpha * grm[idx] + (1.0f - a.alpha) * swa);
+    }
+    // the step's key and value replace the oldest slot of this unit's ring
+    constexpr int PC = D * (int)sizeof(Tin) / 16;   // 16-byte pieces per row
+    if (tid < 2 * PC) {
+      const int which = tid / PC, piece = tid % PC;
+      Tin* dst = static_cast<Tin*>(a.ring) + ((size_t)u * 2 + which) * w * D + (size_t)(p % w) * D;
+      const Tin* src = which ? vin : kin;
+      reinterpret_cast<uint4*>(dst)[piece] = reinterpret_cast<const uint4*>(src)[piece];
+    }
+    sm100::mbar_arrive(&cons[s]);
+  }
+}
+
+}  // namespace kvs
 }  // namespace liger

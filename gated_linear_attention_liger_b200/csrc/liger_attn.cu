@@ -198,8 +198,31 @@ liger_status launch_decode(const liger::DecodeArgs& a, unsigned blocks, cudaStre
   return cuda_check("decode launch");
 }
 
+// Error word of the streamed shared-state decode (bit 0: a bounded wait gave up;
+// word 1: the first site), one per device; read and cleared by
+// liger_attn_decode_kvshared_status().
+__device__ uint32_t g_decode_err[2];
+
 template <typename Tin, int D, int G>
 liger_status launch_decode_kvshared(const liger::DecodeArgs& a, unsigned blocks, cudaStream_t s) {
+  if constexpr (liger::kvs::fits<Tin, D, G>()) {   // the persistent two-stage stream
+    constexpr size_t smem = liger::kvs::Layout<Tin, D, G>::BYTES;
+    auto kern = liger::kvs::decode_kvshared_stream_kernel<Tin, D, G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return cuda_check("cudaFuncSetAttribute(decode_kvshared_stream)");
+    void* err = nullptr;
+    const cudaError_t ge = cudaGetSymbolAddress(&err, g_decode_err);
+    if (ge != cudaSuccess) return fail(LIGER_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(ge));
+    liger::kvs::Args c{a, (int)blocks, static_cast<uint32_t*>(err), liger::tc::wait_limit_ns()};
+    const int sms = liger::tc::num_sms();
+    const unsigned grid = blocks < (unsigned)sms ? blocks : (unsigned)sms;   // one CTA per SM
+    mark_start(s);
+    if (launch_pdl(kern, dim3(grid), dim3(liger::kvs::kThreads), smem, s, c) != cudaSuccess)
+      return cuda_check("decode_kvshared_stream launch");
+    mark_stop(s);
+    ++g_launches;
+    return cuda_check("decode_kvshared_stream launch");
+  }
   constexpr size_t smem = liger::decode_smem_bytes<Tin, D>();
   auto kern = liger::decode_kvshared_kernel<Tin, D, G>;
   // static + dynamic shared memory can exceed the default 48 KiB: always raise the limit
@@ -646,6 +669,20 @@ liger_status liger_attn_full_causal(const void* q, const void* k, const void* v,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_full_attn<64>(mq, mk, mv, prm, Hq, n_seqs, s)
                  : launch_full_attn<128>(mq, mk, mv, prm, Hq, n_seqs, s);
+}
+
+liger_status liger_attn_decode_kvshared_status(void) {
+  g_last_error.clear();
+  uint32_t hdr[2] = {0u, 0u};
+  cudaError_t e = cudaMemcpyFromSymbol(hdr, g_decode_err, sizeof hdr);
+  if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "reading the decode's error word: %s", cudaGetErrorString(e));
+  const uint32_t zero[2] = {0u, 0u};
+  e = cudaMemcpyToSymbol(g_decode_err, zero, sizeof zero);
+  if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "clearing the decode's error word: %s", cudaGetErrorString(e));
+  if (hdr[0] & 1u)
+    return fail(LIGER_ERR_TIMEOUT, "a shared-state decode kernel gave up waiting (site 0x%08x: role %u, barrier %u, unit %u)",
+                hdr[1], hdr[1] >> 28, (hdr[1] >> 20) & 0xFFu, hdr[1] & 0xFFFFFu);
+  return LIGER_OK;
 }
 
 liger_status liger_attn_full_causal_status(void) {

@@ -53,6 +53,7 @@ SIGNATURES = {
                                            _i, _vp]),
     "liger_attn_full_causal": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp]),
     "liger_attn_full_causal_status": (_i, []),
+    "liger_attn_decode_kvshared_status": (_i, []),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }
@@ -304,6 +305,11 @@ def full_causal_attention(q, k, v, cu_seqlens=None, max_seqlen=None, out=None, s
 def full_causal_status() -> int:
     """LIGER_OK, or LIGER_ERR_TIMEOUT if a causal attention call gave up waiting since the last query."""
     return int(load().liger_attn_full_causal_status())
+
+
+def decode_kvshared_status() -> int:
+    """LIGER_OK, or LIGER_ERR_TIMEOUT if a shared-state decode gave up waiting since the last query."""
+    return int(load().liger_attn_decode_kvshared_status())
 
 
 def prefill_backward_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:

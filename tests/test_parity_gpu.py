@@ -293,8 +293,12 @@ def test_full_llama8b_decode(cuda_device):
     (torch.bfloat16, 64, 64, 0, 2, 3),
     (torch.bfloat16, 64, 16, 5, 1, 3),
     (torch.float32, 128, 64, 100, 4, 3),
-    # more (sequence, kv head) units than SMs
+    # more (sequence, kv head) units than SMs: each CTA of the streamed kernel takes
+    # several units and reuses its two stages
     (torch.bfloat16, 64, 64, 30, 4, 170),
+    # ring wrapped (prefix longer than the window), w < 64, several units per CTA
+    (torch.bfloat16, 128, 32, 50, 2, 160),
+    (torch.float32, 64, 48, 60, 4, 90),
 ])
 def test_decode_kvshared_parity(dtype, d, w, T0, G, B, cuda_device):
     """One state per kv head: the oracle runs with that state copied to every q head of
@@ -324,6 +328,7 @@ def test_decode_kvshared_parity(dtype, d, w, T0, G, B, cuda_device):
     assert_close(np64(g_state), st[:, ::G], dtype, "kv-shared state")
     np.testing.assert_array_equal(np64(g_ring), rg)
     np.testing.assert_array_equal(g_pos.cpu().numpy(), ps)
+    assert ops.decode_kvshared_status() == ops.LIGER_OK
 
 
 def test_decode_kvshared_matches_per_head_decode_full_shape(cuda_device):
