@@ -537,11 +537,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_kvshared_kernel(Deco
 namespace liger {
 namespace kvs {
 
-// Shared-state decode as a persistent stream.  One CTA per SM walks the
-// (sequence, kv head) units blockIdx.x, blockIdx.x + gridDim.x, ...  A producer
-// warp moves each unit's fp32 state, its window ring (keys, then values, w slots
-// each, in slot order) and the step's rows q_h (G of them), k and v into one of
-// two shared-memory stages by bulk copies, so that the next unit's bytes are in
+// Decode as a persistent stream.  One CTA per SM walks the units blockIdx.x,
+// blockIdx.x + gridDim.x, ...: (sequence, kv head) with one state read out by the
+// group's G heads (NH = G), or (sequence, q head) with a state per head (NH = 1,
+// PER_HEAD; the group's heads read the same window ring, and the group's first
+// head writes the step's key and value into it).  A producer warp moves each
+// unit's fp32 state, its window ring (keys, then values, w slots each, in slot
+// order) and the step's rows q_h (NH of them), k and v into one of two
+// shared-memory stages by bulk copies, so that the next unit's bytes are in
 // flight while eight consumer warps compute this one.  The updated state goes
 // back to HBM by bulk copies as soon as the consumers have written it, before
 // they run the window branch.  Every wait is bounded; a wait that gives up
@@ -552,7 +555,7 @@ constexpr int kConsumers = 256;               // eight consumer warps
 constexpr int kThreads = kConsumers + 32;     // and the producer warp
 constexpr int kStages = 2;
 
-template <typename Tin, int D, int G>
+template <typename Tin, int D, int G>   // G: heads read out per unit
 struct Layout {
   static constexpr uint32_t STATE = D * D * 4;
   static constexpr uint32_t RING = 2 * 64 * D * sizeof(Tin);    // room for w = 64
@@ -572,7 +575,8 @@ struct Layout {
   static constexpr uint32_t OFF_FK = OFF_GRM + G * D * 4;        // [D] phi(k)
   static constexpr uint32_t OFF_KS = OFF_FK + D * 4;             // [D] k in fp32
   static constexpr uint32_t OFF_VS = OFF_KS + D * 4;             // [D] v in fp32
-  static constexpr uint32_t OFF_SC = OFF_VS + D * 4;             // [G][64] window scores
+  static constexpr uint32_t OFF_GV = OFF_VS + D * 4;             // [D] per-row gates (vector gate)
+  static constexpr uint32_t OFF_SC = OFF_GV + D * 4;             // [G][64] window scores
   static constexpr uint32_t OFF_MISC = OFF_SC + G * 64 * 4;      // barriers, gate, positions, abort
   static constexpr uint32_t BYTES = OFF_MISC + 128;
   static_assert(STAGE % 16 == 0 && STATE % 4096 == 0, "bulk copies need 16-byte sizes");
@@ -587,13 +591,41 @@ constexpr bool fits() {
 
 struct Args {
   DecodeArgs d;
-  int units;           // B * Hkv
+  int units;           // B * Hkv, or B * Hq per head
   uint32_t* err;       // device error word (timeouts)
   uint64_t wait_ns;    // give-up time of each wait
 };
 
-template <typename Tin, int D, int G>
-__global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Args c) {
+// Offsets (in elements) of one unit's rows.
+struct UnitRows {
+  size_t state, ring, q, kv;   // q: the first of the unit's q rows (also its first out row)
+  bool writes_ring;
+};
+template <int G, bool PER_HEAD>
+__device__ __forceinline__ UnitRows unit_rows(long u, int Hq, int Hkv, int D, int w) {
+  UnitRows r;
+  if (PER_HEAD) {
+    const long b = u / Hq, h = u % Hq, grp = Hq / Hkv;
+    const long kvi = b * Hkv + h / grp;
+    r.state = (size_t)u * D * D;
+    r.ring = (size_t)kvi * 2 * w * D;
+    r.q = (size_t)u * D;
+    r.kv = (size_t)kvi * D;
+    r.writes_ring = h % grp == 0;
+  } else {
+    const long b = u / Hkv, kv = u % Hkv;
+    r.state = (size_t)u * D * D;
+    r.ring = (size_t)u * 2 * w * D;
+    r.q = ((size_t)b * Hq + kv * G) * D;
+    r.kv = (size_t)u * D;
+    r.writes_ring = true;
+  }
+  return r;
+}
+
+template <typename Tin, int D, int G, bool PER_HEAD>
+__global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
+  static_assert(!PER_HEAD || G == 1, "a per-head unit reads out one head");
   using L = Layout<Tin, D, G>;
   using sm100::mbar_wait;
   extern __shared__ __align__(128) unsigned char sm[];
@@ -603,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
   float* fk = reinterpret_cast<float*>(sm + L::OFF_FK);
   float* ks = reinterpret_cast<float*>(sm + L::OFF_KS);
   float* vs = reinterpret_cast<float*>(sm + L::OFF_VS);
+  float* gv = reinterpret_cast<float*>(sm + L::OFF_GV);
   float(*sc)[64] = reinterpret_cast<float(*)[64]>(sm + L::OFF_SC);
   float(*part)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
   float(*wsum)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
@@ -640,23 +673,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
     auto issue = [&](int i) {
       const int s = i % kStages;
       const long u = (long)blockIdx.x + (long)i * gridDim.x;
-      const long b = u / Hkv, kv = u % Hkv;
+      const UnitRows r = unit_rows<G, PER_HEAD>(u, Hq, Hkv, D, w);
       unsigned char* st = stage(s);
-      pos_s[s] = max(a.pos[b], 0);   // a negative position is read as 0
+      pos_s[s] = max(a.pos[u / (PER_HEAD ? Hq : Hkv)], 0);   // a negative position is read as 0
       sm100::mbar_arrive_expect_tx(&full[s], L::STATE + ring_bytes + L::QKV);
-      const float* S = a.state + (size_t)u * D * D;
+      const float* S = a.state + r.state;
 #pragma unroll
       for (int piece = 0; piece < 4; ++piece)
         sm100::bulk_load(st + piece * (L::STATE / 4), S + piece * (D * D / 4), L::STATE / 4, &full[s]);
-      sm100::bulk_load(st + L::STATE, static_cast<const Tin*>(a.ring) + (size_t)u * 2 * w * D, ring_bytes,
-                       &full[s]);
+      sm100::bulk_load(st + L::STATE, static_cast<const Tin*>(a.ring) + r.ring, ring_bytes, &full[s]);
       unsigned char* qkv = st + L::STATE + L::RING;
-      sm100::bulk_load(qkv, static_cast<const Tin*>(a.q) + ((size_t)b * Hq + kv * G) * D, G * D * sizeof(Tin),
+      sm100::bulk_load(qkv, static_cast<const Tin*>(a.q) + r.q, G * D * sizeof(Tin), &full[s]);
+      sm100::bulk_load(qkv + G * D * sizeof(Tin), static_cast<const Tin*>(a.k) + r.kv, D * sizeof(Tin), &full[s]);
+      sm100::bulk_load(qkv + (G + 1) * D * sizeof(Tin), static_cast<const Tin*>(a.v) + r.kv, D * sizeof(Tin),
                        &full[s]);
-      sm100::bulk_load(qkv + G * D * sizeof(Tin), static_cast<const Tin*>(a.k) + (size_t)u * D, D * sizeof(Tin),
-                       &full[s]);
-      sm100::bulk_load(qkv + (G + 1) * D * sizeof(Tin), static_cast<const Tin*>(a.v) + (size_t)u * D,
-                       D * sizeof(Tin), &full[s]);
     };
     int issued = 0;
     for (; issued < kStages && issued < n_local; ++issued) issue(issued);
@@ -693,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
     const bool ok = mbar_wait(&full[s], ph, wc, sm100::wsite(6, 1, i));
     if (sm100::named_bar_or(1, kConsumers, !ok)) break;
     const long u = (long)blockIdx.x + (long)i * gridDim.x;
-    const long b = u / Hkv, kv = u % Hkv;
+    const UnitRows ur = unit_rows<G, PER_HEAD>(u, Hq, Hkv, D, w);
     unsigned char* st = stage(s);
     float* Ss = reinterpret_cast<float*>(st);
     const Tin* rk = reinterpret_cast<const Tin*>(st + L::STATE);
@@ -717,6 +747,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
 #pragma unroll
       for (int j = 0; j < EPL; ++j) fk[lane + 32 * j] = x[j] / z;
       if (lane == 0) *gsh = expf(log_sigmoid(sum / (float)D));
+      if (PER_HEAD && a.vector_gate) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) gv[lane + 32 * j] = expf(log_sigmoid(io<Tin>::ld(kin + lane + 32 * j)));
+      }
     } else if (warp <= G) {
       const int hh = warp - 1;
       float x[EPL], m = -INFINITY, z = 0.f;
@@ -742,9 +776,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
     // state update in place, readout for every head of the group; the producer sends
     // the state back as soon as every consumer has written its rows
     {
+      const bool vgate = PER_HEAD && a.vector_gate;
       const float g = *gsh;
       const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
-      const float2 g2 = make_float2(g, g), v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
+      const float2 v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
       float2 a01[G], a23[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) a01[hh] = a23[hh] = make_float2(0.f, 0.f);
@@ -753,6 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
       for (int r4 = 0; r4 < L::RPT; r4 += 4) {
         const int row4 = rg * L::RPT + r4;
         const float4 k4 = *reinterpret_cast<const float4*>(fk + row4);   // phi(k) of four rows
+        const float4 g4 = vgate ? *reinterpret_cast<const float4*>(gv + row4) : make_float4(g, g, g, g);
         float4 q4[G];
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) q4[hh] = *reinterpret_cast<const float4*>(fq + hh * D + row4);
@@ -761,7 +797,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
           float4* sp = reinterpret_cast<float4*>(Ss + (size_t)(row4 + r) * D + 4 * cq);
           const float4 sv = *sp;
           const float kr = r == 0 ? k4.x : r == 1 ? k4.y : r == 2 ? k4.z : k4.w;
-          const float2 k2 = make_float2(kr, kr);
+          const float gr = r == 0 ? g4.x : r == 1 ? g4.y : r == 2 ? g4.z : g4.w;
+          const float2 k2 = make_float2(kr, kr), g2 = make_float2(gr, gr);
           const float2 x01 = ffma2(g2, make_float2(sv.x, sv.y), fmul2(k2, v01));
           const float2 x23 = ffma2(g2, make_float2(sv.z, sv.w), fmul2(k2, v23));
 #pragma unroll
@@ -805,14 +842,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kvshared_stream_kernel(Arg
       float swa = 0.f;
 #pragma unroll
       for (int r = 0; r < L::WV::NW; ++r) swa += wsum[r][hh][e];
-      Tin* orow = static_cast<Tin*>(a.out) + ((size_t)b * Hq + kv * G + hh) * D;
+      Tin* orow = static_cast<Tin*>(a.out) + ur.q + (size_t)hh * D;
       io<Tin>::st(orow + e, a.alpha * grm[idx] + (1.0f - a.alpha) * swa);
     }
-    // the step's key and value replace the oldest slot of this unit's ring
+    // the step's key and value replace the oldest slot of this unit's ring (no unit of
+    // the step reads that slot: it holds the position that just left every window)
     constexpr int PC = D * (int)sizeof(Tin) / 16;   // 16-byte pieces per row
-    if (tid < 2 * PC) {
+    if (ur.writes_ring && tid < 2 * PC) {
       const int which = tid / PC, piece = tid % PC;
-      Tin* dst = static_cast<Tin*>(a.ring) + ((size_t)u * 2 + which) * w * D + (size_t)(p % w) * D;
+      Tin* dst = static_cast<Tin*>(a.ring) + ur.ring + (size_t)which * w * D + (size_t)(p % w) * D;
       const Tin* src = which ? vin : kin;
       reinterpret_cast<uint4*>(dst)[piece] = reinterpret_cast<const uint4*>(src)[piece];
     }

@@ -183,8 +183,34 @@ liger_status launch_ring(const void* k, const void* v, void* ring, int32_t* pos,
   return cuda_check("prefill_ring launch");
 }
 
+// Error word of the streamed decode kernels (bit 0: a bounded wait gave up; word 1:
+// the first site), one per device; read and cleared by liger_attn_decode_status().
+__device__ uint32_t g_decode_err[2];
+
+// The persistent stream (one CTA per SM) over `units` units of G heads each.
+template <typename Tin, int D, int G, bool PER_HEAD>
+liger_status launch_decode_stream(const liger::DecodeArgs& a, unsigned units, cudaStream_t s) {
+  constexpr size_t smem = liger::kvs::Layout<Tin, D, G>::BYTES;
+  auto kern = liger::kvs::decode_stream_kernel<Tin, D, G, PER_HEAD>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return cuda_check("cudaFuncSetAttribute(decode_stream)");
+  void* err = nullptr;
+  const cudaError_t ge = cudaGetSymbolAddress(&err, g_decode_err);
+  if (ge != cudaSuccess) return fail(LIGER_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(ge));
+  liger::kvs::Args c{a, (int)units, static_cast<uint32_t*>(err), liger::tc::wait_limit_ns()};
+  const int sms = liger::tc::num_sms();
+  const unsigned grid = units < (unsigned)sms ? units : (unsigned)sms;   // one CTA per SM
+  mark_start(s);
+  if (launch_pdl(kern, dim3(grid), dim3(liger::kvs::kThreads), smem, s, c) != cudaSuccess)
+    return cuda_check("decode_stream launch");
+  mark_stop(s);
+  ++g_launches;
+  return cuda_check("decode_stream launch");
+}
+
 template <typename Tin, int D>
 liger_status launch_decode(const liger::DecodeArgs& a, unsigned blocks, cudaStream_t s) {
+  if constexpr (liger::kvs::fits<Tin, D, 1>()) return launch_decode_stream<Tin, D, 1, true>(a, blocks, s);
   constexpr size_t smem = liger::decode_smem_bytes<Tin, D>();
   auto kern = liger::decode_kernel<Tin, D>;
   if (smem > 48 * 1024 &&
@@ -198,31 +224,9 @@ liger_status launch_decode(const liger::DecodeArgs& a, unsigned blocks, cudaStre
   return cuda_check("decode launch");
 }
 
-// Error word of the streamed shared-state decode (bit 0: a bounded wait gave up;
-// word 1: the first site), one per device; read and cleared by
-// liger_attn_decode_kvshared_status().
-__device__ uint32_t g_decode_err[2];
-
 template <typename Tin, int D, int G>
 liger_status launch_decode_kvshared(const liger::DecodeArgs& a, unsigned blocks, cudaStream_t s) {
-  if constexpr (liger::kvs::fits<Tin, D, G>()) {   // the persistent two-stage stream
-    constexpr size_t smem = liger::kvs::Layout<Tin, D, G>::BYTES;
-    auto kern = liger::kvs::decode_kvshared_stream_kernel<Tin, D, G>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return cuda_check("cudaFuncSetAttribute(decode_kvshared_stream)");
-    void* err = nullptr;
-    const cudaError_t ge = cudaGetSymbolAddress(&err, g_decode_err);
-    if (ge != cudaSuccess) return fail(LIGER_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(ge));
-    liger::kvs::Args c{a, (int)blocks, static_cast<uint32_t*>(err), liger::tc::wait_limit_ns()};
-    const int sms = liger::tc::num_sms();
-    const unsigned grid = blocks < (unsigned)sms ? blocks : (unsigned)sms;   // one CTA per SM
-    mark_start(s);
-    if (launch_pdl(kern, dim3(grid), dim3(liger::kvs::kThreads), smem, s, c) != cudaSuccess)
-      return cuda_check("decode_kvshared_stream launch");
-    mark_stop(s);
-    ++g_launches;
-    return cuda_check("decode_kvshared_stream launch");
-  }
+  if constexpr (liger::kvs::fits<Tin, D, G>()) return launch_decode_stream<Tin, D, G, false>(a, blocks, s);
   constexpr size_t smem = liger::decode_smem_bytes<Tin, D>();
   auto kern = liger::decode_kvshared_kernel<Tin, D, G>;
   // static + dynamic shared memory can exceed the default 48 KiB: always raise the limit
@@ -671,7 +675,7 @@ liger_status liger_attn_full_causal(const void* q, const void* k, const void* v,
                  : launch_full_attn<128>(mq, mk, mv, prm, Hq, n_seqs, s);
 }
 
-liger_status liger_attn_decode_kvshared_status(void) {
+liger_status liger_attn_decode_status(void) {
   g_last_error.clear();
   uint32_t hdr[2] = {0u, 0u};
   cudaError_t e = cudaMemcpyFromSymbol(hdr, g_decode_err, sizeof hdr);
@@ -680,7 +684,7 @@ liger_status liger_attn_decode_kvshared_status(void) {
   e = cudaMemcpyToSymbol(g_decode_err, zero, sizeof zero);
   if (e != cudaSuccess) return fail(LIGER_ERR_CUDA, "clearing the decode's error word: %s", cudaGetErrorString(e));
   if (hdr[0] & 1u)
-    return fail(LIGER_ERR_TIMEOUT, "a shared-state decode kernel gave up waiting (site 0x%08x: role %u, barrier %u, unit %u)",
+    return fail(LIGER_ERR_TIMEOUT, "a decode kernel gave up waiting (site 0x%08x: role %u, barrier %u, unit %u)",
                 hdr[1], hdr[1] >> 28, (hdr[1] >> 20) & 0xFFu, hdr[1] & 0xFFFFFu);
   return LIGER_OK;
 }

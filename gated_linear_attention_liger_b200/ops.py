@@ -53,7 +53,7 @@ SIGNATURES = {
                                            _i, _vp]),
     "liger_attn_full_causal": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp]),
     "liger_attn_full_causal_status": (_i, []),
-    "liger_attn_decode_kvshared_status": (_i, []),
+    "liger_attn_decode_status": (_i, []),
     "liger_set_timing_events": (None, [_vp, _vp]),
     "liger_kernel_launches": (ctypes.c_uint64, []),
 }
@@ -307,9 +307,9 @@ def full_causal_status() -> int:
     return int(load().liger_attn_full_causal_status())
 
 
-def decode_kvshared_status() -> int:
-    """LIGER_OK, or LIGER_ERR_TIMEOUT if a shared-state decode gave up waiting since the last query."""
-    return int(load().liger_attn_decode_kvshared_status())
+def decode_status() -> int:
+    """LIGER_OK, or LIGER_ERR_TIMEOUT if a decode step gave up waiting since the last query."""
+    return int(load().liger_attn_decode_status())
 
 
 def prefill_backward_workspace_size(B, Hq, Hkv, T, d, n_seqs, dtype=torch.bfloat16) -> int:

@@ -179,16 +179,21 @@ liger_status liger_attn_decode(const void* q, const void* k, const void* v, floa
  *   state  [B, Hkv, d, d] fp32 (in/out): S <- g S + phi(k)^T v once per group
  *   swa_ring, pos: as for liger_attn_decode.
  * Supported: G in {1, 2, 4} (other group sizes return LIGER_ERR_UNSUPPORTED).
- * Except for fp32 at d = 128, the step runs as one persistent CTA per SM whose
- * internal waits are bounded (as for the prefill); a wait that gives up leaves
- * the step's outputs incomplete, and liger_attn_decode_kvshared_status()
- * reports whether any call on the current device gave up since the last query
- * (synchronous read; call it after the stream has completed; it clears the report).
  */
 liger_status liger_attn_decode_kvshared(const void* q, const void* k, const void* v, float* state,
                                         void* swa_ring, void* out, int32_t* pos, int B, int Hq, int Hkv,
                                         int d, int w, float alpha, liger_dtype dt, void* stream);
-liger_status liger_attn_decode_kvshared_status(void);
+
+/*
+ * Timeout report of the decodes.  Except for fp32 at d = 128, every decode step
+ * (liger_attn_decode, liger_attn_decode_kvshared, liger_attn_decode_vector_gate)
+ * runs as one persistent CTA per SM whose internal waits are bounded (as for the
+ * prefill); a wait that gives up leaves that step's outputs incomplete.  Returns
+ * LIGER_ERR_TIMEOUT if any decode on the current device gave up since the last
+ * query, else LIGER_OK (synchronous read; call it after the stream has completed;
+ * it clears the report).
+ */
+liger_status liger_attn_decode_status(void);
 
 /*
  * Prefill without caller-provided scratch (the pages have no counterpart; this

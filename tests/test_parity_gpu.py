@@ -190,16 +190,20 @@ def test_full_tiny_fp32(cuda_device):
 
 # ----------------------------------------------------------------- decode
 
-@pytest.mark.parametrize("dtype,d,w,T0,G", [
-    (torch.bfloat16, 128, 64, 70, 4),
-    (torch.bfloat16, 64, 64, 0, 2),
-    (torch.bfloat16, 64, 16, 5, 1),
-    (torch.float32, 128, 64, 100, 2),
-    (torch.float32, 64, 64, 3, 4),
+@pytest.mark.parametrize("dtype,d,w,T0,G,B", [
+    (torch.bfloat16, 128, 64, 70, 4, 3),
+    (torch.bfloat16, 64, 64, 0, 2, 3),
+    (torch.bfloat16, 64, 16, 5, 1, 3),
+    (torch.float32, 128, 64, 100, 2, 3),
+    (torch.float32, 64, 64, 3, 4, 3),
+    # more (sequence, head) units than SMs, ring wrapped, w < 64: each CTA of the
+    # streamed kernel takes several units and reuses its two stages
+    (torch.bfloat16, 128, 40, 90, 4, 40),
+    (torch.float32, 64, 64, 70, 2, 50),
 ])
-def test_decode_steps_parity(dtype, d, w, T0, G, cuda_device):
+def test_decode_steps_parity(dtype, d, w, T0, G, B, cuda_device):
     """Oracle prefix -> identical state/ring/pos on both sides -> several decode steps."""
-    B, Hkv, steps = 3, 2, 12
+    Hkv, steps = 2, 12
     Hq = Hkv * G
     wl = inputs.small("dec", B=B, Hq=Hq, Hkv=Hkv, T=T0 + steps, d=d, dtype=dtype, seed=17)
     q, k, v = inputs.prefill_inputs(wl)
@@ -223,6 +227,7 @@ def test_decode_steps_parity(dtype, d, w, T0, G, cuda_device):
     assert_close(np64(g_state), st, dtype, "decode state")
     np.testing.assert_array_equal(np64(g_ring), rg)
     np.testing.assert_array_equal(g_pos.cpu().numpy(), ps)
+    assert ops.decode_status() == ops.LIGER_OK
 
 
 def test_prefill_then_decode_matches_longer_prefill(cuda_device):
@@ -328,7 +333,7 @@ def test_decode_kvshared_parity(dtype, d, w, T0, G, B, cuda_device):
     assert_close(np64(g_state), st[:, ::G], dtype, "kv-shared state")
     np.testing.assert_array_equal(np64(g_ring), rg)
     np.testing.assert_array_equal(g_pos.cpu().numpy(), ps)
-    assert ops.decode_kvshared_status() == ops.LIGER_OK
+    assert ops.decode_status() == ops.LIGER_OK
 
 
 def test_decode_kvshared_matches_per_head_decode_full_shape(cuda_device):
