@@ -552,7 +552,7 @@ namespace kvs {
 // copy in flight.
 
 constexpr int kConsumers = 256;               // eight consumer warps
-constexpr int kThreads = kConsumers + 32;     // and the producer warp
+constexpr int kThreads = kConsumers + 64;     // and the producer and feature warps
 constexpr int kStages = 2;
 
 template <typename Tin, int D, int G>   // G: heads read out per unit
@@ -568,18 +568,20 @@ struct Layout {
   static constexpr uint32_t PART = RGN * G * D * 4;              // readout partial sums
   static constexpr uint32_t WSUM = WV::NW * G * D * 4;           // window partial sums (same room)
   static constexpr uint32_t SCRATCH = PART > WSUM ? PART : WSUM;
+  // per stage, written by the feature warp: phi(q_h) [G][D], q_h in fp32 [G][D], phi(k),
+  // k and v in fp32, the per-row gates [D] each, the scalar gate
+  // (q_h, k and v in fp32 are contiguous: one converted copy of the stage's rows)
+  static constexpr uint32_t F_FQ = 0, F_FK = F_FQ + G * D * 4, F_GV = F_FK + D * 4;
+  static constexpr uint32_t F_QF = F_GV + D * 4, F_KS = F_QF + G * D * 4, F_VS = F_KS + D * 4;
+  static constexpr uint32_t F_G = F_VS + D * 4;
+  static constexpr uint32_t FEAT = F_G + 16;
   static constexpr uint32_t OFF_SCRATCH = kStages * STAGE;
-  static constexpr uint32_t OFF_FQ = OFF_SCRATCH + SCRATCH;      // [G][D] phi(q_h)
-  static constexpr uint32_t OFF_QF = OFF_FQ + G * D * 4;         // [G][D] q_h in fp32
-  static constexpr uint32_t OFF_GRM = OFF_QF + G * D * 4;        // [G][D] recurrent readout
-  static constexpr uint32_t OFF_FK = OFF_GRM + G * D * 4;        // [D] phi(k)
-  static constexpr uint32_t OFF_KS = OFF_FK + D * 4;             // [D] k in fp32
-  static constexpr uint32_t OFF_VS = OFF_KS + D * 4;             // [D] v in fp32
-  static constexpr uint32_t OFF_GV = OFF_VS + D * 4;             // [D] per-row gates (vector gate)
-  static constexpr uint32_t OFF_SC = OFF_GV + D * 4;             // [G][64] window scores
-  static constexpr uint32_t OFF_MISC = OFF_SC + G * 64 * 4;      // barriers, gate, positions, abort
+  static constexpr uint32_t OFF_FEAT = OFF_SCRATCH + SCRATCH;    // kStages feature buffers
+  static constexpr uint32_t OFF_GRM = OFF_FEAT + kStages * FEAT; // [G][D] recurrent readout
+  static constexpr uint32_t OFF_SC = OFF_GRM + G * D * 4;        // [G][64] window scores
+  static constexpr uint32_t OFF_MISC = OFF_SC + G * 64 * 4;      // barriers, positions, abort
   static constexpr uint32_t BYTES = OFF_MISC + 128;
-  static_assert(STAGE % 16 == 0 && STATE % 4096 == 0, "bulk copies need 16-byte sizes");
+  static_assert(STAGE % 16 == 0 && STATE % 4096 == 0 && FEAT % 16 == 0, "16-byte pieces");
   static_assert(RGN * RPT == D && RPT >= 1, "row split");
 };
 
@@ -587,6 +589,24 @@ struct Layout {
 template <typename Tin, int D, int G>
 constexpr bool fits() {
   return Layout<Tin, D, G>::BYTES <= 227u * 1024u;
+}
+
+// A lane's EPL consecutive floats (EPL = 2 or 4) in one shared-memory access.
+template <int EPL>
+__device__ __forceinline__ void lane_slice_ld(const float* p, float* x) {
+  if constexpr (EPL == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+  } else {
+    static_assert(EPL == 2, "d = 64 or 128");
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    x[0] = t.x; x[1] = t.y;
+  }
+}
+template <int EPL>
+__device__ __forceinline__ void lane_slice_st(float* p, const float* x) {
+  if constexpr (EPL == 4) *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  else *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
 }
 
 struct Args {
@@ -629,21 +649,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
   using L = Layout<Tin, D, G>;
   using sm100::mbar_wait;
   extern __shared__ __align__(128) unsigned char sm[];
-  float* fq = reinterpret_cast<float*>(sm + L::OFF_FQ);
-  float* qf = reinterpret_cast<float*>(sm + L::OFF_QF);
   float* grm = reinterpret_cast<float*>(sm + L::OFF_GRM);
-  float* fk = reinterpret_cast<float*>(sm + L::OFF_FK);
-  float* ks = reinterpret_cast<float*>(sm + L::OFF_KS);
-  float* vs = reinterpret_cast<float*>(sm + L::OFF_VS);
-  float* gv = reinterpret_cast<float*>(sm + L::OFF_GV);
   float(*sc)[64] = reinterpret_cast<float(*)[64]>(sm + L::OFF_SC);
   float(*part)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
   float(*wsum)[G][D] = reinterpret_cast<float(*)[G][D]>(sm + L::OFF_SCRATCH);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::OFF_MISC);   // [2] stage loaded
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::OFF_MISC);   // [2] ring and q/k/v loaded
   uint64_t* sdone = full + 2;                                        // [2] state updated in place
   uint64_t* cons = full + 4;                                         // [2] stage no longer read
-  float* gsh = reinterpret_cast<float*>(full + 6);
-  int* pos_s = reinterpret_cast<int*>(gsh + 1);                      // [2]
+  uint64_t* featb = full + 6;                                        // [2] stage's features written
+  uint64_t* fullS = full + 8;                                        // [2] state loaded
+  int* pos_s = reinterpret_cast<int*>(full + 10);                    // [2]
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(pos_s + 2);
 
   const DecodeArgs& a = c.d;
@@ -651,12 +666,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
   const int Hkv = a.Hkv, Hq = a.Hq, w = a.w;
   const uint32_t ring_bytes = 2u * (uint32_t)w * D * sizeof(Tin);
   auto stage = [&](int s) { return sm + (size_t)s * L::STAGE; };
+  auto feat = [&](int s, uint32_t off) { return reinterpret_cast<float*>(sm + L::OFF_FEAT + s * L::FEAT + off); };
+  constexpr int EPL = D / 32;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       sm100::mbar_init(&full[s], 1);
       sm100::mbar_init(&sdone[s], kConsumers);
       sm100::mbar_init(&cons[s], kConsumers);
+      sm100::mbar_init(&featb[s], 32);
+      sm100::mbar_init(&fullS[s], 1);
     }
     *abort_flag = 0u;
     sm100::fence_mbar_init();
@@ -670,17 +689,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
   if (warp == kConsumers / 32) {
     // ---------------------------------------------------------------- producer
     if (lane != 0) return;
+    // the state part of a stage is reloaded as soon as the previous unit's state has
+    // left it (mid-unit); the ring and q/k/v part once the consumers release the stage
+    auto issue_state = [&](int i) {
+      const int s = i % kStages;
+      const long u = (long)blockIdx.x + (long)i * gridDim.x;
+      const float* S = a.state + unit_rows<G, PER_HEAD>(u, Hq, Hkv, D, w).state;
+      sm100::mbar_arrive_expect_tx(&fullS[s], L::STATE);
+#pragma unroll
+      for (int piece = 0; piece < 4; ++piece)
+        sm100::bulk_load(stage(s) + piece * (L::STATE / 4), S + piece * (D * D / 4), L::STATE / 4, &fullS[s]);
+    };
     auto issue = [&](int i) {
       const int s = i % kStages;
       const long u = (long)blockIdx.x + (long)i * gridDim.x;
       const UnitRows r = unit_rows<G, PER_HEAD>(u, Hq, Hkv, D, w);
       unsigned char* st = stage(s);
       pos_s[s] = max(a.pos[u / (PER_HEAD ? Hq : Hkv)], 0);   // a negative position is read as 0
-      sm100::mbar_arrive_expect_tx(&full[s], L::STATE + ring_bytes + L::QKV);
-      const float* S = a.state + r.state;
-#pragma unroll
-      for (int piece = 0; piece < 4; ++piece)
-        sm100::bulk_load(st + piece * (L::STATE / 4), S + piece * (D * D / 4), L::STATE / 4, &full[s]);
+      sm100::mbar_arrive_expect_tx(&full[s], ring_bytes + L::QKV);
       sm100::bulk_load(st + L::STATE, static_cast<const Tin*>(a.ring) + r.ring, ring_bytes, &full[s]);
       unsigned char* qkv = st + L::STATE + L::RING;
       sm100::bulk_load(qkv, static_cast<const Tin*>(a.q) + r.q, G * D * sizeof(Tin), &full[s]);
@@ -688,8 +714,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
       sm100::bulk_load(qkv + (G + 1) * D * sizeof(Tin), static_cast<const Tin*>(a.v) + r.kv, D * sizeof(Tin),
                        &full[s]);
     };
-    int issued = 0;
-    for (; issued < kStages && issued < n_local; ++issued) issue(issued);
+    int issued = 0, issued_state = 0;   // units whose ring and q/k/v (state) copies are issued
+    for (; issued < kStages && issued < n_local; ++issued, ++issued_state) {
+      issue_state(issued);
+      issue(issued);
+    }
     for (int i = 0; i < n_local; ++i) {
       const int s = i % kStages;
       const uint32_t ph = (uint32_t)(i / kStages) & 1u;
@@ -701,17 +730,84 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
         sm100::bulk_store(S + piece * (D * D / 4), stage(s) + piece * (L::STATE / 4), L::STATE / 4);
       sm100::bulk_commit();
       if (i + kStages < n_local) {
-        if (!mbar_wait(&cons[s], ph, wc, sm100::wsite(7, 2, i))) break;
         sm100::bulk_wait_read_all();   // this unit's state has left the stage
+        issue_state(issued_state++);
+        if (!mbar_wait(&cons[s], ph, wc, sm100::wsite(7, 2, i))) break;
         issue(issued++);
       }
     }
     // never leave with copies in flight: the last load of each stage, then the stores
     volatile uint32_t never = 0u;
     const sm100::WaitCtx drain{&never, nullptr, c.wait_ns};
+    for (int i = issued_state > kStages ? issued_state - kStages : 0; i < issued_state; ++i)
+      mbar_wait(&fullS[i % kStages], (uint32_t)(i / kStages) & 1u, drain);
     for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
       mbar_wait(&full[i % kStages], (uint32_t)(i / kStages) & 1u, drain);
     sm100::bulk_wait_all();
+    return;
+  }
+
+  if (warp == kConsumers / 32 + 1) {
+    // ---------------------------------------------------------------- features
+    // phi(k), the gate(s) and phi(q_h) of each unit, and fp32 copies of its q, k and v,
+    // into the stage's feature buffer, one unit ahead of the consumers where the copies
+    // allow.  The buffer of stage s is rewritten only after the producer has reloaded
+    // stage s, i.e. after the consumers have released it.
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i % kStages;
+      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+      if (!sm100::warp_all(mbar_wait(&full[s], ph, wc, sm100::wsite(8, 1, i)))) break;
+      const Tin* qin = reinterpret_cast<const Tin*>(stage(s) + L::STATE + L::RING);
+      // fp32 copies of the q rows, k and v (contiguous on both sides), 16 bytes a step
+      constexpr int EPP = 16 / (int)sizeof(Tin);
+      float* rows = feat(s, L::F_QF);
+      for (int pc = lane; pc < (G + 2) * D / EPP; pc += 32) {
+        float xv[EPP];
+        ld16_vals<Tin>(qin + pc * EPP, xv);
+#pragma unroll
+        for (int e = 0; e < EPP; e += 4)
+          *reinterpret_cast<float4*>(rows + pc * EPP + e) = make_float4(xv[e], xv[e + 1], xv[e + 2], xv[e + 3]);
+      }
+      __syncwarp();
+      // one softmax over d per row (row 0 the key, rows 1..G the queries), EPL consecutive
+      // elements per lane
+      float x[G + 1][EPL], m[G + 1], z[G + 1], sum = 0.f;
+#pragma unroll
+      for (int r = 0; r <= G; ++r) {
+        const float* src = (r == 0 ? rows + G * D : rows + (r - 1) * D) + lane * EPL;
+        m[r] = -INFINITY;
+        z[r] = 0.f;
+        lane_slice_ld<EPL>(src, x[r]);
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) m[r] = fmaxf(m[r], x[r][j]);
+      }
+      if (PER_HEAD && a.vector_gate) {
+        float* gv = feat(s, L::F_GV) + lane * EPL;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) gv[j] = expf(log_sigmoid(x[0][j]));
+      }
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) sum += x[0][j];
+#pragma unroll
+      for (int r = 0; r <= G; ++r) m[r] = warp_max(m[r]);
+      sum = warp_sum(sum);
+#pragma unroll
+      for (int r = 0; r <= G; ++r)
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) { x[r][j] = expf(x[r][j] - m[r]); z[r] += x[r][j]; }
+#pragma unroll
+      for (int r = 0; r <= G; ++r) z[r] = warp_sum(z[r]);
+#pragma unroll
+      for (int r = 0; r <= G; ++r) {
+        float* dst = (r == 0 ? feat(s, L::F_FK) : feat(s, L::F_FQ) + (r - 1) * D) + lane * EPL;
+        float y[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) y[j] = x[r][j] / z[r];
+        lane_slice_st<EPL>(dst, y);
+      }
+      if (lane == 0) *feat(s, L::F_G) = expf(log_sigmoid(sum / (float)D));
+      sm100::mbar_arrive(&featb[s]);   // every lane: its own writes are released
+    }
     return;
   }
 
@@ -720,7 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
   for (int i = 0; i < n_local; ++i) {
     const int s = i % kStages;
     const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-    const bool ok = mbar_wait(&full[s], ph, wc, sm100::wsite(6, 1, i));
+    const bool ok = mbar_wait(&featb[s], ph, wc, sm100::wsite(6, 1, i)) &&
+                    mbar_wait(&fullS[s], ph, wc, sm100::wsite(6, 2, i));
     if (sm100::named_bar_or(1, kConsumers, !ok)) break;
     const long u = (long)blockIdx.x + (long)i * gridDim.x;
     const UnitRows ur = unit_rows<G, PER_HEAD>(u, Hq, Hkv, D, w);
@@ -728,56 +825,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
     float* Ss = reinterpret_cast<float*>(st);
     const Tin* rk = reinterpret_cast<const Tin*>(st + L::STATE);
     const Tin* rv = rk + (size_t)w * D;
-    const Tin* qin = reinterpret_cast<const Tin*>(st + L::STATE + L::RING);
-    const Tin* kin = qin + G * D;
+    const Tin* kin = reinterpret_cast<const Tin*>(st + L::STATE + L::RING) + G * D;
     const Tin* vin = kin + D;
+    const float* fq = feat(s, L::F_FQ);
+    const float* qf = feat(s, L::F_QF);
+    const float* fk = feat(s, L::F_FK);
+    const float* ks = feat(s, L::F_KS);
+    const float* vs = feat(s, L::F_VS);
+    const float* gv = feat(s, L::F_GV);
     const int p = pos_s[s];
-
-    // phi(k) and the gate (warp 0), phi(q_h) (warps 1..G), fp32 copies of q, k, v (the rest)
-    constexpr int EPL = D / 32;
-    if (warp == 0) {
-      float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = io<Tin>::ld(kin + lane + 32 * j); m = fmaxf(m, x[j]); sum += x[j]; }
-      m = warp_max(m);
-      sum = warp_sum(sum);
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
-      z = warp_sum(z);
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) fk[lane + 32 * j] = x[j] / z;
-      if (lane == 0) *gsh = expf(log_sigmoid(sum / (float)D));
-      if (PER_HEAD && a.vector_gate) {
-#pragma unroll
-        for (int j = 0; j < EPL; ++j) gv[lane + 32 * j] = expf(log_sigmoid(io<Tin>::ld(kin + lane + 32 * j)));
-      }
-    } else if (warp <= G) {
-      const int hh = warp - 1;
-      float x[EPL], m = -INFINITY, z = 0.f;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = io<Tin>::ld(qin + hh * D + lane + 32 * j); m = fmaxf(m, x[j]); }
-      m = warp_max(m);
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
-      z = warp_sum(z);
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) fq[hh * D + lane + 32 * j] = x[j] / z;
-    } else {
-      constexpr int first = 32 * (G + 1), nconv = kConsumers - first;
-      for (int idx = tid - first; idx < (G + 2) * D; idx += nconv) {
-        const float x = io<Tin>::ld(qin + idx);   // q rows, then k, then v
-        if (idx < G * D) qf[idx] = x;
-        else if (idx < (G + 1) * D) ks[idx - G * D] = x;
-        else vs[idx - (G + 1) * D] = x;
-      }
-    }
-    sm100::named_bar(1, kConsumers);
 
     // state update in place, readout for every head of the group; the producer sends
     // the state back as soon as every consumer has written its rows
     {
       const bool vgate = PER_HEAD && a.vector_gate;
-      const float g = *gsh;
+      const float g = *feat(s, L::F_G);
       const float4 vv = *reinterpret_cast<const float4*>(vs + 4 * cq);
       const float2 v01 = make_float2(vv.x, vv.y), v23 = make_float2(vv.z, vv.w);
       float2 a01[G], a23[G];
@@ -817,9 +879,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
     }
     sm100::fence_proxy_async_smem();   // the rows written above are read by the bulk copy out
     sm100::mbar_arrive(&sdone[s]);
-    sm100::named_bar(1, kConsumers);
 
-    // window scores on the ring in slot order (window position jj is slot (p+1+jj) mod w)
+    // window scores on the ring in slot order (window position jj is slot (p+1+jj) mod w);
+    // they read only this phase's inputs, so no barrier separates them from the update
     const int row0 = (p + 1) % w;
     window_scores<Tin, D, G, D>(reinterpret_cast<const float(*)[D]>(qf), ks, rk, sc, p, w, tid, row0, w);
     sm100::named_bar(1, kConsumers);
