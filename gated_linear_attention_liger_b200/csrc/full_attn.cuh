@@ -23,6 +23,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "liger_attn.h"
 #include "sm100.cuh"
@@ -36,6 +38,7 @@ constexpr int BM = 128;                 // query rows (tokens) per tile; two til
 constexpr int BN = 128;                 // keys per block
 constexpr int kThreads = 320;           // warps 0-3 softmax A, 4-7 softmax B, 8 TMA, 9 MMA
 constexpr float kRescaleLog2 = 8.f;     // raise the running maximum only beyond 2^8
+constexpr int kPolyPairs = 2;           // of every 8 column pairs off the diagonal: 2^x by polynomial
 
 struct Params {
   void* out;
@@ -220,13 +223,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       const bool diag = j == diag_blk;
       float bm = -INFINITY;
+      if (diag) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        x[c] *= sl2;
-        if (diag && c > r) x[c] = -INFINITY;
+        for (int c = 0; c < BN; ++c)
+          if (c > r) x[c] = -INFINITY;
       }
 #pragma unroll
       for (int c = 0; c < BN; c += 2) bm = fmax3(bm, x[c], x[c + 1]);
+      bm *= sl2;   // the scale is positive: the maximum of the scaled scores
       // raise the running maximum (and rescale this row's O and sum) only when the block's
       // maximum exceeds it by more than 2^8; decided per row, entered warp-wide
       const bool raise = bm > m + kRescaleLog2;
@@ -251,23 +255,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= f;
         m = mn;
       }
-      const float2 nm2 = make_float2(-m, -m);
+      const float2 nm2 = make_float2(-m, -m), s2 = make_float2(sl2, sl2);
       float2 ls = make_float2(0.f, 0.f);
       // P over the first 64 columns of the tile's score buffer (the scores are in
-      // registers), written eight columns at a time so that fewer values are live at once
+      // registers), written eight columns at a time so that fewer values are live at once.
+      // Off the diagonal block, kPolyPairs of every eight column pairs take 2^x from the
+      // FMA pipes (exp2_poly2) instead of the special-function unit, the busier of the two
+      // here; the diagonal block (with its masked -inf scores) stays on the unit.
+      auto write_p = [&](auto poly) {
 #pragma unroll
-      for (int h4 = 0; h4 < 8; ++h4) {
-        uint32_t pk[8];
+        for (int h4 = 0; h4 < 8; ++h4) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-          float2 y = fadd2(make_float2(x[h4 * 16 + c], x[h4 * 16 + c + 1]), nm2);
-          y.x = ex2(y.x);
-          y.y = ex2(y.y);
-          ls = fadd2(ls, y);
-          pk[c / 2] = pack_bf16(y.x, y.y);
+          for (int c = 0; c < 16; c += 2) {
+            float2 y = ffma2(make_float2(x[h4 * 16 + c], x[h4 * 16 + c + 1]), s2, nm2);
+            if (decltype(poly)::value && c >= 16 - 2 * kPolyPairs) {
+              y = exp2_poly2(y);
+            } else {
+              y.x = ex2(y.x);
+              y.y = ex2(y.y);
+            }
+            ls = fadd2(ls, y);
+            pk[c / 2] = pack_bf16(y.x, y.y);
+          }
+          tmem_st8u(sb + h4 * 8, pk);
         }
-        tmem_st8u(sb + h4 * 8, pk);
-      }
+      };
+      if (diag) write_p(std::false_type{});
+      else write_p(std::true_type{});
       l += ls.x + ls.y;
       tmem_wait_st();
       tc_fence_before();
