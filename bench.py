@@ -821,8 +821,8 @@ def run_decode(args, world, dev, stream, pk, windows, kvshared=False):
             "gpu_launches": per_graph_launches * reps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"],
-                         "traffic": measured_traffic("decode_kvshared_kernel<bf16,128,4>" if kvshared
-                                                     else "decode_kernel<bf16,128>"),
+                         "traffic": measured_traffic("decode_stream_kernel<bf16,128,4,kv-shared>" if kvshared
+                                                     else "decode_stream_kernel<bf16,128,1,per-head>"),
                          "kernel": "decode state stream" + (" (kv-shared)" if kvshared else ""), "kernel_ms": kms,
                          "kernel_timing": "events in graph" if kernel_events else "graph step average",
                          "algorithmic_bytes": alg, "peak_source": pk["source"]}}
