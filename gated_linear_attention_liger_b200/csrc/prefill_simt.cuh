@@ -61,36 +61,52 @@ constexpr int kMaxWindow = 64;
 template <int D>
 constexpr int simt_ring_stride() { return D + 4; }
 
+// The recurrence's thread tile: thread = a row group of RPG key rows x one quad of value
+// columns; the NRG row groups of a column quad are adjacent lanes.  phi(k), phi(q) and the
+// per-row gates of a token are stored by row group, each group's RPG values padded to a
+// stride of an odd number of 16-byte units, so that the row groups a warp reads in one
+// vector load sit in different bank groups.
+template <int D>
+struct SimtRows {
+  static constexpr int CQN = D / 4;                 // column quads
+  static constexpr int NRG = kSimtThreads / CQN;    // row groups
+  static constexpr int RPG = D / NRG;               // rows per group
+  static constexpr int RGS = ((RPG / 4 + 1) % 2) ? RPG + 4 : RPG + 8;   // padded group stride (floats)
+  static constexpr int FS = NRG * RGS;              // floats per token
+  static_assert(NRG >= 8 && NRG <= 32 && RPG % 4 == 0, "row groups of a quad within one warp");
+  __device__ __forceinline__ static int at(int e) { return (e / RPG) * RGS + e % RPG; }
+};
+
 // VG: one gate per key dimension, sigmoid(k_t[r]) on row r of the state (the
 // per-dimension form of the pooled key gate); otherwise the pooled scalar gate.
 template <int D, bool VG = false>
 constexpr size_t simt_prefill_smem_bytes() {
-  constexpr int RG = kSimtThreads / D;
-  return sizeof(float) * (size_t)(2 * kSimtRing * simt_ring_stride<D>() + 3 * kSimtChunk * D + kSimtChunk * RG * D +
-                                  kSimtChunk * kSimtRing + kSimtChunk + (VG ? kSimtChunk * D : 0));
+  constexpr int FS = SimtRows<D>::FS;
+  return sizeof(float) * (size_t)(2 * kSimtRing * simt_ring_stride<D>() + kSimtChunk * D + 2 * kSimtChunk * FS +
+                                  kSimtChunk * D + kSimtChunk * kSimtRing + kSimtChunk + (VG ? kSimtChunk * FS : 0));
 }
 
 template <typename Tin, int D, bool VG = false>
 __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillArgs a) {
   constexpr int NT = kSimtThreads, C = kSimtChunk, RING = kSimtRing;
   constexpr int RS = simt_ring_stride<D>();
-  constexpr int RG = NT / D;      // row groups
-  constexpr int RPT = D / RG;     // key rows per thread
+  using RT = SimtRows<D>;
+  constexpr int NRG = RT::NRG, RPG = RT::RPG, RGS = RT::RGS, FS = RT::FS;
   constexpr int EPL = D / 32;     // elements per lane for row-wise work
   constexpr int TPW = C / (NT / 32);   // window: tokens per warp
   constexpr int XPL = RING / 32;       // window: ring positions per lane
-  static_assert(RING == C + kMaxWindow && RING % 32 == 0 && C % (NT / 32) == 0 && RPT % 4 == 0 &&
-                (EPL == 2 || EPL == 4), "window and row tiling");
+  static_assert(RING == C + kMaxWindow && RING % 32 == 0 && C % (NT / 32) == 0 && (EPL == 2 || EPL == 4),
+                "window and row tiling");
   extern __shared__ float smem[];
   float* ring_k = smem;                     // [RING][RS]
   float* ring_v = ring_k + RING * RS;       // [RING][RS]
   float* qbuf = ring_v + RING * RS;         // [C][D]  raw q, later the window output
-  float* fq = qbuf + C * D;                 // [C][D]  phi(q)
-  float* fk = fq + C * D;                   // [C][D]  phi(k)
-  float* part = fk + C * D;                 // [C][RG][D] partial readouts
-  float* sc = part + C * RG * D;            // [C][RING] window probabilities over the ring positions
+  float* fq = qbuf + C * D;                 // [C][FS] phi(q), by row group
+  float* fk = fq + C * FS;                  // [C][FS] phi(k), by row group
+  float* grm = fk + C * FS;                 // [C][D] recurrent readouts
+  float* sc = grm + C * D;                  // [C][RING] window probabilities over the ring positions
   float* gate = sc + C * RING;              // [C]
-  float* gvec = gate + C;                   // [C][D] per-dimension gates (VG only)
+  float* gvec = gate + C;                   // [C][FS] per-dimension gates by row group (VG only)
 
   const Tin* __restrict__ q = static_cast<const Tin*>(a.q);
   const Tin* __restrict__ k = static_cast<const Tin*>(a.k);
@@ -118,16 +134,18 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
   if (a.only_flagged && a.only_flagged[(size_t)seq * Hkv + kv] == 0u) return;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = tid % D, rg = tid / D;
+  const int rg = tid % NRG, cq = tid / NRG;   // recurrence tile: rows rg*RPG.., columns 4cq..4cq+3
   const float inv_sqrt_d = 1.0f / sqrtf((float)D);
   const float alpha = a.alpha, beta = 1.0f - a.alpha;
 
-  float s[RPT];
+  float4 s[RPG];   // s[r] = row rg*RPG + r, columns 4cq .. 4cq+3
   const size_t st_off = ((size_t)seq * Hq + h) * D * D;
   const float* s_in = first ? (a.init_state ? a.init_state + st_off : nullptr)
                             : a.seg_state + ((size_t)unit * Hkv + kv) * D * D;
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) s[r] = s_in ? s_in[(size_t)(rg * RPT + r) * D + c] : 0.f;
+  for (int r = 0; r < RPG; ++r)
+    s[r] = s_in ? *reinterpret_cast<const float4*>(s_in + (size_t)(rg * RPG + r) * D + 4 * cq)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
 
   // the window's keys and values before the first token (segmented mode)
   for (long idx = tid; idx < (sb - max(tb, sb - (w - 1))) * D; idx += NT) {
@@ -164,10 +182,11 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
       z = warp_sum(z);
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) fk[i * D + lane + 32 * j] = x[j] / z;
+      for (int j = 0; j < EPL; ++j) fk[i * FS + RT::at(lane + 32 * j)] = x[j] / z;
       if (VG) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) gvec[i * D + lane + 32 * j] = expf(log_sigmoid(ring_k[slot * RS + lane + 32 * j]));
+        for (int j = 0; j < EPL; ++j)
+          gvec[i * FS + RT::at(lane + 32 * j)] = expf(log_sigmoid(ring_k[slot * RS + lane + 32 * j]));
       } else if (lane == 0) {
         gate[i] = expf(log_sigmoid(sum / (float)D));
       }
@@ -180,7 +199,7 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
       for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
       z = warp_sum(z);
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) fq[i * D + lane + 32 * j] = x[j] / z;
+      for (int j = 0; j < EPL; ++j) fq[i * FS + RT::at(lane + 32 * j)] = x[j] / z;
     }
     __syncthreads();   // features and gates of every token (phase 2 rows are spread over the warps)
     // 3. window branch over the ring, which holds positions t0 - 64 .. t0 + C - 1 (ring
@@ -277,48 +296,66 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
 #pragma unroll
         for (int q = 0; q < EPL; ++q) qbuf[(i0 + tt) * D + EPL * lane + q] = o[tt][q];
     }
-    // 4. token-serial recurrence on the register-resident state (no syncs); rows in fours
-    //    from shared memory, pairs of rows in packed multiply-adds
-    for (int i = 0; i < n; ++i) {
-      const float g = VG ? 1.f : gate[i];
-      const float vc = ring_v[((int)((t0 + i - tb) % RING)) * RS + c];
-      const float* fki = fk + i * D + rg * RPT;
-      const float* fqi = fq + i * D + rg * RPT;
-      const float* gvi = gvec + i * D + rg * RPT;
-      const float2 vc2 = make_float2(vc, vc), g2 = make_float2(g, g);
-      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+    // 4. token-serial recurrence on the register-resident state (no syncs): each thread
+    //    updates its RPG x 4 tile in packed pairs, then the readout's partial sums over the
+    //    row groups are added by a reduce-scatter among the NRG adjacent lanes (after it,
+    //    each lane holds the total of one of the quad's four columns)
+    {
+      const int slot_c = (int)((t0 - tb) % RING);
+      for (int i = 0; i < n; ++i) {
+        const float g = VG ? 1.f : gate[i];
+        int slot = slot_c + i;
+        slot = slot >= RING ? slot - RING : slot;
+        const float4 v4 = *reinterpret_cast<const float4*>(ring_v + slot * RS + 4 * cq);
+        const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
+        const float* fki = fk + i * FS + rg * RGS;
+        const float* fqi = fq + i * FS + rg * RGS;
+        const float* gvi = gvec + i * FS + rg * RGS;
+        float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int r = 0; r < RPT; r += 4) {
-        const float4 kf = *reinterpret_cast<const float4*>(fki + r);
-        const float4 qf = *reinterpret_cast<const float4*>(fqi + r);
-        float2 ga = g2, gb = g2;
-        if (VG) {
-          const float4 gf = *reinterpret_cast<const float4*>(gvi + r);
-          ga = make_float2(gf.x, gf.y);
-          gb = make_float2(gf.z, gf.w);
+        for (int r4 = 0; r4 < RPG; r4 += 4) {
+          const float4 kf = *reinterpret_cast<const float4*>(fki + r4);
+          const float4 qf = *reinterpret_cast<const float4*>(fqi + r4);
+          const float4 gf = VG ? *reinterpret_cast<const float4*>(gvi + r4) : make_float4(g, g, g, g);
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            const float kr = rr == 0 ? kf.x : rr == 1 ? kf.y : rr == 2 ? kf.z : kf.w;
+            const float qr = rr == 0 ? qf.x : rr == 1 ? qf.y : rr == 2 ? qf.z : qf.w;
+            const float gr = rr == 0 ? gf.x : rr == 1 ? gf.y : rr == 2 ? gf.z : gf.w;
+            const float2 k2 = make_float2(kr, kr), g2 = make_float2(gr, gr), q2 = make_float2(qr, qr);
+            float4& sr = s[r4 + rr];
+            const float2 s01 = sm100::ffma2(g2, make_float2(sr.x, sr.y), sm100::fmul2(k2, v01));
+            const float2 s23 = sm100::ffma2(g2, make_float2(sr.z, sr.w), sm100::fmul2(k2, v23));
+            sr = make_float4(s01.x, s01.y, s23.x, s23.y);
+            a01 = sm100::ffma2(q2, s01, a01);
+            a23 = sm100::ffma2(q2, s23, a23);
+          }
         }
-        const float2 s01 = sm100::ffma2(ga, make_float2(s[r], s[r + 1]), sm100::fmul2(make_float2(kf.x, kf.y), vc2));
-        const float2 s23 = sm100::ffma2(gb, make_float2(s[r + 2], s[r + 3]), sm100::fmul2(make_float2(kf.z, kf.w), vc2));
-        s[r] = s01.x; s[r + 1] = s01.y; s[r + 2] = s23.x; s[r + 3] = s23.y;
-        a01 = sm100::ffma2(make_float2(qf.x, qf.y), s01, a01);
-        a23 = sm100::ffma2(make_float2(qf.z, qf.w), s23, a23);
+        // reduce-scatter over the row groups (lane bits below NRG)
+        const bool up1 = (rg & (NRG / 2)) != 0;
+        float2 keep = up1 ? a23 : a01;
+        const float2 send = up1 ? a01 : a23;
+        keep.x += __shfl_xor_sync(0xffffffffu, send.x, NRG / 2);
+        keep.y += __shfl_xor_sync(0xffffffffu, send.y, NRG / 2);
+        const bool up2 = (rg & (NRG / 4)) != 0;
+        float t = (up2 ? keep.y : keep.x) + __shfl_xor_sync(0xffffffffu, up2 ? keep.x : keep.y, NRG / 4);
+#pragma unroll
+        for (int o = NRG / 8; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if ((rg & (NRG / 4 - 1)) == 0) grm[i * D + 4 * cq + (up1 ? 2 : 0) + (up2 ? 1 : 0)] = t;
       }
-      part[(i * RG + rg) * D + c] = (a01.x + a01.y) + (a23.x + a23.y);
     }
     __syncthreads();
     // 5. mix and store
     for (int idx = tid; idx < n * D; idx += NT) {
       const int i = idx / D, e = idx % D;
-      float grm = 0.f;
-#pragma unroll
-      for (int r = 0; r < RG; ++r) grm += part[(i * RG + r) * D + e];
-      io<Tin>::st(out + ((size_t)(t0 + i) * Hq + h) * D + e, alpha * grm + beta * qbuf[idx]);
+      io<Tin>::st(out + ((size_t)(t0 + i) * Hq + h) * D + e, alpha * grm[idx] + beta * qbuf[idx]);
     }
     __syncthreads();
   }
   if (a.final_state && last) {
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) a.final_state[st_off + (size_t)(rg * RPT + r) * D + c] = s[r];
+    for (int r = 0; r < RPG; ++r)
+      *reinterpret_cast<float4*>(a.final_state + st_off + (size_t)(rg * RPG + r) * D + 4 * cq) = s[r];
   }
 }
 
