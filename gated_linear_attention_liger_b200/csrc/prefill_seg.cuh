@@ -58,46 +58,52 @@ __global__ void plan_kernel(const int32_t* cu, long T, int n_seqs, long T_total,
   *n_segs = (int)n;
 }
 
-// Per (segment slot, kv head), 256 threads: thread (column c, row group rg) owns
-// rows rg*RPT .. rg*RPT+RPT-1 of column c of dS.  Tokens are staged 64 at a time,
-// last to first: lam[r] = B - B_j (the gates after token j) is then known when j is
-// reached, and w_j[r] = e^{lam[r]} phi(k_j)[r] <= phi(k_j)[r].
+// Per (segment slot, kv head), 256 threads: thread (row group rg, column quad cq) owns
+// the tile of rows rg*RPG .. rg*RPG+RPG-1 and columns 4cq .. 4cq+3 of dS (the general
+// kernel's recurrence tile; the keys and weights are stored in its padded row-group
+// layout, so a thread's RPG rows are float4 loads without bank conflicts).  Tokens are
+// staged 64 at a time, last to first: lam[r] = B - B_j (the gates after token j) is then
+// known when j is reached, and w_j[r] = e^{lam[r]} phi(k_j)[r] <= phi(k_j)[r].
 template <typename Tin, int D, bool VG>
 __global__ void __launch_bounds__(kSegThreads) seg_state_kernel(const Tin* __restrict__ k,
                                                                 const Tin* __restrict__ v, int Hkv,
                                                                 const SimtSeg* segs, const int* n_segs,
                                                                 float* __restrict__ ds, float* __restrict__ lam_out) {
   constexpr int NT = kSegThreads, S = kStage;
-  constexpr int RG = NT / D, RPT = D / RG, EPL = D / 32;
+  using RT = SimtRows<D>;
+  static_assert(kSegThreads == kSimtThreads, "the general kernel's tile");
+  constexpr int RPG = RT::RPG, RGS = RT::RGS, FS = RT::FS, NRG = RT::NRG, EPL = D / 32;
   extern __shared__ __align__(16) float seg_smem[];
-  float (*kw)[D] = reinterpret_cast<float (*)[D]>(seg_smem);            // [S][D] raw keys, then the weights w_j
-  float (*vs)[D] = reinterpret_cast<float (*)[D]>(seg_smem + S * D);    // [S][D]
-  float (*lg)[VG ? D : 1] = reinterpret_cast<float (*)[VG ? D : 1]>(seg_smem + 2 * S * D);   // [S] log gates
+  float (*kw)[FS] = reinterpret_cast<float (*)[FS]>(seg_smem);           // [S][FS] raw keys, then the weights w_j
+  float (*vs)[D] = reinterpret_cast<float (*)[D]>(seg_smem + S * FS);    // [S][D]
+  float (*lg)[VG ? D : 1] = reinterpret_cast<float (*)[VG ? D : 1]>(seg_smem + S * (FS + D));   // [S] log gates
   __shared__ float lam[D];                   // gates after the staged block
   const int slot = blockIdx.x / Hkv, kv = blockIdx.x % Hkv;
   if (slot >= *n_segs) return;
   const SimtSeg sg = segs[slot];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = tid % D, rg = tid / D;
-  float acc[RPT];
+  const int rg = tid % NRG, cq = tid / NRG;
+  float4 acc[RPG];
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) acc[r] = 0.f;
+  for (int r = 0; r < RPG; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tid < D) lam[tid] = 0.f;
   for (long t1 = sg.t_end; t1 > sg.t_begin; t1 -= S) {
     const long t0 = max(sg.t_begin, t1 - S);
     const int n = (int)(t1 - t0);
     __syncthreads();   // the previous block's weights are consumed
-    for (int idx = tid; idx < n * D; idx += NT) {
-      const int i = idx / D, e = idx % D;
-      kw[i][e] = io<Tin>::ld(k + ((size_t)(t0 + i) * Hkv + kv) * D + e);
-      vs[i][e] = io<Tin>::ld(v + ((size_t)(t0 + i) * Hkv + kv) * D + e);
+    {   // every load of a thread in flight before its first store
+      RowPieces<Tin, D, S, NT> pk, pv;
+      pk.load(k + ((size_t)t0 * Hkv + kv) * D, (size_t)Hkv * D, n, tid);
+      pv.load(v + ((size_t)t0 * Hkv + kv) * D, (size_t)Hkv * D, n, tid);
+      pk.store(n, tid, [=](int i, int e) { return &kw[i][RT::at(e)]; });
+      pv.store(n, tid, [=](int i, int e) { return &vs[i][e]; });
     }
     __syncthreads();
     // phi(k) and the log gates, one warp per token
     for (int i = warp; i < n; i += NT / 32) {
       float x[EPL], m = -INFINITY, sum = 0.f, z = 0.f;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) { x[j] = kw[i][lane + 32 * j]; m = fmaxf(m, x[j]); sum += x[j]; }
+      for (int j = 0; j < EPL; ++j) { x[j] = kw[i][RT::at(lane + 32 * j)]; m = fmaxf(m, x[j]); sum += x[j]; }
       m = warp_max(m);
       sum = warp_sum(sum);
       if (VG) {
@@ -110,34 +116,49 @@ __global__ void __launch_bounds__(kSegThreads) seg_state_kernel(const Tin* __res
       for (int j = 0; j < EPL; ++j) { x[j] = expf(x[j] - m); z += x[j]; }
       z = warp_sum(z);
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) kw[i][lane + 32 * j] = x[j] / z;
+      for (int j = 0; j < EPL; ++j) kw[i][RT::at(lane + 32 * j)] = x[j] / z;
     }
     __syncthreads();
     // weights, last token first: one thread per key dimension
     if (tid < D) {
       float l = lam[tid];
+      const int at = RT::at(tid);
       for (int i = n - 1; i >= 0; --i) {
-        kw[i][tid] *= expf(l);
+        kw[i][at] *= expf(l);
         l += lg[i][VG ? tid : 0];
       }
       lam[tid] = l;
     }
     __syncthreads();
     for (int i = 0; i < n; ++i) {
-      const float vc = vs[i][c];
+      const float4 v4 = *reinterpret_cast<const float4*>(&vs[i][4 * cq]);
+      const float2 v01 = make_float2(v4.x, v4.y), v23 = make_float2(v4.z, v4.w);
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) acc[r] = fmaf(kw[i][rg * RPT + r], vc, acc[r]);
+      for (int r4 = 0; r4 < RPG; r4 += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(&kw[i][rg * RGS + r4]);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const float wr = rr == 0 ? w4.x : rr == 1 ? w4.y : rr == 2 ? w4.z : w4.w;
+          const float2 w2 = make_float2(wr, wr);
+          float4& a = acc[r4 + rr];
+          const float2 a01 = sm100::ffma2(w2, v01, make_float2(a.x, a.y));
+          const float2 a23 = sm100::ffma2(w2, v23, make_float2(a.z, a.w));
+          a = make_float4(a01.x, a01.y, a23.x, a23.y);
+        }
+      }
     }
   }
   float* dst = ds + ((size_t)slot * Hkv + kv) * D * D;
 #pragma unroll
-  for (int r = 0; r < RPT; ++r) dst[(size_t)(rg * RPT + r) * D + c] = acc[r];
+  for (int r = 0; r < RPG; ++r) *reinterpret_cast<float4*>(dst + (size_t)(rg * RPG + r) * D + 4 * cq) = acc[r];
   __syncthreads();
   if (tid < D) lam_out[((size_t)slot * Hkv + kv) * D + tid] = lam[tid];
 }
 
 template <int D, bool VG>
-constexpr size_t seg_state_smem_bytes() { return sizeof(float) * (size_t)kStage * (2 * D + (VG ? D : 1)); }
+constexpr size_t seg_state_smem_bytes() {
+  return sizeof(float) * (size_t)kStage * (SimtRows<D>::FS + D + (VG ? D : 1));
+}
 
 // Per (sequence, kv head, block of 256 state elements): folds the segments'
 // contributions in order, overwriting each segment's dS with the state entering it
@@ -165,19 +186,38 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const SimtSeg* segs,
     if (__syncthreads_or(differ) && threadIdx.x == 0) atomicOr(&flags[(size_t)seq * Hkv + kv], 1u);
   }
   // the segments of one sequence are consecutive in the table, which is sorted by
-  // sequence: the first is found by bisection
+  // sequence: both ends are found by bisection, so the loop below knows its length
   const int n = *n_segs;
-  int first = 0, hi = n;
-  while (first < hi) {
-    const int mid = (first + hi) >> 1;
-    if (segs[mid].seq < seq) first = mid + 1;
-    else hi = mid;
-  }
-  for (int slot = first; slot < n && segs[slot].seq == seq; ++slot) {
-    float* pp = ds + ((size_t)slot * Hkv + kv) * D * D + e;
-    const float d = *pp;
-    *pp = s;
-    s = fmaf(expf(lam[((size_t)slot * Hkv + kv) * D + r]), s, d);
+  auto lower = [&](int key) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (segs[mid].seq < key) lo = mid + 1;
+      else hi = mid;
+    }
+    return lo;
+  };
+  const int first = lower(seq), last = lower(seq + 1);
+  // PF segments' dS and log gates are loaded before their serial multiply-adds, so that
+  // the loads of a batch are in flight together
+  constexpr int PF = 8;
+  for (int base = first; base < last; base += PF) {
+    float dv[PF], lv[PF];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (base + u < last) {
+        const size_t su = (size_t)(base + u) * Hkv + kv;
+        dv[u] = ds[su * D * D + e];
+        lv[u] = lam[su * D + r];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (base + u < last) {
+        ds[((size_t)(base + u) * Hkv + kv) * D * D + e] = s;
+        s = fmaf(expf(lv[u]), s, dv[u]);
+      }
+    }
   }
 }
 

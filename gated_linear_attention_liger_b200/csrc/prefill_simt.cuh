@@ -77,6 +77,52 @@ struct SimtRows {
   __device__ __forceinline__ static int at(int e) { return (e / RPG) * RGS + e % RPG; }
 };
 
+// Up to MAXR rows of one head of a [token][head][D] tensor, staged into shared memory in
+// 16-byte pieces: load() issues every load of the calling thread (read-only path), store()
+// converts to fp32 and writes each piece as float4s at dst(row, element).  Calling the
+// load() of several tensors before their store() puts all of a thread's loads in flight
+// together, so a chunk's rows arrive in about one memory latency.
+template <typename Tin, int D, int MAXR, int NT>
+struct RowPieces {
+  static constexpr int EPP = 16 / (int)sizeof(Tin);          // elements per piece
+  static constexpr int PPR = D / EPP;                        // pieces per row
+  static constexpr int MAXP = (MAXR * PPR + NT - 1) / NT;    // pieces per thread
+  uint4 raw[MAXP];
+  __device__ __forceinline__ void load(const Tin* __restrict__ src, size_t row_stride, int n, int tid) {
+#pragma unroll
+    for (int u = 0; u < MAXP; ++u) {
+      const int idx = tid + u * NT;
+      if (idx < n * PPR)
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)(idx / PPR) * row_stride + (idx % PPR) * EPP));
+    }
+  }
+  template <typename Dst>
+  __device__ __forceinline__ void store(int n, int tid, Dst dst) const {
+#pragma unroll
+    for (int u = 0; u < MAXP; ++u) {
+      const int idx = tid + u * NT;
+      if (idx < n * PPR) {
+        float x[EPP];
+        if constexpr (sizeof(Tin) == 2) {
+          const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            x[2 * q] = __uint_as_float(w4[q] << 16);
+            x[2 * q + 1] = __uint_as_float(w4[q] & 0xFFFF0000u);
+          }
+        } else {
+          x[0] = __uint_as_float(raw[u].x); x[1] = __uint_as_float(raw[u].y);
+          x[2] = __uint_as_float(raw[u].z); x[3] = __uint_as_float(raw[u].w);
+        }
+        const int i = idx / PPR, e0 = (idx % PPR) * EPP;
+#pragma unroll
+        for (int e = 0; e < EPP; e += 4)
+          *reinterpret_cast<float4*>(dst(i, e0 + e)) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+      }
+    }
+  }
+};
+
 // VG: one gate per key dimension, sigmoid(k_t[r]) on row r of the state (the
 // per-dimension form of the pooled key gate); otherwise the pooled scalar gate.
 template <int D, bool VG = false>
@@ -148,24 +194,44 @@ __global__ void __launch_bounds__(kSimtThreads) prefill_simt_kernel(SimtPrefillA
                 : make_float4(0.f, 0.f, 0.f, 0.f);
 
   // the window's keys and values before the first token (segmented mode)
-  for (long idx = tid; idx < (sb - max(tb, sb - (w - 1))) * D; idx += NT) {
-    const long t = max(tb, sb - (w - 1)) + idx / D;
-    const int e = (int)(idx % D);
-    const int slot = (int)((t - tb) % RING);
-    ring_k[slot * RS + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
-    ring_v[slot * RS + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
+  {
+    const long tp = max(tb, sb - (w - 1));
+    const int np = (int)(sb - tp);
+    const int slot_p = (int)((tp - tb) % RING);
+    auto ring_row = [&](float* ring) {
+      return [=](int i, int e) {
+        int sl = slot_p + i;
+        sl = sl >= RING ? sl - RING : sl;
+        return ring + sl * RS + e;
+      };
+    };
+    RowPieces<Tin, D, kMaxWindow - 1, NT> pk, pv;
+    pk.load(k + ((size_t)tp * Hkv + kv) * D, (size_t)Hkv * D, np, tid);
+    pv.load(v + ((size_t)tp * Hkv + kv) * D, (size_t)Hkv * D, np, tid);
+    pk.store(np, tid, ring_row(ring_k));
+    pv.store(np, tid, ring_row(ring_v));
   }
 
   for (long t0 = sb; t0 < te; t0 += C) {
     const int n = (int)min((long)C, te - t0);
-    // 1. stage the chunk: q rows, and k/v rows into the window ring
-    for (int idx = tid; idx < n * D; idx += NT) {
-      const int i = idx / D, e = idx % D;
-      const long t = t0 + i;
-      const int slot = (int)((t - tb) % RING);
-      qbuf[idx] = io<Tin>::ld(q + ((size_t)t * Hq + h) * D + e);
-      ring_k[slot * RS + e] = io<Tin>::ld(k + ((size_t)t * Hkv + kv) * D + e);
-      ring_v[slot * RS + e] = io<Tin>::ld(v + ((size_t)t * Hkv + kv) * D + e);
+    // 1. stage the chunk: q rows, and k/v rows into the window ring (every load of a
+    //    thread in flight before its first store)
+    {
+      const int slot_c = (int)((t0 - tb) % RING);
+      auto ring_row = [&](float* ring) {
+        return [=](int i, int e) {
+          int sl = slot_c + i;
+          sl = sl >= RING ? sl - RING : sl;
+          return ring + sl * RS + e;
+        };
+      };
+      RowPieces<Tin, D, C, NT> pq, pk, pv;
+      pq.load(q + ((size_t)t0 * Hq + h) * D, (size_t)Hq * D, n, tid);
+      pk.load(k + ((size_t)t0 * Hkv + kv) * D, (size_t)Hkv * D, n, tid);
+      pv.load(v + ((size_t)t0 * Hkv + kv) * D, (size_t)Hkv * D, n, tid);
+      pq.store(n, tid, [=](int i, int e) { return qbuf + i * D + e; });
+      pk.store(n, tid, ring_row(ring_k));
+      pv.store(n, tid, ring_row(ring_v));
     }
     __syncthreads();
     // 2. feature maps and gate, one warp per token
