@@ -200,6 +200,8 @@ def test_full_tiny_fp32(cuda_device):
     # streamed kernel takes several units and reuses its two stages
     (torch.bfloat16, 128, 40, 90, 4, 40),
     (torch.float32, 64, 64, 70, 2, 50),
+    # w = 1: the window is the current token alone
+    (torch.bfloat16, 128, 1, 20, 2, 7),
 ])
 def test_decode_steps_parity(dtype, d, w, T0, G, B, cuda_device):
     """Oracle prefix -> identical state/ring/pos on both sides -> several decode steps."""
@@ -304,6 +306,7 @@ def test_full_llama8b_decode(cuda_device):
     # ring wrapped (prefix longer than the window), w < 64, several units per CTA
     (torch.bfloat16, 128, 32, 50, 2, 160),
     (torch.float32, 64, 48, 60, 4, 90),
+    (torch.bfloat16, 64, 1, 9, 4, 5),
 ])
 def test_decode_kvshared_parity(dtype, d, w, T0, G, B, cuda_device):
     """One state per kv head: the oracle runs with that state copied to every q head of
