@@ -251,8 +251,8 @@ liger_status liger_attn_prefill_noalloc_status(void);
  */
 
 /*
- * The gated recurrent branch with one gate per key dimension (the survey's
- * vector gate; Paper-Notes page, section 统一的门控线性循环框架: Liger adapts to
+ * The gated recurrent branch with one gate per key dimension (a vector gate;
+ * Paper-Notes page, section 统一的门控线性循环框架: Liger adapts to
  * GLA, Mamba2, mLSTM, HGRN2 and RWKV6 through the form of the gate G_t in
  * S_t = G_t (.) S_{t-1} + phi(k_t)^T v_t).  The pooling of the key is taken per
  * element: G_t[r] = sigmoid(k_t[r]) scales row r (key dimension) of the state,
