@@ -19,6 +19,8 @@
 // Liger Attention; constant-memory decoding: same page, section 亮点与洞察.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -552,7 +554,11 @@ namespace kvs {
 // copy in flight.
 
 constexpr int kConsumers = 256;               // eight consumer warps
-constexpr int kThreads = kConsumers + 64;     // and the producer and feature warps
+// feature warps: the key and half of the queries on one, the other queries on a second
+template <int G>
+constexpr int feature_warps() { return G >= 2 ? 2 : 1; }
+template <int G>
+constexpr int threads() { return kConsumers + 32 + 32 * feature_warps<G>(); }   // + producer, features
 constexpr int kStages = 2;
 
 template <typename Tin, int D, int G>   // G: heads read out per unit
@@ -644,7 +650,7 @@ __device__ __forceinline__ UnitRows unit_rows(long u, int Hq, int Hkv, int D, in
 }
 
 template <typename Tin, int D, int G, bool PER_HEAD>
-__global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
+__global__ void __launch_bounds__(threads<G>(), 1) decode_stream_kernel(Args c) {
   static_assert(!PER_HEAD || G == 1, "a per-head unit reads out one head");
   using L = Layout<Tin, D, G>;
   using sm100::mbar_wait;
@@ -674,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
       sm100::mbar_init(&full[s], 1);
       sm100::mbar_init(&sdone[s], kConsumers);
       sm100::mbar_init(&cons[s], kConsumers);
-      sm100::mbar_init(&featb[s], 32);
+      sm100::mbar_init(&featb[s], 32 * feature_warps<G>());
       sm100::mbar_init(&fullS[s], 1);
     }
     *abort_flag = 0u;
@@ -747,65 +753,90 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(Args c) {
     return;
   }
 
-  if (warp == kConsumers / 32 + 1) {
+  if (warp > kConsumers / 32) {
     // ---------------------------------------------------------------- features
     // phi(k), the gate(s) and phi(q_h) of each unit, and fp32 copies of its q, k and v,
     // into the stage's feature buffer, one unit ahead of the consumers where the copies
-    // allow.  The buffer of stage s is rewritten only after the producer has reloaded
-    // stage s, i.e. after the consumers have released it.
-    for (int i = 0; i < n_local; ++i) {
-      const int s = i % kStages;
-      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-      if (!sm100::warp_all(mbar_wait(&full[s], ph, wc, sm100::wsite(8, 1, i)))) break;
+    // allow.  Feature row 0 is the key (with the gates and the copy of v), rows 1..G the
+    // queries; with two feature warps the first takes rows 0 .. G/2, the second the rest,
+    // each converting the rows it reads.  The buffer of stage s is rewritten only after
+    // the producer has reloaded stage s, i.e. after the consumers have released it.
+    constexpr int EPP = 16 / (int)sizeof(Tin), PPR = D / EPP;
+    auto feature_rows = [&](int s, auto r0c, auto r1c) {
+      constexpr int R0 = decltype(r0c)::value, R1 = decltype(r1c)::value, NR = R1 - R0;
+      constexpr int Q0 = R0 > 0 ? R0 : 1;   // first query row of this warp
       const Tin* qin = reinterpret_cast<const Tin*>(stage(s) + L::STATE + L::RING);
-      // fp32 copies of the q rows, k and v (contiguous on both sides), 16 bytes a step
-      constexpr int EPP = 16 / (int)sizeof(Tin);
-      float* rows = feat(s, L::F_QF);
-      for (int pc = lane; pc < (G + 2) * D / EPP; pc += 32) {
+      float* rows = feat(s, L::F_QF);       // q rows, then k, then v (as in the stage)
+      // fp32 copies, 16 bytes a step: this warp's query rows, and k and v with the key
+      for (int pc = (Q0 - 1) * PPR + lane; pc < (R1 - 1) * PPR; pc += 32) {
         float xv[EPP];
         ld16_vals<Tin>(qin + pc * EPP, xv);
 #pragma unroll
         for (int e = 0; e < EPP; e += 4)
           *reinterpret_cast<float4*>(rows + pc * EPP + e) = make_float4(xv[e], xv[e + 1], xv[e + 2], xv[e + 3]);
       }
+      if (R0 == 0) {
+        for (int pc = G * PPR + lane; pc < (G + 2) * PPR; pc += 32) {
+          float xv[EPP];
+          ld16_vals<Tin>(qin + pc * EPP, xv);
+#pragma unroll
+          for (int e = 0; e < EPP; e += 4)
+            *reinterpret_cast<float4*>(rows + pc * EPP + e) = make_float4(xv[e], xv[e + 1], xv[e + 2], xv[e + 3]);
+        }
+      }
       __syncwarp();
-      // one softmax over d per row (row 0 the key, rows 1..G the queries), EPL consecutive
-      // elements per lane
-      float x[G + 1][EPL], m[G + 1], z[G + 1], sum = 0.f;
+      // one softmax over d per row, EPL consecutive elements per lane
+      float x[NR][EPL], m[NR], z[NR], sum = 0.f;
 #pragma unroll
-      for (int r = 0; r <= G; ++r) {
+      for (int rr = 0; rr < NR; ++rr) {
+        const int r = R0 + rr;
         const float* src = (r == 0 ? rows + G * D : rows + (r - 1) * D) + lane * EPL;
-        m[r] = -INFINITY;
-        z[r] = 0.f;
-        lane_slice_ld<EPL>(src, x[r]);
+        m[rr] = -INFINITY;
+        z[rr] = 0.f;
+        lane_slice_ld<EPL>(src, x[rr]);
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) m[r] = fmaxf(m[r], x[r][j]);
+        for (int j = 0; j < EPL; ++j) m[rr] = fmaxf(m[rr], x[rr][j]);
       }
-      if (PER_HEAD && a.vector_gate) {
-        float* gv = feat(s, L::F_GV) + lane * EPL;
+      if (R0 == 0) {
+        if (PER_HEAD && a.vector_gate) {
+          float* gv = feat(s, L::F_GV) + lane * EPL;
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) gv[j] = expf(log_sigmoid(x[0][j]));
+          for (int j = 0; j < EPL; ++j) gv[j] = expf(log_sigmoid(x[0][j]));
+        }
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) sum += x[0][j];
+        sum = warp_sum(sum);
       }
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) sum += x[0][j];
+      for (int rr = 0; rr < NR; ++rr) m[rr] = warp_max(m[rr]);
 #pragma unroll
-      for (int r = 0; r <= G; ++r) m[r] = warp_max(m[r]);
-      sum = warp_sum(sum);
+      for (int rr = 0; rr < NR; ++rr)
 #pragma unroll
-      for (int r = 0; r <= G; ++r)
+        for (int j = 0; j < EPL; ++j) { x[rr][j] = expf(x[rr][j] - m[rr]); z[rr] += x[rr][j]; }
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) { x[r][j] = expf(x[r][j] - m[r]); z[r] += x[r][j]; }
+      for (int rr = 0; rr < NR; ++rr) z[rr] = warp_sum(z[rr]);
 #pragma unroll
-      for (int r = 0; r <= G; ++r) z[r] = warp_sum(z[r]);
-#pragma unroll
-      for (int r = 0; r <= G; ++r) {
+      for (int rr = 0; rr < NR; ++rr) {
+        const int r = R0 + rr;
         float* dst = (r == 0 ? feat(s, L::F_FK) : feat(s, L::F_FQ) + (r - 1) * D) + lane * EPL;
         float y[EPL];
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) y[j] = x[r][j] / z[r];
+        for (int j = 0; j < EPL; ++j) y[j] = x[rr][j] / z[rr];
         lane_slice_st<EPL>(dst, y);
       }
-      if (lane == 0) *feat(s, L::F_G) = expf(log_sigmoid(sum / (float)D));
+      if (R0 == 0 && lane == 0) *feat(s, L::F_G) = expf(log_sigmoid(sum / (float)D));
+    };
+    constexpr int RSPLIT = feature_warps<G>() == 2 ? 1 + G / 2 : G + 1;   // rows of the first warp
+    const int fw = warp - kConsumers / 32 - 1;
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i % kStages;
+      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+      if (!sm100::warp_all(mbar_wait(&full[s], ph, wc, sm100::wsite(8, 1 + fw, i)))) break;
+      if (fw == 0) {
+        feature_rows(s, std::integral_constant<int, 0>{}, std::integral_constant<int, RSPLIT>{});
+      } else if constexpr (feature_warps<G>() == 2) {
+        feature_rows(s, std::integral_constant<int, RSPLIT>{}, std::integral_constant<int, G + 1>{});
+      }
       sm100::mbar_arrive(&featb[s]);   // every lane: its own writes are released
     }
     return;

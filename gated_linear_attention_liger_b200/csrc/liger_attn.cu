@@ -201,7 +201,7 @@ liger_status launch_decode_stream(const liger::DecodeArgs& a, unsigned units, cu
   const int sms = liger::tc::num_sms();
   const unsigned grid = units < (unsigned)sms ? units : (unsigned)sms;   // one CTA per SM
   mark_start(s);
-  if (launch_pdl(kern, dim3(grid), dim3(liger::kvs::kThreads), smem, s, c) != cudaSuccess)
+  if (launch_pdl(kern, dim3(grid), dim3(liger::kvs::threads<G>()), smem, s, c) != cudaSuccess)
     return cuda_check("decode_stream launch");
   mark_stop(s);
   ++g_launches;
