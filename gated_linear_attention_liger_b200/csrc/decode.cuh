@@ -547,7 +547,8 @@ namespace kvs {
 // unit's fp32 state, its window ring (keys, then values, w slots each, in slot
 // order) and the step's rows q_h (NH of them), k and v into one of two
 // shared-memory stages by bulk copies, so that the next unit's bytes are in
-// flight while eight consumer warps compute this one.  The updated state goes
+// flight while eight consumer warps compute this one; one or two feature warps
+// prepare each unit's feature maps and gates ahead of them.  The updated state goes
 // back to HBM by bulk copies as soon as the consumers have written it, before
 // they run the window branch.  Every wait is bounded; a wait that gives up
 // records the timeout in the device error word and the CTA winds down with no
@@ -574,7 +575,7 @@ struct Layout {
   static constexpr uint32_t PART = RGN * G * D * 4;              // readout partial sums
   static constexpr uint32_t WSUM = WV::NW * G * D * 4;           // window partial sums (same room)
   static constexpr uint32_t SCRATCH = PART > WSUM ? PART : WSUM;
-  // per stage, written by the feature warp: phi(q_h) [G][D], q_h in fp32 [G][D], phi(k),
+  // per stage, written by the feature warps: phi(q_h) [G][D], q_h in fp32 [G][D], phi(k),
   // k and v in fp32, the per-row gates [D] each, the scalar gate
   // (q_h, k and v in fp32 are contiguous: one converted copy of the stage's rows)
   static constexpr uint32_t F_FQ = 0, F_FK = F_FQ + G * D * 4, F_GV = F_FK + D * 4;
